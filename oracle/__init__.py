@@ -1,0 +1,24 @@
+"""CPU oracle for query-aware top-k selective attention (ESA and MoBA forms).
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package. The CUDA library never
+calls it, and it never calls the CUDA library: the two share no code, headers,
+helpers or constants. Both receive their inputs from
+``query_aware_selective_b200.synthetic``.
+
+Everything here is plain numpy in float64: slow, literal, and written so that it
+can be checked against the pages by eye.
+
+* ``oracle.esa``  - Efficient Selective Attention ("Efficient Selective Attention"
+  article, implementation section): compression, importance score, score
+  correction, chunk sum, neighbour influence, top-k, attention over
+  initial + selected + local tokens.
+* ``oracle.moba`` - Mixture of Block Attention (MoBA article, sections 1-3):
+  block mean pooling, gate, causal top-k, block attention.
+
+Pins: every function here is checked by ``tests/test_oracle_*.py`` against
+closed forms, library routines (torch SDPA in float64), brute force on tiny
+inputs, hand-worked examples and invariants. Parity that the pages cannot fix
+(the clamp constant C, the region boundary, MoBA's off-by-one) is stated as a
+reading in the docstrings of the functions concerned.
+"""

@@ -1,0 +1,235 @@
+"""Seeded synthetic inputs for query-aware selective attention.
+
+This module only draws random tensors and fixes the workload shapes. It is
+imported by the tests, the benchmark and the smoke check, and it is the one
+module that both the CUDA path and the CPU oracle receive their inputs from.
+It computes none of the method's steps: no compression of stored tensors, no
+scoring, no selection and no attention. The single piece of linear algebra in
+here aims the planted needle keys (see ``plant_needles``), which is part of how
+the input is built, not something any output is checked against.
+
+Shapes follow the attention layers the ESA write-up evaluates on
+(Llama-3-8B-Instruct / Mistral-7B-Instruct-v0.2: 32 query heads, 8 KV heads,
+head dim 128, hidden 4096; "Efficient Selective Attention" article, experiment
+section) and the MoBA article's 64-block setting (MoBA article, "experiments",
+the fixed-sparsity scaling figure). The benchmarks those pages use (LongBench,
+InfiniteBench, NeedleBench) are not available; these tensors stand in for them.
+
+Recipe, for every workload: one ``torch.Generator`` seeded with the workload's
+seed draws, in this order, Q, K, V (standard normal, in the workload dtype),
+then W_q and W_k (normal with variance 1/in_dim, fp32), then the needle
+positions. Needle keys overwrite K at those positions.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class EsaWorkload:
+    """Shape and parameters of one ESA workload (decode or chunked prefill)."""
+
+    name: str
+    batch: int
+    hq: int
+    hkv: int
+    head_dim: int
+    n_ctx: int          # tokens in the KV cache when the step runs
+    chunk: int          # prefill chunk length; 1 for decode
+    d_c: int            # compressed dimension d'
+    n_init: int
+    window: int
+    topk: int
+    eps: int
+    clamp_c: float      # +inf disables the clamp
+    n_needles: int
+    dtype: str          # "f32" or "bf16"
+    seed: int
+    mode: str           # "decode" or "prefill"
+
+    @property
+    def hidden(self) -> int:
+        return self.hq * self.head_dim
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+
+@dataclasses.dataclass(frozen=True)
+class MobaWorkload:
+    """Shape and parameters of one MoBA causal prefill workload."""
+
+    name: str
+    batch: int
+    heads: int
+    head_dim: int
+    seq: int
+    block: int
+    topk: int           # past blocks selected per (query, head); the current block is extra
+    dtype: str
+    seed: int
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+
+def default_clamp(d_c: int) -> float:
+    """Default clamp bound C of the score correction: 4 * sqrt(d')."""
+    return 4.0 * math.sqrt(d_c)
+
+
+TINY_DECODE = EsaWorkload("esa_tiny_decode_n2048_f32", 1, 4, 4, 64, 2048, 1, 16,
+                          16, 256, 128, 2, default_clamp(16), 3, "f32", 0, "decode")
+PREFILL_32K = EsaWorkload("esa_prefill_llama3_8b_ctx32768_chunk512", 1, 32, 8, 128, 32768, 512,
+                          128, 128, 4096, 2048, 2, default_clamp(128), 0, "bf16", 1, "prefill")
+DECODE_128K = EsaWorkload("esa_decode_llama3_8b_b16_ctx131072", 16, 32, 8, 128, 131072, 1,
+                          128, 128, 4096, 2048, 2, default_clamp(128), 8, "bf16", 2, "decode")
+MOBA_64K = MobaWorkload("moba_prefill_h32_seq65536_block1024_top3", 1, 32, 128, 65536, 1024, 3,
+                        "bf16", 3)
+DECODE_1M = EsaWorkload("esa_decode_mistral_7b_b4_ctx1048576", 4, 32, 8, 128, 1048576, 1,
+                        128, 128, 4096, 2048, 2, default_clamp(128), 16, "bf16", 4, "decode")
+
+WORKLOADS = {w.name: w for w in (TINY_DECODE, PREFILL_32K, DECODE_128K, MOBA_64K, DECODE_1M)}
+
+
+def local_start(c0: int, n_init: int, window: int) -> int:
+    """First position of the local part for a chunk starting at c0 (region rule).
+
+    Initial = [0, min(n_init, lo)), middle = [n_init, lo), local = [lo, c1),
+    lo = min(c0, max(n_init, c0 - window)). This is a shape rule shared by the
+    generator (needle placement) and callers; it involves no data.
+    """
+    return min(c0, max(n_init, c0 - window))
+
+
+def _randn(shape, dtype, gen, device):
+    return torch.randn(shape, generator=gen, device=device, dtype=torch.float32).to(dtype) \
+        if dtype == torch.float32 else torch.randn(shape, generator=gen, device=device, dtype=dtype)
+
+
+def make_esa_inputs(w: EsaWorkload, device="cpu", n_ctx: Optional[int] = None,
+                    batch: Optional[int] = None) -> dict:
+    """Draw Q, K, V, W_q, W_k (and plant needles) for an ESA workload.
+
+    Decode: q is [B, 1, Hq, D] for position N-1; k, v are [B, N, Hkv, D].
+    Prefill: q is [B, N, Hq, D] for every position; k, v as above.
+    ``n_ctx``/``batch`` shrink the workload for small tests (same recipe).
+    """
+    n = n_ctx or w.n_ctx
+    b = batch or w.batch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed)
+    dt = w.torch_dtype
+    lq = 1 if w.mode == "decode" else n
+    q = _randn((b, lq, w.hq, w.head_dim), dt, gen, device)
+    k = _randn((b, n, w.hkv, w.head_dim), dt, gen, device)
+    v = _randn((b, n, w.hkv, w.head_dim), dt, gen, device)
+    std = 1.0 / math.sqrt(w.hidden)
+    wq = torch.randn((w.hidden, w.d_c), generator=gen, device=device, dtype=torch.float32) * std
+    wk = torch.randn((w.hidden, w.d_c), generator=gen, device=device, dtype=torch.float32) * std
+    out = dict(q=q, k=k, v=v, wq=wq, wk=wk, needles=None)
+    if w.n_needles and w.mode == "decode":
+        out["needles"] = plant_needles(w, q, k, wq, wk, gen)
+    return out
+
+
+def needle_positions(w: EsaWorkload, n_ctx: int, gen: torch.Generator) -> torch.Tensor:
+    """Needle positions per sequence: one per equal segment of the middle,
+    at least eps from either edge of the segment (hence >= 2*eps+1 apart)."""
+    c0 = n_ctx - 1
+    lo = local_start(c0, w.n_init, w.window)
+    mid0, mid1 = w.n_init, lo
+    seg = (mid1 - mid0) // w.n_needles
+    assert seg >= 2 * w.eps + 2, "middle too short for the needles"
+    r = torch.randint(0, seg - 2 * w.eps, (w.n_needles,), generator=gen,
+                      device=gen.device).cpu()
+    base = torch.arange(w.n_needles) * seg + mid0 + w.eps
+    return base + r
+
+
+def plant_needles(w: EsaWorkload, q, k, wq, wk, gen) -> torch.Tensor:
+    """Overwrite K at the needle positions with keys aimed at the query.
+
+    A needle key (the same vector for every KV head's slot of its group layout)
+    is beta * u / |u| with u the direction in raw key space along which the
+    compressed score of the decode query grows fastest: u = d(score)/d(key).
+    beta = 3 * sqrt(Hkv * D). Returns the positions, [B, n_needles] int64.
+    """
+    b, n = k.shape[0], k.shape[1]
+    g = w.hq // w.hkv
+    pos = torch.empty((b, w.n_needles), dtype=torch.int64)
+    beta = 3.0 * math.sqrt(w.hkv * w.head_dim)
+    for s in range(b):
+        p = needle_positions(w, n, gen)
+        pos[s] = p
+        qf = q[s, 0].reshape(-1).float()                          # [Hq*D]
+        qc = qf @ wq                                              # aim point in compressed space
+        grad_expanded = (wk @ qc).reshape(w.hq, w.head_dim)       # d score / d expanded key
+        u = grad_expanded.reshape(w.hkv, g, w.head_dim).sum(1)    # fold the GQA copies
+        key = (beta * u / u.norm()).to(k.dtype)
+        k[s, p.to(k.device)] = key.unsqueeze(0).expand(len(p), -1, -1)
+    return pos
+
+
+def make_moba_inputs(w: MobaWorkload, device="cpu", seq: Optional[int] = None,
+                     heads: Optional[int] = None, batch: Optional[int] = None) -> dict:
+    """Draw Q, K, V ([B, S, H, D]) for a MoBA workload."""
+    s = seq or w.seq
+    h = heads or w.heads
+    b = batch or w.batch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed)
+    dt = w.torch_dtype
+    q = _randn((b, s, h, w.head_dim), dt, gen, device)
+    k = _randn((b, s, h, w.head_dim), dt, gen, device)
+    v = _randn((b, s, h, w.head_dim), dt, gen, device)
+    return dict(q=q, k=k, v=v)
+
+
+def random_index_list(batch: int, mid0: int, mid1: int, topk: int, seed: int) -> tuple:
+    """A valid selection result drawn at random: per sequence, min(topk, |mid|)
+    distinct middle positions, ascending, padded with -1. Used to test the
+    attention call on its own. Returns (idx [B, topk] int32, count [B] int32)."""
+    gen = torch.Generator()
+    gen.manual_seed(seed)
+    n = max(0, mid1 - mid0)
+    cnt = min(topk, n)
+    idx = torch.full((batch, topk), -1, dtype=torch.int32)
+    for b in range(batch):
+        sel = torch.randperm(n, generator=gen)[:cnt].sort().values + mid0
+        idx[b, :cnt] = sel.to(torch.int32)
+    return idx, torch.full((batch,), cnt, dtype=torch.int32)
+
+
+def random_block_lists(batch: int, seq: int, heads: int, block: int, topk: int,
+                       seed: int) -> torch.Tensor:
+    """Valid MoBA block lists drawn at random: for a query in block c, min(topk, c)
+    distinct past blocks, ascending, then c, then -1 padding.
+    Returns [B, S, H, topk+1] int16."""
+    gen = torch.Generator()
+    gen.manual_seed(seed)
+    out = torch.full((batch, seq, heads, topk + 1), -1, dtype=torch.int16)
+    cur = torch.arange(seq) // block
+    keys = torch.rand((batch, seq, heads, max(1, (seq + block - 1) // block)), generator=gen)
+    nb = keys.shape[-1]
+    blk = torch.arange(nb)
+    # past blocks only: push current and future blocks to the end
+    keys = keys.masked_fill(blk.view(1, 1, 1, nb) >= cur.view(1, seq, 1, 1), 2.0)
+    order = keys.argsort(dim=-1)[..., :topk]
+    cnt = torch.clamp(cur, max=topk)
+    valid = torch.arange(topk).view(1, 1, 1, topk) < cnt.view(1, seq, 1, 1)
+    order = torch.where(valid, order, torch.full_like(order, 1 << 14))
+    order = order.sort(dim=-1).values
+    order = torch.where(order == (1 << 14), torch.full_like(order, -1), order)
+    out[..., :topk] = order.to(torch.int16)
+    # the current block goes right after the last valid past block
+    for c in range(topk + 1):
+        mask = cnt == c
+        out[:, mask, :, c] = cur[mask].to(torch.int16).view(1, -1, 1)
+    return out
