@@ -1,0 +1,204 @@
+/*
+ * esa.h - C ABI of libesa: query-aware top-k selective attention on B200 (sm_100a).
+ *
+ * Two forms of the method:
+ *   ESA  - Efficient Selective Attention (Huawei Noah's Ark write-up, arXiv 2502.14477):
+ *          compress query and key with a one-layer linear map, score every middle
+ *          cached token against the current chunk's queries in that low-dimensional
+ *          space, correct each query's scores, sum over the chunk, lift each score by
+ *          its neighbours, keep the top-k, and attend exactly over initial + selected +
+ *          local tokens.
+ *   MoBA - Mixture of Block Attention (MoBA article, arXiv 2502.13189): a gate picks
+ *          the top-k past blocks by <q, mean-pooled block keys>, the current block is
+ *          always added with a causal mask, and attention runs over those blocks.
+ *
+ * Conventions for every call:
+ *   - Every tensor pointer is DEVICE memory owned by the caller. The library never
+ *     allocates, frees or keeps a pointer after the call returns. Scratch memory is
+ *     passed in through `workspace`; its size comes from the matching *_workspace_size
+ *     call, and it needs 256-byte alignment.
+ *   - Tensors are dense and row-major in the order the shapes are written. q, k, v, o
+ *     need 16-byte aligned base pointers; compressed tensors (q_c, k_c) too.
+ *   - `stream` is a cudaStream_t passed as an opaque pointer (NULL = legacy default
+ *     stream). Every call only enqueues work on it and returns; none synchronises.
+ *   - Arguments are checked on the host before anything is launched. A bad argument
+ *     returns ESA_ERR_INVALID_ARG (or ESA_ERR_WORKSPACE / ESA_ERR_UNSUPPORTED) and
+ *     launches nothing. A failed launch returns ESA_ERR_CUDA. esa_last_error() then
+ *     gives a message (thread-local, valid until the next call on the same thread).
+ *   - Kernels that wait on barriers wait a bounded time. If a wait runs out, the
+ *     kernel records ESA_ERR_TIMEOUT in a device status word and returns without
+ *     hanging; esa_device_status() reads and clears that word.
+ *   - Calls are thread-compatible: calls on different streams may overlap only if
+ *     they use different workspaces and write different outputs.
+ *
+ * Citations name the page and passage each operation follows.
+ */
+#ifndef ESA_H_
+#define ESA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ESA_OK = 0,
+  ESA_ERR_INVALID_ARG = 1,  /* a shape, pointer, alignment or parameter is wrong */
+  ESA_ERR_UNSUPPORTED = 2,  /* valid, but this build has no kernel for it (e.g. head_dim 96) */
+  ESA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  ESA_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out (see esa_device_status) */
+  ESA_ERR_WORKSPACE = 5     /* workspace is NULL, misaligned or smaller than required */
+} esa_status_t;
+
+typedef enum { ESA_F32 = 0, ESA_BF16 = 1 } esa_dtype_t;
+
+/* ESA selection parameters.
+ *   n_init  - initial tokens always attended (ESA write-up, implementation paragraph:
+ *             the sequence is split into initial, middle, local and current parts)
+ *   window  - local tokens before the chunk that are always attended
+ *   topk    - middle tokens kept (ESA write-up, core steps: a fixed number of tokens)
+ *   eps     - neighbour radius of the neighbour-influence step (ESA write-up,
+ *             neighbour-influence paragraph; read as a max over +-eps)
+ *   clamp_c - lower bound -C of each query's max-shifted score (ESA write-up,
+ *             score-correction paragraph); +INFINITY disables the clamp.
+ * Regions of a chunk [c0, c1) (c1 = c0 + lq):
+ *   lo = min(c0, max(n_init, c0 - window));
+ *   initial = [0, min(n_init, lo)), middle = [n_init, lo), local = [lo, c1) (causal). */
+typedef struct {
+  int32_t n_init;
+  int32_t window;
+  int32_t topk;
+  int32_t eps;
+  float clamp_c;
+} esa_params_t;
+
+/* ---------------------------------------------------------------- ESA calls -- */
+
+/* esa_compress - one-layer linear map of the merged heads (ESA write-up, core-steps
+ * and implementation paragraphs: q and k pass through a one-layer MLP, 4096 -> 128).
+ *   y[r, :] = concat_{h < n_heads_out} x[r, h / G, :] @ W,   G = n_heads_out / n_heads_in
+ * i.e. under GQA each query head h reads KV head h / G (keys are expanded to the
+ * query-head count before the map). No bias, no activation.
+ *   x:  rows of [n_heads_in, head_dim], dtype x_dtype (ESA_F32 or ESA_BF16); row r starts
+ *       at element r * x_row_stride (x_row_stride >= n_heads_in * head_dim, a multiple of 8),
+ *       so one call can read the new key of every sequence of a batched cache
+ *   w:  [n_heads_out * head_dim, d_out] fp32
+ *   y:  rows of d_out fp32, row r at y + r * y_row_stride (y_row_stride >= d_out), so a
+ *       call can write straight into a compressed key cache at any row offset.
+ * Requires head_dim in {64, 128}, d_out % 16 == 0, d_out <= 256, rows >= 0 (0 = no-op).
+ * Accumulates in fp32. */
+esa_status_t esa_compress(const void* x, esa_dtype_t x_dtype, int64_t rows, int64_t x_row_stride,
+                          int32_t n_heads_in, int32_t n_heads_out, int32_t head_dim,
+                          const float* w, int32_t d_out, float* y, int64_t y_row_stride,
+                          void* stream);
+
+/* esa_score_select - importance score, correction, chunk sum, neighbour max-pool and
+ * top-k for one chunk of every sequence in a batch (ESA write-up, implementation,
+ * score-correction and neighbour-influence paragraphs).
+ *   S_ij = q_c[b, i] . k_c[b, j]                 for i < lq, j in middle
+ *   m_i  = max_j S_ij
+ *   s_j  = sum_i max(S_ij - m_i, -clamp_c)
+ *   s'_j = max_{m in middle, |m - j| <= eps} s_m
+ *   keep min(topk, |middle|) tokens by (s' descending, position ascending)
+ *   q_c:       [batch, lq, d_c] fp32, compressed queries at positions [c0, c0 + lq)
+ *   k_c:       [batch, n_cap, d_c] fp32, compressed key cache; rows [0, c0 + lq) valid
+ *   idx_out:   [batch, topk] int32 absolute positions, ascending, -1 after count
+ *   count_out: [batch] int32 = min(topk, |middle|) (the same for every sequence)
+ *   score_out: NULL, or [batch, |middle|] fp32 receiving s' (for checking)
+ * Requires d_c % 16 == 0 and d_c <= 256, 1 <= lq <= 4096, c0 + lq <= n_cap,
+ * topk >= 1, 0 <= eps <= 64. An empty middle gives count 0 and all -1. */
+esa_status_t esa_score_select(const float* q_c, const float* k_c, int32_t batch, int32_t lq,
+                              int64_t n_cap, int64_t c0, int32_t d_c, esa_params_t p,
+                              int32_t* idx_out, int32_t* count_out, float* score_out,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+size_t esa_score_select_workspace_size(int32_t batch, int32_t lq, int64_t n_cap, int64_t c0,
+                                       int32_t d_c, esa_params_t p);
+
+/* esa_sparse_attn - exact attention over initial + selected + local tokens (ESA
+ * write-up, implementation and final-attention paragraphs: initial and selected
+ * tokens form the global part, local tokens the window part, fused into one output
+ * with the full queries, keys and values). One softmax over the union; causal inside
+ * the local part; GQA: query head h reads KV head h / (hq / hkv).
+ *   q:     [batch, lq, hq, head_dim]   queries at positions [c0, c0 + lq)
+ *   k, v:  [batch, n_cap, hkv, head_dim]; rows [0, c0 + lq) valid
+ *   idx:   [batch, >= p.topk] int32 selected middle positions, ascending (as
+ *          esa_score_select writes them); count: [batch] int32 entries used
+ *   o:     [batch, lq, hq, head_dim], dtype dt
+ *   lse:   NULL or [batch, lq, hq] fp32, natural log of the softmax denominator
+ *   scale: softmax scale; <= 0 means 1/sqrt(head_dim)
+ * Requires head_dim in {64, 128}, hq % hkv == 0, c0 + lq <= n_cap. The selected
+ * positions must lie in the middle region; entries are not re-checked on the device. */
+esa_status_t esa_sparse_attn(const void* q, const void* k, const void* v, esa_dtype_t dt,
+                             int32_t batch, int32_t lq, int64_t n_cap, int64_t c0,
+                             int32_t hq, int32_t hkv, int32_t head_dim,
+                             const int32_t* idx, const int32_t* count, esa_params_t p,
+                             float scale, void* o, float* lse,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+size_t esa_sparse_attn_workspace_size(int32_t batch, int32_t lq, int64_t c0, int32_t hq,
+                                      int32_t hkv, int32_t head_dim, esa_dtype_t dt,
+                                      esa_params_t p);
+
+/* --------------------------------------------------------------- MoBA calls -- */
+
+/* moba_block_gate - block choice of MoBA (MoBA article, section 3: blocks of size
+ * `block`, gate s_i = <q, mean_pool(K[block i])>, top-k gate, causality).
+ * Block b covers [b*block, min((b+1)*block, seq)). For a query at position p in block
+ * c = p / block, the candidates are the past blocks 0..c-1 (reading: "strictly before
+ * the query's block"); the kept ones are the top min(topk, c) by (score descending,
+ * block ascending); the current block c is always added.
+ *   q, k:       [batch, seq, heads, head_dim], dtype dt
+ *   blocks_out: [batch, seq, heads, topk + 1] int16: attended blocks ascending (the
+ *               current block last), then -1.
+ * Requires head_dim in {64, 128}, block >= 16 and a multiple of 16,
+ * 0 <= topk <= 15, seq / block <= 1024 blocks. Means and scores are fp32. */
+esa_status_t moba_block_gate(const void* q, const void* k, esa_dtype_t dt, int32_t batch,
+                             int64_t seq, int32_t heads, int32_t head_dim, int32_t block,
+                             int32_t topk, int16_t* blocks_out,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* moba_block_attn - attention of each (query, head) over the blocks listed for it
+ * (MoBA article, section 2: MoBA(q, K, V) = Softmax(q K[I]^T) V[I]); the current
+ * block is cut causally at the query (section 3, causality). Scale as esa_sparse_attn.
+ *   blocks: [batch, seq, heads, topk + 1] int16 as moba_block_gate writes them.
+ *   o:      [batch, seq, heads, head_dim] dtype dt; lse: NULL or [batch, seq, heads] fp32. */
+esa_status_t moba_block_attn(const void* q, const void* k, const void* v, esa_dtype_t dt,
+                             int32_t batch, int64_t seq, int32_t heads, int32_t head_dim,
+                             int32_t block, int32_t topk, const int16_t* blocks, float scale,
+                             void* o, float* lse, void* workspace, size_t ws_bytes,
+                             void* stream);
+
+/* moba_block_gate_attn - the whole MoBA causal prefill: moba_block_gate then
+ * moba_block_attn. blocks_out may be NULL (the lists then live in the workspace). */
+esa_status_t moba_block_gate_attn(const void* q, const void* k, const void* v, esa_dtype_t dt,
+                                  int32_t batch, int64_t seq, int32_t heads, int32_t head_dim,
+                                  int32_t block, int32_t topk, float scale, void* o, float* lse,
+                                  int16_t* blocks_out, void* workspace, size_t ws_bytes,
+                                  void* stream);
+
+/* Workspace bytes for moba_block_gate (which = 0), moba_block_attn (1) and
+ * moba_block_gate_attn (2). */
+size_t moba_workspace_size(int32_t which, int32_t batch, int64_t seq, int32_t heads,
+                           int32_t head_dim, int32_t block, int32_t topk);
+
+/* ------------------------------------------------------------------- status -- */
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char* esa_last_error(void);
+
+/* Waits for `stream`, then reads and clears the device status word of the current
+ * device. Returns ESA_OK, or ESA_ERR_TIMEOUT if a kernel's bounded wait ran out since
+ * the last read (the message names the kernel and the wait). */
+esa_status_t esa_device_status(void* stream);
+
+/* Library version string. */
+const char* esa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ESA_H_ */

@@ -207,17 +207,17 @@ def sparse_attn(q, k, v, c0, idx, count, n_init, window, scale=None, rows=None):
         keys = attended_keys(c0, lq, n_init, window, idx[b], int(count[b]))
         kk = np.asarray(k[b, keys], dtype=np.float64)     # [L, Hkv, D]
         vv = np.asarray(v[b, keys], dtype=np.float64)
-        kh = kk[:, head_map, :]                           # [L, Hq, D]
-        vh = vv[:, head_map, :]
+        kh = np.ascontiguousarray(kk[:, head_map, :].transpose(1, 0, 2))   # [Hq, L, D]
+        vh = np.ascontiguousarray(vv[:, head_map, :].transpose(1, 0, 2))
         for i in items:
             p = c0 + i
             vis = keys <= p
             qi = np.asarray(q[b, i], dtype=np.float64)    # [Hq, D]
-            logits = np.einsum("hd,lhd->hl", qi, kh[vis]) * scale
+            logits = np.matmul(kh[:, vis, :], qi[:, :, None])[:, :, 0] * scale   # [Hq, L']
             mx = logits.max(axis=1, keepdims=True)
             e = np.exp(logits - mx)
             den = e.sum(axis=1, keepdims=True)
-            o[b, i] = np.einsum("hl,lhd->hd", e / den, vh[vis])
+            o[b, i] = np.matmul((e / den)[:, None, :], vh[:, vis, :])[:, 0, :]
             lse[b, i] = (mx + np.log(den))[:, 0]
     return o, lse
 

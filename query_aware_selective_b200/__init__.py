@@ -1,0 +1,12 @@
+"""Query-aware top-k selective attention (ESA and MoBA forms) on B200 (sm_100a).
+
+The compute path is libesa.so (C ABI in include/esa.h, CUDA kernels in csrc/);
+this package only marshals torch tensors into it. ``synthetic`` draws the seeded
+benchmark inputs; ``cost`` holds the algorithmic byte and flop counts used for
+rooflines.
+"""
+from ._abi import (EsaError, EsaParams, compress, device_status, load, moba_block_attn, moba_block_gate,
+                   moba_block_gate_attn, params, score_select, sparse_attn)
+
+__all__ = ["EsaError", "EsaParams", "compress", "device_status", "load", "moba_block_attn", "moba_block_gate",
+           "moba_block_gate_attn", "params", "score_select", "sparse_attn"]

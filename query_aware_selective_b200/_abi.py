@@ -1,0 +1,260 @@
+"""Thin ctypes binding of libesa (include/esa.h).
+
+Argument marshalling only: every step of the path runs in libesa's CUDA kernels.
+Outputs and workspaces are torch tensors (the caller's device memory); a function
+allocates them when the caller passes none. There is no CPU fallback: without the
+built library, or without a CUDA device, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libesa.so")
+
+ESA_OK, ESA_ERR_INVALID_ARG, ESA_ERR_UNSUPPORTED, ESA_ERR_CUDA, ESA_ERR_TIMEOUT, ESA_ERR_WORKSPACE = range(6)
+ESA_F32, ESA_BF16 = 0, 1
+
+# Every exported function of include/esa.h: name -> (restype, argtypes)
+_vp, _i32, _i64, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+
+
+class EsaParams(ctypes.Structure):
+    """esa_params_t: n_init, window, topk, eps, clamp_c (+inf = no clamp)."""
+
+    _fields_ = [("n_init", ctypes.c_int32), ("window", ctypes.c_int32), ("topk", ctypes.c_int32),
+                ("eps", ctypes.c_int32), ("clamp_c", ctypes.c_float)]
+
+
+SIGNATURES = {
+    "esa_compress": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i32, _i32, _i32, _vp, _i32, _vp, _i64, _vp]),
+    "esa_score_select": (ctypes.c_int, [_vp, _vp, _i32, _i32, _i64, _i64, _i32, EsaParams, _vp, _vp, _vp,
+                                        _vp, _sz, _vp]),
+    "esa_score_select_workspace_size": (_sz, [_i32, _i32, _i64, _i64, _i32, EsaParams]),
+    "esa_sparse_attn": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i64, _i64, _i32, _i32, _i32,
+                                       _vp, _vp, EsaParams, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "esa_sparse_attn_workspace_size": (_sz, [_i32, _i32, _i64, _i32, _i32, _i32, ctypes.c_int, EsaParams]),
+    "moba_block_gate": (ctypes.c_int, [_vp, _vp, ctypes.c_int, _i32, _i64, _i32, _i32, _i32, _i32, _vp, _vp,
+                                       _sz, _vp]),
+    "moba_block_attn": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i64, _i32, _i32, _i32, _i32, _vp,
+                                       _f32, _vp, _vp, _vp, _sz, _vp]),
+    "moba_block_gate_attn": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i64, _i32, _i32, _i32, _i32,
+                                            _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moba_workspace_size": (_sz, [_i32, _i32, _i64, _i32, _i32, _i32, _i32]),
+    "esa_last_error": (ctypes.c_char_p, []),
+    "esa_device_status": (ctypes.c_int, [_vp]),
+    "esa_version": (ctypes.c_char_p, []),
+}
+
+_lib = None
+
+
+class EsaError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        super().__init__(f"{where}: status {status}: {message}")
+        self.status = status
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libesa and declare every signature. Raises if the library is missing."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libesa is not built ({path} missing); run __graft_entry__.build()")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def _check(status: int, where: str):
+    if status != ESA_OK:
+        raise EsaError(status, where, load().esa_last_error().decode())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return ESA_F32
+    if t.dtype == torch.bfloat16:
+        return ESA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _dev(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("libesa takes CUDA tensors (no CPU path)")
+            if not t.is_contiguous():
+                raise ValueError("libesa takes contiguous tensors")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _workspace(nbytes: int, device, ws: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
+    if nbytes == 0:
+        return ws
+    if ws is not None and ws.numel() * ws.element_size() >= nbytes:
+        return ws
+    return torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+
+
+def _ws_ptr(ws: Optional[torch.Tensor]) -> tuple:
+    if ws is None:
+        return None, 0
+    p = ws.data_ptr()
+    pad = (-p) % 256
+    return p + pad, ws.numel() * ws.element_size() - pad
+
+
+def params(n_init: int, window: int, topk: int, eps: int, clamp_c: float = math.inf) -> EsaParams:
+    return EsaParams(n_init, window, topk, eps, clamp_c)
+
+
+def compress(x: torch.Tensor, w: torch.Tensor, n_heads_out: int, out: Optional[torch.Tensor] = None,
+             out_row_stride: Optional[int] = None) -> torch.Tensor:
+    """esa_compress. x: [rows, Hin, D] (f32 or bf16; each row contiguous, rows may be
+    strided); w: [Hout*D, d'] f32 -> [rows, d'] f32. With `out` given, rows are written
+    at out + r * out_row_stride (default d')."""
+    if not x.is_cuda or not w.is_cuda or not w.is_contiguous():
+        raise ValueError("libesa takes CUDA tensors (no CPU path); w must be contiguous")
+    rows, hin, d = x.shape
+    if x.stride(2) != 1 or x.stride(1) != d:
+        raise ValueError("each row of x must be contiguous [Hin, D]")
+    dout = w.shape[1]
+    if out is None:
+        out = torch.empty((rows, dout), dtype=torch.float32, device=x.device)
+        stride = dout
+    else:
+        stride = out_row_stride or dout
+    _check(load().esa_compress(_ptr(x), _dtype_code(x), rows, x.stride(0) if rows > 1 else hin * d, hin,
+                               n_heads_out, d, _ptr(w), dout, _ptr(out), stride, _stream()), "esa_compress")
+    return out
+
+
+def score_select_workspace_size(batch, lq, n_cap, c0, d_c, p: EsaParams) -> int:
+    return load().esa_score_select_workspace_size(batch, lq, n_cap, c0, d_c, p)
+
+
+def score_select(q_c: torch.Tensor, k_c: torch.Tensor, c0: int, p: EsaParams, want_scores: bool = False,
+                 idx: Optional[torch.Tensor] = None, count: Optional[torch.Tensor] = None,
+                 scores: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None):
+    """esa_score_select. q_c [B, Lq, d'] f32, k_c [B, n_cap, d'] f32.
+    Returns (idx [B, topk] int32, count [B] int32, s' [B, n_mid] f32 or None)."""
+    _dev(q_c, k_c)
+    b, lq, dc = q_c.shape
+    n_cap = k_c.shape[1]
+    dev = q_c.device
+    if idx is None:
+        idx = torch.empty((b, p.topk), dtype=torch.int32, device=dev)
+    if count is None:
+        count = torch.empty((b,), dtype=torch.int32, device=dev)
+    if want_scores and scores is None:
+        lo = min(c0, max(p.n_init, c0 - p.window))
+        scores = torch.empty((b, max(0, lo - p.n_init)), dtype=torch.float32, device=dev)
+    ws = _workspace(score_select_workspace_size(b, lq, n_cap, c0, dc, p), dev, workspace)
+    wp, wn = _ws_ptr(ws)
+    _check(load().esa_score_select(_ptr(q_c), _ptr(k_c), b, lq, n_cap, c0, dc, p, _ptr(idx), _ptr(count),
+                                   _ptr(scores) if want_scores else None, wp, wn, _stream()), "esa_score_select")
+    return idx, count, (scores if want_scores else None)
+
+
+def sparse_attn_workspace_size(batch, lq, c0, hq, hkv, d, dtype_code, p: EsaParams) -> int:
+    return load().esa_sparse_attn_workspace_size(batch, lq, c0, hq, hkv, d, dtype_code, p)
+
+
+def sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, c0: int, idx: torch.Tensor,
+                count: torch.Tensor, p: EsaParams, scale: float = 0.0, want_lse: bool = False,
+                out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None):
+    """esa_sparse_attn. q [B, Lq, Hq, D]; k, v [B, n_cap, Hkv, D]; idx [B, >=topk] int32.
+    Returns (o [B, Lq, Hq, D], lse [B, Lq, Hq] f32 or None)."""
+    _dev(q, k, v, idx, count)
+    b, lq, hq, d = q.shape
+    n_cap, hkv = k.shape[1], k.shape[2]
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((b, lq, hq), dtype=torch.float32, device=q.device)
+    ws = _workspace(sparse_attn_workspace_size(b, lq, c0, hq, hkv, d, dt, p), q.device, workspace)
+    wp, wn = _ws_ptr(ws)
+    _check(load().esa_sparse_attn(_ptr(q), _ptr(k), _ptr(v), dt, b, lq, n_cap, c0, hq, hkv, d, _ptr(idx),
+                                  _ptr(count), p, scale, _ptr(out), _ptr(lse) if want_lse else None, wp, wn,
+                                  _stream()), "esa_sparse_attn")
+    return out, (lse if want_lse else None)
+
+
+def moba_workspace_size(which, batch, seq, heads, d, block, topk) -> int:
+    return load().moba_workspace_size(which, batch, seq, heads, d, block, topk)
+
+
+def moba_block_gate(q, k, block: int, topk: int, out=None, workspace=None) -> torch.Tensor:
+    """moba_block_gate -> blocks [B, S, H, topk+1] int16."""
+    _dev(q, k)
+    b, s, h, d = q.shape
+    if out is None:
+        out = torch.empty((b, s, h, topk + 1), dtype=torch.int16, device=q.device)
+    ws = _workspace(moba_workspace_size(0, b, s, h, d, block, topk), q.device, workspace)
+    wp, wn = _ws_ptr(ws)
+    _check(load().moba_block_gate(_ptr(q), _ptr(k), _dtype_code(q), b, s, h, d, block, topk, _ptr(out), wp, wn,
+                                  _stream()), "moba_block_gate")
+    return out
+
+
+def moba_block_attn(q, k, v, block: int, topk: int, blocks: torch.Tensor, scale: float = 0.0,
+                    want_lse: bool = False, out=None, lse=None, workspace=None):
+    """moba_block_attn -> (o [B, S, H, D], lse [B, S, H] or None)."""
+    _dev(q, k, v, blocks)
+    b, s, h, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((b, s, h), dtype=torch.float32, device=q.device)
+    ws = _workspace(moba_workspace_size(1, b, s, h, d, block, topk), q.device, workspace)
+    wp, wn = _ws_ptr(ws)
+    _check(load().moba_block_attn(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), b, s, h, d, block, topk, _ptr(blocks),
+                                  scale, _ptr(out), _ptr(lse) if want_lse else None, wp, wn, _stream()),
+           "moba_block_attn")
+    return out, (lse if want_lse else None)
+
+
+def moba_block_gate_attn(q, k, v, block: int, topk: int, scale: float = 0.0, want_blocks: bool = False,
+                         want_lse: bool = False, out=None, lse=None, blocks=None, workspace=None):
+    """moba_block_gate_attn -> (o, lse or None, blocks or None)."""
+    _dev(q, k, v)
+    b, s, h, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((b, s, h), dtype=torch.float32, device=q.device)
+    if want_blocks and blocks is None:
+        blocks = torch.empty((b, s, h, topk + 1), dtype=torch.int16, device=q.device)
+    ws = _workspace(moba_workspace_size(2, b, s, h, d, block, topk), q.device, workspace)
+    wp, wn = _ws_ptr(ws)
+    _check(load().moba_block_gate_attn(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), b, s, h, d, block, topk, scale,
+                                       _ptr(out), _ptr(lse) if want_lse else None,
+                                       _ptr(blocks) if want_blocks else None, wp, wn, _stream()),
+           "moba_block_gate_attn")
+    return out, (lse if want_lse else None), (blocks if want_blocks else None)
+
+
+def device_status() -> None:
+    """Raise EsaError if a kernel's bounded wait ran out since the last check."""
+    _check(load().esa_device_status(_stream()), "esa_device_status")

@@ -1,0 +1,365 @@
+// attn_tc.cuh - tensor-core attention over an indexed key list (sm_100a tcgen05).
+//
+// One CTA computes 128 query rows against a list of key rows, 128 keys per step:
+//   S_j  = Q K_j^T          tcgen05.mma kind::f16 (bf16 in, fp32 accumulate), TMEM
+//   P_j  = exp2(S_j * c - m) softmax warps read S_j from TMEM, write bf16 P_j to smem
+//   PV_j = P_j V_j          tcgen05.mma into a second TMEM buffer
+//   o    = o * alpha + PV_j the softmax warps accumulate o in registers (one row each)
+// Roles (224 threads): warps 0-3 softmax (thread = row = TMEM lane), warp 4 issues
+// the MMAs (one lane), warp 5 loads Q and the K rows, warp 6 loads the V rows.
+// K/V rows are gathered by cp.async (16-byte pieces) straight into the 128-byte
+// swizzled layout the MMA descriptors name; loaders wait for their own copies and
+// fence to the async proxy before arriving on the "full" barrier.
+//
+// Shared memory: Q 32 KB, K 2 x 32 KB, V 2 x 32 KB, P 2 x 32 KB (each operand tile is
+// two 16 KB column blocks of 128 rows x 128 bytes). TMEM: S double buffer (2 x 128
+// columns) and PV double buffer (2 x 128 columns) = 512 columns.
+//
+// The problem policy P says which rows and keys a CTA owns:
+//   bool setup(): per-CTA fields; false = nothing to do
+//   const bf16* q_row(int r): row r's query (nullptr: padding row)
+//   int64_t kv_row(int64_t t): element offset of key t's K/V row (t < n_keys())
+//   int64_t n_keys(); int64_t limit(int r): last key index row r may attend
+//   void store(int r, const float* o, float m2, float l): o is unnormalised,
+//        m2 the running max in log2 units, l the denominator
+#pragma once
+#include "common.cuh"
+#include "keylist.cuh"
+
+namespace esa {
+
+constexpr int kTcThreads = 224;
+constexpr int kTcRows = 128;
+constexpr int kTcKeys = 128;
+constexpr int kTcD = 128;
+constexpr uint32_t kTileBytes = 128 * 256;            // 128 rows x 128 bf16
+constexpr uint32_t kBlkBytes = 128 * 128;             // one 64-column block of a tile
+constexpr uint32_t kTcSmemBytes = 7 * kTileBytes + 1024 /*align*/ + 512 /*barriers*/;
+
+struct TcSmem {
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
+  uint64_t pv_full[2], pv_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// Copy one 128 x 128 bf16 tile (rows given by a functor returning the element offset
+// of the row or -1) into swizzled shared memory. 32 threads; lane owns chunk lane % 16
+// of rows lane / 16, lane / 16 + 2, ...
+template <typename RowFn>
+__device__ __forceinline__ void load_tile_rows(uint32_t dst, const __nv_bfloat16* base, RowFn row_off, int lane) {
+  const int ch = lane & 15;
+  const uint32_t blk = (ch >> 3) * kBlkBytes;
+  const uint32_t cc = ch & 7;
+#pragma unroll 4
+  for (int r = lane >> 4; r < 128; r += 2) {
+    const int64_t off = row_off(r);
+    const void* src = off >= 0 ? (const void*)(base + off + ch * 8) : (const void*)base;
+    cp_async16(dst + blk + sw128_off(r, cc), src, off >= 0 ? 16u : 0u);
+  }
+}
+
+template <class Problem>
+__global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(Problem prob) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sQ = smem_u32(smem);
+  const uint32_t sK = sQ + kTileBytes;       // 2 stages
+  const uint32_t sV = sK + 2 * kTileBytes;   // 2 stages
+  const uint32_t sP = sV + 2 * kTileBytes;   // 2 buffers
+  TcSmem& sm = *reinterpret_cast<TcSmem*>(smem + 7 * kTileBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (!prob.setup()) return;
+  const int64_t n_keys = prob.n_keys();
+  const int nt = (int)((n_keys + kTcKeys - 1) / kTcKeys);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.q_full, 32);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.k_full[s], 32);
+      mbar_init(&sm.v_full[s], 32);
+      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
+      mbar_init(&sm.s_full[s], 1);
+      mbar_init(&sm.s_empty[s], 128);
+      mbar_init(&sm.p_full[s], 128);
+      mbar_init(&sm.p_empty[s], 1);
+      mbar_init(&sm.pv_full[s], 1);
+      mbar_init(&sm.pv_empty[s], 128);
+    }
+    mbar_init(&sm.mma_done, 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+
+  if (warp == 5) {
+    // ---------------------------------------------------------------- Q + K loader
+    load_tile_rows(sQ, prob.q_base(), [&](int r) -> int64_t { return prob.q_row(r); }, lane);
+    cp_async_commit();
+    cp_async_wait_all();
+    fence_proxy_async();
+    mbar_arrive(&sm.q_full);
+    bool ok = true;
+    for (int j = 0; j < nt && ok; ++j) {
+      const int s = j & 1;
+      ok = mbar_wait(&sm.k_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, 101);
+      if (!ok) break;
+      const int64_t t0 = (int64_t)j * kTcKeys;
+      load_tile_rows(sK + s * kTileBytes, prob.kv_base_k(),
+                     [&](int r) -> int64_t { return t0 + r < n_keys ? prob.kv_row(t0 + r) : -1; }, lane);
+      cp_async_commit();
+      if (j >= 1) {
+        cp_async_wait<1>();
+        fence_proxy_async();
+        mbar_arrive(&sm.k_full[(j - 1) & 1]);
+      }
+    }
+    cp_async_wait_all();
+    if (ok && nt > 0) {
+      fence_proxy_async();
+      mbar_arrive(&sm.k_full[(nt - 1) & 1]);
+    }
+  } else if (warp == 6) {
+    // ---------------------------------------------------------------- V loader
+    bool ok = true;
+    for (int j = 0; j < nt && ok; ++j) {
+      const int s = j & 1;
+      ok = mbar_wait(&sm.v_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, 102);
+      if (!ok) break;
+      const int64_t t0 = (int64_t)j * kTcKeys;
+      load_tile_rows(sV + s * kTileBytes, prob.kv_base_v(),
+                     [&](int r) -> int64_t { return t0 + r < n_keys ? prob.kv_row(t0 + r) : -1; }, lane);
+      cp_async_commit();
+      if (j >= 1) {
+        cp_async_wait<1>();
+        fence_proxy_async();
+        mbar_arrive(&sm.v_full[(j - 1) & 1]);
+      }
+    }
+    cp_async_wait_all();
+    if (ok && nt > 0) {
+      fence_proxy_async();
+      mbar_arrive(&sm.v_full[(nt - 1) & 1]);
+    }
+  } else if (warp == 4) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = umma_idesc(kFmtBF16, 128, 128, 0, 0);
+      constexpr uint32_t idesc_pv = umma_idesc(kFmtBF16, 128, 128, 0, 1);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j & 1;
+        if (!mbar_wait(&sm.k_full[s], (j >> 1) & 1, abort_flag, 103)) return false;
+        if (!mbar_wait(&sm.s_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, 104)) return false;
+        tc_fence_after();
+        const uint32_t kt = sK + s * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (kk >> 2) * kBlkBytes + (kk & 3) * 32;
+          umma_f16_ss(tmem + s * 128, sdesc_sw128(sQ + koff, 16, 1024), sdesc_sw128(kt + koff, 16, 1024),
+                      idesc_qk, kk > 0);
+        }
+        umma_commit(&sm.s_full[s]);
+        umma_commit(&sm.k_empty[s]);
+        return true;
+      };
+      bool ok = nt == 0 || mbar_wait(&sm.q_full, 0, abort_flag, 105);
+      if (ok && nt > 0) ok = issue_s(0);
+      for (int j = 0; j < nt && ok; ++j) {
+        const int s = j & 1;
+        if (j + 1 < nt && !(ok = issue_s(j + 1))) break;
+        if (!(ok = mbar_wait(&sm.p_full[s], (j >> 1) & 1, abort_flag, 106))) break;
+        if (!(ok = mbar_wait(&sm.v_full[s], (j >> 1) & 1, abort_flag, 107))) break;
+        if (!(ok = mbar_wait(&sm.pv_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, 108))) break;
+        tc_fence_after();
+        const uint32_t pt = sP + s * kTileBytes;
+        const uint32_t vt = sV + s * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          // A = P (K-major: keys along the 128-byte rows); B = V (MN-major: 8-key row
+          // groups of 1024 bytes, d blocks of 64 columns 16 KB apart)
+          const uint32_t poff = (kk >> 2) * kBlkBytes + (kk & 3) * 32;
+          umma_f16_ss(tmem + 256 + s * 128, sdesc_sw128(pt + poff, 16, 1024),
+                      sdesc_sw128(vt + kk * 2048, kBlkBytes, 1024), idesc_pv, kk > 0);
+        }
+        umma_commit(&sm.pv_full[s]);
+        umma_commit(&sm.p_empty[s]);
+        umma_commit(&sm.v_empty[s]);
+      }
+      // every MMA issued so far has completed before TMEM is released
+      umma_commit(&sm.mma_done);
+      mbar_wait(&sm.mma_done, 0, abort_flag, 109, /*respect_abort=*/false);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- softmax (rows)
+    const int r = threadIdx.x;                 // 0..127 = TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const int64_t lim = prob.limit(r);
+    const float sl2 = prob.scale_log2();
+    float o[kTcD];
+#pragma unroll
+    for (int e = 0; e < kTcD; ++e) o[e] = 0.f;
+    float m = -INFINITY, l = 0.f, alpha_pend = 0.f;
+    bool ok = true;
+    auto consume_pv = [&](int j) -> bool {
+      const int s = j & 1;
+      if (!mbar_wait_warp(&sm.pv_full[s], (j >> 1) & 1, abort_flag, 110)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float x[32];
+        tmem_ld32(lane_base + 256 + s * 128 + c * 32, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[c * 32 + e] = fmaf(o[c * 32 + e], alpha_pend, x[e]);
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.pv_empty[s]);
+      return true;
+    };
+    for (int j = 0; j < nt; ++j) {
+      const int s = j & 1;
+      if (!(ok = mbar_wait_warp(&sm.s_full[s], (j >> 1) & 1, abort_flag, 111))) break;
+      tc_fence_after();
+      const int64_t t0 = (int64_t)j * kTcKeys;
+      const uint32_t sa = lane_base + s * 128;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float x[32];
+        tmem_ld32(sa + c * 32, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int64_t t = t0 + c * 32 + e;
+          mx = fmaxf(mx, t <= lim ? x[e] * sl2 : -INFINITY);
+        }
+      }
+      const float m_new = fmaxf(m, mx);
+      const float m_use = m_new == -INFINITY ? 0.f : m_new;
+      const float alpha = fast_exp2(m - m_use);
+      if (!(ok = mbar_wait_warp(&sm.p_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, 112))) break;
+      const uint32_t pt = sP + s * kTileBytes;
+      float lsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float x[32];
+        tmem_ld32(sa + c * 32, x);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int64_t t = t0 + c * 32 + e;
+          const float p0 = t <= lim ? fast_exp2(x[e] * sl2 - m_use) : 0.f;
+          const float p1 = t + 1 <= lim ? fast_exp2(x[e + 1] * sl2 - m_use) : 0.f;
+          lsum += p0 + p1;
+          pk[e / 2] = pack_bf16x2(p0, p1);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int chunk = c * 4 + q;                 // 16-byte chunk of the 256-byte row
+          const uint32_t dst = pt + (chunk >> 3) * kBlkBytes + sw128_off(r, chunk & 7);
+          st_shared_v4(dst, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.s_empty[s]);
+      fence_proxy_async();
+      mbar_arrive(&sm.p_full[s]);
+      l = l * alpha + lsum;
+      m = m_new;
+      if (j >= 1 && !(ok = consume_pv(j - 1))) break;
+      alpha_pend = alpha;
+    }
+    if (ok && nt > 0) ok = consume_pv(nt - 1);
+    if (ok) prob.store(r, o, m, l);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 4) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ ESA problem --
+// CTA (row tile, KV head g, sequence b). Row R = tile * 128 + r packs (query i, head
+// in group hl) as i = R / G, hl = R % G, so each loaded K/V row serves G query heads.
+struct EsaTcProblem {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  __nv_bfloat16* o;
+  float* lse;
+  KeyList keys;
+  int64_t n_cap, c0;
+  int lq, hq, hkv, G;
+  float sl2;
+  // per CTA
+  int b, g, tile, cnt;
+  int64_t n_prior, nk;
+
+  __device__ bool setup() {
+    tile = blockIdx.x;
+    g = blockIdx.y;
+    b = blockIdx.z;
+    cnt = min(max(keys.count[b], 0), (int)keys.idx_stride);
+    n_prior = keys.ni + cnt + (c0 - keys.lo);
+    const int rows = lq * G;
+    if (tile * kTcRows >= rows) return false;
+    const int imax = min(lq - 1, (tile * kTcRows + kTcRows - 1) / G);
+    nk = n_prior + imax + 1;
+    return true;
+  }
+  __device__ const __nv_bfloat16* q_base() const { return q; }
+  __device__ const __nv_bfloat16* kv_base_k() const { return k; }
+  __device__ const __nv_bfloat16* kv_base_v() const { return v; }
+  __device__ int64_t q_row(int r) const {
+    const int R = tile * kTcRows + r;
+    if (R >= lq * G) return -1;
+    const int i = R / G, hl = R % G;
+    return (((int64_t)b * lq + i) * hq + g * G + hl) * kTcD;
+  }
+  __device__ int64_t kv_row(int64_t t) const {
+    const int64_t p = keys.pos(b, cnt, t);
+    return (((int64_t)b * n_cap + p) * hkv + g) * kTcD;
+  }
+  __device__ int64_t n_keys() const { return nk; }
+  __device__ int64_t limit(int r) const {
+    const int R = tile * kTcRows + r;
+    return n_prior + min(R / G, lq - 1);
+  }
+  __device__ float scale_log2() const { return sl2; }
+  __device__ void store(int r, const float* acc, float m2, float l) {
+    const int R = tile * kTcRows + r;
+    if (R >= lq * G) return;
+    const int i = R / G, hl = R % G;
+    const int64_t row = ((int64_t)b * lq + i) * hq + g * G + hl;
+    const float inv = 1.f / l;
+    uint4* dst = reinterpret_cast<uint4*>(o + row * kTcD);
+#pragma unroll
+    for (int c = 0; c < kTcD / 8; ++c) {
+      uint4 w;
+      w.x = pack_bf16x2(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
+      w.y = pack_bf16x2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
+      w.z = pack_bf16x2(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv);
+      w.w = pack_bf16x2(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
+      dst[c] = w;
+    }
+    if (lse) lse[row] = (m2 + __log2f(l)) * 0.69314718055994531f;
+  }
+};
+
+}  // namespace esa

@@ -1,0 +1,634 @@
+// esa_lib.cu - the C ABI of libesa (include/esa.h): argument checks, workspace
+// layout and kernel launches. Every kernel lives in the .cuh files included here, so
+// the library is one translation unit with one copy of the device status word.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "../../include/esa.h"
+#include "attn_simt.cuh"
+#include "attn_tc.cuh"
+#include "common.cuh"
+#include "compress.cuh"
+#include "moba.cuh"
+#include "score.cuh"
+#include "topk.cuh"
+
+namespace {
+
+thread_local std::string g_err;
+
+esa_status_t fail(esa_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
+esa_status_t ok() {
+  g_err.clear();
+  return ESA_OK;
+}
+
+esa_status_t check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ESA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return ESA_OK;
+}
+
+#define ESA_LAUNCH_CHECK(what)                         \
+  do {                                                 \
+    const esa_status_t st_ = check_launch(what);       \
+    if (st_ != ESA_OK) return st_;                     \
+  } while (0)
+
+#define ESA_CUDA(call)                                                               \
+  do {                                                                               \
+    const cudaError_t e_ = (call);                                                   \
+    if (e_ != cudaSuccess) return fail(ESA_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Region rule of a chunk [c0, c1): lo = min(c0, max(n_init, c0 - window)).
+struct Regions {
+  int64_t lo, ni, mid0, n_mid;
+};
+Regions regions(int64_t c0, const esa_params_t& p) {
+  Regions r;
+  r.lo = std::min<int64_t>(c0, std::max<int64_t>(p.n_init, c0 - p.window));
+  r.ni = std::min<int64_t>(p.n_init, r.lo);
+  r.mid0 = p.n_init;
+  r.n_mid = std::max<int64_t>(0, r.lo - p.n_init);
+  return r;
+}
+
+// Carves a workspace into 256-byte aligned regions in a fixed order.
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  template <typename T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += up256(count * sizeof(T));
+    return p;
+  }
+};
+
+template <typename K>
+esa_status_t set_max_smem(K kernel, int bytes) {
+  ESA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  return ESA_OK;
+}
+
+esa_status_t check_params(const esa_params_t& p) {
+  if (p.n_init < 0 || p.window < 0) return fail(ESA_ERR_INVALID_ARG, "n_init and window must be >= 0");
+  if (p.topk < 1) return fail(ESA_ERR_INVALID_ARG, "topk must be >= 1 (got %d)", p.topk);
+  if (p.eps < 0 || p.eps > 64) return fail(ESA_ERR_INVALID_ARG, "eps must be in [0, 64] (got %d)", p.eps);
+  if (std::isnan(p.clamp_c) || p.clamp_c < 0.f) return fail(ESA_ERR_INVALID_ARG, "clamp_c must be >= 0 or +inf");
+  return ESA_OK;
+}
+
+// ------------------------------------------------------------------ score_select --
+struct SelWs {
+  float* S;
+  float* s;
+  uint32_t* u;
+  uint32_t* m_key;
+  uint32_t* hist;
+  esa::SelState* st;
+  uint2* tiles;
+  size_t bytes;
+  size_t zero_bytes;   // m_key + hist are contiguous and cleared together
+};
+
+SelWs carve_select(void* ws, int32_t batch, int32_t lq, int64_t n_mid) {
+  Carver c{reinterpret_cast<uint8_t*>(ws)};
+  SelWs w;
+  const int64_t n_tiles = cdiv(std::max<int64_t>(n_mid, 1), esa::kTkTile);
+  w.m_key = c.take<uint32_t>((size_t)batch * lq);
+  const size_t zero_start = 0;
+  w.hist = c.take<uint32_t>((size_t)batch * 3 * esa::kTkBins);
+  w.zero_bytes = c.off - zero_start;
+  w.S = c.take<float>((size_t)batch * lq * n_mid);
+  w.s = c.take<float>((size_t)batch * n_mid);
+  w.u = c.take<uint32_t>((size_t)batch * n_mid);
+  w.st = c.take<esa::SelState>((size_t)batch);
+  w.tiles = c.take<uint2>((size_t)batch * n_tiles);
+  w.bytes = c.off;
+  return w;
+}
+
+template <int DC>
+void launch_score_small(const float* q_c, const float* k_c, int lq, int64_t n_cap, int64_t mid0, int64_t n_mid,
+                        int batch, float* S, uint32_t* m_key, cudaStream_t s) {
+  const int64_t keys_per_cta = 512;
+  dim3 grid((unsigned)cdiv(n_mid, keys_per_cta), batch);
+  if (lq == 1)
+    esa::score_small_kernel<DC, 1><<<grid, 256, 0, s>>>(q_c, k_c, lq, n_cap, mid0, n_mid, keys_per_cta, S, m_key);
+  else
+    esa::score_small_kernel<DC, esa::kScoreSmallLq><<<grid, 256, 0, s>>>(q_c, k_c, lq, n_cap, mid0, n_mid,
+                                                                         keys_per_cta, S, m_key);
+}
+
+}  // namespace
+
+// Every exported function below is declared extern "C" in esa.h, which gives these
+// definitions C linkage.
+
+const char* esa_version(void) { return "libesa 0.1 (sm_100a)"; }
+
+const char* esa_last_error(void) { return g_err.c_str(); }
+
+esa_status_t esa_device_status(void* stream) {
+  ESA_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  unsigned long long v = 0;
+  ESA_CUDA(cudaMemcpyFromSymbol(&v, esa::g_status, sizeof(v)));
+  if (v == 0) return ok();
+  const unsigned long long zero = 0;
+  ESA_CUDA(cudaMemcpyToSymbol(esa::g_status, &zero, sizeof(zero)));
+  return fail(ESA_ERR_TIMEOUT, "device wait ran out at site %u (status %u)", (unsigned)(v & 0xffffffffu),
+              (unsigned)(v >> 32));
+}
+
+// ------------------------------------------------------------------ esa_compress --
+esa_status_t esa_compress(const void* x, esa_dtype_t x_dtype, int64_t rows, int64_t x_row_stride,
+                          int32_t n_heads_in, int32_t n_heads_out, int32_t head_dim, const float* w, int32_t d_out,
+                          float* y, int64_t y_row_stride, void* stream) {
+  if (rows < 0) return fail(ESA_ERR_INVALID_ARG, "rows must be >= 0");
+  if (rows == 0) return ok();
+  if (!x || !w || !y) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  if (x_dtype != ESA_F32 && x_dtype != ESA_BF16) return fail(ESA_ERR_INVALID_ARG, "bad dtype %d", (int)x_dtype);
+  if (n_heads_in <= 0 || n_heads_out <= 0 || n_heads_out % n_heads_in)
+    return fail(ESA_ERR_INVALID_ARG, "n_heads_out (%d) must be a positive multiple of n_heads_in (%d)", n_heads_out,
+                n_heads_in);
+  if (head_dim != 64 && head_dim != 128) return fail(ESA_ERR_UNSUPPORTED, "head_dim %d (64 or 128)", head_dim);
+  if (d_out <= 0 || d_out % 16 || d_out > 256) return fail(ESA_ERR_UNSUPPORTED, "d_out %d (multiple of 16, <= 256)", d_out);
+  if (y_row_stride < d_out) return fail(ESA_ERR_INVALID_ARG, "y_row_stride < d_out");
+  if (x_row_stride < (int64_t)n_heads_in * head_dim || x_row_stride % 8)
+    return fail(ESA_ERR_INVALID_ARG, "x_row_stride must be >= n_heads_in * head_dim and a multiple of 8");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int ct = d_out % 32 == 0 ? 32 : 16;
+  dim3 grid((unsigned)cdiv(rows, esa::kCmpRT), d_out / ct);
+  if (x_dtype == ESA_F32) {
+    if (ct == 32)
+      esa::compress_kernel<float, 32><<<grid, esa::kCmpThreads, 0, s>>>(static_cast<const float*>(x), rows, x_row_stride, n_heads_in,
+                                                                       n_heads_out, head_dim, w, d_out, y, y_row_stride);
+    else
+      esa::compress_kernel<float, 16><<<grid, esa::kCmpThreads, 0, s>>>(static_cast<const float*>(x), rows, x_row_stride, n_heads_in,
+                                                                       n_heads_out, head_dim, w, d_out, y, y_row_stride);
+  } else {
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+    if (ct == 32)
+      esa::compress_kernel<__nv_bfloat16, 32><<<grid, esa::kCmpThreads, 0, s>>>(xb, rows, x_row_stride, n_heads_in, n_heads_out,
+                                                                               head_dim, w, d_out, y, y_row_stride);
+    else
+      esa::compress_kernel<__nv_bfloat16, 16><<<grid, esa::kCmpThreads, 0, s>>>(xb, rows, x_row_stride, n_heads_in, n_heads_out,
+                                                                               head_dim, w, d_out, y, y_row_stride);
+  }
+  ESA_LAUNCH_CHECK("compress_kernel");
+  return ok();
+}
+
+// ------------------------------------------------------------------ score_select --
+size_t esa_score_select_workspace_size(int32_t batch, int32_t lq, int64_t n_cap, int64_t c0, int32_t d_c,
+                                       esa_params_t p) {
+  (void)n_cap;
+  (void)d_c;
+  if (batch <= 0 || lq <= 0) return 0;
+  const Regions r = regions(c0, p);
+  return carve_select(nullptr, batch, lq, r.n_mid).bytes;
+}
+
+esa_status_t esa_score_select(const float* q_c, const float* k_c, int32_t batch, int32_t lq, int64_t n_cap,
+                              int64_t c0, int32_t d_c, esa_params_t p, int32_t* idx_out, int32_t* count_out,
+                              float* score_out, void* workspace, size_t ws_bytes, void* stream) {
+  esa_status_t st = check_params(p);
+  if (st != ESA_OK) return st;
+  if (batch <= 0) return fail(ESA_ERR_INVALID_ARG, "batch must be >= 1");
+  if (lq < 1 || lq > 4096) return fail(ESA_ERR_INVALID_ARG, "lq must be in [1, 4096] (got %d)", lq);
+  if (c0 < 0 || c0 + lq > n_cap) return fail(ESA_ERR_INVALID_ARG, "need 0 <= c0 and c0 + lq <= n_cap");
+  if (d_c <= 0 || d_c % 16 || d_c > 256) return fail(ESA_ERR_UNSUPPORTED, "d_c %d (multiple of 16, <= 256)", d_c);
+  if (!q_c || !k_c || !idx_out || !count_out) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(q_c, 16) || !aligned(k_c, 16)) return fail(ESA_ERR_INVALID_ARG, "q_c and k_c need 16-byte alignment");
+  const Regions r = regions(c0, p);
+  if (r.n_mid > (int64_t)1 << 30) return fail(ESA_ERR_UNSUPPORTED, "middle longer than 2^30 tokens");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t kk = std::min<int64_t>(p.topk, r.n_mid);
+  const bool need_scores = r.n_mid > p.topk || (score_out && r.n_mid > 0);
+  if (need_scores) {
+    const SelWs need = carve_select(nullptr, batch, lq, r.n_mid);
+    if (!workspace || ws_bytes < need.bytes || !aligned(workspace, 256))
+      return fail(ESA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need.bytes, ws_bytes);
+    const SelWs w = carve_select(workspace, batch, lq, r.n_mid);
+    ESA_CUDA(cudaMemsetAsync(w.m_key, 0, w.zero_bytes, s));
+    const bool small = lq <= esa::kScoreSmallLq && (d_c == 16 || d_c == 32 || d_c == 64 || d_c == 128 || d_c == 256);
+    if (small) {
+      switch (d_c) {
+        case 16: launch_score_small<16>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, w.S, w.m_key, s); break;
+        case 32: launch_score_small<32>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, w.S, w.m_key, s); break;
+        case 64: launch_score_small<64>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, w.S, w.m_key, s); break;
+        case 128: launch_score_small<128>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, w.S, w.m_key, s); break;
+        default: launch_score_small<256>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, w.S, w.m_key, s); break;
+      }
+    } else {
+      dim3 grid((unsigned)cdiv(r.n_mid, esa::kScT), (unsigned)cdiv(lq, esa::kScT), batch);
+      esa::score_tiled_kernel<<<grid, 256, 0, s>>>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, d_c, w.S, w.m_key);
+    }
+    ESA_LAUNCH_CHECK("score kernel");
+    esa::clamp_sum_kernel<<<dim3((unsigned)cdiv(r.n_mid, 256), batch), 256, 0, s>>>(w.S, w.m_key, lq, r.n_mid,
+                                                                                    p.clamp_c, w.s);
+    ESA_LAUNCH_CHECK("clamp_sum_kernel");
+    const int n_tiles = (int)cdiv(r.n_mid, esa::kTkTile);
+    const dim3 tgrid(n_tiles, batch);
+    esa::pool_hist_kernel<<<tgrid, esa::kTkThreads, 0, s>>>(w.s, r.n_mid, p.eps, w.u, score_out, w.hist);
+    ESA_LAUNCH_CHECK("pool_hist_kernel");
+    if (r.n_mid > p.topk) {
+      for (int level = 0; level < 3; ++level) {
+        if (level > 0) {
+          esa::radix_hist_kernel<<<tgrid, esa::kTkThreads, 0, s>>>(w.u, r.n_mid, level, w.st, w.hist);
+          ESA_LAUNCH_CHECK("radix_hist_kernel");
+        }
+        esa::radix_select_kernel<<<batch, 1024, 0, s>>>(w.hist, level, (uint32_t)kk, w.st);
+        ESA_LAUNCH_CHECK("radix_select_kernel");
+      }
+      esa::compact_count_kernel<<<tgrid, esa::kTkThreads, 0, s>>>(w.u, r.n_mid, w.st, w.tiles, n_tiles);
+      ESA_LAUNCH_CHECK("compact_count_kernel");
+      esa::compact_write_kernel<<<tgrid, esa::kTkThreads, 0, s>>>(w.u, r.n_mid, w.st, w.tiles, n_tiles, r.mid0,
+                                                                  p.topk, idx_out);
+      ESA_LAUNCH_CHECK("compact_write_kernel");
+    }
+  }
+  const bool all_mid = r.n_mid <= p.topk;
+  esa::fill_selection_kernel<<<dim3((unsigned)std::max<int64_t>(1, cdiv(p.topk, 256)), batch), 256, 0, s>>>(
+      idx_out, count_out, p.topk, (int)kk, r.mid0, all_mid ? 1 : 0);
+  ESA_LAUNCH_CHECK("fill_selection_kernel");
+  return ok();
+}
+
+// ------------------------------------------------------------------ sparse_attn --
+namespace {
+
+struct AttnPlan {
+  bool tc;
+  int nsplit;
+  int64_t keys_per_split;
+  size_t ws_bytes;
+};
+
+AttnPlan plan_attn(int32_t batch, int32_t lq, int64_t c0, int32_t hq, int32_t hkv, int32_t head_dim, esa_dtype_t dt,
+                   const esa_params_t& p) {
+  AttnPlan pl{};
+  const Regions r = regions(c0, p);
+  const int g = hq / hkv;
+  pl.tc = dt == ESA_BF16 && head_dim == 128 && (int64_t)lq * g >= 64;
+  if (pl.tc) return pl;
+  const int64_t n_keys_max = r.ni + std::min<int64_t>(p.topk, r.n_mid) + (c0 - r.lo) + lq;
+  const int64_t base = (int64_t)batch * lq * hkv;
+  const int64_t want_ctas = 4 * 148;
+  int64_t per = std::max<int64_t>(256, cdiv(n_keys_max, std::max<int64_t>(1, want_ctas / base)));
+  per = cdiv(per, 64) * 64;
+  pl.keys_per_split = per;
+  pl.nsplit = (int)cdiv(n_keys_max, per);
+  pl.ws_bytes = pl.nsplit > 1 ? up256((size_t)batch * lq * hq * pl.nsplit * (head_dim + 2) * sizeof(float)) : 0;
+  return pl;
+}
+
+template <typename T, int D, int G>
+void launch_simt(const esa::SimtAttnArgs& a, int batch, cudaStream_t s) {
+  dim3 grid(a.nsplit, a.hkv, batch * a.lq);
+  esa::attn_simt_kernel<T, D, G><<<grid, esa::kSimtWarps * 32, 0, s>>>(a);
+}
+
+template <typename T, int D>
+bool dispatch_simt_g(const esa::SimtAttnArgs& a, int g, int batch, cudaStream_t s) {
+  switch (g) {
+    case 1: launch_simt<T, D, 1>(a, batch, s); return true;
+    case 2: launch_simt<T, D, 2>(a, batch, s); return true;
+    case 4: launch_simt<T, D, 4>(a, batch, s); return true;
+    case 8: launch_simt<T, D, 8>(a, batch, s); return true;
+    default: return false;
+  }
+}
+
+}  // namespace
+
+size_t esa_sparse_attn_workspace_size(int32_t batch, int32_t lq, int64_t c0, int32_t hq, int32_t hkv,
+                                      int32_t head_dim, esa_dtype_t dt, esa_params_t p) {
+  if (batch <= 0 || lq <= 0 || hkv <= 0 || hq <= 0 || hq % hkv) return 0;
+  return plan_attn(batch, lq, c0, hq, hkv, head_dim, dt, p).ws_bytes;
+}
+
+esa_status_t esa_sparse_attn(const void* q, const void* k, const void* v, esa_dtype_t dt, int32_t batch, int32_t lq,
+                             int64_t n_cap, int64_t c0, int32_t hq, int32_t hkv, int32_t head_dim,
+                             const int32_t* idx, const int32_t* count, esa_params_t p, float scale, void* o,
+                             float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  esa_status_t st = check_params(p);
+  if (st != ESA_OK) return st;
+  if (dt != ESA_F32 && dt != ESA_BF16) return fail(ESA_ERR_INVALID_ARG, "bad dtype %d", (int)dt);
+  if (batch <= 0 || lq <= 0) return fail(ESA_ERR_INVALID_ARG, "batch and lq must be >= 1");
+  if (hq <= 0 || hkv <= 0 || hq % hkv) return fail(ESA_ERR_INVALID_ARG, "hq must be a positive multiple of hkv");
+  if (head_dim != 64 && head_dim != 128) return fail(ESA_ERR_UNSUPPORTED, "head_dim %d (64 or 128)", head_dim);
+  const int g = hq / hkv;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return fail(ESA_ERR_UNSUPPORTED, "GQA group %d (1, 2, 4 or 8)", g);
+  if (c0 < 0 || c0 + lq > n_cap) return fail(ESA_ERR_INVALID_ARG, "need 0 <= c0 and c0 + lq <= n_cap");
+  if (!q || !k || !v || !o || !idx || !count) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16))
+    return fail(ESA_ERR_INVALID_ARG, "q, k, v, o need 16-byte alignment");
+  const Regions r = regions(c0, p);
+  const AttnPlan pl = plan_attn(batch, lq, c0, hq, hkv, head_dim, dt, p);
+  if (pl.ws_bytes && (!workspace || ws_bytes < pl.ws_bytes || !aligned(workspace, 256)))
+    return fail(ESA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", pl.ws_bytes, ws_bytes);
+  if (scale <= 0.f) scale = 1.f / std::sqrt((float)head_dim);
+  const float sl2 = scale * 1.4426950408889634f;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  esa::KeyList keys{idx, p.topk, r.ni, r.lo, n_cap, count};
+  if (pl.tc) {
+    static bool attr_set[64] = {};
+    int dev = 0;
+    ESA_CUDA(cudaGetDevice(&dev));
+    if (dev < 64 && !attr_set[dev]) {
+      st = set_max_smem(esa::attn_tc_kernel<esa::EsaTcProblem>, esa::kTcSmemBytes);
+      if (st != ESA_OK) return st;
+      attr_set[dev] = true;
+    }
+    esa::EsaTcProblem pr{};
+    pr.q = static_cast<const __nv_bfloat16*>(q);
+    pr.k = static_cast<const __nv_bfloat16*>(k);
+    pr.v = static_cast<const __nv_bfloat16*>(v);
+    pr.o = static_cast<__nv_bfloat16*>(o);
+    pr.lse = lse;
+    pr.keys = keys;
+    pr.n_cap = n_cap;
+    pr.c0 = c0;
+    pr.lq = lq;
+    pr.hq = hq;
+    pr.hkv = hkv;
+    pr.G = g;
+    pr.sl2 = sl2;
+    dim3 grid((unsigned)cdiv((int64_t)lq * g, esa::kTcRows), hkv, batch);
+    esa::attn_tc_kernel<esa::EsaTcProblem><<<grid, esa::kTcThreads, esa::kTcSmemBytes, s>>>(pr);
+    ESA_LAUNCH_CHECK("attn_tc_kernel<esa>");
+    return ok();
+  }
+  esa::SimtAttnArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.part = static_cast<float*>(workspace);
+  a.keys = keys;
+  a.n_cap = n_cap;
+  a.c0 = c0;
+  a.lq = lq;
+  a.hq = hq;
+  a.hkv = hkv;
+  a.nsplit = pl.nsplit;
+  a.keys_per_split = pl.keys_per_split;
+  a.scale_log2 = sl2;
+  bool launched;
+  if (dt == ESA_BF16)
+    launched = head_dim == 128 ? dispatch_simt_g<__nv_bfloat16, 128>(a, g, batch, s)
+                               : dispatch_simt_g<__nv_bfloat16, 64>(a, g, batch, s);
+  else
+    launched = head_dim == 128 ? dispatch_simt_g<float, 128>(a, g, batch, s) : dispatch_simt_g<float, 64>(a, g, batch, s);
+  if (!launched) return fail(ESA_ERR_UNSUPPORTED, "GQA group %d", g);
+  ESA_LAUNCH_CHECK("attn_simt_kernel");
+  if (pl.nsplit > 1) {
+    const int64_t rows = (int64_t)batch * lq * hq;
+    const dim3 cgrid((unsigned)cdiv(rows, 8));
+    if (dt == ESA_BF16) {
+      if (head_dim == 128)
+        esa::attn_combine_kernel<__nv_bfloat16, 128><<<cgrid, 256, 0, s>>>(a.part, rows, pl.nsplit,
+                                                                          static_cast<__nv_bfloat16*>(o), lse);
+      else
+        esa::attn_combine_kernel<__nv_bfloat16, 64><<<cgrid, 256, 0, s>>>(a.part, rows, pl.nsplit,
+                                                                         static_cast<__nv_bfloat16*>(o), lse);
+    } else {
+      if (head_dim == 128)
+        esa::attn_combine_kernel<float, 128><<<cgrid, 256, 0, s>>>(a.part, rows, pl.nsplit, static_cast<float*>(o),
+                                                                  lse);
+      else
+        esa::attn_combine_kernel<float, 64><<<cgrid, 256, 0, s>>>(a.part, rows, pl.nsplit, static_cast<float*>(o),
+                                                                 lse);
+    }
+    ESA_LAUNCH_CHECK("attn_combine_kernel");
+  }
+  return ok();
+}
+
+// ------------------------------------------------------------------ MoBA --
+namespace {
+
+struct MobaWs {
+  float* kbar;
+  int16_t* blocks;
+  uint32_t* cnt;    // cnt, fill contiguous (cleared together)
+  uint32_t* fill;
+  uint32_t* off;
+  uint32_t* tile_off;
+  uint32_t* totals;
+  uint32_t* list;
+  float* part_o;
+  float* part_lse;
+  size_t zero_bytes;
+  size_t bytes;
+  int64_t n_lists, pairs, max_tiles;
+};
+
+int64_t moba_pairs(int64_t seq, int block, int topk) {
+  const int64_t nb = cdiv(seq, block);
+  int64_t pairs = 0;
+  for (int64_t c = 0; c < nb; ++c) pairs += std::min<int64_t>(block, seq - c * block) * std::min<int64_t>(topk, c);
+  return pairs;
+}
+
+// which: 0 gate only, 1 attention only, 2 both (blocks live in the workspace)
+MobaWs carve_moba(void* ws, int which, int32_t batch, int64_t seq, int32_t heads, int32_t d, int32_t block,
+                  int32_t topk) {
+  Carver c{reinterpret_cast<uint8_t*>(ws)};
+  MobaWs w{};
+  const int64_t nb = cdiv(seq, block);
+  w.n_lists = (int64_t)batch * heads * nb;
+  w.pairs = moba_pairs(seq, block, topk) * batch * heads;
+  w.max_tiles = cdiv(w.pairs, esa::kTcRows) + w.n_lists;
+  if (which == 0 || which == 2) w.kbar = c.take<float>((size_t)batch * heads * nb * d);
+  if (which == 2) w.blocks = c.take<int16_t>((size_t)batch * seq * heads * (topk + 1));
+  if (which >= 1) {
+    const size_t z0 = c.off;
+    w.cnt = c.take<uint32_t>(w.n_lists);
+    w.fill = c.take<uint32_t>(w.n_lists);
+    w.zero_bytes = c.off - z0;
+    w.off = c.take<uint32_t>(w.n_lists);
+    w.tile_off = c.take<uint32_t>(w.n_lists + 1);
+    w.totals = c.take<uint32_t>(2);
+    w.list = c.take<uint32_t>(std::max<int64_t>(1, w.pairs));
+    w.part_o = c.take<float>((size_t)batch * seq * heads * (topk + 1) * d);
+    w.part_lse = c.take<float>((size_t)batch * seq * heads * (topk + 1));
+  }
+  w.bytes = c.off;
+  return w;
+}
+
+esa_status_t moba_check(const void* q, const void* k, esa_dtype_t dt, int32_t batch, int64_t seq, int32_t heads,
+                        int32_t head_dim, int32_t block, int32_t topk) {
+  if (dt != ESA_BF16) return fail(ESA_ERR_UNSUPPORTED, "MoBA kernels take bf16 tensors");
+  if (batch <= 0 || seq <= 0 || heads <= 0) return fail(ESA_ERR_INVALID_ARG, "batch, seq, heads must be >= 1");
+  if (head_dim != 128) return fail(ESA_ERR_UNSUPPORTED, "MoBA head_dim %d (128)", head_dim);
+  if (block < 16 || block % 16) return fail(ESA_ERR_INVALID_ARG, "block must be a multiple of 16, >= 16");
+  if (topk < 0 || topk > esa::kMobaMaxTopk) return fail(ESA_ERR_INVALID_ARG, "topk must be in [0, 15]");
+  if (cdiv(seq, block) > 1024) return fail(ESA_ERR_UNSUPPORTED, "more than 1024 blocks");
+  if (seq >= ((int64_t)1 << 27)) return fail(ESA_ERR_UNSUPPORTED, "seq must be < 2^27");
+  if (!q || !k) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(q, 16) || !aligned(k, 16)) return fail(ESA_ERR_INVALID_ARG, "16-byte alignment required");
+  return ESA_OK;
+}
+
+esa_status_t moba_gate_launch(const MobaWs& w, const void* q, const void* k, int32_t batch, int64_t seq, int32_t heads,
+                              int32_t block, int32_t topk, int16_t* blocks_out, cudaStream_t s) {
+  const int nb = (int)cdiv(seq, block);
+  esa::moba_mean_kernel<__nv_bfloat16><<<dim3(nb, heads, batch), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(k), seq, heads, 128, block, w.kbar);
+  ESA_LAUNCH_CHECK("moba_mean_kernel");
+  esa::moba_gate_kernel<__nv_bfloat16, 128><<<dim3((unsigned)cdiv(seq, 128), heads, batch), 128, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(q), w.kbar, seq, heads, block, nb, topk, blocks_out);
+  ESA_LAUNCH_CHECK("moba_gate_kernel");
+  return ESA_OK;
+}
+
+esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, const void* v, int32_t batch,
+                              int64_t seq, int32_t heads, int32_t block, int32_t topk, const int16_t* blocks,
+                              float scale, void* o, float* lse, cudaStream_t s) {
+  const int nb = (int)cdiv(seq, block);
+  if (scale <= 0.f) scale = 1.f / std::sqrt(128.f);
+  const float sl2 = scale * 1.4426950408889634f;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  ESA_CUDA(cudaGetDevice(&dev));
+  if (dev < 64 && !attr_set[dev]) {
+    esa_status_t st = set_max_smem(esa::attn_tc_kernel<esa::MobaPastProblem>, esa::kTcSmemBytes);
+    if (st != ESA_OK) return st;
+    st = set_max_smem(esa::attn_tc_kernel<esa::MobaCurrentProblem>, esa::kTcSmemBytes);
+    if (st != ESA_OK) return st;
+    attr_set[dev] = true;
+  }
+  ESA_CUDA(cudaMemsetAsync(w.cnt, 0, w.zero_bytes, s));
+  const dim3 lgrid((unsigned)cdiv(seq * heads, 256), batch);
+  if (topk > 0 && w.pairs > 0) {
+    esa::moba_list_kernel<<<lgrid, 256, 0, s>>>(blocks, seq, heads, block, nb, topk, 0, w.cnt, w.off, w.fill, w.list);
+    ESA_LAUNCH_CHECK("moba_list_kernel(count)");
+    esa::moba_scan_kernel<<<1, 1024, 0, s>>>(w.cnt, w.n_lists, w.off, w.tile_off, w.totals);
+    ESA_LAUNCH_CHECK("moba_scan_kernel");
+    esa::moba_list_kernel<<<lgrid, 256, 0, s>>>(blocks, seq, heads, block, nb, topk, 1, w.cnt, w.off, w.fill, w.list);
+    ESA_LAUNCH_CHECK("moba_list_kernel(fill)");
+    esa::MobaPastProblem pp{};
+    pp.q = static_cast<const __nv_bfloat16*>(q);
+    pp.k = static_cast<const __nv_bfloat16*>(k);
+    pp.v = static_cast<const __nv_bfloat16*>(v);
+    pp.part_o = w.part_o;
+    pp.part_lse = w.part_lse;
+    pp.tile_off = w.tile_off;
+    pp.off = w.off;
+    pp.cnt = w.cnt;
+    pp.list = w.list;
+    pp.seq = seq;
+    pp.heads = heads;
+    pp.n_blocks = nb;
+    pp.block = block;
+    pp.topk = topk;
+    pp.n_lists = w.n_lists;
+    pp.sl2 = sl2;
+    esa::attn_tc_kernel<esa::MobaPastProblem><<<(unsigned)w.max_tiles, esa::kTcThreads, esa::kTcSmemBytes, s>>>(pp);
+    ESA_LAUNCH_CHECK("attn_tc_kernel<moba past>");
+  }
+  esa::MobaCurrentProblem cp{};
+  cp.q = static_cast<const __nv_bfloat16*>(q);
+  cp.k = static_cast<const __nv_bfloat16*>(k);
+  cp.v = static_cast<const __nv_bfloat16*>(v);
+  cp.part_o = w.part_o;
+  cp.part_lse = w.part_lse;
+  cp.seq = seq;
+  cp.heads = heads;
+  cp.n_blocks = nb;
+  cp.block = block;
+  cp.topk = topk;
+  cp.tiles_per_block = (int)cdiv(block, esa::kTcRows);
+  cp.sl2 = sl2;
+  esa::attn_tc_kernel<esa::MobaCurrentProblem>
+      <<<dim3(cp.tiles_per_block * nb, heads, batch), esa::kTcThreads, esa::kTcSmemBytes, s>>>(cp);
+  ESA_LAUNCH_CHECK("attn_tc_kernel<moba current>");
+  const int64_t rows = (int64_t)batch * seq * heads;
+  esa::moba_combine_kernel<128><<<(unsigned)cdiv(rows, 8), 256, 0, s>>>(
+      w.part_o, w.part_lse, seq, heads, block, topk, rows, static_cast<__nv_bfloat16*>(o), lse);
+  ESA_LAUNCH_CHECK("moba_combine_kernel");
+  return ESA_OK;
+}
+
+}  // namespace
+
+size_t moba_workspace_size(int32_t which, int32_t batch, int64_t seq, int32_t heads, int32_t head_dim, int32_t block,
+                           int32_t topk) {
+  if (which < 0 || which > 2 || batch <= 0 || seq <= 0 || heads <= 0 || block <= 0 || topk < 0) return 0;
+  return carve_moba(nullptr, which, batch, seq, heads, head_dim, block, topk).bytes;
+}
+
+esa_status_t moba_block_gate(const void* q, const void* k, esa_dtype_t dt, int32_t batch, int64_t seq, int32_t heads,
+                             int32_t head_dim, int32_t block, int32_t topk, int16_t* blocks_out, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  esa_status_t st = moba_check(q, k, dt, batch, seq, heads, head_dim, block, topk);
+  if (st != ESA_OK) return st;
+  if (!blocks_out) return fail(ESA_ERR_INVALID_ARG, "null blocks_out");
+  const MobaWs need = carve_moba(nullptr, 0, batch, seq, heads, head_dim, block, topk);
+  if (!workspace || ws_bytes < need.bytes || !aligned(workspace, 256))
+    return fail(ESA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need.bytes, ws_bytes);
+  const MobaWs w = carve_moba(workspace, 0, batch, seq, heads, head_dim, block, topk);
+  st = moba_gate_launch(w, q, k, batch, seq, heads, block, topk, blocks_out, reinterpret_cast<cudaStream_t>(stream));
+  return st == ESA_OK ? ok() : st;
+}
+
+esa_status_t moba_block_attn(const void* q, const void* k, const void* v, esa_dtype_t dt, int32_t batch, int64_t seq,
+                             int32_t heads, int32_t head_dim, int32_t block, int32_t topk, const int16_t* blocks,
+                             float scale, void* o, float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  esa_status_t st = moba_check(q, k, dt, batch, seq, heads, head_dim, block, topk);
+  if (st != ESA_OK) return st;
+  if (!v || !o || !blocks) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(v, 16) || !aligned(o, 16)) return fail(ESA_ERR_INVALID_ARG, "16-byte alignment required");
+  const MobaWs need = carve_moba(nullptr, 1, batch, seq, heads, head_dim, block, topk);
+  if (!workspace || ws_bytes < need.bytes || !aligned(workspace, 256))
+    return fail(ESA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need.bytes, ws_bytes);
+  const MobaWs w = carve_moba(workspace, 1, batch, seq, heads, head_dim, block, topk);
+  st = moba_attn_launch(w, q, k, v, batch, seq, heads, block, topk, blocks, scale, o, lse,
+                        reinterpret_cast<cudaStream_t>(stream));
+  return st == ESA_OK ? ok() : st;
+}
+
+esa_status_t moba_block_gate_attn(const void* q, const void* k, const void* v, esa_dtype_t dt, int32_t batch,
+                                  int64_t seq, int32_t heads, int32_t head_dim, int32_t block, int32_t topk,
+                                  float scale, void* o, float* lse, int16_t* blocks_out, void* workspace,
+                                  size_t ws_bytes, void* stream) {
+  esa_status_t st = moba_check(q, k, dt, batch, seq, heads, head_dim, block, topk);
+  if (st != ESA_OK) return st;
+  if (!v || !o) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(v, 16) || !aligned(o, 16)) return fail(ESA_ERR_INVALID_ARG, "16-byte alignment required");
+  const MobaWs need = carve_moba(nullptr, 2, batch, seq, heads, head_dim, block, topk);
+  if (!workspace || ws_bytes < need.bytes || !aligned(workspace, 256))
+    return fail(ESA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need.bytes, ws_bytes);
+  const MobaWs w = carve_moba(workspace, 2, batch, seq, heads, head_dim, block, topk);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int16_t* blocks = blocks_out ? blocks_out : w.blocks;
+  st = moba_gate_launch(w, q, k, batch, seq, heads, block, topk, blocks, s);
+  if (st != ESA_OK) return st;
+  st = moba_attn_launch(w, q, k, v, batch, seq, heads, block, topk, blocks, scale, o, lse, s);
+  return st == ESA_OK ? ok() : st;
+}
+

@@ -1,0 +1,347 @@
+// moba.cuh - Mixture of Block Attention (MoBA article, sections 2-3).
+//
+//   block means   Kbar[b, h, blk] = mean of K over block blk (fp32)
+//   gate          s_blk = <q, Kbar[blk]> for past blocks blk < cur; keep the top
+//                 min(topk, cur) by (score desc, block asc); add the current block
+//   attention     softmax over the kept blocks, the current block cut causally
+//
+// The attention is grouped by key block instead of by query: for every (sequence,
+// head, past block) the queries that chose that block form a list, and one tensor-core
+// CTA attends 128 listed queries to the block's contiguous keys. Each (query, head)
+// thereby gets one partial (o, lse) per attended block, written to its slot (the
+// block's rank in the query's list); the current block is one more partial, and a
+// final kernel merges the partials by log-sum-exp. The work is exactly the selected
+// (query, block) pairs, so no key is attended that the gate did not keep.
+#pragma once
+#include <cub/block/block_scan.cuh>
+
+#include "attn_tc.cuh"
+#include "common.cuh"
+
+namespace esa {
+
+constexpr int kMobaMaxTopk = 15;
+
+// ------------------------------------------------------------------ block means --
+// grid (n_blocks, H, B), 256 threads: thread = (d pair, row phase); fixed order sums.
+template <typename T>
+__global__ void __launch_bounds__(256) moba_mean_kernel(const T* __restrict__ k, int64_t seq, int heads, int d,
+                                                        int block, float* __restrict__ kbar) {
+  __shared__ float part[256][2];
+  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int pairs = d / 2;
+  const int dp = threadIdx.x % pairs;
+  const int ph = threadIdx.x / pairs;
+  const int nph = 256 / pairs;
+  const int64_t r0 = (int64_t)blk * block;
+  const int64_t r1 = min(seq, r0 + block);
+  float a0 = 0.f, a1 = 0.f;
+  for (int64_t r = r0 + ph; r < r1; r += nph) {
+    const T* p = k + ((b * seq + r) * heads + h) * d + 2 * dp;
+    a0 += static_cast<float>(p[0]);
+    a1 += static_cast<float>(p[1]);
+  }
+  part[threadIdx.x][0] = a0;
+  part[threadIdx.x][1] = a1;
+  __syncthreads();
+  if (threadIdx.x < pairs) {
+    float s0 = 0.f, s1 = 0.f;
+    for (int q = 0; q < nph; ++q) {
+      s0 += part[q * pairs + threadIdx.x][0];
+      s1 += part[q * pairs + threadIdx.x][1];
+    }
+    const float inv = 1.f / (float)(r1 - r0);
+    float* o = kbar + (((int64_t)b * heads + h) * gridDim.x + blk) * d + 2 * threadIdx.x;
+    o[0] = s0 * inv;
+    o[1] = s1 * inv;
+  }
+}
+
+// ------------------------------------------------------------------ gate --
+// grid (ceil(seq / 128), H, B), 128 threads; thread = query position. The query row
+// lives in registers; block means are staged 32 blocks at a time in shared memory and
+// read as broadcasts. Kept list: insertion that never moves an element past an equal
+// one, visiting blocks in ascending order -> ties go to the lower block.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) moba_gate_kernel(const T* __restrict__ q, const float* __restrict__ kbar,
+                                                        int64_t seq, int heads, int block, int n_blocks, int topk,
+                                                        int16_t* __restrict__ blocks_out) {
+  constexpr int CB = 32;
+  __shared__ float4 kb[CB][D / 4];
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int64_t p = (int64_t)blockIdx.x * 128 + threadIdx.x;
+  const bool valid = p < seq;
+  const int cur = valid ? (int)(p / block) : 0;
+  const int64_t p_last = min(seq - 1, (int64_t)blockIdx.x * 128 + 127);
+  const int cur_max = (int)(p_last / block);
+  float qv[D];
+  if (valid) {
+    const T* qp = q + ((b * seq + p) * heads + h) * D;
+#pragma unroll
+    for (int e = 0; e < D; e += 16 / sizeof(T)) load_vec(qp + e, &qv[e]);
+  }
+  float vals[kMobaMaxTopk];
+  int ids[kMobaMaxTopk];
+#pragma unroll
+  for (int i = 0; i < kMobaMaxTopk; ++i) { vals[i] = -INFINITY; ids[i] = -1; }
+  const float* kbh = kbar + ((int64_t)b * heads + h) * n_blocks * D;
+  for (int c0 = 0; c0 < cur_max; c0 += CB) {
+    __syncthreads();
+    for (int t = threadIdx.x; t < CB * D / 4; t += 128) {
+      const int c = t / (D / 4), e = t % (D / 4);
+      kb[c][e] = (c0 + c < n_blocks) ? reinterpret_cast<const float4*>(kbh + (int64_t)(c0 + c) * D)[e]
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();
+    if (!valid) continue;
+    const int cend = min(CB, cur - c0);
+    for (int c = 0; c < cend; ++c) {
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < D / 4; ++e) {
+        const float4 w = kb[c][e];
+        acc = fmaf(qv[4 * e], w.x, acc);
+        acc = fmaf(qv[4 * e + 1], w.y, acc);
+        acc = fmaf(qv[4 * e + 2], w.z, acc);
+        acc = fmaf(qv[4 * e + 3], w.w, acc);
+      }
+      float v = acc;
+      int id = c0 + c;
+#pragma unroll
+      for (int i = 0; i < kMobaMaxTopk; ++i) {
+        if (i < topk && v > vals[i]) {
+          const float tv = vals[i]; vals[i] = v; v = tv;
+          const int ti = ids[i]; ids[i] = id; id = ti;
+        }
+      }
+    }
+  }
+  if (!valid) return;
+  // ascending block order: small unrolled exchange sort on the kept ids (-1 last)
+#pragma unroll
+  for (int i = 0; i < kMobaMaxTopk; ++i)
+#pragma unroll
+    for (int j = 0; j + 1 < kMobaMaxTopk - i; ++j) {
+      const int a = ids[j], c = ids[j + 1];
+      const bool swap = (a < 0 && c >= 0) || (a >= 0 && c >= 0 && c < a);
+      ids[j] = swap ? c : a;
+      ids[j + 1] = swap ? a : c;
+    }
+  int16_t* out = blocks_out + ((b * seq + p) * heads + h) * (topk + 1);
+  int n = 0;
+#pragma unroll
+  for (int i = 0; i < kMobaMaxTopk; ++i)
+    if (i < topk && ids[i] >= 0) out[n++] = (int16_t)ids[i];
+  out[n++] = (int16_t)cur;
+  for (; n < topk + 1; ++n) out[n] = -1;
+}
+
+// ------------------------------------------------------------------ query lists --
+// For each (b, p, h) and each past block in its list (the first min(topk, p / block)
+// entries), count (pass 0) or append (pass 1) the pair (p, slot) to the list of
+// (b, h, block). The order inside a list is not fixed, but every pair owns its own
+// output slot, so the results do not depend on it.
+__global__ void moba_list_kernel(const int16_t* __restrict__ blocks, int64_t seq, int heads, int block,
+                                 int n_blocks, int topk, int pass, uint32_t* __restrict__ cnt,
+                                 const uint32_t* __restrict__ off, uint32_t* __restrict__ fill,
+                                 uint32_t* __restrict__ list) {
+  const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // (p, h) of sequence b
+  const int b = blockIdx.y;
+  if (row >= seq * heads) return;
+  const int64_t p = row / heads;
+  const int h = (int)(row % heads);
+  const int n_past = min(topk, (int)(p / block));
+  const int16_t* lst = blocks + ((int64_t)b * seq * heads + row) * (topk + 1);
+  for (int s = 0; s < n_past; ++s) {
+    const int blk = lst[s];
+    if (blk < 0 || blk >= n_blocks) break;
+    const int64_t li = ((int64_t)b * heads + h) * n_blocks + blk;
+    if (pass == 0) {
+      atomicAdd(&cnt[li], 1u);
+    } else {
+      const uint32_t at = atomicAdd(&fill[li], 1u);
+      list[off[li] + at] = ((uint32_t)p << 4) | (uint32_t)s;
+    }
+  }
+}
+
+// Exclusive scans over all lists: entry offsets and 128-row tile offsets. One CTA.
+__global__ void __launch_bounds__(1024) moba_scan_kernel(const uint32_t* __restrict__ cnt, int64_t n_lists,
+                                                         uint32_t* __restrict__ off, uint32_t* __restrict__ tile_off,
+                                                         uint32_t* __restrict__ totals) {
+  using Scan = cub::BlockScan<uint32_t, 1024>;
+  __shared__ typename Scan::TempStorage t1, t2;
+  __shared__ uint32_t carry_e, carry_t;
+  if (threadIdx.x == 0) { carry_e = 0; carry_t = 0; }
+  __syncthreads();
+  for (int64_t base = 0; base < n_lists; base += 1024) {
+    const int64_t i = base + threadIdx.x;
+    const uint32_t c = i < n_lists ? cnt[i] : 0u;
+    const uint32_t t = (c + kTcRows - 1) / kTcRows;
+    uint32_t ec, tc, es, ts;
+    Scan(t1).ExclusiveSum(c, ec, es);
+    Scan(t2).ExclusiveSum(t, tc, ts);
+    if (i < n_lists) {
+      off[i] = carry_e + ec;
+      tile_off[i] = carry_t + tc;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) { carry_e += es; carry_t += ts; }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    tile_off[n_lists] = carry_t;
+    totals[0] = carry_e;
+    totals[1] = carry_t;
+  }
+}
+
+// ------------------------------------------------------------------ TC problems --
+// Partials: part_o [B, seq, H, topk+1, D] fp32 (normalised), part_lse [B, seq, H, topk+1].
+struct MobaPastProblem {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  float* part_o;
+  float* part_lse;
+  const uint32_t* tile_off;   // [n_lists + 1]
+  const uint32_t* off;        // [n_lists]
+  const uint32_t* cnt;        // [n_lists]
+  const uint32_t* list;       // packed (p << 4 | slot)
+  int64_t seq;
+  int heads, n_blocks, block, topk;
+  int64_t n_lists;
+  float sl2;
+  // per CTA
+  int b, h, blk;
+  uint32_t e0, n_rows;
+
+  __device__ bool setup() {
+    const uint32_t tile = blockIdx.x;
+    if (tile >= tile_off[n_lists]) return false;
+    int64_t lo = 0, hi = n_lists - 1;       // last list with tile_off <= tile
+    while (lo < hi) {
+      const int64_t mid = (lo + hi + 1) / 2;
+      if (tile_off[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    const int64_t li = lo;
+    blk = (int)(li % n_blocks);
+    h = (int)((li / n_blocks) % heads);
+    b = (int)(li / ((int64_t)n_blocks * heads));
+    const uint32_t t_in = tile - tile_off[li];
+    e0 = off[li] + t_in * kTcRows;
+    n_rows = min((uint32_t)kTcRows, cnt[li] - t_in * kTcRows);
+    return true;
+  }
+  __device__ const __nv_bfloat16* q_base() const { return q; }
+  __device__ const __nv_bfloat16* kv_base_k() const { return k; }
+  __device__ const __nv_bfloat16* kv_base_v() const { return v; }
+  __device__ int64_t q_row(int r) const {
+    if ((uint32_t)r >= n_rows) return -1;
+    const int64_t p = list[e0 + r] >> 4;
+    return (((int64_t)b * seq + p) * heads + h) * kTcD;
+  }
+  __device__ int64_t n_keys() const { return min((int64_t)block, seq - (int64_t)blk * block); }
+  __device__ int64_t kv_row(int64_t t) const {
+    return (((int64_t)b * seq + (int64_t)blk * block + t) * heads + h) * kTcD;
+  }
+  __device__ int64_t limit(int) const { return n_keys() - 1; }
+  __device__ float scale_log2() const { return sl2; }
+  __device__ void store(int r, const float* acc, float m2, float l) {
+    if ((uint32_t)r >= n_rows) return;
+    const uint32_t e = list[e0 + r];
+    const int64_t p = e >> 4;
+    const int slot = e & 15;
+    const int64_t row = (((int64_t)b * seq + p) * heads + h) * (topk + 1) + slot;
+    const float inv = 1.f / l;
+    float4* dst = reinterpret_cast<float4*>(part_o + row * kTcD);
+#pragma unroll
+    for (int c = 0; c < kTcD / 4; ++c)
+      dst[c] = make_float4(acc[4 * c] * inv, acc[4 * c + 1] * inv, acc[4 * c + 2] * inv, acc[4 * c + 3] * inv);
+    part_lse[row] = (m2 + __log2f(l)) * 0.69314718055994531f;
+  }
+};
+
+// Current block: grid (tiles_per_block * n_blocks, H, B); rows = 128 consecutive
+// queries of one head inside one block; keys = the block up to each query (causal).
+struct MobaCurrentProblem {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  float* part_o;
+  float* part_lse;
+  int64_t seq;
+  int heads, n_blocks, block, topk, tiles_per_block;
+  float sl2;
+  int b, h, blk;
+  int64_t p0, kb0, nrows;
+
+  __device__ bool setup() {
+    blk = blockIdx.x / tiles_per_block;
+    const int t = blockIdx.x % tiles_per_block;
+    h = blockIdx.y;
+    b = blockIdx.z;
+    kb0 = (int64_t)blk * block;
+    p0 = kb0 + (int64_t)t * kTcRows;
+    const int64_t bend = min(seq, kb0 + block);
+    if (p0 >= bend) return false;
+    nrows = min((int64_t)kTcRows, bend - p0);
+    return true;
+  }
+  __device__ const __nv_bfloat16* q_base() const { return q; }
+  __device__ const __nv_bfloat16* kv_base_k() const { return k; }
+  __device__ const __nv_bfloat16* kv_base_v() const { return v; }
+  __device__ int64_t q_row(int r) const {
+    if (r >= nrows) return -1;
+    return (((int64_t)b * seq + p0 + r) * heads + h) * kTcD;
+  }
+  __device__ int64_t n_keys() const { return p0 + nrows - kb0; }
+  __device__ int64_t kv_row(int64_t t) const { return (((int64_t)b * seq + kb0 + t) * heads + h) * kTcD; }
+  __device__ int64_t limit(int r) const { return p0 + min((int64_t)r, nrows - 1) - kb0; }
+  __device__ float scale_log2() const { return sl2; }
+  __device__ void store(int r, const float* acc, float m2, float l) {
+    if (r >= nrows) return;
+    const int64_t p = p0 + r;
+    const int slot = min(topk, blk);
+    const int64_t row = (((int64_t)b * seq + p) * heads + h) * (topk + 1) + slot;
+    const float inv = 1.f / l;
+    float4* dst = reinterpret_cast<float4*>(part_o + row * kTcD);
+#pragma unroll
+    for (int c = 0; c < kTcD / 4; ++c)
+      dst[c] = make_float4(acc[4 * c] * inv, acc[4 * c + 1] * inv, acc[4 * c + 2] * inv, acc[4 * c + 3] * inv);
+    part_lse[row] = (m2 + __log2f(l)) * 0.69314718055994531f;
+  }
+};
+
+// Merge the min(topk, cur) + 1 partials of each (b, p, h). One warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) moba_combine_kernel(const float* __restrict__ part_o,
+                                                           const float* __restrict__ part_lse, int64_t seq, int heads,
+                                                           int block, int topk, int64_t n_rows,
+                                                           __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);   // (b, p, h) flattened
+  const int lane = threadIdx.x & 31;
+  if (row >= n_rows) return;
+  const int64_t p = (row / heads) % seq;
+  const int ns = min(topk, (int)(p / block)) + 1;
+  const float* lr = part_lse + row * (topk + 1);
+  float M = -INFINITY;
+  for (int s = 0; s < ns; ++s) M = fmaxf(M, lr[s]);
+  float L = 0.f;
+  float acc[D / 32];
+#pragma unroll
+  for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
+  for (int s = 0; s < ns; ++s) {
+    const float w = __expf(lr[s] - M);
+    L += w;
+    const float* po = part_o + (row * (topk + 1) + s) * D;
+#pragma unroll
+    for (int e = 0; e < D / 32; ++e) acc[e] = fmaf(w, po[lane + 32 * e], acc[e]);
+  }
+  const float inv = 1.f / L;
+#pragma unroll
+  for (int e = 0; e < D / 32; ++e) o[row * D + lane + 32 * e] = __float2bfloat16_rn(acc[e] * inv);
+  if (lane == 0 && lse) lse[row] = M + __logf(L);
+}
+
+}  // namespace esa

@@ -1,0 +1,139 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+The library must load, export every function include/esa.h declares, and reject
+bad arguments on the host before anything is launched (no CUDA call happens on
+these paths). The Python binding must refuse CPU tensors: there is no CPU path.
+"""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+import torch
+
+import query_aware_selective_b200 as qas
+from query_aware_selective_b200 import _abi
+from query_aware_selective_b200 import build as qbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "esa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    qbuild.build()
+    return _abi.load()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:esa_status_t|size_t|const char\*)\s+(\w+)\s*\(", text, flags=re.M)
+
+
+def test_header_declares_the_boundary():
+    names = set(header_functions())
+    for required in ["esa_compress", "esa_score_select", "esa_sparse_attn", "moba_block_gate_attn",
+                     "esa_last_error", "esa_device_status"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+        assert name in _abi.SIGNATURES, f"binding does not declare {name}"
+
+
+def test_params_struct_layout():
+    assert ctypes.sizeof(_abi.EsaParams) == 20
+    assert [f[0] for f in _abi.EsaParams._fields_] == ["n_init", "window", "topk", "eps", "clamp_c"]
+
+
+FAKE = 0x10000  # a 256-byte aligned non-null value: never dereferenced on the rejected paths
+
+
+def _err(lib):
+    return lib.esa_last_error().decode()
+
+
+def test_compress_rejects_bad_arguments(lib):
+    f = lib.esa_compress
+    xs = 8 * 128
+    assert f(FAKE, 1, -1, xs, 8, 32, 128, FAKE, 128, FAKE, 128, None) == _abi.ESA_ERR_INVALID_ARG
+    assert "rows" in _err(lib)
+    assert f(None, 1, 4, xs, 8, 32, 128, FAKE, 128, FAKE, 128, None) == _abi.ESA_ERR_INVALID_ARG
+    assert f(FAKE, 7, 4, xs, 8, 32, 128, FAKE, 128, FAKE, 128, None) == _abi.ESA_ERR_INVALID_ARG
+    assert f(FAKE, 1, 4, xs, 8, 30, 128, FAKE, 128, FAKE, 128, None) == _abi.ESA_ERR_INVALID_ARG
+    assert f(FAKE, 1, 4, xs, 8, 32, 96, FAKE, 128, FAKE, 128, None) == _abi.ESA_ERR_UNSUPPORTED
+    assert f(FAKE, 1, 4, xs, 8, 32, 128, FAKE, 24, FAKE, 24, None) == _abi.ESA_ERR_UNSUPPORTED
+    assert f(FAKE, 1, 4, xs, 8, 32, 128, FAKE, 128, FAKE, 64, None) == _abi.ESA_ERR_INVALID_ARG
+    assert f(FAKE, 1, 4, xs - 8, 8, 32, 128, FAKE, 128, FAKE, 128, None) == _abi.ESA_ERR_INVALID_ARG
+    assert f(FAKE, 1, 4, xs + 4, 8, 32, 128, FAKE, 128, FAKE, 128, None) == _abi.ESA_ERR_INVALID_ARG
+    # zero rows is a no-op that launches nothing
+    assert f(FAKE, 1, 0, xs, 8, 32, 128, FAKE, 128, FAKE, 128, None) == _abi.ESA_OK
+
+
+def test_score_select_rejects_bad_arguments(lib):
+    f = lib.esa_score_select
+    good = _abi.params(128, 4096, 2048, 2, 45.25)
+    args = lambda p, lq=1, n_cap=131072, c0=131071, dc=128, ws=FAKE, wsn=1 << 40: (
+        FAKE, FAKE, 16, lq, n_cap, c0, dc, p, FAKE, FAKE, None, ws, wsn, None)
+    assert f(*args(_abi.params(128, 4096, 0, 2, 1.0))) == _abi.ESA_ERR_INVALID_ARG      # topk 0
+    assert f(*args(_abi.params(128, 4096, 16, 65, 1.0))) == _abi.ESA_ERR_INVALID_ARG    # eps too large
+    assert f(*args(_abi.params(128, 4096, 16, 2, -1.0))) == _abi.ESA_ERR_INVALID_ARG    # negative clamp
+    assert f(*args(_abi.params(128, 4096, 16, 2, math.nan))) == _abi.ESA_ERR_INVALID_ARG
+    assert f(*args(good, c0=131072)) == _abi.ESA_ERR_INVALID_ARG                          # c0 + lq > n_cap
+    assert f(*args(good, lq=0)) == _abi.ESA_ERR_INVALID_ARG
+    assert f(*args(good, dc=24)) == _abi.ESA_ERR_UNSUPPORTED
+    assert f(*args(good, ws=None)) == _abi.ESA_ERR_WORKSPACE
+    assert f(*args(good, wsn=16)) == _abi.ESA_ERR_WORKSPACE
+    assert f(*args(good, ws=FAKE + 8)) == _abi.ESA_ERR_WORKSPACE                          # misaligned
+    assert "workspace" in _err(lib)
+
+
+def test_sparse_attn_rejects_bad_arguments(lib):
+    f = lib.esa_sparse_attn
+    p = _abi.params(128, 4096, 2048, 2, 45.25)
+    a = lambda hq=32, hkv=8, d=128, dt=1, q=FAKE, o=FAKE: (
+        q, FAKE, FAKE, dt, 16, 1, 131072, 131071, hq, hkv, d, FAKE, FAKE, p, 0.0, o, None, FAKE, 1 << 40, None)
+    assert f(*a(hq=12, hkv=4)) == _abi.ESA_ERR_UNSUPPORTED        # group of 3
+    assert f(*a(hq=30, hkv=8)) == _abi.ESA_ERR_INVALID_ARG
+    assert f(*a(d=80)) == _abi.ESA_ERR_UNSUPPORTED
+    assert f(*a(dt=5)) == _abi.ESA_ERR_INVALID_ARG
+    assert f(*a(q=FAKE + 2)) == _abi.ESA_ERR_INVALID_ARG           # misaligned
+    assert f(*a(o=None)) == _abi.ESA_ERR_INVALID_ARG
+
+
+def test_moba_rejects_bad_arguments(lib):
+    f = lib.moba_block_gate_attn
+    a = lambda dt=1, block=1024, topk=3, d=128: (FAKE, FAKE, FAKE, dt, 1, 65536, 32, d, block, topk, 0.0, FAKE,
+                                                 None, None, FAKE, 1 << 40, None)
+    assert f(*a(dt=0)) == _abi.ESA_ERR_UNSUPPORTED
+    assert f(*a(block=100)) == _abi.ESA_ERR_INVALID_ARG
+    assert f(*a(topk=16)) == _abi.ESA_ERR_INVALID_ARG
+    assert f(*a(d=64)) == _abi.ESA_ERR_UNSUPPORTED
+    assert f(*a(block=16)) == _abi.ESA_ERR_UNSUPPORTED              # 4096 blocks > 1024
+
+
+def test_workspace_sizes(lib):
+    p = _abi.params(128, 4096, 2048, 2, 45.25)
+    small = _abi.score_select_workspace_size(1, 1, 32768, 16384, 128, p)
+    big = _abi.score_select_workspace_size(16, 1, 131072, 131071, 128, p)
+    assert 0 < small < big
+    assert _abi.score_select_workspace_size(0, 1, 10, 5, 128, p) == 0
+    assert _abi.moba_workspace_size(0, 1, 65536, 32, 128, 1024, 3) < _abi.moba_workspace_size(2, 1, 65536, 32, 128,
+                                                                                              1024, 3)
+    assert _abi.moba_workspace_size(7, 1, 65536, 32, 128, 1024, 3) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    x = torch.zeros(4, 8, 128, dtype=torch.bfloat16)
+    w = torch.zeros(4096, 128)
+    with pytest.raises(ValueError, match="CUDA"):
+        qas.compress(x, w, 32)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="not built"):
+        _abi.load(str(tmp_path / "libesa.so"))
