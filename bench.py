@@ -1,0 +1,455 @@
+"""Throughput of query-aware top-k selective attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the hot path over one batch of synthetic input:
+  headline  ESA chunked prefill of a Llama-3-8B attention layer, 32768 tokens in
+            chunks of 512 (compress keys and queries, score, correct, chunk-sum,
+            neighbour max-pool, top-k, attention over initial + selected + local);
+  also      ESA decode at 128K context, batch 16, and MoBA causal prefill at 64K
+            (32 heads, 64 blocks of 1024, top-3 + current), each timed the same way.
+Every rank runs its own replica (weak scaling, no collective on the data path);
+time is the max over ranks of the CUDA-event time. L2 is flushed (256 MB write)
+between timed steps, outside the events. Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (oracle/, float64 numpy on the host cores)
+on a bounded sample of the same workload per step; it needs no GPU.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "ESA decode tok/s @128K & chunked-prefill tok/s; % of HBM/tensor roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true", help="time the headline workload only")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--prefill-ctx", type=int, default=0,
+                    help="shorter prefill context (profiling a small case); the line then names that workload")
+    return ap.parse_args()
+
+
+def load_peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "query_aware_selective_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, sources):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    kernel as it is now (same source hash); else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        t = json.load(f)
+    e = t.get(kernel)
+    if not e or e.get("source_hash") != source_hash(*sources):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while running (clocks, power, throttle reasons)."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "utilization.gpu", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id, self.proc, self.lines = gpu_id, None, []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [[x.strip() for x in ln.split(",")] for ln in out.strip().splitlines() if ln.strip()]
+        rows = [r for r in rows if len(r) == len(self.FIELDS)]
+        if not rows:
+            return None
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        busy = [r for r in rows if (num(r[3]) or 0) >= 50] or rows
+        sm = [num(r[0]) for r in busy if num(r[0]) is not None]
+        reasons = set()
+        for r in busy:
+            for name, val in zip(["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"],
+                                 r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(rows[0][1]),
+                "power_w_max": max((num(r[2]) or 0) for r in rows), "samples": len(rows),
+                "samples_under_load": len(busy), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- timing
+
+def time_steps(fn, steps, warmup, flush, dist_max):
+    """Warm up, then time each of `steps` calls with CUDA events (L2 flushed between
+    steps, outside the events). Returns per-step ms (after max over ranks)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    dist_barrier()
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(steps):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    dist_barrier()
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    total = dist_max(sum(ms))
+    return ms, total
+
+
+_dist = None
+
+
+def dist_barrier():
+    if _dist is not None:
+        _dist.barrier()
+
+
+def make_dist_max():
+    import torch
+    if _dist is None:
+        return lambda x: x
+
+    def f(x):
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        _dist.all_reduce(t, op=_dist.ReduceOp.MAX)
+        return float(t.item())
+    return f
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import query_aware_selective_b200 as qas
+    from query_aware_selective_b200 import cost, pipeline, synthetic
+
+    global _dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus > 1 and world == 1:
+        raise SystemExit("--gpus N > 1 runs under torch.distributed.run (one process per GPU)")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        _dist = dist
+    dist_max = make_dist_max()
+    qas.load()
+    dev = torch.device("cuda", local)
+    props = torch.cuda.get_device_properties(dev)
+    peaks, peak_src = load_peaks()
+    flush_buf = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MB > 126 MB L2
+    flush = lambda: flush_buf.zero_()
+    sampler = ClockSampler("GPU-" + str(props.uuid)).start()
+
+    # ---------------------------------------------------------------- headline: prefill
+    w = synthetic.PREFILL_32K
+    if args.prefill_ctx:
+        import dataclasses
+        w = dataclasses.replace(w, n_ctx=args.prefill_ctx, name=f"esa_prefill_llama3_8b_ctx{args.prefill_ctx}_chunk512")
+    p = qas.params(w.n_init, w.window, w.topk, w.eps, w.clamp_c)
+    inp = synthetic.make_esa_inputs(w, device=dev)
+    pf = pipeline.EsaPrefill(w.batch, w.n_ctx, w.chunk, w.hq, w.hkv, w.head_dim, w.d_c, p, device=dev)
+    attn_events = []
+    state = {"collect": False}
+
+    def prefill_step():
+        ev = attn_events if state["collect"] else None
+        pf.run(inp["q"], inp["k"], inp["v"], inp["wq"], inp["wk"], attn_events=ev)
+
+    for _ in range(args.warmup):
+        prefill_step()
+    torch.cuda.synchronize()
+    state["collect"] = True
+    launches0 = qas._abi.launch_count()
+    ms, total_ms = time_steps(prefill_step, args.steps, 0, flush, dist_max)
+    launches = qas._abi.launch_count() - launches0
+    state["collect"] = False
+    tokens = w.batch * w.n_ctx
+    value = world * tokens * args.steps / (total_ms / 1e3)
+    fl = cost.prefill_flops(w.n_ctx, w.chunk, w.hq, w.head_dim, w.d_c, w.n_init, w.window, w.topk)
+    attn_ms = [a.elapsed_time(b) for a, b in attn_events]
+    n_attn = len(attn_ms)
+    attn_time_s = sum(attn_ms) / 1e3
+    achieved = fl["attention"] * args.steps / attn_time_s / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    roofline = {"bound": "tensor", "kernel": "attn_tc_kernel<EsaTcProblem>", "achieved": round(achieved, 1),
+                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "traffic": traffic_for("attn_tc_kernel<EsaTcProblem>", ["attn_tc.cuh", "common.cuh", "keylist.cuh"]),
+                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+                "flops_per_launch": fl["attention"] // (n_attn // args.steps),
+                "launches": n_attn, "avg_launch_us": round(1e3 * sum(attn_ms) / n_attn, 2),
+                "share_of_step": round(sum(attn_ms) / sum(ms), 3)}
+
+    # ---------------------------------------------------------------- e2e through host buffers
+    host = {n: inp[n].cpu().pin_memory() for n in ("q", "k", "v")}
+    out_host = torch.empty(pf.out.shape, dtype=pf.out.dtype).pin_memory()
+    dbuf = {n: torch.empty_like(inp[n]) for n in ("q", "k", "v")}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for n in ("q", "k", "v"):
+            dbuf[n].copy_(host[n], non_blocking=True)
+        o = pf.run(dbuf["q"], dbuf["k"], dbuf["v"], inp["wq"], inp["wk"])
+        out_host.copy_(o, non_blocking=True)
+
+    e_ms, e_total = time_steps(e2e_step, args.e2e_steps, 1, flush, dist_max)
+    e2e = {"value": round(world * tokens * args.e2e_steps / (e_total / 1e3), 1), "unit": "tok/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del host, out_host, dbuf
+
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "model": "llama-3-8b attention layer (random weights)",
+                       "global_batch": w.batch * world, "seq_len": w.n_ctx, "chunk": w.chunk, "hq": w.hq,
+                       "hkv": w.hkv, "head_dim": w.head_dim, "d_c": w.d_c, "n_init": w.n_init,
+                       "window": w.window, "topk": w.topk, "eps": w.eps, "clamp_c": w.clamp_c,
+                       "parallelism": f"replicas x{world}", "l2": "flushed between timed steps (256 MB write)",
+                       "precision": "bf16 attention (fp32 accumulate), fp32 selection"},
+            "roofline": roofline, "e2e": e2e, "gpu_launches": launches}
+
+    # ---------------------------------------------------------------- also: decode, MoBA
+    if not args.no_extras:
+        del inp, pf
+        torch.cuda.empty_cache()
+        line["also"] = {"esa_decode_128k": bench_decode(args, dev, flush, dist_max, peaks, peak_src, world),
+                        "moba_prefill_64k": bench_moba(args, dev, flush, dist_max, peaks, peak_src, world)}
+    line["clocks"] = sampler.stop()
+    line["gpu"] = props.name
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_prefill(seconds_hint=10.0)
+    if _dist is not None:
+        _dist.barrier()
+        _dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def bench_decode(args, dev, flush, dist_max, peaks, peak_src, world):
+    import torch
+    import query_aware_selective_b200 as qas
+    from query_aware_selective_b200 import cost, pipeline, synthetic
+    w = synthetic.DECODE_128K
+    p = qas.params(w.n_init, w.window, w.topk, w.eps, w.clamp_c)
+    inp = synthetic.make_esa_inputs(w, device=dev)
+    dec = pipeline.EsaDecode(w.batch, w.n_ctx, w.hq, w.hkv, w.head_dim, w.d_c, p, device=dev)
+    dec.fill_cache(inp["k"], inp["wk"])
+    torch.cuda.synchronize()
+    phases = []
+    state = {"collect": False}
+
+    def step():
+        ev = None
+        if state["collect"]:
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            phases.append(ev)
+        dec.step(inp["q"], inp["k"], inp["v"], inp["wq"], inp["wk"], phase_events=ev)
+
+    for _ in range(args.warmup):
+        step()
+    state["collect"] = True
+    steps = max(args.steps, 20)
+    ms, total = time_steps(step, steps, 0, flush, dist_max)
+    by = cost.decode_bytes(w.batch, w.n_ctx, w.hq, w.hkv, w.head_dim, w.d_c, w.n_init, w.window, w.topk)
+    sel_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in phases)
+    att_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in phases)
+    hbm = peaks["hbm_gbs"]
+    step_gbs = by["total"] / (total / steps / 1e3) / 1e9
+    sel_gbs = (by["compressed_keys"]) / (sel_ms / 1e3) / 1e9
+    att_gbs = (by["kv_rows"]) / (att_ms / 1e3) / 1e9
+    return {"workload": w.name, "value": round(world * w.batch * steps / (total / 1e3), 1), "unit": "tok/s",
+            "ms_per_step": round(total / steps, 4), "steps": steps,
+            "roofline": {"bound": "hbm", "achieved": round(step_gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(step_gbs / hbm, 4), "bytes_per_step": by["total"],
+                         "peak_source": f"{peak_src} HBM copy"},
+            "phases": {"score_select_ms": round(sel_ms, 4), "score_select_gbs": round(sel_gbs, 1),
+                       "sparse_attn_ms": round(att_ms, 4), "sparse_attn_gbs": round(att_gbs, 1)}}
+
+
+def bench_moba(args, dev, flush, dist_max, peaks, peak_src, world):
+    import torch
+    from query_aware_selective_b200 import cost, pipeline, synthetic
+    w = synthetic.MOBA_64K
+    inp = synthetic.make_moba_inputs(w, device=dev)
+    mb = pipeline.MobaPrefill(w.batch, w.seq, w.heads, w.head_dim, w.block, w.topk, device=dev)
+    step = lambda: mb.run(inp["q"], inp["k"], inp["v"])
+    steps = max(3, args.steps // 2)
+    ms, total = time_steps(step, steps, args.warmup, flush, dist_max)
+    fl = cost.moba_flops(w.seq, w.heads, w.head_dim, w.block, w.topk)
+    ach = fl["total"] / (total / steps / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    return {"workload": w.name, "value": round(world * w.batch * w.seq * steps / (total / 1e3), 1),
+            "unit": "tok/s", "ms_per_step": round(total / steps, 3), "steps": steps,
+            "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(ach / peak, 4), "flops_per_step": fl["total"],
+                         "peak_source": f"{peak_src} bf16 sustained"}}
+
+
+# ----------------------------------------------------------------------------- oracle arm
+
+def oracle_prefill_sample(w, inp_np, c0, rows):
+    """One chunk of the oracle's chunked prefill: compress the chunk's keys and
+    queries, select over the middle, attend `rows` of the chunk's queries.
+    Returns (seconds, tokens-equivalent)."""
+    import numpy as np
+    from oracle import esa as oesa
+    lq = w.chunk
+    t0 = time.perf_counter()
+    kc_new = oesa.compress(inp_np["k"][0, c0:c0 + lq], inp_np["wk"], w.hq)
+    inp_np["k_c"][0, c0:c0 + lq] = kc_new
+    q_c = oesa.compress(inp_np["q"][0, c0:c0 + lq], inp_np["wq"], w.hq)[None]
+    idx, cnt, _ = oesa.score_select(q_c, inp_np["k_c"], c0, w.n_init, w.window, w.topk, w.eps, w.clamp_c)
+    t_sel = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    oesa.sparse_attn(inp_np["q"][:, c0:c0 + lq], inp_np["k"], inp_np["v"], c0, idx, cnt, w.n_init, w.window,
+                     rows=[(0, i) for i in range(rows)])
+    t_att = time.perf_counter() - t1
+    per_token = t_sel / lq + t_att / rows
+    return t_sel + t_att, 1.0 / per_token
+
+
+def oracle_setup(device="cpu"):
+    import numpy as np
+    from oracle import esa as oesa
+    from query_aware_selective_b200 import synthetic
+    w = synthetic.PREFILL_32K
+    inp = synthetic.make_esa_inputs(w, device=device)
+    c0 = (w.n_ctx // 2 // w.chunk) * w.chunk                     # the middle chunk (c0 = 16384)
+    inp_np = {"q": inp["q"][:, c0:c0 + w.chunk].float().cpu().numpy(), "k": inp["k"].float().cpu().numpy(),
+              "v": inp["v"].float().cpu().numpy(), "wq": inp["wq"].cpu().numpy(), "wk": inp["wk"].cpu().numpy()}
+    # queries outside the sampled chunk are not needed: re-index so the chunk sits at c0
+    q_full = np.zeros((1, c0 + w.chunk) + inp_np["q"].shape[2:], dtype=np.float32)
+    q_full[:, c0:] = inp_np["q"]
+    inp_np["q"] = q_full
+    inp_np["k_c"] = np.zeros((1, w.n_ctx, w.d_c))
+    inp_np["k_c"][0, :c0] = oesa.compress(inp_np["k"][0, :c0], inp_np["wk"], w.hq)   # cache state (untimed)
+    return w, inp_np, c0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline_prefill(seconds_hint=10.0):
+    w, inp_np, c0 = oracle_setup()
+    rows = 16
+    secs, tps = oracle_prefill_sample(w, inp_np, c0, rows)
+    return {"value": round(tps, 3), "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"one 512-token chunk at c0={c0} of the 32768-token prefill: compress its keys and queries, "
+                      f"select over its {c0 - w.window - w.n_init}-token middle, attend {rows} of its query rows; "
+                      f"tok/s = 1 / (select time / 512 + attention time / {rows}); {secs:.1f} s of CPU work"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w, inp_np, c0 = oracle_setup()
+    rows = 8
+    for _ in range(args.warmup):
+        oracle_prefill_sample(w, inp_np, c0, rows)
+    vals, secs = [], 0.0
+    for _ in range(args.steps):
+        s, tps = oracle_prefill_sample(w, inp_np, c0, rows)
+        vals.append(tps)
+        secs += s
+    per_tok = sum(1.0 / v for v in vals) / len(vals)
+    value = 1.0 / per_tok
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tok/s",
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * secs / args.steps, 1), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "seq_len": w.n_ctx, "chunk": w.chunk, "global_batch": w.batch},
+            "cpu_baseline": {"kind": "oracle", "cores": blas_threads(), "value": round(value, 3), "unit": "tok/s",
+                             "sample": f"per step: one 512-token chunk at c0={c0} (compress, select) plus "
+                                       f"attention for {rows} of its query rows"},
+            "e2e": {"value": round(value, 3), "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -194,6 +194,10 @@ const char* esa_last_error(void);
  * the last read (the message names the kernel and the wait). */
 esa_status_t esa_device_status(void* stream);
 
+/* Number of kernels this library has launched in this process, all devices and
+ * threads together (accounting only). */
+uint64_t esa_launch_count(void);
+
 /* Library version string. */
 const char* esa_version(void);
 

@@ -41,15 +41,15 @@ def compress(x, w, n_heads_out):
 
     x: [rows, n_heads_in, D]; w: [n_heads_out * D, d']. Returns [rows, d'].
     """
-    x = np.asarray(x, dtype=np.float64)
     w = np.asarray(w, dtype=np.float64)
     rows, n_in, d = x.shape
     assert n_heads_out % n_in == 0
     g = n_heads_out // n_in
     out = np.empty((rows, w.shape[1]), dtype=np.float64)
-    step = 4096
+    step = 4096                                              # row blocks bound the host memory used
     for r0 in range(0, rows, step):
-        xe = np.repeat(x[r0:r0 + step], g, axis=1)          # [r, Hq, D]: head h <- x[:, h // g]
+        xb = np.asarray(x[r0:r0 + step], dtype=np.float64)
+        xe = np.repeat(xb, g, axis=1)                        # [r, Hq, D]: head h <- x[:, h // g]
         out[r0:r0 + step] = xe.reshape(xe.shape[0], n_heads_out * d) @ w
     return out
 

@@ -49,6 +49,7 @@ SIGNATURES = {
     "esa_last_error": (ctypes.c_char_p, []),
     "esa_device_status": (ctypes.c_int, [_vp]),
     "esa_version": (ctypes.c_char_p, []),
+    "esa_launch_count": (ctypes.c_uint64, []),
 }
 
 _lib = None
@@ -253,6 +254,11 @@ def moba_block_gate_attn(q, k, v, block: int, topk: int, scale: float = 0.0, wan
                                        _ptr(blocks) if want_blocks else None, wp, wn, _stream()),
            "moba_block_gate_attn")
     return out, (lse if want_lse else None), (blocks if want_blocks else None)
+
+
+def launch_count() -> int:
+    """Kernels libesa has launched in this process."""
+    return int(load().esa_launch_count())
 
 
 def device_status() -> None:

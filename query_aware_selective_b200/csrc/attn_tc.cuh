@@ -17,8 +17,9 @@
 //
 // The problem policy P says which rows and keys a CTA owns:
 //   bool setup(): per-CTA fields; false = nothing to do
-//   const bf16* q_row(int r): row r's query (nullptr: padding row)
-//   int64_t kv_row(int64_t t): element offset of key t's K/V row (t < n_keys())
+//   int64_t q_row(int r): element offset of row r's query from q_base() (-1: padding)
+//   int64_t kv_pos(int64_t t): row id of key t (t < n_keys()); kv_off(id): its element
+//        offset from kv_base_k() / kv_base_v()
 //   int64_t n_keys(); int64_t limit(int r): last key index row r may attend
 //   void store(int r, const float* o, float m2, float l): o is unnormalised,
 //        m2 the running max in log2 units, l the denominator
@@ -34,7 +35,9 @@ constexpr int kTcKeys = 128;
 constexpr int kTcD = 128;
 constexpr uint32_t kTileBytes = 128 * 256;            // 128 rows x 128 bf16
 constexpr uint32_t kBlkBytes = 128 * 128;             // one 64-column block of a tile
-constexpr uint32_t kTcSmemBytes = 7 * kTileBytes + 1024 /*align*/ + 512 /*barriers*/;
+constexpr uint32_t kTcCtrlBytes = 2048;                       // barriers, TMEM address, key positions
+constexpr uint32_t kTcSmemBytes = 7 * kTileBytes + 1024 /*align*/ + kTcCtrlBytes;
+static_assert(kTcSmemBytes <= 232448, "exceeds the 227 KB of shared memory per CTA");
 
 struct TcSmem {
   uint64_t q_full;
@@ -44,21 +47,69 @@ struct TcSmem {
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
+  int32_t kpos[2][128];      // key rows of the tile being issued, one buffer per loader warp
 };
+static_assert(sizeof(TcSmem) <= kTcCtrlBytes, "control block overflows its reservation");
 
-// Copy one 128 x 128 bf16 tile (rows given by a functor returning the element offset
-// of the row or -1) into swizzled shared memory. 32 threads; lane owns chunk lane % 16
-// of rows lane / 16, lane / 16 + 2, ...
-template <typename RowFn>
-__device__ __forceinline__ void load_tile_rows(uint32_t dst, const __nv_bfloat16* base, RowFn row_off, int lane) {
+// Copy one 128 x 128 bf16 tile into swizzled shared memory: row r comes from element
+// offset off(r) of base (off < 0: zero fill). 32 threads; lane owns the 16-byte chunk
+// lane % 16 of rows lane / 16, lane / 16 + 2, ...
+template <typename OffFn>
+__device__ __forceinline__ void load_tile_rows(uint32_t dst, const __nv_bfloat16* base, OffFn off_of, int lane) {
   const int ch = lane & 15;
   const uint32_t blk = (ch >> 3) * kBlkBytes;
   const uint32_t cc = ch & 7;
-#pragma unroll 4
+#pragma unroll 8
   for (int r = lane >> 4; r < 128; r += 2) {
-    const int64_t off = row_off(r);
+    const int64_t off = off_of(r);
     const void* src = off >= 0 ? (const void*)(base + off + ch * 8) : (const void*)base;
     cp_async16(dst + blk + sw128_off(r, cc), src, off >= 0 ? 16u : 0u);
+  }
+}
+
+// One loader warp streams the key tiles of one operand (K or V) through the two
+// stages. The 128 key positions of tile j + 1 are fetched into registers (4 per lane,
+// consecutive, so gathered index lists are read coalesced) while tile j is issued;
+// they pass through shared memory to the lanes that copy each row. Tile j - 1 is
+// signalled once its copies have landed (own copies waited, then a proxy fence).
+template <class Problem>
+__device__ __forceinline__ void stream_kv(const Problem& prob, const __nv_bfloat16* base, uint32_t stage0,
+                                          uint64_t* full, uint64_t* empty, int32_t* pos_buf, int nt,
+                                          int64_t n_keys, int lane, volatile int* abort_flag, unsigned site) {
+  int32_t pn[4];
+  auto fetch = [&](int j) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int64_t t = (int64_t)j * kTcKeys + lane * 4 + q;
+      pn[q] = t < n_keys ? (int32_t)prob.kv_pos(t) : -1;
+    }
+  };
+  if (nt > 0) fetch(0);
+  bool ok = true;
+  for (int j = 0; j < nt; ++j) {
+    const int s = j & 1;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) pos_buf[lane * 4 + q] = pn[q];
+    __syncwarp();
+    if (j + 1 < nt) fetch(j + 1);
+    ok = mbar_wait(&empty[s], ((j >> 1) & 1) ^ 1, abort_flag, site);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) break;
+    load_tile_rows(stage0 + s * kTileBytes, base,
+                   [&](int r) -> int64_t { const int32_t p = pos_buf[r]; return p >= 0 ? prob.kv_off(p) : -1; },
+                   lane);
+    cp_async_commit();
+    __syncwarp();
+    if (j >= 1) {
+      cp_async_wait<1>();
+      fence_proxy_async();
+      mbar_arrive(&full[(j - 1) & 1]);
+    }
+  }
+  cp_async_wait_all();
+  if (ok && nt > 0) {
+    fence_proxy_async();
+    mbar_arrive(&full[(nt - 1) & 1]);
   }
 }
 
@@ -112,48 +163,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(Problem prob) {
     cp_async_wait_all();
     fence_proxy_async();
     mbar_arrive(&sm.q_full);
-    bool ok = true;
-    for (int j = 0; j < nt && ok; ++j) {
-      const int s = j & 1;
-      ok = mbar_wait(&sm.k_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, 101);
-      if (!ok) break;
-      const int64_t t0 = (int64_t)j * kTcKeys;
-      load_tile_rows(sK + s * kTileBytes, prob.kv_base_k(),
-                     [&](int r) -> int64_t { return t0 + r < n_keys ? prob.kv_row(t0 + r) : -1; }, lane);
-      cp_async_commit();
-      if (j >= 1) {
-        cp_async_wait<1>();
-        fence_proxy_async();
-        mbar_arrive(&sm.k_full[(j - 1) & 1]);
-      }
-    }
-    cp_async_wait_all();
-    if (ok && nt > 0) {
-      fence_proxy_async();
-      mbar_arrive(&sm.k_full[(nt - 1) & 1]);
-    }
+    stream_kv(prob, prob.kv_base_k(), sK, sm.k_full, sm.k_empty, sm.kpos[0], nt, n_keys, lane, abort_flag, 101);
   } else if (warp == 6) {
     // ---------------------------------------------------------------- V loader
-    bool ok = true;
-    for (int j = 0; j < nt && ok; ++j) {
-      const int s = j & 1;
-      ok = mbar_wait(&sm.v_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, 102);
-      if (!ok) break;
-      const int64_t t0 = (int64_t)j * kTcKeys;
-      load_tile_rows(sV + s * kTileBytes, prob.kv_base_v(),
-                     [&](int r) -> int64_t { return t0 + r < n_keys ? prob.kv_row(t0 + r) : -1; }, lane);
-      cp_async_commit();
-      if (j >= 1) {
-        cp_async_wait<1>();
-        fence_proxy_async();
-        mbar_arrive(&sm.v_full[(j - 1) & 1]);
-      }
-    }
-    cp_async_wait_all();
-    if (ok && nt > 0) {
-      fence_proxy_async();
-      mbar_arrive(&sm.v_full[(nt - 1) & 1]);
-    }
+    stream_kv(prob, prob.kv_base_v(), sV, sm.v_full, sm.v_empty, sm.kpos[1], nt, n_keys, lane, abort_flag, 102);
   } else if (warp == 4) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
@@ -332,10 +345,8 @@ struct EsaTcProblem {
     const int i = R / G, hl = R % G;
     return (((int64_t)b * lq + i) * hq + g * G + hl) * kTcD;
   }
-  __device__ int64_t kv_row(int64_t t) const {
-    const int64_t p = keys.pos(b, cnt, t);
-    return (((int64_t)b * n_cap + p) * hkv + g) * kTcD;
-  }
+  __device__ int64_t kv_pos(int64_t t) const { return keys.pos(b, cnt, t); }
+  __device__ int64_t kv_off(int64_t p) const { return (((int64_t)b * n_cap + p) * hkv + g) * kTcD; }
   __device__ int64_t n_keys() const { return nk; }
   __device__ int64_t limit(int r) const {
     const int R = tile * kTcRows + r;

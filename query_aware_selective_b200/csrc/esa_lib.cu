@@ -1,9 +1,12 @@
 // esa_lib.cu - the C ABI of libesa (include/esa.h): argument checks, workspace
 // layout and kernel launches. Every kernel lives in the .cuh files included here, so
 // the library is one translation unit with one copy of the device status word.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -16,11 +19,13 @@
 #include "compress.cuh"
 #include "moba.cuh"
 #include "score.cuh"
+#include "score_tc.cuh"
 #include "topk.cuh"
 
 namespace {
 
 thread_local std::string g_err;
+std::atomic<unsigned long long> g_launches{0};
 
 esa_status_t fail(esa_status_t st, const char* fmt, ...) {
   char buf[512];
@@ -38,6 +43,7 @@ esa_status_t ok() {
 }
 
 esa_status_t check_launch(const char* what) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ESA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
   return ESA_OK;
@@ -99,6 +105,19 @@ esa_status_t check_params(const esa_params_t& p) {
 }
 
 // ------------------------------------------------------------------ score_select --
+// Scoring path: few queries -> registers (S stored); a prefill chunk -> tensor cores
+// (two passes, S never stored); anything else -> SIMT tiles (S stored).
+enum class ScorePath { Small, TensorCore, Tiled };
+
+ScorePath score_path(int32_t batch, int32_t lq, int64_t n_cap, int32_t d_c) {
+  if (lq <= esa::kScoreSmallLq && (d_c == 16 || d_c == 32 || d_c == 64 || d_c == 128 || d_c == 256))
+    return ScorePath::Small;
+  // TMA row coordinates are 32-bit
+  const bool rows_fit = (int64_t)batch * n_cap < ((int64_t)1 << 31) && (int64_t)batch * lq < ((int64_t)1 << 31);
+  if (lq >= 16 && rows_fit && (d_c == 32 || d_c == 64 || d_c == 128)) return ScorePath::TensorCore;
+  return ScorePath::Tiled;
+}
+
 struct SelWs {
   float* S;
   float* s;
@@ -111,21 +130,42 @@ struct SelWs {
   size_t zero_bytes;   // m_key + hist are contiguous and cleared together
 };
 
-SelWs carve_select(void* ws, int32_t batch, int32_t lq, int64_t n_mid) {
+SelWs carve_select(void* ws, int32_t batch, int32_t lq, int64_t n_mid, ScorePath path) {
   Carver c{reinterpret_cast<uint8_t*>(ws)};
   SelWs w;
   const int64_t n_tiles = cdiv(std::max<int64_t>(n_mid, 1), esa::kTkTile);
   w.m_key = c.take<uint32_t>((size_t)batch * lq);
-  const size_t zero_start = 0;
   w.hist = c.take<uint32_t>((size_t)batch * 3 * esa::kTkBins);
-  w.zero_bytes = c.off - zero_start;
-  w.S = c.take<float>((size_t)batch * lq * n_mid);
+  w.zero_bytes = c.off;
+  w.S = path == ScorePath::TensorCore ? nullptr : c.take<float>((size_t)batch * lq * n_mid);
   w.s = c.take<float>((size_t)batch * n_mid);
   w.u = c.take<uint32_t>((size_t)batch * n_mid);
   w.st = c.take<esa::SelState>((size_t)batch);
   w.tiles = c.take<uint2>((size_t)batch * n_tiles);
   w.bytes = c.off;
   return w;
+}
+
+// 2D tensor map over a row-major fp32 matrix [rows, cols], 32 x 128 boxes, 128-byte
+// swizzle (the shared-memory layout the tf32 MMA descriptors expect).
+esa_status_t make_tmap_f32(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    ESA_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+    if (q != cudaDriverEntryPointSuccess || !fn) return fail(ESA_ERR_CUDA, "cuTensorMapEncodeTiled not available");
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * sizeof(float)};
+  cuuint32_t box[2] = {32, 128};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ESA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return ESA_OK;
 }
 
 template <int DC>
@@ -148,6 +188,8 @@ void launch_score_small(const float* q_c, const float* k_c, int lq, int64_t n_ca
 const char* esa_version(void) { return "libesa 0.1 (sm_100a)"; }
 
 const char* esa_last_error(void) { return g_err.c_str(); }
+
+uint64_t esa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 esa_status_t esa_device_status(void* stream) {
   ESA_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
@@ -206,7 +248,7 @@ size_t esa_score_select_workspace_size(int32_t batch, int32_t lq, int64_t n_cap,
   (void)d_c;
   if (batch <= 0 || lq <= 0) return 0;
   const Regions r = regions(c0, p);
-  return carve_select(nullptr, batch, lq, r.n_mid).bytes;
+  return carve_select(nullptr, batch, lq, r.n_mid, score_path(batch, lq, n_cap, d_c)).bytes;
 }
 
 esa_status_t esa_score_select(const float* q_c, const float* k_c, int32_t batch, int32_t lq, int64_t n_cap,
@@ -226,13 +268,13 @@ esa_status_t esa_score_select(const float* q_c, const float* k_c, int32_t batch,
   const int64_t kk = std::min<int64_t>(p.topk, r.n_mid);
   const bool need_scores = r.n_mid > p.topk || (score_out && r.n_mid > 0);
   if (need_scores) {
-    const SelWs need = carve_select(nullptr, batch, lq, r.n_mid);
+    const ScorePath path = score_path(batch, lq, n_cap, d_c);
+    const SelWs need = carve_select(nullptr, batch, lq, r.n_mid, path);
     if (!workspace || ws_bytes < need.bytes || !aligned(workspace, 256))
       return fail(ESA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need.bytes, ws_bytes);
-    const SelWs w = carve_select(workspace, batch, lq, r.n_mid);
+    const SelWs w = carve_select(workspace, batch, lq, r.n_mid, path);
     ESA_CUDA(cudaMemsetAsync(w.m_key, 0, w.zero_bytes, s));
-    const bool small = lq <= esa::kScoreSmallLq && (d_c == 16 || d_c == 32 || d_c == 64 || d_c == 128 || d_c == 256);
-    if (small) {
+    if (path == ScorePath::Small) {
       switch (d_c) {
         case 16: launch_score_small<16>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, w.S, w.m_key, s); break;
         case 32: launch_score_small<32>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, w.S, w.m_key, s); break;
@@ -240,14 +282,39 @@ esa_status_t esa_score_select(const float* q_c, const float* k_c, int32_t batch,
         case 128: launch_score_small<128>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, w.S, w.m_key, s); break;
         default: launch_score_small<256>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, w.S, w.m_key, s); break;
       }
-    } else {
+      ESA_LAUNCH_CHECK("score_small_kernel");
+    } else if (path == ScorePath::Tiled) {
       dim3 grid((unsigned)cdiv(r.n_mid, esa::kScT), (unsigned)cdiv(lq, esa::kScT), batch);
       esa::score_tiled_kernel<<<grid, 256, 0, s>>>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, d_c, w.S, w.m_key);
+      ESA_LAUNCH_CHECK("score_tiled_kernel");
     }
-    ESA_LAUNCH_CHECK("score kernel");
-    esa::clamp_sum_kernel<<<dim3((unsigned)cdiv(r.n_mid, 256), batch), 256, 0, s>>>(w.S, w.m_key, lq, r.n_mid,
-                                                                                    p.clamp_c, w.s);
-    ESA_LAUNCH_CHECK("clamp_sum_kernel");
+    if (path == ScorePath::TensorCore) {
+      CUtensorMap tm_k, tm_q;
+      st = make_tmap_f32(&tm_k, k_c, (uint64_t)batch * n_cap, d_c);
+      if (st != ESA_OK) return st;
+      st = make_tmap_f32(&tm_q, q_c, (uint64_t)batch * lq, d_c);
+      if (st != ESA_OK) return st;
+      esa::ScoreTcArgs a{lq, d_c, n_cap, r.mid0, r.n_mid, w.m_key, w.s, p.clamp_c};
+      const int smem = 1024 + 3 * esa::kStRows * d_c * 4 + 256 + lq * 4;
+      static bool attr_set[64] = {};
+      int dev = 0;
+      ESA_CUDA(cudaGetDevice(&dev));
+      if (dev < 64 && !attr_set[dev]) {
+        const int max_smem = 1024 + 3 * esa::kStRows * 128 * 4 + 256 + 4096 * 4;
+        if ((st = set_max_smem(esa::score_tc_kernel<1>, max_smem)) != ESA_OK) return st;
+        if ((st = set_max_smem(esa::score_tc_kernel<2>, max_smem)) != ESA_OK) return st;
+        attr_set[dev] = true;
+      }
+      const dim3 grid((unsigned)cdiv(r.n_mid, esa::kStRows), batch);
+      esa::score_tc_kernel<1><<<grid, esa::kStThreads, smem, s>>>(tm_k, tm_q, a);
+      ESA_LAUNCH_CHECK("score_tc_kernel<1>");
+      esa::score_tc_kernel<2><<<grid, esa::kStThreads, smem, s>>>(tm_k, tm_q, a);
+      ESA_LAUNCH_CHECK("score_tc_kernel<2>");
+    } else {
+      esa::clamp_sum_kernel<<<dim3((unsigned)cdiv(r.n_mid, 256), batch), 256, 0, s>>>(w.S, w.m_key, lq, r.n_mid,
+                                                                                      p.clamp_c, w.s);
+      ESA_LAUNCH_CHECK("clamp_sum_kernel");
+    }
     const int n_tiles = (int)cdiv(r.n_mid, esa::kTkTile);
     const dim3 tgrid(n_tiles, batch);
     esa::pool_hist_kernel<<<tgrid, esa::kTkThreads, 0, s>>>(w.s, r.n_mid, p.eps, w.u, score_out, w.hist);
@@ -341,6 +408,7 @@ esa_status_t esa_sparse_attn(const void* q, const void* k, const void* v, esa_dt
   const int g = hq / hkv;
   if (g != 1 && g != 2 && g != 4 && g != 8) return fail(ESA_ERR_UNSUPPORTED, "GQA group %d (1, 2, 4 or 8)", g);
   if (c0 < 0 || c0 + lq > n_cap) return fail(ESA_ERR_INVALID_ARG, "need 0 <= c0 and c0 + lq <= n_cap");
+  if (n_cap >= ((int64_t)1 << 31)) return fail(ESA_ERR_UNSUPPORTED, "n_cap must be < 2^31");
   if (!q || !k || !v || !o || !idx || !count) return fail(ESA_ERR_INVALID_ARG, "null pointer");
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16))
     return fail(ESA_ERR_INVALID_ARG, "q, k, v, o need 16-byte alignment");

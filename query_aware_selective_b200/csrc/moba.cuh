@@ -242,9 +242,8 @@ struct MobaPastProblem {
     return (((int64_t)b * seq + p) * heads + h) * kTcD;
   }
   __device__ int64_t n_keys() const { return min((int64_t)block, seq - (int64_t)blk * block); }
-  __device__ int64_t kv_row(int64_t t) const {
-    return (((int64_t)b * seq + (int64_t)blk * block + t) * heads + h) * kTcD;
-  }
+  __device__ int64_t kv_pos(int64_t t) const { return (int64_t)blk * block + t; }
+  __device__ int64_t kv_off(int64_t p) const { return (((int64_t)b * seq + p) * heads + h) * kTcD; }
   __device__ int64_t limit(int) const { return n_keys() - 1; }
   __device__ float scale_log2() const { return sl2; }
   __device__ void store(int r, const float* acc, float m2, float l) {
@@ -296,7 +295,8 @@ struct MobaCurrentProblem {
     return (((int64_t)b * seq + p0 + r) * heads + h) * kTcD;
   }
   __device__ int64_t n_keys() const { return p0 + nrows - kb0; }
-  __device__ int64_t kv_row(int64_t t) const { return (((int64_t)b * seq + kb0 + t) * heads + h) * kTcD; }
+  __device__ int64_t kv_pos(int64_t t) const { return kb0 + t; }
+  __device__ int64_t kv_off(int64_t p) const { return (((int64_t)b * seq + p) * heads + h) * kTcD; }
   __device__ int64_t limit(int r) const { return p0 + min((int64_t)r, nrows - 1) - kb0; }
   __device__ float scale_log2() const { return sl2; }
   __device__ void store(int r, const float* acc, float m2, float l) {

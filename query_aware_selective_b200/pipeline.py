@@ -1,0 +1,146 @@
+"""Host drivers of the hot path: ESA chunked prefill, ESA decode, MoBA prefill.
+
+ESA write-up, implementation paragraph: key and value are cached chunk by chunk;
+each chunk's queries select the important middle tokens (all queries of the chunk
+count), and in decoding the single current query does. These classes hold the
+caller-side state (compressed key cache, index buffers, workspaces, outputs) and
+issue the C-ABI calls in order on the current stream. They allocate everything up
+front, so a step launches kernels only and can be captured in a CUDA graph.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import torch
+
+from . import _abi
+
+
+def _region_lo(c0: int, n_init: int, window: int) -> int:
+    return min(c0, max(n_init, c0 - window))
+
+
+class EsaPrefill:
+    """Chunked prefill of one attention layer: for every chunk [c0, c0 + chunk),
+    compress the chunk's keys into the compressed cache, compress its queries,
+    select middle tokens, attend over initial + selected + local."""
+
+    def __init__(self, batch: int, n_ctx: int, chunk: int, hq: int, hkv: int, head_dim: int, d_c: int,
+                 p: _abi.EsaParams, dtype=torch.bfloat16, device="cuda"):
+        self.batch, self.n_ctx, self.chunk = batch, n_ctx, chunk
+        self.hq, self.hkv, self.d, self.d_c, self.p = hq, hkv, head_dim, d_c, p
+        self.device = torch.device(device)
+        self.k_c = torch.zeros((batch, n_ctx, d_c), dtype=torch.float32, device=device)
+        self.q_c = torch.empty((batch, chunk, d_c), dtype=torch.float32, device=device)
+        self.idx = torch.empty((batch, p.topk), dtype=torch.int32, device=device)
+        self.count = torch.empty((batch,), dtype=torch.int32, device=device)
+        self.out = torch.empty((batch, n_ctx, hq, head_dim), dtype=dtype, device=device)
+        code = _abi.ESA_BF16 if dtype == torch.bfloat16 else _abi.ESA_F32
+        ws_sel = max(_abi.score_select_workspace_size(batch, min(chunk, n_ctx - c0), n_ctx, c0, d_c, p)
+                     for c0 in range(0, n_ctx, chunk))
+        ws_att = max(_abi.sparse_attn_workspace_size(batch, min(chunk, n_ctx - c0), c0, hq, hkv, head_dim, code, p)
+                     for c0 in range(0, n_ctx, chunk))
+        self.ws_sel = torch.empty(ws_sel + 256, dtype=torch.uint8, device=device)
+        self.ws_att = torch.empty(ws_att + 256, dtype=torch.uint8, device=device) if ws_att else None
+        self.out_views = []
+
+    def chunks(self):
+        return [(c0, min(self.chunk, self.n_ctx - c0)) for c0 in range(0, self.n_ctx, self.chunk)]
+
+    def run_chunk(self, c0: int, lq: int, q, k, v, wq, wk, attn_events=None):
+        b = self.batch
+        for s in range(b):
+            _abi.compress(k[s, c0:c0 + lq], wk, self.hq, out=self.k_c[s, c0:c0 + lq])
+            _abi.compress(q[s, c0:c0 + lq], wq, self.hq, out=self.q_c[s, :lq])
+        q_c = self.q_c[:, :lq] if lq == self.chunk else self.q_c[:, :lq].contiguous()
+        _abi.score_select(q_c, self.k_c, c0, self.p, idx=self.idx, count=self.count, workspace=self.ws_sel)
+        qv = q[:, c0:c0 + lq]
+        if not qv.is_contiguous():
+            qv = qv.contiguous()
+        ov = self.out[:, c0:c0 + lq]
+        target = ov if ov.is_contiguous() else torch.empty_like(ov)
+        if attn_events is not None:
+            attn_events[0].record()
+        _abi.sparse_attn(qv, k, v, c0, self.idx, self.count, self.p, out=target, workspace=self.ws_att)
+        if attn_events is not None:
+            attn_events[1].record()
+        if target is not ov:
+            ov.copy_(target)
+
+    def run(self, q, k, v, wq, wk, attn_events=None):
+        """q [B, N, Hq, D], k, v [B, N, Hkv, D] (device), wq, wk [Hq*D, d'].
+        attn_events: optional list that receives one (start, end) CUDA event pair per
+        attention launch. Returns the output [B, N, Hq, D]."""
+        for c0, lq in self.chunks():
+            ev = None
+            if attn_events is not None:
+                ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                attn_events.append(ev)
+            self.run_chunk(c0, lq, q, k, v, wq, wk, ev)
+        return self.out
+
+
+class EsaDecode:
+    """One decode step for a batch: compress the new query and the new key (written
+    into the compressed cache), select over the middle, attend. The KV cache holds
+    n_ctx tokens; the query sits at position n_ctx - 1."""
+
+    def __init__(self, batch: int, n_ctx: int, hq: int, hkv: int, head_dim: int, d_c: int, p: _abi.EsaParams,
+                 dtype=torch.bfloat16, device="cuda"):
+        self.batch, self.n_ctx, self.hq, self.hkv, self.d, self.d_c, self.p = batch, n_ctx, hq, hkv, head_dim, d_c, p
+        self.k_c = torch.zeros((batch, n_ctx, d_c), dtype=torch.float32, device=device)
+        self.q_c = torch.empty((batch, 1, d_c), dtype=torch.float32, device=device)
+        self.idx = torch.empty((batch, p.topk), dtype=torch.int32, device=device)
+        self.count = torch.empty((batch,), dtype=torch.int32, device=device)
+        self.out = torch.empty((batch, 1, hq, head_dim), dtype=dtype, device=device)
+        code = _abi.ESA_BF16 if dtype == torch.bfloat16 else _abi.ESA_F32
+        c0 = n_ctx - 1
+        self.ws_sel = torch.empty(_abi.score_select_workspace_size(batch, 1, n_ctx, c0, d_c, p) + 256,
+                                  dtype=torch.uint8, device=device)
+        nb = _abi.sparse_attn_workspace_size(batch, 1, c0, hq, hkv, head_dim, code, p)
+        self.ws_att = torch.empty(nb + 256, dtype=torch.uint8, device=device) if nb else None
+
+    def fill_cache(self, k, wk, upto: Optional[int] = None):
+        """Compress cached keys [0, upto) of every sequence (prefill state)."""
+        upto = self.n_ctx - 1 if upto is None else upto
+        step = 1 << 16
+        for s in range(self.batch):
+            for r0 in range(0, upto, step):
+                r1 = min(upto, r0 + step)
+                _abi.compress(k[s, r0:r1], wk, self.hq, out=self.k_c[s, r0:r1])
+
+    def step(self, q, k, v, wq, wk, phase_events=None):
+        """q [B, 1, Hq, D]; k, v [B, n_ctx, Hkv, D] with the new token at n_ctx - 1."""
+        pos = self.n_ctx - 1
+        ev = phase_events
+        if ev is not None:
+            ev[0].record()
+        _abi.compress(q[:, 0], wq, self.hq, out=self.q_c.view(self.batch, self.d_c))
+        _abi.compress(k[:, pos], wk, self.hq, out=self.k_c[:, pos], out_row_stride=self.n_ctx * self.d_c)
+        if ev is not None:
+            ev[1].record()
+        _abi.score_select(self.q_c, self.k_c, pos, self.p, idx=self.idx, count=self.count, workspace=self.ws_sel)
+        if ev is not None:
+            ev[2].record()
+        _abi.sparse_attn(q, k, v, pos, self.idx, self.count, self.p, out=self.out, workspace=self.ws_att)
+        if ev is not None:
+            ev[3].record()
+        return self.out
+
+
+class MobaPrefill:
+    """MoBA causal prefill of one layer: gate, then block attention."""
+
+    def __init__(self, batch: int, seq: int, heads: int, head_dim: int, block: int, topk: int,
+                 dtype=torch.bfloat16, device="cuda"):
+        self.batch, self.seq, self.heads, self.d, self.block, self.topk = batch, seq, heads, head_dim, block, topk
+        self.out = torch.empty((batch, seq, heads, head_dim), dtype=dtype, device=device)
+        self.blocks = torch.empty((batch, seq, heads, topk + 1), dtype=torch.int16, device=device)
+        self.ws = torch.empty(_abi.moba_workspace_size(2, batch, seq, heads, head_dim, block, topk) + 256,
+                              dtype=torch.uint8, device=device)
+
+    def run(self, q, k, v):
+        _abi.moba_block_gate_attn(q, k, v, self.block, self.topk, out=self.out, blocks=self.blocks,
+                                  want_blocks=True, workspace=self.ws)
+        return self.out

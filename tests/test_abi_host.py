@@ -29,7 +29,7 @@ def lib():
 def header_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return re.findall(r"^\s*(?:esa_status_t|size_t|const char\*)\s+(\w+)\s*\(", text, flags=re.M)
+    return re.findall(r"^\s*(?:esa_status_t|size_t|uint64_t|const char\*)\s+(\w+)\s*\(", text, flags=re.M)
 
 
 def test_header_declares_the_boundary():
@@ -132,6 +132,13 @@ def test_binding_refuses_cpu_tensors():
     w = torch.zeros(4096, 128)
     with pytest.raises(ValueError, match="CUDA"):
         qas.compress(x, w, 32)
+
+
+def test_rejected_calls_launch_nothing(lib):
+    before = lib.esa_launch_count()
+    lib.esa_compress(None, 1, 4, 1024, 8, 32, 128, FAKE, 128, FAKE, 128, None)
+    lib.esa_compress(FAKE, 1, 0, 1024, 8, 32, 128, FAKE, 128, FAKE, 128, None)
+    assert lib.esa_launch_count() == before
 
 
 def test_missing_library_fails_loudly(tmp_path):

@@ -1,0 +1,110 @@
+"""Parity at the full benchmark sizes, in the launch configuration bench.py times
+(the same pipeline drivers), on outputs the oracle computes one by one: whole
+sequences for decode, sampled chunks and rows for prefill, sampled positions for
+MoBA."""
+import numpy as np
+import pytest
+import torch
+
+import query_aware_selective_b200 as qas
+from oracle import esa as oesa
+from oracle import moba as omoba
+from query_aware_selective_b200 import pipeline, synthetic
+from tests.parity import ATOL_BF16, check_selection, max_abs
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _f64(t):
+    return t.detach().cpu().double().numpy()
+
+
+def _decode_full(w, seqs):
+    p = qas.params(w.n_init, w.window, w.topk, w.eps, w.clamp_c)
+    inp = synthetic.make_esa_inputs(w, device=DEV)
+    dec = pipeline.EsaDecode(w.batch, w.n_ctx, w.hq, w.hkv, w.head_dim, w.d_c, p, device=DEV)
+    dec.fill_cache(inp["k"], inp["wk"])
+    o = dec.step(inp["q"], inp["k"], inp["v"], inp["wq"], inp["wk"]).clone()
+    idx, cnt = dec.idx.cpu().numpy(), dec.count.cpu().numpy()
+    qas.device_status()
+    _, (m0, _), _ = oesa.regions(w.n_ctx - 1, w.n_ctx, w.n_init, w.window)
+    wq, wk = inp["wq"].cpu().numpy(), inp["wk"].cpu().numpy()
+    for b in seqs:
+        qb = inp["q"][b:b + 1].float().cpu().numpy()
+        kb = inp["k"][b:b + 1].float().cpu().numpy()
+        vb = inp["v"][b:b + 1].float().cpu().numpy()
+        ref = oesa.decode_step(qb, kb, vb, wq, wk, w.n_init, w.window, w.topk, w.eps, w.clamp_c)
+        check_selection(idx[b], cnt[b], ref["idx"][0], ref["count"][0], ref["s_prime"][0], m0, w.topk)
+        chosen = set(idx[b, :cnt[b]].tolist())
+        for pos in inp["needles"][b].tolist():
+            assert all(j in chosen for j in range(pos - w.eps, pos + w.eps + 1)), pos
+        assert max_abs(_f64(o[b:b + 1]), ref["o"]) <= ATOL_BF16
+    del inp, dec
+    torch.cuda.empty_cache()
+
+
+def test_decode_128k_batch16():
+    _decode_full(synthetic.DECODE_128K, seqs=(0, 15))
+
+
+def test_decode_1m_batch4():
+    _decode_full(synthetic.DECODE_1M, seqs=(0,))
+
+
+def test_prefill_32k_sampled_chunks():
+    w = synthetic.PREFILL_32K
+    p = qas.params(w.n_init, w.window, w.topk, w.eps, w.clamp_c)
+    inp = synthetic.make_esa_inputs(w, device=DEV)
+    pf = pipeline.EsaPrefill(w.batch, w.n_ctx, w.chunk, w.hq, w.hkv, w.head_dim, w.d_c, p, device=DEV)
+    sampled = {0: None, 13: None, 40: None, 63: None}
+    for ci, (c0, lq) in enumerate(pf.chunks()):
+        pf.run_chunk(c0, lq, inp["q"], inp["k"], inp["v"], inp["wq"], inp["wk"])
+        if ci in sampled:
+            sampled[ci] = (pf.idx.cpu().numpy().copy(), pf.count.cpu().numpy().copy())
+    out = pf.out
+    qas.device_status()
+    qn = inp["q"].float().cpu().numpy()
+    kn = inp["k"].float().cpu().numpy()
+    vn = inp["v"].float().cpu().numpy()
+    wq, wk = inp["wq"].cpu().numpy(), inp["wk"].cpu().numpy()
+    k_c = oesa.compress(kn[0], wk, w.hq)[None]
+    rng = np.random.default_rng(0)
+    for ci, (idx, cnt) in sampled.items():
+        c0 = ci * w.chunk
+        rows = sorted(set(rng.integers(0, w.chunk, 6).tolist()) | {0, w.chunk - 1})
+        ref = oesa.prefill_chunk(qn[:, c0:c0 + w.chunk], kn, vn, k_c, wq, c0, w.n_init, w.window, w.topk, w.eps,
+                                 w.clamp_c, rows=[(0, i) for i in rows])
+        _, (m0, _), _ = oesa.regions(c0, c0 + w.chunk, w.n_init, w.window)
+        check_selection(idx[0], cnt[0], ref["idx"][0], ref["count"][0], ref["s_prime"][0], m0, w.topk)
+        got = _f64(out[:, c0:c0 + w.chunk])
+        assert max_abs(got[:, rows], ref["o"][:, rows]) <= ATOL_BF16
+
+
+def test_moba_64k_sampled_positions():
+    w = synthetic.MOBA_64K
+    inp = synthetic.make_moba_inputs(w, device=DEV)
+    mb = pipeline.MobaPrefill(w.batch, w.seq, w.heads, w.head_dim, w.block, w.topk, device=DEV)
+    out = mb.run(inp["q"], inp["k"], inp["v"])
+    blocks = mb.blocks.cpu().numpy().astype(np.int64)
+    qas.device_status()
+    kn = inp["k"].float().cpu().numpy()
+    kbar = omoba.block_means(kn, w.block)
+    qn = inp["q"].float().cpu().numpy()
+    vn = inp["v"].float().cpu().numpy()
+    rng = np.random.default_rng(1)
+    pos = sorted(set(rng.integers(0, w.seq, 20).tolist()) | {0, w.block - 1, w.block, 3 * w.block + 5, w.seq - 1})
+    ref_blocks = omoba.gate(qn, kbar, w.block, w.topk, positions=pos)
+    got_blocks = blocks[:, pos]
+    same = np.all(got_blocks == ref_blocks, axis=-1)
+    for b, r, h in zip(*np.nonzero(~same)):
+        p_ = pos[r]
+        cur = p_ // w.block
+        sc = kbar[b, h, :cur] @ qn[b, p_, h]
+        kth = np.sort(sc)[::-1][min(w.topk, cur) - 1]
+        for blk in set(got_blocks[b, r, h].tolist()) ^ set(ref_blocks[b, r, h].tolist()):
+            assert abs(sc[blk] - kth) <= 1e-3 * abs(kth) + 1e-6
+    assert same.mean() > 0.97
+    ref_o, _ = omoba.attend(qn, kn, vn, ref_blocks, w.block, positions=pos)
+    got = _f64(out[:, pos])
+    assert max_abs(got[same], ref_o[same]) <= ATOL_BF16

@@ -16,7 +16,7 @@ from tests import test_oracle_moba as pm
 
 MUTATIONS = [
     # (module, function, snippet, replacement, pin)
-    (esa, "compress", "np.repeat(x[r0:r0 + step], g, axis=1)", "np.tile(x[r0:r0 + step], (1, g, 1))",
+    (esa, "compress", "np.repeat(xb, g, axis=1)", "np.tile(xb, (1, g, 1))",
      pe.check_identity_compression_is_multihead_dot),                      # GQA head order
     (esa, "importance", "corrected = np.maximum(corrected, -float(clamp_c))", "pass",
      pe.check_worked_example),                                             # clamp dropped
