@@ -3,8 +3,10 @@
 // One CTA computes 128 query rows against a list of key rows, 128 keys per step:
 //   S_j  = Q K_j^T          tcgen05.mma kind::f16 (bf16 in, fp32 accumulate), TMEM
 //   P_j  = exp2(S_j * c - m) softmax warps read S_j from TMEM, write bf16 P_j to smem
-//   PV_j = P_j V_j          tcgen05.mma into a second TMEM buffer
-//   o    = o * alpha + PV_j the softmax warps accumulate o in registers (one row each)
+//   O   += P_j V_j          tcgen05.mma accumulating in TMEM
+// m is the running row maximum used for the exponentials; it is raised (and O, l
+// rescaled in place) only when a tile's maximum exceeds it by more than 2^8, so most
+// tiles skip the rescale and P stays <= 2^8 (exact softmax either way: o = O / l).
 // Roles (224 threads): warps 0-3 softmax (thread = row = TMEM lane), warp 4 issues
 // the MMAs (one lane), warp 5 loads Q and the K rows, warp 6 loads the V rows.
 // K/V rows are gathered by cp.async (16-byte pieces) straight into the 128-byte
@@ -13,7 +15,7 @@
 //
 // Shared memory: Q 32 KB, K 2 x 32 KB, V 2 x 32 KB, P 2 x 32 KB (each operand tile is
 // two 16 KB column blocks of 128 rows x 128 bytes). TMEM: S double buffer (2 x 128
-// columns) and PV double buffer (2 x 128 columns) = 512 columns.
+// columns) and the O accumulator (128 columns).
 //
 // The problem policy P says which rows and keys a CTA owns:
 //   bool setup(): per-CTA fields; false = nothing to do
@@ -43,7 +45,7 @@ struct TcSmem {
   uint64_t q_full;
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
   uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
-  uint64_t pv_full[2], pv_empty[2];
+  uint64_t pv_full[2];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -140,7 +142,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(Problem prob) {
       mbar_init(&sm.p_full[s], 128);
       mbar_init(&sm.p_empty[s], 1);
       mbar_init(&sm.pv_full[s], 1);
-      mbar_init(&sm.pv_empty[s], 128);
     }
     mbar_init(&sm.mma_done, 1);
     sm.abort_flag = 0;
@@ -195,7 +196,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(Problem prob) {
         if (j + 1 < nt && !(ok = issue_s(j + 1))) break;
         if (!(ok = mbar_wait(&sm.p_full[s], (j >> 1) & 1, abort_flag, 106))) break;
         if (!(ok = mbar_wait(&sm.v_full[s], (j >> 1) & 1, abort_flag, 107))) break;
-        if (!(ok = mbar_wait(&sm.pv_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, 108))) break;
         tc_fence_after();
         const uint32_t pt = sP + s * kTileBytes;
         const uint32_t vt = sV + s * kTileBytes;
@@ -204,8 +204,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(Problem prob) {
           // A = P (K-major: keys along the 128-byte rows); B = V (MN-major: 8-key row
           // groups of 1024 bytes, d blocks of 64 columns 16 KB apart)
           const uint32_t poff = (kk >> 2) * kBlkBytes + (kk & 3) * 32;
-          umma_f16_ss(tmem + 256 + s * 128, sdesc_sw128(pt + poff, 16, 1024),
-                      sdesc_sw128(vt + kk * 2048, kBlkBytes, 1024), idesc_pv, kk > 0);
+          umma_f16_ss(tmem + 256, sdesc_sw128(pt + poff, 16, 1024), sdesc_sw128(vt + kk * 2048, kBlkBytes, 1024),
+                      idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&sm.pv_full[s]);
         umma_commit(&sm.p_empty[s]);
@@ -220,85 +220,81 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(Problem prob) {
     // ---------------------------------------------------------------- softmax (rows)
     const int r = threadIdx.x;                 // 0..127 = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t o_addr = lane_base + 256;
     const int64_t lim = prob.limit(r);
     const float sl2 = prob.scale_log2();
-    float o[kTcD];
-#pragma unroll
-    for (int e = 0; e < kTcD; ++e) o[e] = 0.f;
-    float m = -INFINITY, l = 0.f, alpha_pend = 0.f;
+    constexpr float kRescale = 8.0f;           // log2 units: rescale when the max grows by > 2^8
+    float m = -INFINITY, l = 0.f;
     bool ok = true;
-    auto consume_pv = [&](int j) -> bool {
-      const int s = j & 1;
-      if (!mbar_wait_warp(&sm.pv_full[s], (j >> 1) & 1, abort_flag, 110)) return false;
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float x[32];
-        tmem_ld32(lane_base + 256 + s * 128 + c * 32, x);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[c * 32 + e] = fmaf(o[c * 32 + e], alpha_pend, x[e]);
-      }
-      tc_fence_before();
-      mbar_arrive(&sm.pv_empty[s]);
-      return true;
-    };
     for (int j = 0; j < nt; ++j) {
       const int s = j & 1;
       if (!(ok = mbar_wait_warp(&sm.s_full[s], (j >> 1) & 1, abort_flag, 111))) break;
       tc_fence_after();
       const int64_t t0 = (int64_t)j * kTcKeys;
-      const uint32_t sa = lane_base + s * 128;
+      float x[kTcKeys];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + s * 128 + c * 32, x + c * 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&sm.s_empty[s]);             // S now lives in registers
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float x[32];
-        tmem_ld32(sa + c * 32, x);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int64_t t = t0 + c * 32 + e;
-          mx = fmaxf(mx, t <= lim ? x[e] * sl2 : -INFINITY);
-        }
+      for (int e = 0; e < kTcKeys; ++e) {
+        x[e] = (t0 + e <= lim) ? x[e] * sl2 : -INFINITY;
+        mx = fmaxf(mx, x[e]);
       }
-      const float m_new = fmaxf(m, mx);
-      const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      const float alpha = fast_exp2(m - m_use);
+      if (mx > m + kRescale || m == -INFINITY) {
+        const float m_new = fmaxf(m, mx);
+        if (j > 0 && m_new > m) {
+          const float alpha = fast_exp2(m - m_new);
+          // O holds PV_0..PV_{j-1}; wait for the last of them, then scale in place
+          if (!(ok = mbar_wait_warp(&sm.pv_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, 110))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float ov[32];
+            tmem_ld32(o_addr + c * 32, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+            tmem_st32(o_addr + c * 32, ov);
+          }
+          tmem_wait_st();
+          l *= alpha;
+        }
+        m = m_new;
+      }
+      const float m_use = m == -INFINITY ? 0.f : m;
       if (!(ok = mbar_wait_warp(&sm.p_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, 112))) break;
       const uint32_t pt = sP + s * kTileBytes;
       float lsum = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float x[32];
-        tmem_ld32(sa + c * 32, x);
-        tmem_wait_ld();
-        uint32_t pk[16];
+      for (int c = 0; c < 16; ++c) {           // 16-byte chunks of the 256-byte P row
+        uint32_t pk[4];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int64_t t = t0 + c * 32 + e;
-          const float p0 = t <= lim ? fast_exp2(x[e] * sl2 - m_use) : 0.f;
-          const float p1 = t + 1 <= lim ? fast_exp2(x[e + 1] * sl2 - m_use) : 0.f;
+        for (int e = 0; e < 8; e += 2) {
+          const float p0 = fast_exp2(x[c * 8 + e] - m_use);
+          const float p1 = fast_exp2(x[c * 8 + e + 1] - m_use);
           lsum += p0 + p1;
           pk[e / 2] = pack_bf16x2(p0, p1);
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int chunk = c * 4 + q;                 // 16-byte chunk of the 256-byte row
-          const uint32_t dst = pt + (chunk >> 3) * kBlkBytes + sw128_off(r, chunk & 7);
-          st_shared_v4(dst, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        }
+        const uint32_t dst = pt + (c >> 3) * kBlkBytes + sw128_off(r, c & 7);
+        st_shared_v4(dst, pk[0], pk[1], pk[2], pk[3]);
       }
-      tc_fence_before();
-      mbar_arrive(&sm.s_empty[s]);
+      l += lsum;
       fence_proxy_async();
+      tc_fence_before();
       mbar_arrive(&sm.p_full[s]);
-      l = l * alpha + lsum;
-      m = m_new;
-      if (j >= 1 && !(ok = consume_pv(j - 1))) break;
-      alpha_pend = alpha;
     }
-    if (ok && nt > 0) ok = consume_pv(nt - 1);
-    if (ok) prob.store(r, o, m, l);
+    if (ok && nt > 0) ok = mbar_wait_warp(&sm.pv_full[(nt - 1) & 1], ((nt - 1) >> 1) & 1, abort_flag, 113);
+    if (ok) {
+      tc_fence_after();
+      float o[kTcD];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(o_addr + c * 32, o + c * 32);
+      tmem_wait_ld();
+      prob.store(r, o, m, l);
+    }
   }
 
   tc_fence_before();

@@ -17,6 +17,7 @@
 #include "attn_tc.cuh"
 #include "common.cuh"
 #include "compress.cuh"
+#include "compress_tc.cuh"
 #include "moba.cuh"
 #include "score.cuh"
 #include "score_tc.cuh"
@@ -219,6 +220,28 @@ esa_status_t esa_compress(const void* x, esa_dtype_t x_dtype, int64_t rows, int6
   if (x_row_stride < (int64_t)n_heads_in * head_dim || x_row_stride % 8)
     return fail(ESA_ERR_INVALID_ARG, "x_row_stride must be >= n_heads_in * head_dim and a multiple of 8");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (x_dtype == ESA_BF16 && d_out == esa::kCtN) {
+    // tensor-core path: 8-CTA clusters split the reduction, 128 rows per cluster
+    static bool attr_set[64] = {};
+    int dev = 0;
+    ESA_CUDA(cudaGetDevice(&dev));
+    if (dev < 64 && !attr_set[dev]) {
+      const esa_status_t st = set_max_smem(esa::compress_tc_kernel, esa::kCtSmemBytes);
+      if (st != ESA_OK) return st;
+      attr_set[dev] = true;
+    }
+    const int g = n_heads_out / n_heads_in;
+    const int64_t max_rows = (int64_t)65535 * esa::kCtRows;
+    for (int64_t r0 = 0; r0 < rows; r0 += max_rows) {
+      const int64_t nr = std::min(rows - r0, max_rows);
+      const dim3 grid(esa::kCtCluster, (unsigned)cdiv(nr, esa::kCtRows));
+      esa::compress_tc_kernel<<<grid, esa::kCtThreads, esa::kCtSmemBytes, s>>>(
+          static_cast<const __nv_bfloat16*>(x) + r0 * x_row_stride, nr, x_row_stride, n_heads_in, g, head_dim, w,
+          y + r0 * y_row_stride, y_row_stride);
+      ESA_LAUNCH_CHECK("compress_tc_kernel");
+    }
+    return ok();
+  }
   const int ct = d_out % 32 == 0 ? 32 : 16;
   dim3 grid((unsigned)cdiv(rows, esa::kCmpRT), d_out / ct);
   if (x_dtype == ESA_F32) {

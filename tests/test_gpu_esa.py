@@ -36,6 +36,8 @@ def _rand(shape, seed, dtype):
     (512, 32, 32, 128, 128, torch.bfloat16),  # one prefill chunk of queries
     (5, 4, 4, 64, 16, torch.float32),         # the tiny fp32 layer, d' = 16
     (1, 2, 8, 64, 48, torch.float32),         # one row, d' = 48
+    (300, 4, 16, 64, 128, torch.bfloat16),    # tensor-core path, head_dim 64, 3 row tiles
+    (1, 8, 32, 128, 128, torch.bfloat16),     # a single row
 ])
 def test_compress_parity(rows, hin, hout, d, dc, dtype):
     x = _rand((rows, hin, d), 1, dtype)
@@ -43,6 +45,20 @@ def test_compress_parity(rows, hin, hout, d, dc, dtype):
     y = qas.compress(x.to(DEV), w.to(DEV), hout)
     ref = oesa.compress(_np(x), _np(w), hout)
     assert max_abs(_np(y), ref) <= ATOL_F32
+
+
+def test_compress_strided_rows_of_a_batched_cache():
+    """One call compresses the new key of every sequence (rows n_ctx apart) and writes
+    each into that sequence's row of the compressed cache."""
+    b, n, hkv, hq, d, dc, pos = 5, 40, 8, 32, 128, 128, 37
+    k = _rand((b, n, hkv, d), 5, torch.bfloat16).to(DEV)
+    w = (_rand((hq * d, dc), 6, torch.float32) / math.sqrt(hq * d)).to(DEV)
+    cache = torch.zeros((b, n, dc), device=DEV)
+    qas.compress(k[:, pos], w, hq, out=cache[:, pos], out_row_stride=n * dc)
+    ref = oesa.compress(_np(k[:, pos].cpu()), _np(w.cpu()), hq)
+    got = cache.cpu().numpy()
+    assert max_abs(got[:, pos], ref) <= ATOL_F32
+    assert np.all(np.delete(got, pos, axis=1) == 0.0)
 
 
 def test_compress_writes_into_a_cache_slice():
@@ -77,7 +93,11 @@ def _selection_case(batch, lq, n_cap, c0, dc, p, seed, planted=False):
             ref_v = ref_sp[b]
             got_v = sp[b].cpu().double().numpy()
             scale = max(1.0, float(np.abs(ref_v).max()))
-            assert float(np.abs(got_v - ref_v).max()) <= 1e-4 * scale   # fp32 scores vs float64
+            # fp32 scoring (few queries) is held to 1e-4 of the scale; the tensor-core
+            # path reads the compressed operands as tf32 (10-bit mantissa), so it is held
+            # to the selection band's own 1e-3
+            rel = 1e-3 if (lq >= 16 and dc in (32, 64, 128)) else 1e-4
+            assert float(np.abs(got_v - ref_v).max()) <= rel * scale
     return swaps
 
 
