@@ -9,9 +9,11 @@
 // tiles skip the rescale and P stays <= 2^8 (exact softmax either way: o = O / l).
 // Roles (224 threads): warps 0-3 softmax (thread = row = TMEM lane), warp 4 issues
 // the MMAs (one lane), warp 5 loads Q and the K rows, warp 6 loads the V rows.
-// K/V rows are gathered by cp.async (16-byte pieces) straight into the 128-byte
-// swizzled layout the MMA descriptors name; loaders wait for their own copies and
-// fence to the async proxy before arriving on the "full" barrier.
+// Rows are gathered by TMA (tile::gather4: 4 arbitrary rows of a [rows, 128] bf16
+// tensor map per instruction, one 64-column half at a time) straight into the
+// 128-byte swizzled layout the MMA descriptors name; each lane of a loader warp
+// issues the gathers for 4 of the tile's 128 rows, and the "full" barrier completes
+// on the transaction count.
 //
 // Shared memory: Q 32 KB, K 2 x 32 KB, V 2 x 32 KB, P 2 x 32 KB (each operand tile is
 // two 16 KB column blocks of 128 rows x 128 bytes). TMEM: S double buffer (2 x 128
@@ -19,13 +21,14 @@
 //
 // The problem policy P says which rows and keys a CTA owns:
 //   bool setup(): per-CTA fields; false = nothing to do
-//   int64_t q_row(int r): element offset of row r's query from q_base() (-1: padding)
-//   int64_t kv_pos(int64_t t): row id of key t (t < n_keys()); kv_off(id): its element
-//        offset from kv_base_k() / kv_base_v()
+//   int32_t q_row(int r): row of the Q tensor map for tile row r (-1: padding)
+//   int32_t kv_row(int64_t t): row of the K / V tensor maps for key t (t < n_keys())
 //   int64_t n_keys(); int64_t limit(int r): last key index row r may attend
 //   void store(int r, const float* o, float m2, float l): o is unnormalised,
 //        m2 the running max in log2 units, l the denominator
 #pragma once
+#include <cuda.h>
+
 #include "common.cuh"
 #include "keylist.cuh"
 
@@ -49,74 +52,57 @@ struct TcSmem {
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
-  int32_t kpos[2][128];      // key rows of the tile being issued, one buffer per loader warp
 };
 static_assert(sizeof(TcSmem) <= kTcCtrlBytes, "control block overflows its reservation");
 
-// Copy one 128 x 128 bf16 tile into swizzled shared memory: row r comes from element
-// offset off(r) of base (off < 0: zero fill). 32 threads; lane owns the 16-byte chunk
-// lane % 16 of rows lane / 16, lane / 16 + 2, ...
-template <typename OffFn>
-__device__ __forceinline__ void load_tile_rows(uint32_t dst, const __nv_bfloat16* base, OffFn off_of, int lane) {
-  const int ch = lane & 15;
-  const uint32_t blk = (ch >> 3) * kBlkBytes;
-  const uint32_t cc = ch & 7;
-#pragma unroll 8
-  for (int r = lane >> 4; r < 128; r += 2) {
-    const int64_t off = off_of(r);
-    const void* src = off >= 0 ? (const void*)(base + off + ch * 8) : (const void*)base;
-    cp_async16(dst + blk + sw128_off(r, cc), src, off >= 0 ? 16u : 0u);
-  }
+// Gather 128 rows of a [rows, 128] bf16 tensor into one swizzled tile (two 64-column
+// blocks). Lane l issues rows 4l..4l+3; row ids < 0 are replaced by `fallback` (a
+// valid row whose data the caller masks out). Caller has set the expected bytes.
+__device__ __forceinline__ void gather_tile(uint32_t dst, const CUtensorMap* tm, const int32_t* rows4,
+                                            int32_t fallback, uint64_t* bar, int lane) {
+  int32_t r[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) r[q] = rows4[q] >= 0 ? rows4[q] : fallback;
+  const uint32_t d = dst + lane * 4 * 128;
+  tma_gather4(d, tm, 0, r[0], r[1], r[2], r[3], bar);
+  tma_gather4(d + kBlkBytes, tm, 64, r[0], r[1], r[2], r[3], bar);
 }
 
 // One loader warp streams the key tiles of one operand (K or V) through the two
-// stages. The 128 key positions of tile j + 1 are fetched into registers (4 per lane,
-// consecutive, so gathered index lists are read coalesced) while tile j is issued;
-// they pass through shared memory to the lanes that copy each row. Tile j - 1 is
-// signalled once its copies have landed (own copies waited, then a proxy fence).
+// stages. The rows of tile j + 1 are looked up (4 per lane, consecutive keys, so a
+// gathered index list is read coalesced) while tile j waits for its stage.
 template <class Problem>
-__device__ __forceinline__ void stream_kv(const Problem& prob, const __nv_bfloat16* base, uint32_t stage0,
-                                          uint64_t* full, uint64_t* empty, int32_t* pos_buf, int nt,
-                                          int64_t n_keys, int lane, volatile int* abort_flag, unsigned site) {
-  int32_t pn[4];
-  auto fetch = [&](int j) {
+__device__ __forceinline__ void stream_kv(const Problem& prob, const CUtensorMap* tm, uint32_t stage0,
+                                          uint64_t* full, uint64_t* empty, int nt, int64_t n_keys, int lane,
+                                          volatile int* abort_flag, unsigned site) {
+  int32_t cur[4], nxt[4];
+  auto fetch = [&](int j, int32_t* out) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int64_t t = (int64_t)j * kTcKeys + lane * 4 + q;
-      pn[q] = t < n_keys ? (int32_t)prob.kv_pos(t) : -1;
+      out[q] = t < n_keys ? prob.kv_row(t) : -1;
     }
   };
-  if (nt > 0) fetch(0);
-  bool ok = true;
+  if (nt == 0) return;
+  const int32_t fallback = prob.kv_row(0);
+  fetch(0, nxt);
   for (int j = 0; j < nt; ++j) {
     const int s = j & 1;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) pos_buf[lane * 4 + q] = pn[q];
+    for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
+    if (j + 1 < nt) fetch(j + 1, nxt);
+    bool ok = mbar_wait(&empty[s], ((j >> 1) & 1) ^ 1, abort_flag, site);
+    if (!__all_sync(0xffffffffu, ok)) return;
+    if (lane == 0) mbar_arrive_expect_tx(&full[s], kTileBytes);
     __syncwarp();
-    if (j + 1 < nt) fetch(j + 1);
-    ok = mbar_wait(&empty[s], ((j >> 1) & 1) ^ 1, abort_flag, site);
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok) break;
-    load_tile_rows(stage0 + s * kTileBytes, base,
-                   [&](int r) -> int64_t { const int32_t p = pos_buf[r]; return p >= 0 ? prob.kv_off(p) : -1; },
-                   lane);
-    cp_async_commit();
-    __syncwarp();
-    if (j >= 1) {
-      cp_async_wait<1>();
-      fence_proxy_async();
-      mbar_arrive(&full[(j - 1) & 1]);
-    }
-  }
-  cp_async_wait_all();
-  if (ok && nt > 0) {
-    fence_proxy_async();
-    mbar_arrive(&full[(nt - 1) & 1]);
+    gather_tile(stage0 + s * kTileBytes, tm, cur, fallback, &full[s], lane);
   }
 }
 
 template <class Problem>
-__global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(Problem prob) {
+__global__ void __launch_bounds__(kTcThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, Problem prob) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sQ = smem_u32(smem);
@@ -131,10 +117,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(Problem prob) {
   const int nt = (int)((n_keys + kTcKeys - 1) / kTcKeys);
 
   if (threadIdx.x == 0) {
-    mbar_init(&sm.q_full, 32);
+    mbar_init(&sm.q_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.k_full[s], 32);
-      mbar_init(&sm.v_full[s], 32);
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
       mbar_init(&sm.v_empty[s], 1);
       mbar_init(&sm.s_full[s], 1);
@@ -159,15 +145,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(Problem prob) {
 
   if (warp == 5) {
     // ---------------------------------------------------------------- Q + K loader
-    load_tile_rows(sQ, prob.q_base(), [&](int r) -> int64_t { return prob.q_row(r); }, lane);
-    cp_async_commit();
-    cp_async_wait_all();
-    fence_proxy_async();
-    mbar_arrive(&sm.q_full);
-    stream_kv(prob, prob.kv_base_k(), sK, sm.k_full, sm.k_empty, sm.kpos[0], nt, n_keys, lane, abort_flag, 101);
+    int32_t qr[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) qr[q] = prob.q_row(lane * 4 + q);
+    const int32_t q_fallback = __shfl_sync(0xffffffffu, qr[0], 0);    // row 0 is always a real query
+    if (lane == 0) mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
+    __syncwarp();
+    gather_tile(sQ, &tm_q, qr, q_fallback, &sm.q_full, lane);
+    stream_kv(prob, &tm_k, sK, sm.k_full, sm.k_empty, nt, n_keys, lane, abort_flag, 101);
   } else if (warp == 6) {
     // ---------------------------------------------------------------- V loader
-    stream_kv(prob, prob.kv_base_v(), sV, sm.v_full, sm.v_empty, sm.kpos[1], nt, n_keys, lane, abort_flag, 102);
+    stream_kv(prob, &tm_v, sV, sm.v_full, sm.v_empty, nt, n_keys, lane, abort_flag, 102);
   } else if (warp == 4) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
@@ -237,12 +225,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(Problem prob) {
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&sm.s_empty[s]);             // S now lives in registers
-      float mx = -INFINITY;
+      float mx8[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) mx8[q] = -INFINITY;
 #pragma unroll
       for (int e = 0; e < kTcKeys; ++e) {
         x[e] = (t0 + e <= lim) ? x[e] * sl2 : -INFINITY;
-        mx = fmaxf(mx, x[e]);
+        mx8[e & 7] = fmaxf(mx8[e & 7], x[e]);
       }
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       if (mx > m + kRescale || m == -INFINITY) {
         const float m_new = fmaxf(m, mx);
         if (j > 0 && m_new > m) {
@@ -267,7 +259,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(Problem prob) {
       const float m_use = m == -INFINITY ? 0.f : m;
       if (!(ok = mbar_wait_warp(&sm.p_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, 112))) break;
       const uint32_t pt = sP + s * kTileBytes;
-      float lsum = 0.f;
+      float ls8[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) ls8[q] = 0.f;
 #pragma unroll
       for (int c = 0; c < 16; ++c) {           // 16-byte chunks of the 256-byte P row
         uint32_t pk[4];
@@ -275,13 +269,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(Problem prob) {
         for (int e = 0; e < 8; e += 2) {
           const float p0 = fast_exp2(x[c * 8 + e] - m_use);
           const float p1 = fast_exp2(x[c * 8 + e + 1] - m_use);
-          lsum += p0 + p1;
+          ls8[e] += p0;
+          ls8[e + 1] += p1;
           pk[e / 2] = pack_bf16x2(p0, p1);
         }
         const uint32_t dst = pt + (c >> 3) * kBlkBytes + sw128_off(r, c & 7);
         st_shared_v4(dst, pk[0], pk[1], pk[2], pk[3]);
       }
-      l += lsum;
+      l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(&sm.p_full[s]);
@@ -332,17 +327,15 @@ struct EsaTcProblem {
     nk = n_prior + imax + 1;
     return true;
   }
-  __device__ const __nv_bfloat16* q_base() const { return q; }
-  __device__ const __nv_bfloat16* kv_base_k() const { return k; }
-  __device__ const __nv_bfloat16* kv_base_v() const { return v; }
-  __device__ int64_t q_row(int r) const {
+  __device__ int32_t q_row(int r) const {
     const int R = tile * kTcRows + r;
     if (R >= lq * G) return -1;
     const int i = R / G, hl = R % G;
-    return (((int64_t)b * lq + i) * hq + g * G + hl) * kTcD;
+    return (int32_t)(((int64_t)b * lq + i) * hq + g * G + hl);
   }
-  __device__ int64_t kv_pos(int64_t t) const { return keys.pos(b, cnt, t); }
-  __device__ int64_t kv_off(int64_t p) const { return (((int64_t)b * n_cap + p) * hkv + g) * kTcD; }
+  __device__ int32_t kv_row(int64_t t) const {
+    return (int32_t)(((int64_t)b * n_cap + keys.pos(b, cnt, t)) * hkv + g);
+  }
   __device__ int64_t n_keys() const { return nk; }
   __device__ int64_t limit(int r) const {
     const int R = tile * kTcRows + r;

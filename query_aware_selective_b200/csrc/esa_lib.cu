@@ -149,7 +149,7 @@ SelWs carve_select(void* ws, int32_t batch, int32_t lq, int64_t n_mid, ScorePath
 
 // 2D tensor map over a row-major fp32 matrix [rows, cols], 32 x 128 boxes, 128-byte
 // swizzle (the shared-memory layout the tf32 MMA descriptors expect).
-esa_status_t make_tmap_f32(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols) {
+esa_status_t get_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   if (!encode) {
     cudaDriverEntryPointQueryResult q;
@@ -158,6 +158,31 @@ esa_status_t make_tmap_f32(CUtensorMap* m, const float* base, uint64_t rows, uin
     if (q != cudaDriverEntryPointSuccess || !fn) return fail(ESA_ERR_CUDA, "cuTensorMapEncodeTiled not available");
     encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
+  *out = encode;
+  return ESA_OK;
+}
+
+// 2D tensor map over bf16 rows of 128 elements [rows, 128], boxes of one row x 64
+// columns with 128-byte swizzle: the form tile::gather4 loads (4 rows per instruction).
+esa_status_t make_tmap_rows_bf16(CUtensorMap* m, const void* base, uint64_t rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode;
+  esa_status_t st = get_encoder(&encode);
+  if (st != ESA_OK) return st;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {128 * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ESA_ERR_CUDA, "cuTensorMapEncodeTiled (rows) failed (%d)", (int)r);
+  return ESA_OK;
+}
+
+esa_status_t make_tmap_f32(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode;
+  esa_status_t st0 = get_encoder(&encode);
+  if (st0 != ESA_OK) return st0;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * sizeof(float)};
   cuuint32_t box[2] = {32, 128};
@@ -466,8 +491,14 @@ esa_status_t esa_sparse_attn(const void* q, const void* k, const void* v, esa_dt
     pr.hkv = hkv;
     pr.G = g;
     pr.sl2 = sl2;
+    if ((int64_t)batch * n_cap * hkv >= ((int64_t)1 << 31) || (int64_t)batch * lq * hq >= ((int64_t)1 << 31))
+      return fail(ESA_ERR_UNSUPPORTED, "more than 2^31 K/V or Q rows");
+    CUtensorMap tq, tk, tv;
+    if ((st = make_tmap_rows_bf16(&tq, q, (uint64_t)batch * lq * hq)) != ESA_OK) return st;
+    if ((st = make_tmap_rows_bf16(&tk, k, (uint64_t)batch * n_cap * hkv)) != ESA_OK) return st;
+    if ((st = make_tmap_rows_bf16(&tv, v, (uint64_t)batch * n_cap * hkv)) != ESA_OK) return st;
     dim3 grid((unsigned)cdiv((int64_t)lq * g, esa::kTcRows), hkv, batch);
-    esa::attn_tc_kernel<esa::EsaTcProblem><<<grid, esa::kTcThreads, esa::kTcSmemBytes, s>>>(pr);
+    esa::attn_tc_kernel<esa::EsaTcProblem><<<grid, esa::kTcThreads, esa::kTcSmemBytes, s>>>(tq, tk, tv, pr);
     ESA_LAUNCH_CHECK("attn_tc_kernel<esa>");
     return ok();
   }
@@ -607,12 +638,17 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
   int dev = 0;
   ESA_CUDA(cudaGetDevice(&dev));
   if (dev < 64 && !attr_set[dev]) {
-    esa_status_t st = set_max_smem(esa::attn_tc_kernel<esa::MobaPastProblem>, esa::kTcSmemBytes);
-    if (st != ESA_OK) return st;
-    st = set_max_smem(esa::attn_tc_kernel<esa::MobaCurrentProblem>, esa::kTcSmemBytes);
-    if (st != ESA_OK) return st;
+    esa_status_t sa = set_max_smem(esa::attn_tc_kernel<esa::MobaPastProblem>, esa::kTcSmemBytes);
+    if (sa != ESA_OK) return sa;
+    sa = set_max_smem(esa::attn_tc_kernel<esa::MobaCurrentProblem>, esa::kTcSmemBytes);
+    if (sa != ESA_OK) return sa;
     attr_set[dev] = true;
   }
+  CUtensorMap tq, tk, tv;
+  esa_status_t st;
+  if ((st = make_tmap_rows_bf16(&tq, q, (uint64_t)batch * seq * heads)) != ESA_OK) return st;
+  if ((st = make_tmap_rows_bf16(&tk, k, (uint64_t)batch * seq * heads)) != ESA_OK) return st;
+  if ((st = make_tmap_rows_bf16(&tv, v, (uint64_t)batch * seq * heads)) != ESA_OK) return st;
   ESA_CUDA(cudaMemsetAsync(w.cnt, 0, w.zero_bytes, s));
   const dim3 lgrid((unsigned)cdiv(seq * heads, 256), batch);
   if (topk > 0 && w.pairs > 0) {
@@ -639,7 +675,8 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
     pp.topk = topk;
     pp.n_lists = w.n_lists;
     pp.sl2 = sl2;
-    esa::attn_tc_kernel<esa::MobaPastProblem><<<(unsigned)w.max_tiles, esa::kTcThreads, esa::kTcSmemBytes, s>>>(pp);
+    esa::attn_tc_kernel<esa::MobaPastProblem><<<(unsigned)w.max_tiles, esa::kTcThreads, esa::kTcSmemBytes, s>>>(
+        tq, tk, tv, pp);
     ESA_LAUNCH_CHECK("attn_tc_kernel<moba past>");
   }
   esa::MobaCurrentProblem cp{};
@@ -656,7 +693,7 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
   cp.tiles_per_block = (int)cdiv(block, esa::kTcRows);
   cp.sl2 = sl2;
   esa::attn_tc_kernel<esa::MobaCurrentProblem>
-      <<<dim3(cp.tiles_per_block * nb, heads, batch), esa::kTcThreads, esa::kTcSmemBytes, s>>>(cp);
+      <<<dim3(cp.tiles_per_block * nb, heads, batch), esa::kTcThreads, esa::kTcSmemBytes, s>>>(tq, tk, tv, cp);
   ESA_LAUNCH_CHECK("attn_tc_kernel<moba current>");
   const int64_t rows = (int64_t)batch * seq * heads;
   esa::moba_combine_kernel<128><<<(unsigned)cdiv(rows, 8), 256, 0, s>>>(

@@ -233,17 +233,15 @@ struct MobaPastProblem {
     n_rows = min((uint32_t)kTcRows, cnt[li] - t_in * kTcRows);
     return true;
   }
-  __device__ const __nv_bfloat16* q_base() const { return q; }
-  __device__ const __nv_bfloat16* kv_base_k() const { return k; }
-  __device__ const __nv_bfloat16* kv_base_v() const { return v; }
-  __device__ int64_t q_row(int r) const {
+  __device__ int32_t q_row(int r) const {
     if ((uint32_t)r >= n_rows) return -1;
     const int64_t p = list[e0 + r] >> 4;
-    return (((int64_t)b * seq + p) * heads + h) * kTcD;
+    return (int32_t)(((int64_t)b * seq + p) * heads + h);
   }
   __device__ int64_t n_keys() const { return min((int64_t)block, seq - (int64_t)blk * block); }
-  __device__ int64_t kv_pos(int64_t t) const { return (int64_t)blk * block + t; }
-  __device__ int64_t kv_off(int64_t p) const { return (((int64_t)b * seq + p) * heads + h) * kTcD; }
+  __device__ int32_t kv_row(int64_t t) const {
+    return (int32_t)(((int64_t)b * seq + (int64_t)blk * block + t) * heads + h);
+  }
   __device__ int64_t limit(int) const { return n_keys() - 1; }
   __device__ float scale_log2() const { return sl2; }
   __device__ void store(int r, const float* acc, float m2, float l) {
@@ -287,16 +285,12 @@ struct MobaCurrentProblem {
     nrows = min((int64_t)kTcRows, bend - p0);
     return true;
   }
-  __device__ const __nv_bfloat16* q_base() const { return q; }
-  __device__ const __nv_bfloat16* kv_base_k() const { return k; }
-  __device__ const __nv_bfloat16* kv_base_v() const { return v; }
-  __device__ int64_t q_row(int r) const {
+  __device__ int32_t q_row(int r) const {
     if (r >= nrows) return -1;
-    return (((int64_t)b * seq + p0 + r) * heads + h) * kTcD;
+    return (int32_t)(((int64_t)b * seq + p0 + r) * heads + h);
   }
   __device__ int64_t n_keys() const { return p0 + nrows - kb0; }
-  __device__ int64_t kv_pos(int64_t t) const { return kb0 + t; }
-  __device__ int64_t kv_off(int64_t p) const { return (((int64_t)b * seq + p) * heads + h) * kTcD; }
+  __device__ int32_t kv_row(int64_t t) const { return (int32_t)(((int64_t)b * seq + kb0 + t) * heads + h); }
   __device__ int64_t limit(int r) const { return p0 + min((int64_t)r, nrows - 1) - kb0; }
   __device__ float scale_log2() const { return sl2; }
   __device__ void store(int r, const float* acc, float m2, float l) {
