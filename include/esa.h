@@ -142,6 +142,33 @@ size_t esa_sparse_attn_workspace_size(int32_t batch, int32_t lq, int64_t c0, int
                                       int32_t hkv, int32_t head_dim, esa_dtype_t dt,
                                       esa_params_t p);
 
+/* esa_score_select_noalloc - esa_score_select without a workspace argument. The pages
+ * have no counterpart of this call: it exists for callers that cannot allocate device
+ * memory - a service that plans all its memory at start-up and allows no allocation
+ * afterwards, a plugin running inside another runtime with no access to that runtime's
+ * allocator, a latency-critical loop where an allocation's stall or failure is not
+ * acceptable. It allocates nothing (no cudaMalloc, no cudaFree, no allocating library
+ * routine): its scratch is a fixed 8 MiB array in device memory
+ * (esa_score_select_noalloc_capacity() bytes) that every GPU loading this library
+ * holds until the process exits.
+ *   - Arguments and results are those of esa_score_select.
+ *   - A selection whose scratch (esa_score_select_workspace_size) exceeds the array
+ *     returns ESA_ERR_WORKSPACE without launching anything.
+ *   - The first call on a device looks up the array's device address with that device
+ *     current (a one-time host call per device); make that first call before any
+ *     stream capture.
+ *   - All calls share the one array, and it keeps the previous call's contents; the
+ *     call clears what must start at zero itself. Calls whose GPU work overlaps (on
+ *     different streams or threads, for the same device) race on the array and give
+ *     wrong results: serialise them. */
+esa_status_t esa_score_select_noalloc(const float* q_c, const float* k_c, int32_t batch, int32_t lq,
+                                      int64_t n_cap, int64_t c0, int32_t d_c, esa_params_t p,
+                                      int32_t* idx_out, int32_t* count_out, float* score_out,
+                                      void* stream);
+
+/* Bytes of the fixed scratch array esa_score_select_noalloc uses. */
+size_t esa_score_select_noalloc_capacity(void);
+
 /* --------------------------------------------------------------- MoBA calls -- */
 
 /* moba_block_gate - block choice of MoBA (MoBA article, section 3: blocks of size

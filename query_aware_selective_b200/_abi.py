@@ -50,6 +50,9 @@ SIGNATURES = {
     "esa_device_status": (ctypes.c_int, [_vp]),
     "esa_version": (ctypes.c_char_p, []),
     "esa_launch_count": (ctypes.c_uint64, []),
+    "esa_score_select_noalloc": (ctypes.c_int, [_vp, _vp, _i32, _i32, _i64, _i64, _i32, EsaParams, _vp, _vp, _vp,
+                                                _vp]),
+    "esa_score_select_noalloc_capacity": (_sz, []),
 }
 
 _lib = None
@@ -173,6 +176,27 @@ def score_select(q_c: torch.Tensor, k_c: torch.Tensor, c0: int, p: EsaParams, wa
     wp, wn = _ws_ptr(ws)
     _check(load().esa_score_select(_ptr(q_c), _ptr(k_c), b, lq, n_cap, c0, dc, p, _ptr(idx), _ptr(count),
                                    _ptr(scores) if want_scores else None, wp, wn, _stream()), "esa_score_select")
+    return idx, count, (scores if want_scores else None)
+
+
+def score_select_noalloc(q_c: torch.Tensor, k_c: torch.Tensor, c0: int, p: EsaParams, want_scores: bool = False,
+                         idx: Optional[torch.Tensor] = None, count: Optional[torch.Tensor] = None,
+                         scores: Optional[torch.Tensor] = None):
+    """esa_score_select_noalloc: the same selection, with the library's fixed scratch
+    instead of a workspace (for callers that cannot allocate device memory)."""
+    _dev(q_c, k_c)
+    b, lq, dc = q_c.shape
+    dev = q_c.device
+    if idx is None:
+        idx = torch.empty((b, p.topk), dtype=torch.int32, device=dev)
+    if count is None:
+        count = torch.empty((b,), dtype=torch.int32, device=dev)
+    if want_scores and scores is None:
+        lo = min(c0, max(p.n_init, c0 - p.window))
+        scores = torch.empty((b, max(0, lo - p.n_init)), dtype=torch.float32, device=dev)
+    _check(load().esa_score_select_noalloc(_ptr(q_c), _ptr(k_c), b, lq, k_c.shape[1], c0, dc, p, _ptr(idx),
+                                           _ptr(count), _ptr(scores) if want_scores else None, _stream()),
+           "esa_score_select_noalloc")
     return idx, count, (scores if want_scores else None)
 
 

@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 #include <string>
 
 #include "../../include/esa.h"
@@ -760,3 +761,50 @@ esa_status_t moba_block_gate_attn(const void* q, const void* k, const void* v, e
   return st == ESA_OK ? ok() : st;
 }
 
+
+// ------------------------------------------------------------------ no-alloc selection --
+// Scratch for esa_score_select_noalloc: a fixed array in device memory that every GPU
+// loading this library holds until the process exits. Host code may not use the name
+// as a device address; the address comes from cudaGetSymbolAddress, once per device.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;     // 8 MiB
+__device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[64] = {};
+
+esa_status_t scratch_for_current_device(void** out) {
+  int dev = 0;
+  ESA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(ESA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    ESA_CUDA(cudaGetSymbolAddress(&p, g_select_scratch));
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return ESA_OK;
+}
+
+}  // namespace
+
+esa_status_t esa_score_select_noalloc(const float* q_c, const float* k_c, int32_t batch, int32_t lq, int64_t n_cap,
+                                      int64_t c0, int32_t d_c, esa_params_t p, int32_t* idx_out, int32_t* count_out,
+                                      float* score_out, void* stream) {
+  if (batch <= 0 || lq <= 0) return fail(ESA_ERR_INVALID_ARG, "batch and lq must be >= 1");
+  const size_t need = esa_score_select_workspace_size(batch, lq, n_cap, c0, d_c, p);
+  if (need > kNoAllocScratchBytes)
+    return fail(ESA_ERR_WORKSPACE,
+                "this selection needs %zu bytes of scratch; the no-alloc entry point has %zu (use esa_score_select "
+                "with a workspace)",
+                need, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  const esa_status_t st = scratch_for_current_device(&scratch);
+  if (st != ESA_OK) return st;
+  return esa_score_select(q_c, k_c, batch, lq, n_cap, c0, d_c, p, idx_out, count_out, score_out, scratch,
+                          kNoAllocScratchBytes, stream);
+}
+
+size_t esa_score_select_noalloc_capacity(void) { return kNoAllocScratchBytes; }
