@@ -7,13 +7,16 @@
 // m is the running row maximum used for the exponentials; it is raised (and O, l
 // rescaled in place) only when a tile's maximum exceeds it by more than 2^8, so most
 // tiles skip the rescale and P stays <= 2^8 (exact softmax either way: o = O / l).
-// Roles (224 threads): warps 0-3 softmax (thread = row = TMEM lane), warp 4 issues
-// the MMAs (one lane), warp 5 loads Q and the K rows, warp 6 loads the V rows.
-// Rows are gathered by TMA (tile::gather4: 4 arbitrary rows of a [rows, 128] bf16
-// tensor map per instruction, one 64-column half at a time) straight into the
-// 128-byte swizzled layout the MMA descriptors name; each lane of a loader warp
-// issues the gathers for 4 of the tile's 128 rows, and the "full" barrier completes
-// on the transaction count.
+// Roles (352 threads): warps 0-7 softmax (warp w owns TMEM lanes 32 (w % 4) .. + 31,
+// i.e. rows, and key columns 64 (w / 4) .. + 63: two threads per row, exchanging the
+// row max and sum through shared memory), warp 8 issues the MMAs (one lane), warp 9
+// loads Q and the K tiles, warp 10 loads the V tiles.
+// Tiles come in by TMA straight into the 128-byte swizzled layout the MMA descriptors
+// name, and the "full" barriers complete on the transaction count. A tile whose 128
+// keys are consecutive tokens (initial tokens, local window, chunk, MoBA blocks) is
+// one 3D box per 64-column half ([tokens, heads, 128] map, one head); a tile of
+// scattered keys (the selected middle tokens) is 32 tile::gather4 loads per half
+// (4 arbitrary rows each; each lane of the loader warp issues its 4 rows).
 //
 // Shared memory: Q 32 KB, K 2 x 32 KB, V 2 x 32 KB, P 2 x 32 KB (each operand tile is
 // two 16 KB column blocks of 128 rows x 128 bytes). TMEM: S double buffer (2 x 128
@@ -21,8 +24,11 @@
 //
 // The problem policy P says which rows and keys a CTA owns:
 //   bool setup(): per-CTA fields; false = nothing to do
-//   int32_t q_row(int r): row of the Q tensor map for tile row r (-1: padding)
-//   int32_t kv_row(int64_t t): row of the K / V tensor maps for key t (t < n_keys())
+//   int32_t q_row(int r): row of the Q row map for tile row r (-1: padding)
+//   bool q_box(int* y, int* z): true if the Q tile is one box of the Q box map at (y, z)
+//   int32_t kv_row(int64_t t): row of the K / V row maps for key t (t < n_keys())
+//   int kv_box(int j, int* y, int* z): 1 if key tile j is one box of the K / V box maps
+//        at (head y, token z), 2 if it is one box of the staged copies, 0 if gathered
 //   int64_t n_keys(); int64_t limit(int r): last key index row r may attend
 //   void store(int r, const float* o, float m2, float l): o is unnormalised,
 //        m2 the running max in log2 units, l the denominator
@@ -34,7 +40,8 @@
 
 namespace esa {
 
-constexpr int kTcThreads = 224;
+constexpr int kTcThreads = 352;
+constexpr int kTcMmaWarp = 8, kTcKWarp = 9, kTcVWarp = 10;
 constexpr int kTcRows = 128;
 constexpr int kTcKeys = 128;
 constexpr int kTcD = 128;
@@ -52,6 +59,7 @@ struct TcSmem {
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
+  float red[2][128];         // per-row partial max / sum of the two column halves
 };
 static_assert(sizeof(TcSmem) <= kTcCtrlBytes, "control block overflows its reservation");
 
@@ -72,8 +80,9 @@ __device__ __forceinline__ void gather_tile(uint32_t dst, const CUtensorMap* tm,
 // stages. The rows of tile j + 1 are looked up (4 per lane, consecutive keys, so a
 // gathered index list is read coalesced) while tile j waits for its stage.
 template <class Problem>
-__device__ __forceinline__ void stream_kv(const Problem& prob, const CUtensorMap* tm, uint32_t stage0,
-                                          uint64_t* full, uint64_t* empty, int nt, int64_t n_keys, int lane,
+__device__ __forceinline__ void stream_kv(const Problem& prob, const CUtensorMap* tm_rows, const CUtensorMap* tm_box,
+                                          const CUtensorMap* tm_staged, uint32_t stage0, uint64_t* full,
+                                          uint64_t* empty, int nt, int64_t n_keys, int lane,
                                           volatile int* abort_flag, unsigned site) {
   int32_t cur[4], nxt[4];
   auto fetch = [&](int j, int32_t* out) {
@@ -85,24 +94,44 @@ __device__ __forceinline__ void stream_kv(const Problem& prob, const CUtensorMap
   };
   if (nt == 0) return;
   const int32_t fallback = prob.kv_row(0);
-  fetch(0, nxt);
+  int by = 0, bz = 0;
+  int box_next = prob.kv_box(0, &by, &bz);        // 0: gather, 1: cache box, 2: staged box
+  if (!box_next) fetch(0, nxt);
   for (int j = 0; j < nt; ++j) {
     const int s = j & 1;
+    const int box = box_next;
+    const int y = by, z = bz;
 #pragma unroll
     for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
-    if (j + 1 < nt) fetch(j + 1, nxt);
+    if (j + 1 < nt) {
+      box_next = prob.kv_box(j + 1, &by, &bz);
+      if (!box_next) fetch(j + 1, nxt);
+    }
     bool ok = mbar_wait(&empty[s], ((j >> 1) & 1) ^ 1, abort_flag, site);
     if (!__all_sync(0xffffffffu, ok)) return;
-    if (lane == 0) mbar_arrive_expect_tx(&full[s], kTileBytes);
-    __syncwarp();
-    gather_tile(stage0 + s * kTileBytes, tm, cur, fallback, &full[s], lane);
+    const uint32_t dst = stage0 + s * kTileBytes;
+    if (box) {
+      if (lane == 0) {
+        const CUtensorMap* tm = box == 2 ? tm_staged : tm_box;
+        mbar_arrive_expect_tx(&full[s], kTileBytes);
+        tma_load_3d(dst, tm, 0, y, z, &full[s]);
+        tma_load_3d(dst + kBlkBytes, tm, 64, y, z, &full[s]);
+      }
+    } else {
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], kTileBytes);
+      __syncwarp();
+      gather_tile(dst, tm_rows, cur, fallback, &full[s], lane);
+    }
   }
 }
 
 template <class Problem>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, Problem prob) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tb_q,
+                   const __grid_constant__ CUtensorMap tb_k, const __grid_constant__ CUtensorMap tb_v,
+                   const __grid_constant__ CUtensorMap ts_k, const __grid_constant__ CUtensorMap ts_v,
+                   Problem prob) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sQ = smem_u32(smem);
@@ -124,8 +153,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&sm.k_empty[s], 1);
       mbar_init(&sm.v_empty[s], 1);
       mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.s_empty[s], 128);
-      mbar_init(&sm.p_full[s], 128);
+      mbar_init(&sm.s_empty[s], 256);
+      mbar_init(&sm.p_full[s], 256);
       mbar_init(&sm.p_empty[s], 1);
       mbar_init(&sm.pv_full[s], 1);
     }
@@ -133,7 +162,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     sm.abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 4) {
+  if (warp == kTcMmaWarp) {
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
@@ -143,20 +172,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
 
-  if (warp == 5) {
+  if (warp == kTcKWarp) {
     // ---------------------------------------------------------------- Q + K loader
-    int32_t qr[4];
+    int qy = 0, qz = 0;
+    if (prob.q_box(&qy, &qz)) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
+        tma_load_3d(sQ, &tb_q, 0, qy, qz, &sm.q_full);
+        tma_load_3d(sQ + kBlkBytes, &tb_q, 64, qy, qz, &sm.q_full);
+      }
+    } else {
+      int32_t qr[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) qr[q] = prob.q_row(lane * 4 + q);
-    const int32_t q_fallback = __shfl_sync(0xffffffffu, qr[0], 0);    // row 0 is always a real query
-    if (lane == 0) mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
-    __syncwarp();
-    gather_tile(sQ, &tm_q, qr, q_fallback, &sm.q_full, lane);
-    stream_kv(prob, &tm_k, sK, sm.k_full, sm.k_empty, nt, n_keys, lane, abort_flag, 101);
-  } else if (warp == 6) {
+      for (int q = 0; q < 4; ++q) qr[q] = prob.q_row(lane * 4 + q);
+      const int32_t q_fallback = __shfl_sync(0xffffffffu, qr[0], 0);    // row 0 is always a real query
+      if (lane == 0) mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
+      __syncwarp();
+      gather_tile(sQ, &tm_q, qr, q_fallback, &sm.q_full, lane);
+    }
+    stream_kv(prob, &tm_k, &tb_k, &ts_k, sK, sm.k_full, sm.k_empty, nt, n_keys, lane, abort_flag, 101);
+  } else if (warp == kTcVWarp) {
     // ---------------------------------------------------------------- V loader
-    stream_kv(prob, &tm_v, sV, sm.v_full, sm.v_empty, nt, n_keys, lane, abort_flag, 102);
-  } else if (warp == 4) {
+    stream_kv(prob, &tm_v, &tb_v, &ts_v, sV, sm.v_full, sm.v_empty, nt, n_keys, lane, abort_flag, 102);
+  } else if (warp == kTcMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc(kFmtBF16, 128, 128, 0, 0);
@@ -206,44 +244,57 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- softmax (rows)
-    const int r = threadIdx.x;                 // 0..127 = TMEM lane
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    const uint32_t o_addr = lane_base + 256;
+    constexpr int HC = kTcKeys / 2;            // key columns per thread
+    const int quad = warp & 3, half = warp >> 2;
+    const int r = quad * 32 + lane;            // row = TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t o_addr = lane_base + 256 + half * HC;
+    const uint32_t pair_bar = 1 + quad;        // named barrier of warps quad and quad + 4
     const int64_t lim = prob.limit(r);
     const float sl2 = prob.scale_log2();
     constexpr float kRescale = 8.0f;           // log2 units: rescale when the max grows by > 2^8
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+    // Every bounded wait is followed by bar_all over the warp pair, so both warps of a
+    // row pair leave together when a wait runs out (a named barrier has no timeout).
     for (int j = 0; j < nt; ++j) {
       const int s = j & 1;
-      if (!(ok = mbar_wait_warp(&sm.s_full[s], (j >> 1) & 1, abort_flag, 111))) break;
-      tc_fence_after();
-      const int64_t t0 = (int64_t)j * kTcKeys;
-      float x[kTcKeys];
+      const bool got = mbar_wait_warp(&sm.s_full[s], (j >> 1) & 1, abort_flag, 111);
+      const int64_t t0 = (int64_t)j * kTcKeys + half * HC;
+      float x[HC];
+      float mx = -INFINITY;
+      if (got) {
+        tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + s * 128 + c * 32, x + c * 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&sm.s_empty[s]);             // S now lives in registers
-      float mx8[8];
+        for (int c = 0; c < HC / 32; ++c) tmem_ld32(lane_base + s * 128 + half * HC + c * 32, x + c * 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&sm.s_empty[s]);           // S now lives in registers
+        float mx8[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) mx8[q] = -INFINITY;
+        for (int q = 0; q < 8; ++q) mx8[q] = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < kTcKeys; ++e) {
-        x[e] = (t0 + e <= lim) ? x[e] * sl2 : -INFINITY;
-        mx8[e & 7] = fmaxf(mx8[e & 7], x[e]);
+        for (int e = 0; e < HC; ++e) {
+          x[e] = (t0 + e <= lim) ? x[e] * sl2 : -INFINITY;
+          mx8[e & 7] = fmaxf(mx8[e & 7], x[e]);
+        }
+        mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       }
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      if (mx > m + kRescale || m == -INFINITY) {
+      sm.red[half][r] = mx;
+      if (!(ok = bar_all(pair_bar, 64, got))) break;
+      mx = fmaxf(mx, sm.red[half ^ 1][r]);
+      asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");   // red[] is reused next
+      if (mx > m + kRescale || m == -INFINITY) {                      // same decision in both halves
         const float m_new = fmaxf(m, mx);
         if (j > 0 && m_new > m) {
           const float alpha = fast_exp2(m - m_new);
-          // O holds PV_0..PV_{j-1}; wait for the last of them, then scale in place
-          if (!(ok = mbar_wait_warp(&sm.pv_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, 110))) break;
+          // O holds PV_0..PV_{j-1}; wait for the last of them, then scale this half in place
+          const bool done = mbar_wait_warp(&sm.pv_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, 110);
+          if (!(ok = bar_all(pair_bar, 64, done))) break;
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < HC / 32; ++c) {
             float ov[32];
             tmem_ld32(o_addr + c * 32, ov);
             tmem_wait_ld();
@@ -257,13 +308,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         m = m_new;
       }
       const float m_use = m == -INFINITY ? 0.f : m;
-      if (!(ok = mbar_wait_warp(&sm.p_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, 112))) break;
-      const uint32_t pt = sP + s * kTileBytes;
+      const bool free_p = mbar_wait_warp(&sm.p_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, 112);
+      if (!(ok = bar_all(pair_bar, 64, free_p))) break;
+      const uint32_t pt = sP + s * kTileBytes + half * kBlkBytes;   // this half's 64-key block
       float ls8[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) ls8[q] = 0.f;
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {           // 16-byte chunks of the 256-byte P row
+      for (int c = 0; c < 8; ++c) {            // 16-byte chunks of the 128-byte half row
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 8; e += 2) {
@@ -273,29 +325,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           ls8[e + 1] += p1;
           pk[e / 2] = pack_bf16x2(p0, p1);
         }
-        const uint32_t dst = pt + (c >> 3) * kBlkBytes + sw128_off(r, c & 7);
-        st_shared_v4(dst, pk[0], pk[1], pk[2], pk[3]);
+        st_shared_v4(pt + sw128_off(r, c), pk[0], pk[1], pk[2], pk[3]);
       }
       l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(&sm.p_full[s]);
     }
-    if (ok && nt > 0) ok = mbar_wait_warp(&sm.pv_full[(nt - 1) & 1], ((nt - 1) >> 1) & 1, abort_flag, 113);
+    bool fin = ok;
+    if (ok && nt > 0) fin = mbar_wait_warp(&sm.pv_full[(nt - 1) & 1], ((nt - 1) >> 1) & 1, abort_flag, 113);
+    ok = bar_all(pair_bar, 64, fin);           // both halves of the pair get here
+    sm.red[half][r] = l;
+    asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+    const float l_row = l + sm.red[half ^ 1][r];
     if (ok) {
       tc_fence_after();
-      float o[kTcD];
+      float o[HC];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(o_addr + c * 32, o + c * 32);
+      for (int c = 0; c < HC / 32; ++c) tmem_ld32(o_addr + c * 32, o + c * 32);
       tmem_wait_ld();
-      prob.store(r, o, m, l);
+      prob.store(r, half * HC, o, m, l_row);
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 4) tmem_dealloc(tmem, 512);
+  if (warp == kTcMmaWarp) tmem_dealloc(tmem, 512);
 }
 
 // ------------------------------------------------------------------ ESA problem --
@@ -311,6 +367,7 @@ struct EsaTcProblem {
   int64_t n_cap, c0;
   int lq, hq, hkv, G;
   float sl2;
+  int staged;            // selected K/V rows were copied to contiguous buffers
   // per CTA
   int b, g, tile, cnt;
   int64_t n_prior, nk;
@@ -336,21 +393,50 @@ struct EsaTcProblem {
   __device__ int32_t kv_row(int64_t t) const {
     return (int32_t)(((int64_t)b * n_cap + keys.pos(b, cnt, t)) * hkv + g);
   }
+  // Q tile = 128 / G consecutive queries x the G heads of group g: one box of the
+  // [B * lq, hq, 128] map (rows past the chunk belong to no stored output)
+  __device__ bool q_box(int* y, int* z) const {
+    *y = g * G;
+    *z = (int)((int64_t)b * lq + (tile * kTcRows) / G);
+    return true;
+  }
+  // a key tile inside the initial tokens or inside the local part (window + chunk) is
+  // 128 consecutive tokens of the cache; one inside the selected tokens is 128
+  // consecutive rows of the staged copy [B, topk, Hkv, D]; keys past n_keys are loaded
+  // but masked by limit()
+  __device__ int kv_box(int j, int* y, int* z) const {
+    const int64_t t0 = (int64_t)j * kTcRows, t1 = t0 + kTcRows - 1;
+    *y = g;
+    if (t1 < keys.ni) {
+      *z = (int)((int64_t)b * n_cap + t0);
+      return 1;
+    }
+    if (t0 >= keys.ni + cnt) {
+      *z = (int)((int64_t)b * n_cap + keys.lo + (t0 - keys.ni - cnt));
+      return 1;
+    }
+    if (staged && t0 >= keys.ni && t1 < keys.ni + cnt) {
+      *z = (int)((int64_t)b * keys.idx_stride + (t0 - keys.ni));
+      return 2;
+    }
+    return 0;
+  }
   __device__ int64_t n_keys() const { return nk; }
   __device__ int64_t limit(int r) const {
     const int R = tile * kTcRows + r;
     return n_prior + min(R / G, lq - 1);
   }
   __device__ float scale_log2() const { return sl2; }
-  __device__ void store(int r, const float* acc, float m2, float l) {
+  // columns [col0, col0 + 64) of row r; the LSE comes with the first half
+  __device__ void store(int r, int col0, const float* acc, float m2, float l) {
     const int R = tile * kTcRows + r;
     if (R >= lq * G) return;
     const int i = R / G, hl = R % G;
     const int64_t row = ((int64_t)b * lq + i) * hq + g * G + hl;
     const float inv = 1.f / l;
-    uint4* dst = reinterpret_cast<uint4*>(o + row * kTcD);
+    uint4* dst = reinterpret_cast<uint4*>(o + row * kTcD + col0);
 #pragma unroll
-    for (int c = 0; c < kTcD / 8; ++c) {
+    for (int c = 0; c < kTcD / 16; ++c) {
       uint4 w;
       w.x = pack_bf16x2(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
       w.y = pack_bf16x2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
@@ -358,8 +444,37 @@ struct EsaTcProblem {
       w.w = pack_bf16x2(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
       dst[c] = w;
     }
-    if (lse) lse[row] = (m2 + __log2f(l)) * 0.69314718055994531f;
+    if (lse && col0 == 0) lse[row] = (m2 + __log2f(l)) * 0.69314718055994531f;
   }
 };
+
+}  // namespace esa
+
+namespace esa {
+
+// Copy the selected K and V rows of every sequence into contiguous buffers
+// [B, topk, Hkv, D] (all heads of a token are one contiguous row of Hkv * D elements),
+// so that the attention kernel loads selected keys as boxes instead of row gathers.
+// One CTA per (selected entry, sequence); 16-byte pieces.
+__global__ void __launch_bounds__(256) gather_selected_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                                              const int32_t* __restrict__ idx,
+                                                              const int32_t* __restrict__ count, int64_t n_cap,
+                                                              int topk, int row_vec, uint4* __restrict__ ks,
+                                                              uint4* __restrict__ vs) {
+  const int b = blockIdx.y;
+  const int cnt = min(max(count[b], 0), topk);
+  for (int t = blockIdx.x; t < cnt; t += gridDim.x) {
+    int64_t p = idx[(int64_t)b * topk + t];
+    p = p < 0 ? 0 : (p >= n_cap ? n_cap - 1 : p);
+    const uint4* ksrc = k + ((int64_t)b * n_cap + p) * row_vec;
+    const uint4* vsrc = v + ((int64_t)b * n_cap + p) * row_vec;
+    uint4* kd = ks + ((int64_t)b * topk + t) * row_vec;
+    uint4* vd = vs + ((int64_t)b * topk + t) * row_vec;
+    for (int e = threadIdx.x; e < row_vec; e += blockDim.x) {
+      kd[e] = ld_stream16(ksrc + e);
+      vd[e] = ld_stream16(vsrc + e);
+    }
+  }
+}
 
 }  // namespace esa

@@ -180,6 +180,24 @@ esa_status_t make_tmap_rows_bf16(CUtensorMap* m, const void* base, uint64_t rows
   return ESA_OK;
 }
 
+// 3D tensor map over bf16 [tokens, heads, 128]; a box is box_tokens consecutive tokens x
+// box_heads consecutive heads x 64 columns, 128-byte swizzle (rows ordered token-major).
+esa_status_t make_tmap_box_bf16(CUtensorMap* m, const void* base, uint64_t heads, uint64_t tokens,
+                                uint32_t box_heads, uint32_t box_tokens) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode;
+  esa_status_t st = get_encoder(&encode);
+  if (st != ESA_OK) return st;
+  cuuint64_t dims[3] = {128, heads, tokens};
+  cuuint64_t strides[2] = {128 * 2, heads * 128 * 2};
+  cuuint32_t box[3] = {64, box_heads, box_tokens};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ESA_ERR_CUDA, "cuTensorMapEncodeTiled (box) failed (%d)", (int)r);
+  return ESA_OK;
+}
+
 esa_status_t make_tmap_f32(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols) {
   PFN_cuTensorMapEncodeTiled_v12000 encode;
   esa_status_t st0 = get_encoder(&encode);
@@ -407,7 +425,11 @@ AttnPlan plan_attn(int32_t batch, int32_t lq, int64_t c0, int32_t hq, int32_t hk
   const Regions r = regions(c0, p);
   const int g = hq / hkv;
   pl.tc = dt == ESA_BF16 && head_dim == 128 && (int64_t)lq * g >= 64;
-  if (pl.tc) return pl;
+  if (pl.tc) {
+    // staged copies of the selected K and V rows: [B, topk, Hkv, D] bf16 each
+    pl.ws_bytes = 2 * up256((size_t)batch * p.topk * hkv * head_dim * 2);
+    return pl;
+  }
   const int64_t n_keys_max = r.ni + std::min<int64_t>(p.topk, r.n_mid) + (c0 - r.lo) + lq;
   const int64_t base = (int64_t)batch * lq * hkv;
   const int64_t want_ctas = 4 * 148;
@@ -494,12 +516,30 @@ esa_status_t esa_sparse_attn(const void* q, const void* k, const void* v, esa_dt
     pr.sl2 = sl2;
     if ((int64_t)batch * n_cap * hkv >= ((int64_t)1 << 31) || (int64_t)batch * lq * hq >= ((int64_t)1 << 31))
       return fail(ESA_ERR_UNSUPPORTED, "more than 2^31 K/V or Q rows");
-    CUtensorMap tq, tk, tv;
+    uint8_t* ks = static_cast<uint8_t*>(workspace);
+    uint8_t* vs = ks + pl.ws_bytes / 2;
+    const int row_vec = hkv * head_dim * 2 / 16;
+    const int64_t max_sel = std::min<int64_t>(p.topk, r.n_mid);
+    pr.staged = max_sel > 0 ? 1 : 0;
+    if (max_sel > 0) {
+      const dim3 ggrid((unsigned)std::min<int64_t>(max_sel, 4096), batch);
+      esa::gather_selected_kernel<<<ggrid, 128, 0, s>>>(
+          static_cast<const uint4*>(k), static_cast<const uint4*>(v), idx, count, n_cap, p.topk, row_vec,
+          reinterpret_cast<uint4*>(ks), reinterpret_cast<uint4*>(vs));
+      ESA_LAUNCH_CHECK("gather_selected_kernel");
+    }
+    CUtensorMap tq, tk, tv, bq, bk, bv, sk, sv;
+    if ((st = make_tmap_box_bf16(&sk, ks, hkv, (uint64_t)batch * p.topk, 1, esa::kTcKeys)) != ESA_OK) return st;
+    if ((st = make_tmap_box_bf16(&sv, vs, hkv, (uint64_t)batch * p.topk, 1, esa::kTcKeys)) != ESA_OK) return st;
     if ((st = make_tmap_rows_bf16(&tq, q, (uint64_t)batch * lq * hq)) != ESA_OK) return st;
     if ((st = make_tmap_rows_bf16(&tk, k, (uint64_t)batch * n_cap * hkv)) != ESA_OK) return st;
     if ((st = make_tmap_rows_bf16(&tv, v, (uint64_t)batch * n_cap * hkv)) != ESA_OK) return st;
+    if ((st = make_tmap_box_bf16(&bq, q, hq, (uint64_t)batch * lq, g, esa::kTcRows / g)) != ESA_OK) return st;
+    if ((st = make_tmap_box_bf16(&bk, k, hkv, (uint64_t)batch * n_cap, 1, esa::kTcKeys)) != ESA_OK) return st;
+    if ((st = make_tmap_box_bf16(&bv, v, hkv, (uint64_t)batch * n_cap, 1, esa::kTcKeys)) != ESA_OK) return st;
     dim3 grid((unsigned)cdiv((int64_t)lq * g, esa::kTcRows), hkv, batch);
-    esa::attn_tc_kernel<esa::EsaTcProblem><<<grid, esa::kTcThreads, esa::kTcSmemBytes, s>>>(tq, tk, tv, pr);
+    esa::attn_tc_kernel<esa::EsaTcProblem><<<grid, esa::kTcThreads, esa::kTcSmemBytes, s>>>(tq, tk, tv, bq, bk, bv,
+                                                                                           sk, sv, pr);
     ESA_LAUNCH_CHECK("attn_tc_kernel<esa>");
     return ok();
   }
@@ -645,11 +685,14 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
     if (sa != ESA_OK) return sa;
     attr_set[dev] = true;
   }
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, bq, bk, bv;
   esa_status_t st;
   if ((st = make_tmap_rows_bf16(&tq, q, (uint64_t)batch * seq * heads)) != ESA_OK) return st;
   if ((st = make_tmap_rows_bf16(&tk, k, (uint64_t)batch * seq * heads)) != ESA_OK) return st;
   if ((st = make_tmap_rows_bf16(&tv, v, (uint64_t)batch * seq * heads)) != ESA_OK) return st;
+  if ((st = make_tmap_box_bf16(&bq, q, heads, (uint64_t)batch * seq, 1, esa::kTcRows)) != ESA_OK) return st;
+  if ((st = make_tmap_box_bf16(&bk, k, heads, (uint64_t)batch * seq, 1, esa::kTcKeys)) != ESA_OK) return st;
+  if ((st = make_tmap_box_bf16(&bv, v, heads, (uint64_t)batch * seq, 1, esa::kTcKeys)) != ESA_OK) return st;
   ESA_CUDA(cudaMemsetAsync(w.cnt, 0, w.zero_bytes, s));
   const dim3 lgrid((unsigned)cdiv(seq * heads, 256), batch);
   if (topk > 0 && w.pairs > 0) {
@@ -677,7 +720,7 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
     pp.n_lists = w.n_lists;
     pp.sl2 = sl2;
     esa::attn_tc_kernel<esa::MobaPastProblem><<<(unsigned)w.max_tiles, esa::kTcThreads, esa::kTcSmemBytes, s>>>(
-        tq, tk, tv, pp);
+        tq, tk, tv, bq, bk, bv, bk, bv, pp);
     ESA_LAUNCH_CHECK("attn_tc_kernel<moba past>");
   }
   esa::MobaCurrentProblem cp{};
@@ -694,7 +737,8 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
   cp.tiles_per_block = (int)cdiv(block, esa::kTcRows);
   cp.sl2 = sl2;
   esa::attn_tc_kernel<esa::MobaCurrentProblem>
-      <<<dim3(cp.tiles_per_block * nb, heads, batch), esa::kTcThreads, esa::kTcSmemBytes, s>>>(tq, tk, tv, cp);
+      <<<dim3(cp.tiles_per_block * nb, heads, batch), esa::kTcThreads, esa::kTcSmemBytes, s>>>(tq, tk, tv, bq, bk, bv,
+                                                                                            bk, bv, cp);
   ESA_LAUNCH_CHECK("attn_tc_kernel<moba current>");
   const int64_t rows = (int64_t)batch * seq * heads;
   esa::moba_combine_kernel<128><<<(unsigned)cdiv(rows, 8), 256, 0, s>>>(

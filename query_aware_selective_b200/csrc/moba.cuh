@@ -242,20 +242,26 @@ struct MobaPastProblem {
   __device__ int32_t kv_row(int64_t t) const {
     return (int32_t)(((int64_t)b * seq + (int64_t)blk * block + t) * heads + h);
   }
+  __device__ bool q_box(int*, int*) const { return false; }        // listed queries: gathered
+  __device__ int kv_box(int j, int* y, int* z) const {              // a block is consecutive tokens
+    *y = h;
+    *z = (int)((int64_t)b * seq + (int64_t)blk * block + (int64_t)j * kTcKeys);
+    return 1;
+  }
   __device__ int64_t limit(int) const { return n_keys() - 1; }
   __device__ float scale_log2() const { return sl2; }
-  __device__ void store(int r, const float* acc, float m2, float l) {
+  __device__ void store(int r, int col0, const float* acc, float m2, float l) {
     if ((uint32_t)r >= n_rows) return;
     const uint32_t e = list[e0 + r];
     const int64_t p = e >> 4;
     const int slot = e & 15;
     const int64_t row = (((int64_t)b * seq + p) * heads + h) * (topk + 1) + slot;
     const float inv = 1.f / l;
-    float4* dst = reinterpret_cast<float4*>(part_o + row * kTcD);
+    float4* dst = reinterpret_cast<float4*>(part_o + row * kTcD + col0);
 #pragma unroll
-    for (int c = 0; c < kTcD / 4; ++c)
+    for (int c = 0; c < kTcD / 8; ++c)
       dst[c] = make_float4(acc[4 * c] * inv, acc[4 * c + 1] * inv, acc[4 * c + 2] * inv, acc[4 * c + 3] * inv);
-    part_lse[row] = (m2 + __log2f(l)) * 0.69314718055994531f;
+    if (col0 == 0) part_lse[row] = (m2 + __log2f(l)) * 0.69314718055994531f;
   }
 };
 
@@ -291,19 +297,29 @@ struct MobaCurrentProblem {
   }
   __device__ int64_t n_keys() const { return p0 + nrows - kb0; }
   __device__ int32_t kv_row(int64_t t) const { return (int32_t)(((int64_t)b * seq + kb0 + t) * heads + h); }
+  __device__ bool q_box(int* y, int* z) const {                     // 128 consecutive queries of head h
+    *y = h;
+    *z = (int)((int64_t)b * seq + p0);
+    return true;
+  }
+  __device__ int kv_box(int j, int* y, int* z) const {
+    *y = h;
+    *z = (int)((int64_t)b * seq + kb0 + (int64_t)j * kTcKeys);
+    return 1;
+  }
   __device__ int64_t limit(int r) const { return p0 + min((int64_t)r, nrows - 1) - kb0; }
   __device__ float scale_log2() const { return sl2; }
-  __device__ void store(int r, const float* acc, float m2, float l) {
+  __device__ void store(int r, int col0, const float* acc, float m2, float l) {
     if (r >= nrows) return;
     const int64_t p = p0 + r;
     const int slot = min(topk, blk);
     const int64_t row = (((int64_t)b * seq + p) * heads + h) * (topk + 1) + slot;
     const float inv = 1.f / l;
-    float4* dst = reinterpret_cast<float4*>(part_o + row * kTcD);
+    float4* dst = reinterpret_cast<float4*>(part_o + row * kTcD + col0);
 #pragma unroll
-    for (int c = 0; c < kTcD / 4; ++c)
+    for (int c = 0; c < kTcD / 8; ++c)
       dst[c] = make_float4(acc[4 * c] * inv, acc[4 * c + 1] * inv, acc[4 * c + 2] * inv, acc[4 * c + 3] * inv);
-    part_lse[row] = (m2 + __log2f(l)) * 0.69314718055994531f;
+    if (col0 == 0) part_lse[row] = (m2 + __log2f(l)) * 0.69314718055994531f;
   }
 };
 
