@@ -270,16 +270,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&sm.s_empty[s]);           // S now lives in registers
+        // keys t0 + e with e <= rem are visible (causal cut); masked scores become -inf
+        const int64_t rem64 = lim - t0;
+        const int rem = rem64 < 0 ? -1 : (rem64 >= HC ? HC : (int)rem64);
         float mx8[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) mx8[q] = -INFINITY;
 #pragma unroll
         for (int e = 0; e < HC; ++e) {
-          x[e] = (t0 + e <= lim) ? x[e] * sl2 : -INFINITY;
+          x[e] = e <= rem ? x[e] : -INFINITY;
           mx8[e & 7] = fmaxf(mx8[e & 7], x[e]);
         }
         mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;   // scale > 0
       }
       sm.red[half][r] = mx;
       if (!(ok = bar_all(pair_bar, 64, got))) break;
@@ -319,8 +322,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 8; e += 2) {
-          const float p0 = fast_exp2(x[c * 8 + e] - m_use);
-          const float p1 = fast_exp2(x[c * 8 + e + 1] - m_use);
+          const float p0 = fast_exp2(fmaf(x[c * 8 + e], sl2, -m_use));
+          const float p1 = fast_exp2(fmaf(x[c * 8 + e + 1], sl2, -m_use));
           ls8[e] += p0;
           ls8[e + 1] += p1;
           pk[e / 2] = pack_bf16x2(p0, p1);

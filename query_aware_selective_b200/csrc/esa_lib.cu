@@ -264,24 +264,34 @@ esa_status_t esa_compress(const void* x, esa_dtype_t x_dtype, int64_t rows, int6
   if (x_row_stride < (int64_t)n_heads_in * head_dim || x_row_stride % 8)
     return fail(ESA_ERR_INVALID_ARG, "x_row_stride must be >= n_heads_in * head_dim and a multiple of 8");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (x_dtype == ESA_BF16 && d_out == esa::kCtN) {
-    // tensor-core path: 8-CTA clusters split the reduction, 128 rows per cluster
+  const int g = n_heads_out / n_heads_in;
+  if (x_dtype == ESA_BF16 && d_out == esa::kCtN && (g == 1 || g == 2 || g == 4)) {
+    // tensor-core path: 8-CTA clusters split the reduction, 128 rows x 64 columns per CTA
     static bool attr_set[64] = {};
     int dev = 0;
     ESA_CUDA(cudaGetDevice(&dev));
     if (dev < 64 && !attr_set[dev]) {
-      const esa_status_t st = set_max_smem(esa::compress_tc_kernel, esa::kCtSmemBytes);
+      esa_status_t st = set_max_smem(esa::compress_tc_kernel<1>, esa::kCtSmemBytes);
+      if (st == ESA_OK) st = set_max_smem(esa::compress_tc_kernel<2>, esa::kCtSmemBytes);
+      if (st == ESA_OK) st = set_max_smem(esa::compress_tc_kernel<4>, esa::kCtSmemBytes);
       if (st != ESA_OK) return st;
       attr_set[dev] = true;
     }
-    const int g = n_heads_out / n_heads_in;
     const int64_t max_rows = (int64_t)65535 * esa::kCtRows;
     for (int64_t r0 = 0; r0 < rows; r0 += max_rows) {
       const int64_t nr = std::min(rows - r0, max_rows);
-      const dim3 grid(esa::kCtCluster, (unsigned)cdiv(nr, esa::kCtRows));
-      esa::compress_tc_kernel<<<grid, esa::kCtThreads, esa::kCtSmemBytes, s>>>(
-          static_cast<const __nv_bfloat16*>(x) + r0 * x_row_stride, nr, x_row_stride, n_heads_in, g, head_dim, w,
-          y + r0 * y_row_stride, y_row_stride);
+      const dim3 grid(esa::kCtCluster, (unsigned)cdiv(nr, esa::kCtRows), esa::kCtN / esa::kCtNS);
+      const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x) + r0 * x_row_stride;
+      float* yb = y + r0 * y_row_stride;
+      if (g == 1)
+        esa::compress_tc_kernel<1><<<grid, esa::kCtThreads, esa::kCtSmemBytes, s>>>(xb, nr, x_row_stride, n_heads_in,
+                                                                                    head_dim, w, yb, y_row_stride);
+      else if (g == 2)
+        esa::compress_tc_kernel<2><<<grid, esa::kCtThreads, esa::kCtSmemBytes, s>>>(xb, nr, x_row_stride, n_heads_in,
+                                                                                    head_dim, w, yb, y_row_stride);
+      else
+        esa::compress_tc_kernel<4><<<grid, esa::kCtThreads, esa::kCtSmemBytes, s>>>(xb, nr, x_row_stride, n_heads_in,
+                                                                                    head_dim, w, yb, y_row_stride);
       ESA_LAUNCH_CHECK("compress_tc_kernel");
     }
     return ok();
