@@ -217,8 +217,9 @@ size_t moba_workspace_size(int32_t which, int32_t batch, int64_t seq, int32_t he
 const char* esa_last_error(void);
 
 /* Waits for `stream`, then reads and clears the device status word of the current
- * device. Returns ESA_OK, or ESA_ERR_TIMEOUT if a kernel's bounded wait ran out since
- * the last read (the message names the kernel and the wait). */
+ * device. Returns ESA_OK, ESA_ERR_TIMEOUT if a kernel's bounded wait ran out since the
+ * last read (the message names the kernel and the wait), or ESA_ERR_CUDA if a kernel
+ * stopped early on a launch-environment check (e.g. misaligned shared memory). */
 esa_status_t esa_device_status(void* stream);
 
 /* Number of kernels this library has launched in this process, all devices and

@@ -7,10 +7,10 @@
 // m is the running row maximum used for the exponentials; it is raised (and O, l
 // rescaled in place) only when a tile's maximum exceeds it by more than 2^8, so most
 // tiles skip the rescale and P stays <= 2^8 (exact softmax either way: o = O / l).
-// Roles (352 threads): warps 0-7 softmax (warp w owns TMEM lanes 32 (w % 4) .. + 31,
-// i.e. rows, and key columns 64 (w / 4) .. + 63: two threads per row, exchanging the
-// row max and sum through shared memory), warp 8 issues the MMAs (one lane), warp 9
-// loads Q and the K tiles, warp 10 loads the V tiles.
+// Roles (608 threads): warps 0-15 softmax (warp w owns TMEM lanes 32 (w % 4) .. + 31,
+// i.e. rows, and key columns 32 (w / 4) .. + 31: four threads per row, exchanging the
+// row max and sum through shared memory), warp 16 issues the MMAs (one lane), warp 17
+// loads Q and the K tiles, warp 18 loads the V tiles.
 // Tiles come in by TMA straight into the 128-byte swizzled layout the MMA descriptors
 // name, and the "full" barriers complete on the transaction count. A tile whose 128
 // keys are consecutive tokens (initial tokens, local window, chunk, MoBA blocks) is
@@ -40,15 +40,18 @@
 
 namespace esa {
 
-constexpr int kTcThreads = 352;
-constexpr int kTcMmaWarp = 8, kTcKWarp = 9, kTcVWarp = 10;
+constexpr int kTcSplit = 4;                                  // softmax threads per row
+constexpr int kTcThreads = (4 * kTcSplit + 3) * 32;
+constexpr int kTcMmaWarp = 4 * kTcSplit, kTcKWarp = kTcMmaWarp + 1, kTcVWarp = kTcMmaWarp + 2;
 constexpr int kTcRows = 128;
 constexpr int kTcKeys = 128;
 constexpr int kTcD = 128;
 constexpr uint32_t kTileBytes = 128 * 256;            // 128 rows x 128 bf16
 constexpr uint32_t kBlkBytes = 128 * 128;             // one 64-column block of a tile
-constexpr uint32_t kTcCtrlBytes = 2048;                       // barriers, TMEM address, key positions
-constexpr uint32_t kTcSmemBytes = 7 * kTileBytes + 1024 /*align*/ + kTcCtrlBytes;
+constexpr uint32_t kTcCtrlBytes = 3072;                       // barriers, TMEM address, row exchange
+// No alignment slack: the kernel checks that the dynamic shared memory starts on a
+// 1024-byte boundary (the 128-byte swizzle atoms need it) and stops with an error if not.
+constexpr uint32_t kTcSmemBytes = 7 * kTileBytes + kTcCtrlBytes;
 static_assert(kTcSmemBytes <= 232448, "exceeds the 227 KB of shared memory per CTA");
 
 struct TcSmem {
@@ -59,7 +62,7 @@ struct TcSmem {
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
-  float red[2][128];         // per-row partial max / sum of the two column halves
+  float red[kTcSplit][128];  // per-row partial max / sum of the column parts
 };
 static_assert(sizeof(TcSmem) <= kTcCtrlBytes, "control block overflows its reservation");
 
@@ -132,8 +135,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                    const __grid_constant__ CUtensorMap tb_k, const __grid_constant__ CUtensorMap tb_v,
                    const __grid_constant__ CUtensorMap ts_k, const __grid_constant__ CUtensorMap ts_v,
                    Problem prob) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) record_status(5u, 100);
+    return;
+  }
   const uint32_t sQ = smem_u32(smem);
   const uint32_t sK = sQ + kTileBytes;       // 2 stages
   const uint32_t sV = sK + 2 * kTileBytes;   // 2 stages
@@ -153,8 +160,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&sm.k_empty[s], 1);
       mbar_init(&sm.v_empty[s], 1);
       mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.s_empty[s], 256);
-      mbar_init(&sm.p_full[s], 256);
+      mbar_init(&sm.s_empty[s], 128 * kTcSplit);
+      mbar_init(&sm.p_full[s], 128 * kTcSplit);
       mbar_init(&sm.p_empty[s], 1);
       mbar_init(&sm.pv_full[s], 1);
     }
@@ -244,29 +251,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- softmax (rows)
-    constexpr int HC = kTcKeys / 2;            // key columns per thread
-    const int quad = warp & 3, half = warp >> 2;
+    constexpr int HC = kTcKeys / kTcSplit;     // key columns per thread
+    constexpr uint32_t kGroup = 32 * kTcSplit; // threads sharing a row set (named barrier size)
+    const int quad = warp & 3, part = warp >> 2;
     const int r = quad * 32 + lane;            // row = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    const uint32_t o_addr = lane_base + 256 + half * HC;
-    const uint32_t pair_bar = 1 + quad;        // named barrier of warps quad and quad + 4
+    const uint32_t o_addr = lane_base + 256 + part * HC;
+    const uint32_t row_bar = 1 + quad;         // named barrier of the kTcSplit warps of this quadrant
     const int64_t lim = prob.limit(r);
     const float sl2 = prob.scale_log2();
     constexpr float kRescale = 8.0f;           // log2 units: rescale when the max grows by > 2^8
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    // Every bounded wait is followed by bar_all over the warp pair, so both warps of a
-    // row pair leave together when a wait runs out (a named barrier has no timeout).
+    // Every bounded wait is followed by bar_all over the row group, so all warps of a
+    // row group leave together when a wait runs out (a named barrier has no timeout).
     for (int j = 0; j < nt; ++j) {
       const int s = j & 1;
       const bool got = mbar_wait_warp(&sm.s_full[s], (j >> 1) & 1, abort_flag, 111);
-      const int64_t t0 = (int64_t)j * kTcKeys + half * HC;
+      const int64_t t0 = (int64_t)j * kTcKeys + part * HC;
       float x[HC];
       float mx = -INFINITY;
       if (got) {
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < HC / 32; ++c) tmem_ld32(lane_base + s * 128 + half * HC + c * 32, x + c * 32);
+        for (int c = 0; c < HC / 32; ++c) tmem_ld32(lane_base + s * 128 + part * HC + c * 32, x + c * 32);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&sm.s_empty[s]);           // S now lives in registers
@@ -276,25 +284,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         float mx8[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) mx8[q] = -INFINITY;
+        if (rem >= HC - 1) {                   // the whole part is visible: no mask
 #pragma unroll
-        for (int e = 0; e < HC; ++e) {
-          x[e] = e <= rem ? x[e] : -INFINITY;
-          mx8[e & 7] = fmaxf(mx8[e & 7], x[e]);
+          for (int e = 0; e < HC; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], x[e]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < HC; ++e) {
+            x[e] = e <= rem ? x[e] : -INFINITY;
+            mx8[e & 7] = fmaxf(mx8[e & 7], x[e]);
+          }
         }
         mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                    fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;   // scale > 0
       }
-      sm.red[half][r] = mx;
-      if (!(ok = bar_all(pair_bar, 64, got))) break;
-      mx = fmaxf(mx, sm.red[half ^ 1][r]);
-      asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");   // red[] is reused next
-      if (mx > m + kRescale || m == -INFINITY) {                      // same decision in both halves
+      sm.red[part][r] = mx;
+      if (!(ok = bar_all(row_bar, kGroup, got))) break;
+#pragma unroll
+      for (int q = 0; q < kTcSplit; ++q) mx = fmaxf(mx, sm.red[q][r]);
+      asm volatile("bar.sync %0, %1;" ::"r"(row_bar), "r"(kGroup) : "memory");   // red[] is reused next
+      if (mx > m + kRescale || m == -INFINITY) {                                  // same in the whole group
         const float m_new = fmaxf(m, mx);
         if (j > 0 && m_new > m) {
           const float alpha = fast_exp2(m - m_new);
-          // O holds PV_0..PV_{j-1}; wait for the last of them, then scale this half in place
+          // O holds PV_0..PV_{j-1}; wait for the last of them, then scale this part in place
           const bool done = mbar_wait_warp(&sm.pv_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, 110);
-          if (!(ok = bar_all(pair_bar, 64, done))) break;
+          if (!(ok = bar_all(row_bar, kGroup, done))) break;
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < HC / 32; ++c) {
@@ -312,23 +326,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       const float m_use = m == -INFINITY ? 0.f : m;
       const bool free_p = mbar_wait_warp(&sm.p_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, 112);
-      if (!(ok = bar_all(pair_bar, 64, free_p))) break;
-      const uint32_t pt = sP + s * kTileBytes + half * kBlkBytes;   // this half's 64-key block
+      if (!(ok = bar_all(row_bar, kGroup, free_p))) break;
+      // this part's keys: 64-key block (part * HC) / 64, first 16-byte chunk ((part * HC) % 64) / 8
+      const uint32_t pt = sP + s * kTileBytes + ((part * HC) >> 6) * kBlkBytes;
+      const int ch0 = ((part * HC) & 63) >> 3;
       float ls8[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) ls8[q] = 0.f;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {            // 16-byte chunks of the 128-byte half row
+      for (int c = 0; c < HC / 8; ++c) {       // 16-byte chunks of this part
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 8; e += 2) {
-          const float p0 = fast_exp2(fmaf(x[c * 8 + e], sl2, -m_use));
-          const float p1 = fast_exp2(fmaf(x[c * 8 + e + 1], sl2, -m_use));
-          ls8[e] += p0;
-          ls8[e + 1] += p1;
-          pk[e / 2] = pack_bf16x2(p0, p1);
+          // P goes to the MMA as bf16 by truncation (integer ops only); the row sum adds
+          // the same truncated values, so the normalisation matches what the MMA sees
+          const uint32_t b0 = __float_as_uint(fast_exp2(fmaf(x[c * 8 + e], sl2, -m_use))) & 0xFFFF0000u;
+          const uint32_t b1 = __float_as_uint(fast_exp2(fmaf(x[c * 8 + e + 1], sl2, -m_use))) & 0xFFFF0000u;
+          ls8[e] += __uint_as_float(b0);
+          ls8[e + 1] += __uint_as_float(b1);
+          pk[e / 2] = __byte_perm(b0, b1, 0x7632);
         }
-        st_shared_v4(pt + sw128_off(r, c), pk[0], pk[1], pk[2], pk[3]);
+        st_shared_v4(pt + sw128_off(r, ch0 + c), pk[0], pk[1], pk[2], pk[3]);
       }
       l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       fence_proxy_async();
@@ -337,17 +355,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     bool fin = ok;
     if (ok && nt > 0) fin = mbar_wait_warp(&sm.pv_full[(nt - 1) & 1], ((nt - 1) >> 1) & 1, abort_flag, 113);
-    ok = bar_all(pair_bar, 64, fin);           // both halves of the pair get here
-    sm.red[half][r] = l;
-    asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
-    const float l_row = l + sm.red[half ^ 1][r];
+    ok = bar_all(row_bar, kGroup, fin);        // every warp of the row group gets here
+    sm.red[part][r] = l;
+    asm volatile("bar.sync %0, %1;" ::"r"(row_bar), "r"(kGroup) : "memory");
+    float l_row = 0.f;
+#pragma unroll
+    for (int q = 0; q < kTcSplit; ++q) l_row += sm.red[q][r];
     if (ok) {
       tc_fence_after();
       float o[HC];
 #pragma unroll
       for (int c = 0; c < HC / 32; ++c) tmem_ld32(o_addr + c * 32, o + c * 32);
       tmem_wait_ld();
-      prob.store(r, half * HC, o, m, l_row);
+      prob.store(r, part * HC, o, m, l_row);
     }
   }
 
@@ -430,7 +450,7 @@ struct EsaTcProblem {
     return n_prior + min(R / G, lq - 1);
   }
   __device__ float scale_log2() const { return sl2; }
-  // columns [col0, col0 + 64) of row r; the LSE comes with the first half
+  // columns [col0, col0 + kTcD / kTcSplit) of row r; the LSE comes with the first part
   __device__ void store(int r, int col0, const float* acc, float m2, float l) {
     const int R = tile * kTcRows + r;
     if (R >= lq * G) return;
@@ -439,7 +459,7 @@ struct EsaTcProblem {
     const float inv = 1.f / l;
     uint4* dst = reinterpret_cast<uint4*>(o + row * kTcD + col0);
 #pragma unroll
-    for (int c = 0; c < kTcD / 16; ++c) {
+    for (int c = 0; c < kTcD / kTcSplit / 8; ++c) {
       uint4 w;
       w.x = pack_bf16x2(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
       w.y = pack_bf16x2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);

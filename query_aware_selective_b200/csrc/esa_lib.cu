@@ -243,8 +243,9 @@ esa_status_t esa_device_status(void* stream) {
   if (v == 0) return ok();
   const unsigned long long zero = 0;
   ESA_CUDA(cudaMemcpyToSymbol(esa::g_status, &zero, sizeof(zero)));
-  return fail(ESA_ERR_TIMEOUT, "device wait ran out at site %u (status %u)", (unsigned)(v & 0xffffffffu),
-              (unsigned)(v >> 32));
+  const unsigned code = (unsigned)(v >> 32), site = (unsigned)(v & 0xffffffffu);
+  if (code == 5u) return fail(ESA_ERR_CUDA, "kernel site %u found its shared memory misaligned and stopped", site);
+  return fail(ESA_ERR_TIMEOUT, "device wait ran out at site %u (status %u)", site, code);
 }
 
 // ------------------------------------------------------------------ esa_compress --

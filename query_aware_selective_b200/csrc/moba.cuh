@@ -259,7 +259,7 @@ struct MobaPastProblem {
     const float inv = 1.f / l;
     float4* dst = reinterpret_cast<float4*>(part_o + row * kTcD + col0);
 #pragma unroll
-    for (int c = 0; c < kTcD / 8; ++c)
+    for (int c = 0; c < kTcD / kTcSplit / 4; ++c)
       dst[c] = make_float4(acc[4 * c] * inv, acc[4 * c + 1] * inv, acc[4 * c + 2] * inv, acc[4 * c + 3] * inv);
     if (col0 == 0) part_lse[row] = (m2 + __log2f(l)) * 0.69314718055994531f;
   }
@@ -317,7 +317,7 @@ struct MobaCurrentProblem {
     const float inv = 1.f / l;
     float4* dst = reinterpret_cast<float4*>(part_o + row * kTcD + col0);
 #pragma unroll
-    for (int c = 0; c < kTcD / 8; ++c)
+    for (int c = 0; c < kTcD / kTcSplit / 4; ++c)
       dst[c] = make_float4(acc[4 * c] * inv, acc[4 * c + 1] * inv, acc[4 * c + 2] * inv, acc[4 * c + 3] * inv);
     if (col0 == 0) part_lse[row] = (m2 + __log2f(l)) * 0.69314718055994531f;
   }
