@@ -18,8 +18,11 @@
 // scattered keys (the selected middle tokens) is 32 tile::gather4 loads per half
 // (4 arbitrary rows each; each lane of the loader warp issues its 4 rows).
 //
-// Shared memory: Q 32 KB, K 2 x 32 KB, V 2 x 32 KB, P 2 x 32 KB (each operand tile is
-// two 16 KB column blocks of 128 rows x 128 bytes). TMEM: S double buffer (2 x 128
+// Shared memory: Q 32 KB, K 3 x 32 KB, V 2 x 32 KB, P 32 KB (each operand tile is
+// two 16 KB column blocks of 128 rows x 128 bytes). K gets the deepest ring because
+// S_{j+1} is issued while P_j is being formed, so K tile j + 2 must already be on its
+// way; P needs one buffer: P_j is written after the row max of S_j is known, by which
+// time PV_{j-1} (the previous reader) has finished. TMEM: S double buffer (2 x 128
 // columns) and the O accumulator (128 columns).
 //
 // The problem policy P says which rows and keys a CTA owns:
@@ -51,13 +54,14 @@ constexpr uint32_t kBlkBytes = 128 * 128;             // one 64-column block of 
 constexpr uint32_t kTcCtrlBytes = 3072;                       // barriers, TMEM address, row exchange
 // No alignment slack: the kernel checks that the dynamic shared memory starts on a
 // 1024-byte boundary (the 128-byte swizzle atoms need it) and stops with an error if not.
-constexpr uint32_t kTcSmemBytes = 7 * kTileBytes + kTcCtrlBytes;
+constexpr int kTcKStages = 3, kTcVStages = 2;
+constexpr uint32_t kTcSmemBytes = (2 + kTcKStages + kTcVStages) * kTileBytes + kTcCtrlBytes;
 static_assert(kTcSmemBytes <= 232448, "exceeds the 227 KB of shared memory per CTA");
 
 struct TcSmem {
   uint64_t q_full;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
+  uint64_t k_full[kTcKStages], k_empty[kTcKStages], v_full[kTcVStages], v_empty[kTcVStages];
+  uint64_t s_full[2], s_empty[2], p_full, p_empty;
   uint64_t pv_full[2];
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -79,10 +83,10 @@ __device__ __forceinline__ void gather_tile(uint32_t dst, const CUtensorMap* tm,
   tma_gather4(d + kBlkBytes, tm, 64, r[0], r[1], r[2], r[3], bar);
 }
 
-// One loader warp streams the key tiles of one operand (K or V) through the two
-// stages. The rows of tile j + 1 are looked up (4 per lane, consecutive keys, so a
+// One loader warp streams the key tiles of one operand (K or V) through its NST
+// stages (tile j in stage j % NST, the barrier's j / NST-th phase). The rows of tile j + 1 are looked up (4 per lane, consecutive keys, so a
 // gathered index list is read coalesced) while tile j waits for its stage.
-template <class Problem>
+template <int NST, class Problem>
 __device__ __forceinline__ void stream_kv(const Problem& prob, const CUtensorMap* tm_rows, const CUtensorMap* tm_box,
                                           const CUtensorMap* tm_staged, uint32_t stage0, uint64_t* full,
                                           uint64_t* empty, int nt, int64_t n_keys, int lane,
@@ -101,7 +105,8 @@ __device__ __forceinline__ void stream_kv(const Problem& prob, const CUtensorMap
   int box_next = prob.kv_box(0, &by, &bz);        // 0: gather, 1: cache box, 2: staged box
   if (!box_next) fetch(0, nxt);
   for (int j = 0; j < nt; ++j) {
-    const int s = j & 1;
+    const int s = j % NST;
+    const int ph = (j / NST) & 1;
     const int box = box_next;
     const int y = by, z = bz;
 #pragma unroll
@@ -110,7 +115,7 @@ __device__ __forceinline__ void stream_kv(const Problem& prob, const CUtensorMap
       box_next = prob.kv_box(j + 1, &by, &bz);
       if (!box_next) fetch(j + 1, nxt);
     }
-    bool ok = mbar_wait(&empty[s], ((j >> 1) & 1) ^ 1, abort_flag, site);
+    bool ok = mbar_wait(&empty[s], ph ^ 1, abort_flag, site);
     if (!__all_sync(0xffffffffu, ok)) return;
     const uint32_t dst = stage0 + s * kTileBytes;
     if (box) {
@@ -142,10 +147,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     return;
   }
   const uint32_t sQ = smem_u32(smem);
-  const uint32_t sK = sQ + kTileBytes;       // 2 stages
-  const uint32_t sV = sK + 2 * kTileBytes;   // 2 stages
-  const uint32_t sP = sV + 2 * kTileBytes;   // 2 buffers
-  TcSmem& sm = *reinterpret_cast<TcSmem*>(smem + 7 * kTileBytes);
+  const uint32_t sK = sQ + kTileBytes;
+  const uint32_t sV = sK + kTcKStages * kTileBytes;
+  const uint32_t sP = sV + kTcVStages * kTileBytes;
+  TcSmem& sm = *reinterpret_cast<TcSmem*>(smem + (2 + kTcKStages + kTcVStages) * kTileBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (!prob.setup()) return;
@@ -154,17 +159,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kTcKStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
-      mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int s = 0; s < kTcVStages; ++s) {
+      mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.s_empty[s], 128 * kTcSplit);
-      mbar_init(&sm.p_full[s], 128 * kTcSplit);
-      mbar_init(&sm.p_empty[s], 1);
+      mbar_init(&sm.s_empty[s], 4 * kTcSplit);       // one arrival per softmax warp
       mbar_init(&sm.pv_full[s], 1);
     }
+    mbar_init(&sm.p_full, 4 * kTcSplit);
+    mbar_init(&sm.p_empty, 1);
     mbar_init(&sm.mma_done, 1);
     sm.abort_flag = 0;
     fence_barrier_init();
@@ -197,21 +206,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncwarp();
       gather_tile(sQ, &tm_q, qr, q_fallback, &sm.q_full, lane);
     }
-    stream_kv(prob, &tm_k, &tb_k, &ts_k, sK, sm.k_full, sm.k_empty, nt, n_keys, lane, abort_flag, 101);
+    stream_kv<kTcKStages>(prob, &tm_k, &tb_k, &ts_k, sK, sm.k_full, sm.k_empty, nt, n_keys, lane, abort_flag, 101);
   } else if (warp == kTcVWarp) {
     // ---------------------------------------------------------------- V loader
-    stream_kv(prob, &tm_v, &tb_v, &ts_v, sV, sm.v_full, sm.v_empty, nt, n_keys, lane, abort_flag, 102);
+    stream_kv<kTcVStages>(prob, &tm_v, &tb_v, &ts_v, sV, sm.v_full, sm.v_empty, nt, n_keys, lane, abort_flag, 102);
   } else if (warp == kTcMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc(kFmtBF16, 128, 128, 0, 0);
       constexpr uint32_t idesc_pv = umma_idesc(kFmtBF16, 128, 128, 0, 1);
       auto issue_s = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!mbar_wait(&sm.k_full[s], (j >> 1) & 1, abort_flag, 103)) return false;
+        const int s = j & 1, ks = j % kTcKStages;
+        if (!mbar_wait(&sm.k_full[ks], (j / kTcKStages) & 1, abort_flag, 103)) return false;
         if (!mbar_wait(&sm.s_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, 104)) return false;
         tc_fence_after();
-        const uint32_t kt = sK + s * kTileBytes;
+        const uint32_t kt = sK + ks * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t koff = (kk >> 2) * kBlkBytes + (kk & 3) * 32;
@@ -219,19 +228,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                       idesc_qk, kk > 0);
         }
         umma_commit(&sm.s_full[s]);
-        umma_commit(&sm.k_empty[s]);
+        umma_commit(&sm.k_empty[ks]);
         return true;
       };
       bool ok = nt == 0 || mbar_wait(&sm.q_full, 0, abort_flag, 105);
       if (ok && nt > 0) ok = issue_s(0);
       for (int j = 0; j < nt && ok; ++j) {
-        const int s = j & 1;
+        const int s = j & 1, vs = j % kTcVStages;
         if (j + 1 < nt && !(ok = issue_s(j + 1))) break;
-        if (!(ok = mbar_wait(&sm.p_full[s], (j >> 1) & 1, abort_flag, 106))) break;
-        if (!(ok = mbar_wait(&sm.v_full[s], (j >> 1) & 1, abort_flag, 107))) break;
+        if (!(ok = mbar_wait(&sm.p_full, j & 1, abort_flag, 106))) break;
+        if (!(ok = mbar_wait(&sm.v_full[vs], (j / kTcVStages) & 1, abort_flag, 107))) break;
         tc_fence_after();
-        const uint32_t pt = sP + s * kTileBytes;
-        const uint32_t vt = sV + s * kTileBytes;
+        const uint32_t pt = sP;
+        const uint32_t vt = sV + vs * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           // A = P (K-major: keys along the 128-byte rows); B = V (MN-major: 8-key row
@@ -241,8 +250,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                       idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&sm.pv_full[s]);
-        umma_commit(&sm.p_empty[s]);
-        umma_commit(&sm.v_empty[s]);
+        umma_commit(&sm.p_empty);
+        umma_commit(&sm.v_empty[vs]);
       }
       // every MMA issued so far has completed before TMEM is released
       umma_commit(&sm.mma_done);
@@ -277,7 +286,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int c = 0; c < HC / 32; ++c) tmem_ld32(lane_base + s * 128 + part * HC + c * 32, x + c * 32);
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(&sm.s_empty[s]);           // S now lives in registers
+        mbar_arrive_warp(&sm.s_empty[s]);      // S now lives in registers
         // keys t0 + e with e <= rem are visible (causal cut); masked scores become -inf
         const int64_t rem64 = lim - t0;
         const int rem = rem64 < 0 ? -1 : (rem64 >= HC ? HC : (int)rem64);
@@ -325,10 +334,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         m = m_new;
       }
       const float m_use = m == -INFINITY ? 0.f : m;
-      const bool free_p = mbar_wait_warp(&sm.p_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, 112);
+      const bool free_p = mbar_wait_warp(&sm.p_empty, (j & 1) ^ 1, abort_flag, 112);
       if (!(ok = bar_all(row_bar, kGroup, free_p))) break;
       // this part's keys: 64-key block (part * HC) / 64, first 16-byte chunk ((part * HC) % 64) / 8
-      const uint32_t pt = sP + s * kTileBytes + ((part * HC) >> 6) * kBlkBytes;
+      const uint32_t pt = sP + ((part * HC) >> 6) * kBlkBytes;
       const int ch0 = ((part * HC) & 63) >> 3;
       float ls8[8];
 #pragma unroll
@@ -351,7 +360,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       fence_proxy_async();
       tc_fence_before();
-      mbar_arrive(&sm.p_full[s]);
+      mbar_arrive_warp(&sm.p_full);
     }
     bool fin = ok;
     if (ok && nt > 0) fin = mbar_wait_warp(&sm.pv_full[(nt - 1) & 1], ((nt - 1) >> 1) & 1, abort_flag, 113);

@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
       mbar_init(&sm.q_full[i], 1);
       mbar_init(&sm.q_empty[i], 1);
       mbar_init(&sm.d_full[i], 1);
-      mbar_init(&sm.d_empty[i], 128);
+      mbar_init(&sm.d_empty[i], 4);                 // one arrival per epilogue warp
     }
     mbar_init(&sm.done, 1);
     sm.abort_flag = 0;
@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
             if (j0 + c * 32 + e < a.n_mid) mx = fmaxf(mx, x[e]);
         }
         tc_fence_before();
-        mbar_arrive(&sm.d_empty[buf]);
+        mbar_arrive_warp(&sm.d_empty[buf]);
         const int q = t * kStRows + r;
         if (q < a.lq && mx > -INFINITY) atomicMax(&a.m_key[(int64_t)b * a.lq + q], order_key(mx));
       } else {
@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
             if (c * 32 + e < qn) acc += fmaxf(x[e] - mt[c * 32 + e], lo);
         }
         tc_fence_before();
-        mbar_arrive(&sm.d_empty[buf]);
+        mbar_arrive_warp(&sm.d_empty[buf]);
       }
     }
     if (PASS == 2 && j_r < a.n_mid) a.s[(int64_t)b * a.n_mid + j_r] = acc;
