@@ -272,8 +272,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr float kRescale = 8.0f;           // log2 units: rescale when the max grows by > 2^8
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    // Every bounded wait is followed by bar_all over the row group, so all warps of a
-    // row group leave together when a wait runs out (a named barrier has no timeout).
+    // The kTcSplit warps of a row group meet once per tile at a bar.red.or: unless some
+    // part's maximum exceeds m by more than 2^8 (or a wait of some warp ran out), m stays
+    // and no exchange is needed. Otherwise they agree on success (bar_all: a named
+    // barrier has no timeout, so all warps of a group leave together), exchange the part
+    // maxima through shared memory and rescale. A failed wait is carried in `ok` to the
+    // next meeting; the warp skips the work that depended on it.
     for (int j = 0; j < nt; ++j) {
       const int s = j & 1;
       const bool got = mbar_wait_warp(&sm.s_full[s], (j >> 1) & 1, abort_flag, 111);
@@ -306,14 +310,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                    fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;   // scale > 0
       }
-      sm.red[part][r] = mx;
-      if (!(ok = bar_all(row_bar, kGroup, got))) break;
+      ok = ok && got;
+      if (bar_any(row_bar, kGroup, !ok || mx > m + kRescale)) {                   // -inf + 8 = -inf
+        if (!(ok = bar_all(row_bar, kGroup, ok))) break;
+        sm.red[part][r] = mx;
+        asm volatile("bar.sync %0, %1;" ::"r"(row_bar), "r"(kGroup) : "memory");
 #pragma unroll
-      for (int q = 0; q < kTcSplit; ++q) mx = fmaxf(mx, sm.red[q][r]);
-      asm volatile("bar.sync %0, %1;" ::"r"(row_bar), "r"(kGroup) : "memory");   // red[] is reused next
-      if (mx > m + kRescale || m == -INFINITY) {                                  // same in the whole group
-        const float m_new = fmaxf(m, mx);
-        if (j > 0 && m_new > m) {
+        for (int q = 0; q < kTcSplit; ++q) mx = fmaxf(mx, sm.red[q][r]);
+        asm volatile("bar.sync %0, %1;" ::"r"(row_bar), "r"(kGroup) : "memory");   // red[] is reused
+        const float m_new = fmaxf(m, mx);    // > m + 2^8 for the whole row group
+        if (m != -INFINITY) {
           const float alpha = fast_exp2(m - m_new);
           // O holds PV_0..PV_{j-1}; wait for the last of them, then scale this part in place
           const bool done = mbar_wait_warp(&sm.pv_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, 110);
@@ -334,30 +340,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         m = m_new;
       }
       const float m_use = m == -INFINITY ? 0.f : m;
-      const bool free_p = mbar_wait_warp(&sm.p_empty, (j & 1) ^ 1, abort_flag, 112);
-      if (!(ok = bar_all(row_bar, kGroup, free_p))) break;
+      if (!mbar_wait_warp(&sm.p_empty, (j & 1) ^ 1, abort_flag, 112)) {
+        ok = false;                            // P is still being read: write nothing
+        continue;
+      }
       // this part's keys: 64-key block (part * HC) / 64, first 16-byte chunk ((part * HC) % 64) / 8
       const uint32_t pt = sP + ((part * HC) >> 6) * kBlkBytes;
       const int ch0 = ((part * HC) & 63) >> 3;
-      float ls8[8];
+      const float2 scale2 = make_float2(sl2, sl2), shift2 = make_float2(-m_use, -m_use);
+      float2 ls2[4];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) ls8[q] = 0.f;
+      for (int q = 0; q < 4; ++q) ls2[q] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < HC / 8; ++c) {       // 16-byte chunks of this part
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 8; e += 2) {
-          // P goes to the MMA as bf16 by truncation (integer ops only); the row sum adds
-          // the same truncated values, so the normalisation matches what the MMA sees
-          const uint32_t b0 = __float_as_uint(fast_exp2(fmaf(x[c * 8 + e], sl2, -m_use))) & 0xFFFF0000u;
-          const uint32_t b1 = __float_as_uint(fast_exp2(fmaf(x[c * 8 + e + 1], sl2, -m_use))) & 0xFFFF0000u;
-          ls8[e] += __uint_as_float(b0);
-          ls8[e + 1] += __uint_as_float(b1);
-          pk[e / 2] = __byte_perm(b0, b1, 0x7632);
+          const float2 t = __ffma2_rn(make_float2(x[c * 8 + e], x[c * 8 + e + 1]), scale2, shift2);
+          const float2 pe = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+          ls2[e / 2] = __fadd2_rn(ls2[e / 2], pe);
+          // P goes to the MMA as bf16, rounded to nearest (unbiased, so l may add the
+          // unrounded values)
+          const __nv_bfloat162 h = __floats2bfloat162_rn(pe.x, pe.y);
+          pk[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
         }
         st_shared_v4(pt + sw128_off(r, ch0 + c), pk[0], pk[1], pk[2], pk[3]);
       }
-      l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
+      const float2 l2 = __fadd2_rn(__fadd2_rn(ls2[0], ls2[1]), __fadd2_rn(ls2[2], ls2[3]));
+      l += l2.x + l2.y;
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive_warp(&sm.p_full);

@@ -211,6 +211,20 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, int3
       : "memory");
 }
 
+// OR of `v` over the `count` threads that meet at named barrier `id` (bar.red).
+__device__ __forceinline__ bool bar_any(uint32_t id, uint32_t count, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
 // AND of `v` over the `count` threads that meet at named barrier `id` (bar.red): every
 // participant gets the same answer, so a group can leave a loop together.
 __device__ __forceinline__ bool bar_all(uint32_t id, uint32_t count, bool v) {
