@@ -2,8 +2,11 @@
 //
 // One CTA computes 128 query rows against a list of key rows, 128 keys per step:
 //   S_j  = Q K_j^T          tcgen05.mma kind::f16 (bf16 in, fp32 accumulate), TMEM
-//   P_j  = exp2(S_j * c - m) softmax warps read S_j from TMEM, write bf16 P_j to smem
+//   P_j  = exp2(S_j * c - m) softmax warps read S_j from TMEM, write bf16 P_j back
+//                            over the first half of S_j's columns
 //   O   += P_j V_j          tcgen05.mma accumulating in TMEM
+// P is the A operand of the second MMA and is read from TMEM (the .kind::f16 form
+// with [a_tmem]).
 // m is the running row maximum used for the exponentials; it is raised (and O, l
 // rescaled in place) only when a tile's maximum exceeds it by more than 2^8, so most
 // tiles skip the rescale and P stays <= 2^8 (exact softmax either way: o = O / l).
@@ -18,12 +21,16 @@
 // scattered keys (the selected middle tokens) is 32 tile::gather4 loads per half
 // (4 arbitrary rows each; each lane of the loader warp issues its 4 rows).
 //
-// Shared memory: Q 32 KB, K 3 x 32 KB, V 2 x 32 KB, P 32 KB (each operand tile is
-// two 16 KB column blocks of 128 rows x 128 bytes). K gets the deepest ring because
-// S_{j+1} is issued while P_j is being formed, so K tile j + 2 must already be on its
-// way; P needs one buffer: P_j is written after the row max of S_j is known, by which
-// time PV_{j-1} (the previous reader) has finished. TMEM: S double buffer (2 x 128
-// columns) and the O accumulator (128 columns).
+// Shared memory: Q 32 KB, K 3 x 32 KB, V 3 x 32 KB (each operand tile is two 16 KB
+// column blocks of 128 rows x 128 bytes). TMEM (512 columns): three S/P buffers at 0,
+// 128 and 256, the O accumulator at 384.
+// A group of MMAs that starts on an idle tensor pipe pays a fill latency of several
+// hundred cycles, so the MMA warp keeps S two tiles ahead: right after PV_j it issues
+// S_{j+3}, and the softmax warps find S_{j+1} ready when they finish P_j.
+// P_j overwrites S_j, and S_{j+3} overwrites P_j. The MMA warp issues S_{j+3} only after
+// PV_j, which it issues only after the softmax warps have signalled (p_full) that they
+// have read S_j and stored P_j; the tensor pipe executes one thread's MMAs in issue
+// order, so PV_j has read P_j before S_{j+3} is written.
 //
 // The problem policy P says which rows and keys a CTA owns:
 //   bool setup(): per-CTA fields; false = nothing to do
@@ -54,14 +61,16 @@ constexpr uint32_t kBlkBytes = 128 * 128;             // one 64-column block of 
 constexpr uint32_t kTcCtrlBytes = 3072;                       // barriers, TMEM address, row exchange
 // No alignment slack: the kernel checks that the dynamic shared memory starts on a
 // 1024-byte boundary (the 128-byte swizzle atoms need it) and stops with an error if not.
-constexpr int kTcKStages = 3, kTcVStages = 2;
-constexpr uint32_t kTcSmemBytes = (2 + kTcKStages + kTcVStages) * kTileBytes + kTcCtrlBytes;
+constexpr int kTcKStages = 3, kTcVStages = 3;
+constexpr uint32_t kTcSmemBytes = (1 + kTcKStages + kTcVStages) * kTileBytes + kTcCtrlBytes;
+constexpr int kTcSBufs = 3;                                   // S/P buffers in TMEM
+constexpr uint32_t kTmemO = 384;                              // O accumulator column
 static_assert(kTcSmemBytes <= 232448, "exceeds the 227 KB of shared memory per CTA");
 
 struct TcSmem {
   uint64_t q_full;
   uint64_t k_full[kTcKStages], k_empty[kTcKStages], v_full[kTcVStages], v_empty[kTcVStages];
-  uint64_t s_full[2], s_empty[2], p_full, p_empty;
+  uint64_t s_full[kTcSBufs], p_full[kTcSBufs];
   uint64_t pv_full[2];
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -149,8 +158,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t sQ = smem_u32(smem);
   const uint32_t sK = sQ + kTileBytes;
   const uint32_t sV = sK + kTcKStages * kTileBytes;
-  const uint32_t sP = sV + kTcVStages * kTileBytes;
-  TcSmem& sm = *reinterpret_cast<TcSmem*>(smem + (2 + kTcKStages + kTcVStages) * kTileBytes);
+  TcSmem& sm = *reinterpret_cast<TcSmem*>(smem + (1 + kTcKStages + kTcVStages) * kTileBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (!prob.setup()) return;
@@ -167,13 +175,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kTcSBufs; ++s) {
       mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.s_empty[s], 4 * kTcSplit);       // one arrival per softmax warp
-      mbar_init(&sm.pv_full[s], 1);
+      mbar_init(&sm.p_full[s], 4 * kTcSplit);        // one arrival per softmax warp
     }
-    mbar_init(&sm.p_full, 4 * kTcSplit);
-    mbar_init(&sm.p_empty, 1);
+    for (int s = 0; s < 2; ++s) mbar_init(&sm.pv_full[s], 1);
     mbar_init(&sm.mma_done, 1);
     sm.abort_flag = 0;
     fence_barrier_init();
@@ -216,9 +222,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       constexpr uint32_t idesc_qk = umma_idesc(kFmtBF16, 128, 128, 0, 0);
       constexpr uint32_t idesc_pv = umma_idesc(kFmtBF16, 128, 128, 0, 1);
       auto issue_s = [&](int j) -> bool {
-        const int s = j & 1, ks = j % kTcKStages;
+        const int s = j % kTcSBufs, ks = j % kTcKStages;
+        // buffer s last held P_{j-3}: PV_{j-3} is already issued (p_full[s] was waited for)
         if (!mbar_wait(&sm.k_full[ks], (j / kTcKStages) & 1, abort_flag, 103)) return false;
-        if (!mbar_wait(&sm.s_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, 104)) return false;
         tc_fence_after();
         const uint32_t kt = sK + ks * kTileBytes;
 #pragma unroll
@@ -232,25 +238,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         return true;
       };
       bool ok = nt == 0 || mbar_wait(&sm.q_full, 0, abort_flag, 105);
-      if (ok && nt > 0) ok = issue_s(0);
+      for (int j = 0; j < kTcSBufs - 1 && j < nt && ok; ++j) ok = issue_s(j);
       for (int j = 0; j < nt && ok; ++j) {
-        const int s = j & 1, vs = j % kTcVStages;
-        if (j + 1 < nt && !(ok = issue_s(j + 1))) break;
-        if (!(ok = mbar_wait(&sm.p_full, j & 1, abort_flag, 106))) break;
+        const int s = j % kTcSBufs, vs = j % kTcVStages;
+        if (j + kTcSBufs - 1 < nt && !(ok = issue_s(j + kTcSBufs - 1))) break;
+        if (!(ok = mbar_wait(&sm.p_full[s], (j / kTcSBufs) & 1, abort_flag, 106))) break;
         if (!(ok = mbar_wait(&sm.v_full[vs], (j / kTcVStages) & 1, abort_flag, 107))) break;
         tc_fence_after();
-        const uint32_t pt = sP;
         const uint32_t vt = sV + vs * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          // A = P (K-major: keys along the 128-byte rows); B = V (MN-major: 8-key row
-          // groups of 1024 bytes, d blocks of 64 columns 16 KB apart)
-          const uint32_t poff = (kk >> 2) * kBlkBytes + (kk & 3) * 32;
-          umma_f16_ss(tmem + 256, sdesc_sw128(pt + poff, 16, 1024), sdesc_sw128(vt + kk * 2048, kBlkBytes, 1024),
+          // A = P from TMEM (keys 16 kk .. + 15 in columns 8 kk .. + 7 of buffer s);
+          // B = V (MN-major: 8-key row groups of 1024 bytes, d blocks 16 KB apart)
+          umma_f16_ts(tmem + kTmemO, tmem + s * 128 + kk * 8, sdesc_sw128(vt + kk * 2048, kBlkBytes, 1024),
                       idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&sm.pv_full[s]);
-        umma_commit(&sm.p_empty);
+        umma_commit(&sm.pv_full[j & 1]);
         umma_commit(&sm.v_empty[vs]);
       }
       // every MMA issued so far has completed before TMEM is released
@@ -265,7 +268,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int quad = warp & 3, part = warp >> 2;
     const int r = quad * 32 + lane;            // row = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    const uint32_t o_addr = lane_base + 256 + part * HC;
+    const uint32_t o_addr = lane_base + kTmemO + part * HC;
     const uint32_t row_bar = 1 + quad;         // named barrier of the kTcSplit warps of this quadrant
     const int64_t lim = prob.limit(r);
     const float sl2 = prob.scale_log2();
@@ -279,8 +282,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // maxima through shared memory and rescale. A failed wait is carried in `ok` to the
     // next meeting; the warp skips the work that depended on it.
     for (int j = 0; j < nt; ++j) {
-      const int s = j & 1;
-      const bool got = mbar_wait_warp(&sm.s_full[s], (j >> 1) & 1, abort_flag, 111);
+      const int s = j % kTcSBufs;
+      const bool got = mbar_wait_warp(&sm.s_full[s], (j / kTcSBufs) & 1, abort_flag, 111);
       const int64_t t0 = (int64_t)j * kTcKeys + part * HC;
       float x[HC];
       float mx = -INFINITY;
@@ -288,9 +291,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < HC / 32; ++c) tmem_ld32(lane_base + s * 128 + part * HC + c * 32, x + c * 32);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive_warp(&sm.s_empty[s]);      // S now lives in registers
+        tmem_wait_ld();                        // S now lives in registers
         // keys t0 + e with e <= rem are visible (causal cut); masked scores become -inf
         const int64_t rem64 = lim - t0;
         const int rem = rem64 < 0 ? -1 : (rem64 >= HC ? HC : (int)rem64);
@@ -340,37 +341,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         m = m_new;
       }
       const float m_use = m == -INFINITY ? 0.f : m;
-      if (!mbar_wait_warp(&sm.p_empty, (j & 1) ^ 1, abort_flag, 112)) {
-        ok = false;                            // P is still being read: write nothing
-        continue;
-      }
-      // this part's keys: 64-key block (part * HC) / 64, first 16-byte chunk ((part * HC) % 64) / 8
-      const uint32_t pt = sP + ((part * HC) >> 6) * kBlkBytes;
-      const int ch0 = ((part * HC) & 63) >> 3;
+      // P_j over S_j: every warp of the row group has read its part of S_j (the
+      // barrier above), so the packed P of keys 32 part .. + 31 may go to columns
+      // 16 part .. + 15 of the buffer
       const float2 scale2 = make_float2(sl2, sl2), shift2 = make_float2(-m_use, -m_use);
       float2 ls2[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) ls2[q] = make_float2(0.f, 0.f);
+      uint32_t pk[HC / 2];
 #pragma unroll
-      for (int c = 0; c < HC / 8; ++c) {       // 16-byte chunks of this part
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          const float2 t = __ffma2_rn(make_float2(x[c * 8 + e], x[c * 8 + e + 1]), scale2, shift2);
-          const float2 pe = make_float2(fast_exp2(t.x), fast_exp2(t.y));
-          ls2[e / 2] = __fadd2_rn(ls2[e / 2], pe);
-          // P goes to the MMA as bf16, rounded to nearest (unbiased, so l may add the
-          // unrounded values)
-          const __nv_bfloat162 h = __floats2bfloat162_rn(pe.x, pe.y);
-          pk[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
-        }
-        st_shared_v4(pt + sw128_off(r, ch0 + c), pk[0], pk[1], pk[2], pk[3]);
+      for (int e = 0; e < HC; e += 2) {
+        const float2 t = __ffma2_rn(make_float2(x[e], x[e + 1]), scale2, shift2);
+        const float2 pe = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+        ls2[(e / 2) & 3] = __fadd2_rn(ls2[(e / 2) & 3], pe);
+        // P goes to the MMA as bf16, rounded to nearest (unbiased, so l may add the
+        // unrounded values)
+        const __nv_bfloat162 h = __floats2bfloat162_rn(pe.x, pe.y);
+        pk[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
       }
+      static_assert(HC == 32, "one 16-column TMEM store per thread");
+      tmem_st16(lane_base + s * 128 + part * 16, pk);
       const float2 l2 = __fadd2_rn(__fadd2_rn(ls2[0], ls2[1]), __fadd2_rn(ls2[2], ls2[3]));
       l += l2.x + l2.y;
-      fence_proxy_async();
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive_warp(&sm.p_full);
+      mbar_arrive_warp(&sm.p_full[s]);
     }
     bool fin = ok;
     if (ok && nt > 0) fin = mbar_wait_warp(&sm.pv_full[(nt - 1) & 1], ((nt - 1) >> 1) & 1, abort_flag, 113);
