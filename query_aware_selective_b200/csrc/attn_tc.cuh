@@ -221,17 +221,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc(kFmtBF16, 128, 128, 0, 0);
       constexpr uint32_t idesc_pv = umma_idesc(kFmtBF16, 128, 128, 0, 1);
+      // This thread shares its issue slots with four busy softmax warps, so the loops
+      // below do as little as possible per MMA: descriptors are built once and only the
+      // low word moves (16-byte units: K step kk of a K-major operand is +2 kk within a
+      // 64-column block and +1024 per block; of the MN-major V tile, +128 kk).
+      const uint64_t dq = sdesc_sw128(sQ, 16, 1024), dk = sdesc_sw128(sK, 16, 1024);
+      const uint64_t dv = sdesc_sw128(sV, kBlkBytes, 1024);
+      const uint32_t q_lo = (uint32_t)dq, q_hi = (uint32_t)(dq >> 32);
+      const uint32_t k_lo = (uint32_t)dk, k_hi = (uint32_t)(dk >> 32);
+      const uint32_t v_lo = (uint32_t)dv, v_hi = (uint32_t)(dv >> 32);
       auto issue_s = [&](int j) -> bool {
         const int s = j % kTcSBufs, ks = j % kTcKStages;
         // buffer s last held P_{j-3}: PV_{j-3} is already issued (p_full[s] was waited for)
         if (!mbar_wait(&sm.k_full[ks], (j / kTcKStages) & 1, abort_flag, 103)) return false;
         tc_fence_after();
-        const uint32_t kt = sK + ks * kTileBytes;
+        const uint32_t kb = k_lo + ks * (kTileBytes >> 4), d = tmem + s * 128;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (kk >> 2) * kBlkBytes + (kk & 3) * 32;
-          umma_f16_ss(tmem + s * 128, sdesc_sw128(sQ + koff, 16, 1024), sdesc_sw128(kt + koff, 16, 1024),
-                      idesc_qk, kk > 0);
+          const uint32_t off = (kk >> 2) * (kBlkBytes >> 4) + (kk & 3) * 2;
+          umma_f16_ss2(d, q_lo + off, q_hi, kb + off, k_hi, idesc_qk, kk > 0);
         }
         umma_commit(&sm.s_full[s]);
         umma_commit(&sm.k_empty[ks]);
@@ -245,13 +253,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!(ok = mbar_wait(&sm.p_full[s], (j / kTcSBufs) & 1, abort_flag, 106))) break;
         if (!(ok = mbar_wait(&sm.v_full[vs], (j / kTcVStages) & 1, abort_flag, 107))) break;
         tc_fence_after();
-        const uint32_t vt = sV + vs * kTileBytes;
+        const uint32_t vb = v_lo + vs * (kTileBytes >> 4), pa = tmem + s * 128;
+        const uint32_t acc0 = j > 0;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           // A = P from TMEM (keys 16 kk .. + 15 in columns 8 kk .. + 7 of buffer s);
           // B = V (MN-major: 8-key row groups of 1024 bytes, d blocks 16 KB apart)
-          umma_f16_ts(tmem + kTmemO, tmem + s * 128 + kk * 8, sdesc_sw128(vt + kk * 2048, kBlkBytes, 1024),
-                      idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_f16_ts2(tmem + kTmemO, pa + kk * 8, vb + kk * 128, v_hi, idesc_pv, kk > 0 ? 1u : acc0);
         }
         umma_commit(&sm.pv_full[j & 1]);
         umma_commit(&sm.v_empty[vs]);
@@ -264,6 +272,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else {
     // ---------------------------------------------------------------- softmax (rows)
     constexpr int HC = kTcKeys / kTcSplit;     // key columns per thread
+    static_assert(HC == 32, "one 32-column TMEM load and two 8-column stores per thread and tile");
     constexpr uint32_t kGroup = 32 * kTcSplit; // threads sharing a row set (named barrier size)
     const int quad = warp & 3, part = warp >> 2;
     const int r = quad * 32 + lane;            // row = TMEM lane
@@ -275,97 +284,147 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr float kRescale = 8.0f;           // log2 units: rescale when the max grows by > 2^8
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+
+    // Keys t0 + e of tile j with e <= rem are visible (causal cut); rem >= HC - 1: all.
+    auto rem_of = [&](int j) -> int {
+      const int64_t rem64 = lim - ((int64_t)j * kTcKeys + part * HC);
+      return rem64 < 0 ? -1 : (rem64 >= HC ? HC : (int)rem64);
+    };
+    // Wait for S_j; then load_s starts loading this thread's scores (complete at
+    // tmem_wait_ld).
+    auto wait_s = [&](int j) -> bool {
+      const bool got = mbar_wait_warp(&sm.s_full[j % kTcSBufs], (j / kTcSBufs) & 1, abort_flag, 111);
+      if (got) tc_fence_after();
+      return got;
+    };
+    auto load_s = [&](int j, float* dst) { tmem_ld32(lane_base + (j % kTcSBufs) * 128 + part * HC, dst); };
+    // Masked scores become -inf; returns this part's maximum in log2 units (scale > 0).
+    auto mask_max = [&](int rem, float* v) -> float {
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (rem >= HC - 1) {
+#pragma unroll
+        for (int e = 0; e < HC; ++e) m4[e & 3] = fmaxf(m4[e & 3], v[e]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < HC; ++e) {
+          v[e] = e <= rem ? v[e] : -INFINITY;
+          m4[e & 3] = fmaxf(m4[e & 3], v[e]);
+        }
+      }
+      return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+    };
     // The kTcSplit warps of a row group meet once per tile at a bar.red.or: unless some
     // part's maximum exceeds m by more than 2^8 (or a wait of some warp ran out), m stays
     // and no exchange is needed. Otherwise they agree on success (bar_all: a named
     // barrier has no timeout, so all warps of a group leave together), exchange the part
-    // maxima through shared memory and rescale. A failed wait is carried in `ok` to the
-    // next meeting; the warp skips the work that depended on it.
-    for (int j = 0; j < nt; ++j) {
-      const int s = j % kTcSBufs;
-      const bool got = mbar_wait_warp(&sm.s_full[s], (j / kTcSBufs) & 1, abort_flag, 111);
-      const int64_t t0 = (int64_t)j * kTcKeys + part * HC;
-      float x[HC];
-      float mx = -INFINITY;
-      if (got) {
+    // maxima through shared memory, and rescale O (which then holds PV_0 .. PV_{j-1})
+    // and l. Returns false when the group has to stop.
+    auto decide = [&](int j, float mx) -> bool {
+      if (!bar_any(row_bar, kGroup, !ok || mx > m + kRescale)) return true;   // -inf + 8 = -inf
+      if (!(ok = bar_all(row_bar, kGroup, ok))) return false;
+      sm.red[part][r] = mx;
+      asm volatile("bar.sync %0, %1;" ::"r"(row_bar), "r"(kGroup) : "memory");
+#pragma unroll
+      for (int q = 0; q < kTcSplit; ++q) mx = fmaxf(mx, sm.red[q][r]);
+      asm volatile("bar.sync %0, %1;" ::"r"(row_bar), "r"(kGroup) : "memory");   // red[] is reused
+      const float m_new = fmaxf(m, mx);        // > m + 2^8 for the whole row group
+      if (m != -INFINITY) {
+        const float alpha = fast_exp2(m - m_new);
+        const bool done = mbar_wait_warp(&sm.pv_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, 110);
+        if (!(ok = bar_all(row_bar, kGroup, done))) return false;
         tc_fence_after();
+        float ov[32];
+        tmem_ld32(o_addr, ov);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < HC / 32; ++c) tmem_ld32(lane_base + s * 128 + part * HC + c * 32, x + c * 32);
-        tmem_wait_ld();                        // S now lives in registers
-        // keys t0 + e with e <= rem are visible (causal cut); masked scores become -inf
-        const int64_t rem64 = lim - t0;
-        const int rem = rem64 < 0 ? -1 : (rem64 >= HC ? HC : (int)rem64);
-        float mx8[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) mx8[q] = -INFINITY;
-        if (rem >= HC - 1) {                   // the whole part is visible: no mask
-#pragma unroll
-          for (int e = 0; e < HC; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], x[e]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < HC; ++e) {
-            x[e] = e <= rem ? x[e] : -INFINITY;
-            mx8[e & 7] = fmaxf(mx8[e & 7], x[e]);
-          }
-        }
-        mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;   // scale > 0
+        for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+        tmem_st32(o_addr, ov);
+        tmem_wait_st();
+        l *= alpha;
       }
-      ok = ok && got;
-      if (bar_any(row_bar, kGroup, !ok || mx > m + kRescale)) {                   // -inf + 8 = -inf
-        if (!(ok = bar_all(row_bar, kGroup, ok))) break;
-        sm.red[part][r] = mx;
-        asm volatile("bar.sync %0, %1;" ::"r"(row_bar), "r"(kGroup) : "memory");
-#pragma unroll
-        for (int q = 0; q < kTcSplit; ++q) mx = fmaxf(mx, sm.red[q][r]);
-        asm volatile("bar.sync %0, %1;" ::"r"(row_bar), "r"(kGroup) : "memory");   // red[] is reused
-        const float m_new = fmaxf(m, mx);    // > m + 2^8 for the whole row group
-        if (m != -INFINITY) {
-          const float alpha = fast_exp2(m - m_new);
-          // O holds PV_0..PV_{j-1}; wait for the last of them, then scale this part in place
-          const bool done = mbar_wait_warp(&sm.pv_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, 110);
-          if (!(ok = bar_all(row_bar, kGroup, done))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < HC / 32; ++c) {
-            float ov[32];
-            tmem_ld32(o_addr + c * 32, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-            tmem_st32(o_addr + c * 32, ov);
-          }
-          tmem_wait_st();
-          l *= alpha;
-        }
-        m = m_new;
-      }
+      m = m_new;
+      return true;
+    };
+    // One tile, software-pipelined: cur holds S_j (masked, m decided). P_j is formed in
+    // two halves (MUFU exp2); S_{j+1} is loaded into nxt after the first half (when half
+    // of cur is no longer needed, which keeps the live registers within the 96 a thread
+    // has here), and its maximum is taken between the exponentials of the second half,
+    // so the ALU reduction hides behind the exp2 unit. P_j goes to
+    // the TMEM buffer over S_j (every warp of the row group has read its part of S_j,
+    // the barrier in decide), keys 32 part .. + 31 to columns 16 part .. + 15. Then the
+    // group decides m for tile j + 1. Returns false when there is no next tile or the
+    // group has to stop.
+    auto step = [&](int j, float* cur, float* nxt) -> bool {
+      const int s = j % kTcSBufs;
+      const bool has_next = j + 1 < nt;
+      const bool got_n = has_next && wait_s(j + 1);
+      const int rem_n = has_next ? rem_of(j + 1) : HC;
       const float m_use = m == -INFINITY ? 0.f : m;
-      // P_j over S_j: every warp of the row group has read its part of S_j (the
-      // barrier above), so the packed P of keys 32 part .. + 31 may go to columns
-      // 16 part .. + 15 of the buffer
       const float2 scale2 = make_float2(sl2, sl2), shift2 = make_float2(-m_use, -m_use);
-      float2 ls2[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) ls2[q] = make_float2(0.f, 0.f);
-      uint32_t pk[HC / 2];
-#pragma unroll
-      for (int e = 0; e < HC; e += 2) {
-        const float2 t = __ffma2_rn(make_float2(x[e], x[e + 1]), scale2, shift2);
+      float2 ls2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      uint32_t pk[8];
+      // P goes to the MMA as bf16, rounded to nearest (unbiased, so l may add the
+      // unrounded values)
+      auto pair = [&](int e) -> uint32_t {
+        const float2 t = __ffma2_rn(make_float2(cur[e], cur[e + 1]), scale2, shift2);
         const float2 pe = make_float2(fast_exp2(t.x), fast_exp2(t.y));
-        ls2[(e / 2) & 3] = __fadd2_rn(ls2[(e / 2) & 3], pe);
-        // P goes to the MMA as bf16, rounded to nearest (unbiased, so l may add the
-        // unrounded values)
+        ls2[(e >> 1) & 1] = __fadd2_rn(ls2[(e >> 1) & 1], pe);
         const __nv_bfloat162 h = __floats2bfloat162_rn(pe.x, pe.y);
-        pk[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
+        return *reinterpret_cast<const uint32_t*>(&h);
+      };
+#pragma unroll
+      for (int e = 0; e < HC / 2; e += 2) pk[e / 2] = pair(e);
+      tmem_st8(lane_base + s * 128 + part * 16, pk);
+      float mx_n = -INFINITY;
+      if (got_n) {
+        load_s(j + 1, nxt);
+        tmem_wait_ld();
       }
-      static_assert(HC == 32, "one 16-column TMEM store per thread");
-      tmem_st16(lane_base + s * 128 + part * 16, pk);
-      const float2 l2 = __fadd2_rn(__fadd2_rn(ls2[0], ls2[1]), __fadd2_rn(ls2[2], ls2[3]));
+      if (__all_sync(0xffffffffu, got_n && rem_n >= HC - 1)) {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int e = HC / 2; e < HC; e += 2) {
+          pk[(e - HC / 2) / 2] = pair(e);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int f = (e - HC / 2) * 2 + q;             // 4 of S_{j+1} per pair of P_j
+            m4[q] = fmaxf(m4[q], nxt[f]);
+          }
+        }
+        mx_n = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+      } else {
+#pragma unroll
+        for (int e = HC / 2; e < HC; e += 2) pk[(e - HC / 2) / 2] = pair(e);
+        if (got_n) mx_n = mask_max(rem_n, nxt);
+      }
+      tmem_st8(lane_base + s * 128 + part * 16 + 8, pk);
+      const float2 l2 = __fadd2_rn(ls2[0], ls2[1]);
       l += l2.x + l2.y;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(&sm.p_full[s]);
+      if (!has_next) return false;
+      ok = ok && got_n;
+      return decide(j + 1, mx_n);
+    };
+
+    float xa[HC], xb[HC];
+    if (nt > 0) {
+      const bool got = wait_s(0);
+      float mx = -INFINITY;
+      if (got) {
+        load_s(0, xa);
+        tmem_wait_ld();
+        mx = mask_max(rem_of(0), xa);
+      }
+      ok = ok && got;
+      if (decide(0, mx)) {
+        for (int j = 0; j < nt; ++j) {
+          if (!step(j, xa, xb)) break;
+#pragma unroll
+          for (int e = 0; e < HC; ++e) xa[e] = xb[e];
+        }
+      }
     }
     bool fin = ok;
     if (ok && nt > 0) fin = mbar_wait_warp(&sm.pv_full[(nt - 1) & 1], ((nt - 1) >> 1) & 1, abort_flag, 113);
@@ -378,13 +437,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (ok) {
       tc_fence_after();
       float o[HC];
-#pragma unroll
-      for (int c = 0; c < HC / 32; ++c) tmem_ld32(o_addr + c * 32, o + c * 32);
+      tmem_ld32(o_addr, o);
       tmem_wait_ld();
       prob.store(r, part * HC, o, m, l_row);
     }
   }
-
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
