@@ -48,6 +48,10 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--prefill-ctx", type=int, default=0,
                     help="shorter prefill context (profiling a small case); the line then names that workload")
+    ap.add_argument("--only", choices=["decode", "moba"], default=None,
+                    help="profiling: run one of the other workloads alone and print its figures")
+    ap.add_argument("--decode-batch", type=int, default=0, help="profiling: decode batch (default: the workload's)")
+    ap.add_argument("--moba-seq", type=int, default=0, help="profiling: MoBA sequence length (default: the workload's)")
     return ap.parse_args()
 
 
@@ -182,6 +186,22 @@ def make_dist_max():
 
 # ----------------------------------------------------------------------------- our arm
 
+def run_only(args):
+    """Profiling helper: one of the secondary workloads alone (optionally smaller), on
+    one GPU, printing its figures as one JSON line."""
+    import torch
+    import query_aware_selective_b200 as qas
+    torch.cuda.set_device(0)
+    qas.load()
+    dev = torch.device("cuda", 0)
+    peaks, peak_src = load_peaks()
+    flush_buf = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    flush = lambda: flush_buf.zero_()
+    fn = bench_decode if args.only == "decode" else bench_moba
+    out = fn(args, dev, flush, make_dist_max(), peaks, peak_src, 1)
+    print(json.dumps({"only": args.only, **out}), flush=True)
+
+
 def run_ours(args):
     import torch
     import query_aware_selective_b200 as qas
@@ -299,6 +319,9 @@ def bench_decode(args, dev, flush, dist_max, peaks, peak_src, world):
     import query_aware_selective_b200 as qas
     from query_aware_selective_b200 import cost, pipeline, synthetic
     w = synthetic.DECODE_128K
+    if args.decode_batch:
+        import dataclasses
+        w = dataclasses.replace(w, batch=args.decode_batch, name=f"esa_decode_llama3_8b_b{args.decode_batch}_ctx{w.n_ctx}")
     p = qas.params(w.n_init, w.window, w.topk, w.eps, w.clamp_c)
     inp = synthetic.make_esa_inputs(w, device=dev)
     dec = pipeline.EsaDecode(w.batch, w.n_ctx, w.hq, w.hkv, w.head_dim, w.d_c, p, device=dev)
@@ -339,6 +362,9 @@ def bench_moba(args, dev, flush, dist_max, peaks, peak_src, world):
     import torch
     from query_aware_selective_b200 import cost, pipeline, synthetic
     w = synthetic.MOBA_64K
+    if args.moba_seq:
+        import dataclasses
+        w = dataclasses.replace(w, seq=args.moba_seq, name=f"moba_prefill_h{w.heads}_seq{args.moba_seq}_block{w.block}_top{w.topk}")
     inp = synthetic.make_moba_inputs(w, device=dev)
     mb = pipeline.MobaPrefill(w.batch, w.seq, w.heads, w.head_dim, w.block, w.topk, device=dev)
     step = lambda: mb.run(inp["q"], inp["k"], inp["v"])
@@ -447,6 +473,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.only:
+        run_only(args)
     else:
         run_ours(args)
 
