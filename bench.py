@@ -139,9 +139,11 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- timing
 
-def time_steps(fn, steps, warmup, flush, dist_max):
+def time_steps(fn, steps, warmup, flush, dist_max, after_step=None):
     """Warm up, then time each of `steps` calls with CUDA events (L2 flushed between
-    steps, outside the events). Returns per-step ms (after max over ranks)."""
+    steps, outside the events). after_step, if given, runs after each step once the
+    device is idle (outside the events; it reads timing events of the step). Returns
+    per-step ms and their sum (the sum after max over ranks)."""
     import torch
     for _ in range(warmup):
         fn()
@@ -156,6 +158,9 @@ def time_steps(fn, steps, warmup, flush, dist_max):
         fn()
         b.record()
         evs.append((a, b))
+        if after_step is not None:
+            torch.cuda.synchronize()
+            after_step()
     torch.cuda.synchronize()
     dist_barrier()
     torch.cuda.synchronize()
@@ -237,25 +242,30 @@ def run_ours(args):
     p = qas.params(w.n_init, w.window, w.topk, w.eps, w.clamp_c)
     inp = synthetic.make_esa_inputs(w, device=dev)
     pf = pipeline.EsaPrefill(w.batch, w.n_ctx, w.chunk, w.hq, w.hkv, w.head_dim, w.d_c, p, device=dev)
+    # The whole step (weight packing + every chunk) is one CUDA graph; the attention
+    # launches carry external timing events, read after each replay.
     attn_events = []
-    state = {"collect": False}
 
-    def prefill_step():
-        ev = attn_events if state["collect"] else None
-        pf.run(inp["q"], inp["k"], inp["v"], inp["wq"], inp["wk"], attn_events=ev)
+    def prefill_run(ev=None):
+        pf.run(inp["q"], inp["k"], inp["v"], inp["wq"], inp["wk"], attn_events=ev, external_events=True)
 
-    for _ in range(args.warmup):
-        prefill_step()
-    torch.cuda.synchronize()
-    state["collect"] = True
     launches0 = qas._abi.launch_count()
-    ms, total_ms = time_steps(prefill_step, args.steps, 0, flush, dist_max)
-    launches = qas._abi.launch_count() - launches0
-    state["collect"] = False
+    prefill_run()
+    torch.cuda.synchronize()
+    launches_per_step = qas._abi.launch_count() - launches0
+
+    def capture_body():
+        attn_events.clear()
+        prefill_run(attn_events)
+
+    graph = pipeline.graph_of(capture_body)
+    attn_ms = []
+    ms, total_ms = time_steps(graph.replay, args.steps, args.warmup, flush, dist_max,
+                              after_step=lambda: attn_ms.extend(a.elapsed_time(b) for a, b in attn_events))
+    launches = launches_per_step * args.steps
     tokens = w.batch * w.n_ctx
     value = world * tokens * args.steps / (total_ms / 1e3)
     fl = cost.prefill_flops(w.n_ctx, w.chunk, w.hq, w.head_dim, w.d_c, w.n_init, w.window, w.topk)
-    attn_ms = [a.elapsed_time(b) for a, b in attn_events]
     n_attn = len(attn_ms)
     attn_time_s = sum(attn_ms) / 1e3
     achieved = fl["attention"] * args.steps / attn_time_s / 1e12
@@ -271,20 +281,20 @@ def run_ours(args):
     # ---------------------------------------------------------------- e2e through host buffers
     host = {n: inp[n].cpu().pin_memory() for n in ("q", "k", "v")}
     out_host = torch.empty(pf.out.shape, dtype=pf.out.dtype).pin_memory()
-    dbuf = {n: torch.empty_like(inp[n]) for n in ("q", "k", "v")}
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_host.numel() * out_host.element_size()
 
     def e2e_step():
+        # the graph reads the input buffers it was captured on: copy the host inputs there
         for n in ("q", "k", "v"):
-            dbuf[n].copy_(host[n], non_blocking=True)
-        o = pf.run(dbuf["q"], dbuf["k"], dbuf["v"], inp["wq"], inp["wk"])
-        out_host.copy_(o, non_blocking=True)
+            inp[n].copy_(host[n], non_blocking=True)
+        graph.replay()
+        out_host.copy_(pf.out, non_blocking=True)
 
     e_ms, e_total = time_steps(e2e_step, args.e2e_steps, 1, flush, dist_max)
     e2e = {"value": round(world * tokens * args.e2e_steps / (e_total / 1e3), 1), "unit": "tok/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    del host, out_host, dbuf
+    del host, out_host
 
     line = {"metric": METRIC, "value": round(value, 1), "unit": "tok/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 3), "higher_is_better": True,
@@ -294,12 +304,13 @@ def run_ours(args):
                        "hkv": w.hkv, "head_dim": w.head_dim, "d_c": w.d_c, "n_init": w.n_init,
                        "window": w.window, "topk": w.topk, "eps": w.eps, "clamp_c": w.clamp_c,
                        "parallelism": f"replicas x{world}", "l2": "flushed between timed steps (256 MB write)",
+                       "execution": "one CUDA graph per step (weight packing and all 64 chunks)",
                        "precision": "bf16 attention (fp32 accumulate), fp32 selection"},
             "roofline": roofline, "e2e": e2e, "gpu_launches": launches}
 
     # ---------------------------------------------------------------- also: decode, MoBA
     if not args.no_extras:
-        del inp, pf
+        del inp, pf, graph
         torch.cuda.empty_cache()
         line["also"] = {"esa_decode_128k": bench_decode(args, dev, flush, dist_max, peaks, peak_src, world),
                         "moba_prefill_64k": bench_moba(args, dev, flush, dist_max, peaks, peak_src, world)}
@@ -327,30 +338,21 @@ def bench_decode(args, dev, flush, dist_max, peaks, peak_src, world):
     dec = pipeline.EsaDecode(w.batch, w.n_ctx, w.hq, w.hkv, w.head_dim, w.d_c, p, device=dev)
     dec.fill_cache(inp["k"], inp["wk"])
     torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+    graph = pipeline.graph_of(lambda: dec.step(inp["q"], inp["k"], inp["v"], inp["wq"], inp["wk"], phase_events=ev))
     phases = []
-    state = {"collect": False}
-
-    def step():
-        ev = None
-        if state["collect"]:
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-            phases.append(ev)
-        dec.step(inp["q"], inp["k"], inp["v"], inp["wq"], inp["wk"], phase_events=ev)
-
-    for _ in range(args.warmup):
-        step()
-    state["collect"] = True
     steps = max(args.steps, 20)
-    ms, total = time_steps(step, steps, 0, flush, dist_max)
+    ms, total = time_steps(graph.replay, steps, args.warmup, flush, dist_max,
+                           after_step=lambda: phases.append((ev[1].elapsed_time(ev[2]), ev[2].elapsed_time(ev[3]))))
     by = cost.decode_bytes(w.batch, w.n_ctx, w.hq, w.hkv, w.head_dim, w.d_c, w.n_init, w.window, w.topk)
-    sel_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in phases)
-    att_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in phases)
+    sel_ms = statistics.mean(e[0] for e in phases)
+    att_ms = statistics.mean(e[1] for e in phases)
     hbm = peaks["hbm_gbs"]
     step_gbs = by["total"] / (total / steps / 1e3) / 1e9
     sel_gbs = (by["compressed_keys"]) / (sel_ms / 1e3) / 1e9
     att_gbs = (by["kv_rows"]) / (att_ms / 1e3) / 1e9
     return {"workload": w.name, "value": round(world * w.batch * steps / (total / 1e3), 1), "unit": "tok/s",
-            "ms_per_step": round(total / steps, 4), "steps": steps,
+            "ms_per_step": round(total / steps, 4), "steps": steps, "execution": "one CUDA graph per step",
             "roofline": {"bound": "hbm", "achieved": round(step_gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(step_gbs / hbm, 4), "bytes_per_step": by["total"],
                          "peak_source": f"{peak_src} HBM copy"},
@@ -367,14 +369,15 @@ def bench_moba(args, dev, flush, dist_max, peaks, peak_src, world):
         w = dataclasses.replace(w, seq=args.moba_seq, name=f"moba_prefill_h{w.heads}_seq{args.moba_seq}_block{w.block}_top{w.topk}")
     inp = synthetic.make_moba_inputs(w, device=dev)
     mb = pipeline.MobaPrefill(w.batch, w.seq, w.heads, w.head_dim, w.block, w.topk, device=dev)
-    step = lambda: mb.run(inp["q"], inp["k"], inp["v"])
+    graph = pipeline.graph_of(lambda: mb.run(inp["q"], inp["k"], inp["v"]))
     steps = max(3, args.steps // 2)
-    ms, total = time_steps(step, steps, args.warmup, flush, dist_max)
+    ms, total = time_steps(graph.replay, steps, args.warmup, flush, dist_max)
     fl = cost.moba_flops(w.seq, w.heads, w.head_dim, w.block, w.topk)
     ach = fl["total"] / (total / steps / 1e3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     return {"workload": w.name, "value": round(world * w.batch * w.seq * steps / (total / 1e3), 1),
             "unit": "tok/s", "ms_per_step": round(total / steps, 3), "steps": steps,
+            "execution": "one CUDA graph per step",
             "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(ach / peak, 4), "flops_per_step": fl["total"],
                          "peak_source": f"{peak_src} bf16 sustained"}}

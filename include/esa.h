@@ -94,6 +94,34 @@ esa_status_t esa_compress(const void* x, esa_dtype_t x_dtype, int64_t rows, int6
                           const float* w, int32_t d_out, float* y, int64_t y_row_stride,
                           void* stream);
 
+/* esa_compress_pack_size / esa_compress_pack / esa_compress_packed - the same map
+ * with the weight prepared once for the tensor cores. The weight is static across
+ * calls (it is the compression layer), so folding the GQA rows and splitting fp32
+ * into bf16 high + low parts (|w - hi - lo| <= 2^-17 |w|; both halves are multiplied,
+ * so the product keeps fp32-level accuracy) is done by esa_compress_pack, and every
+ * later esa_compress_packed call only streams x and the packed weight.
+ *   esa_compress_pack_size: bytes of the packed weight for a reduction length
+ *       K = n_heads_in * head_dim and d_out; 0 if the packed path does not support the
+ *       shape (it needs d_out == 128 and K a multiple of 512).
+ *   esa_compress_pack: w as for esa_compress ([n_heads_out * head_dim, d_out] fp32,
+ *       n_heads_out a multiple of n_heads_in) -> packed (device, caller-owned,
+ *       packed_bytes >= esa_compress_pack_size, 16-byte aligned). The packed layout is
+ *       the library's own; it is only valid as input to esa_compress_packed with the
+ *       same n_heads_in, head_dim and d_out.
+ *   esa_compress_packed: y = the map of x (bf16 rows of [n_heads_in, head_dim], row r at
+ *       x + r * x_row_stride, x_row_stride a multiple of 8, base 16-byte aligned) with
+ *       the packed weight; y as for esa_compress (fp32, y_row_stride >= 128, base and
+ *       y_row_stride giving 16-byte aligned rows). rows >= 0 (0 = no-op).
+ * Results equal esa_compress's up to fp32 summation order (both split the weight the
+ * same way and accumulate in fp32). Errors: ESA_ERR_UNSUPPORTED for shapes the packed
+ * path does not take, ESA_ERR_INVALID_ARG for null, misaligned or short buffers. */
+size_t esa_compress_pack_size(int32_t n_heads_in, int32_t head_dim, int32_t d_out);
+esa_status_t esa_compress_pack(const float* w, int32_t n_heads_in, int32_t n_heads_out, int32_t head_dim,
+                               int32_t d_out, void* packed, size_t packed_bytes, void* stream);
+esa_status_t esa_compress_packed(const void* x, int64_t rows, int64_t x_row_stride, int32_t n_heads_in,
+                                 int32_t head_dim, const void* packed, int32_t d_out, float* y,
+                                 int64_t y_row_stride, void* stream);
+
 /* esa_score_select - importance score, correction, chunk sum, neighbour max-pool and
  * top-k for one chunk of every sequence in a batch (ESA write-up, implementation,
  * score-correction and neighbour-influence paragraphs).

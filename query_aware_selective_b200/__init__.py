@@ -5,8 +5,9 @@ this package only marshals torch tensors into it. ``synthetic`` draws the seeded
 benchmark inputs; ``cost`` holds the algorithmic byte and flop counts used for
 rooflines.
 """
-from ._abi import (EsaError, EsaParams, compress, device_status, load, moba_block_attn, moba_block_gate,
-                   moba_block_gate_attn, params, score_select, sparse_attn)
+from ._abi import (EsaError, EsaParams, compress, compress_pack, compress_pack_size, compress_packed, device_status,
+                   load, moba_block_attn, moba_block_gate, moba_block_gate_attn, params, score_select, sparse_attn)
 
-__all__ = ["EsaError", "EsaParams", "compress", "device_status", "load", "moba_block_attn", "moba_block_gate",
-           "moba_block_gate_attn", "params", "score_select", "sparse_attn"]
+__all__ = ["EsaError", "EsaParams", "compress", "compress_pack", "compress_pack_size", "compress_packed",
+           "device_status", "load", "moba_block_attn", "moba_block_gate", "moba_block_gate_attn", "params",
+           "score_select", "sparse_attn"]

@@ -33,6 +33,9 @@ class EsaParams(ctypes.Structure):
 
 SIGNATURES = {
     "esa_compress": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i32, _i32, _i32, _vp, _i32, _vp, _i64, _vp]),
+    "esa_compress_pack_size": (_sz, [_i32, _i32, _i32]),
+    "esa_compress_pack": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, _sz, _vp]),
+    "esa_compress_packed": (ctypes.c_int, [_vp, _i64, _i64, _i32, _i32, _vp, _i32, _vp, _i64, _vp]),
     "esa_score_select": (ctypes.c_int, [_vp, _vp, _i32, _i32, _i64, _i64, _i32, EsaParams, _vp, _vp, _vp,
                                         _vp, _sz, _vp]),
     "esa_score_select_workspace_size": (_sz, [_i32, _i32, _i64, _i64, _i32, EsaParams]),
@@ -149,6 +152,48 @@ def compress(x: torch.Tensor, w: torch.Tensor, n_heads_out: int, out: Optional[t
         stride = out_row_stride or dout
     _check(load().esa_compress(_ptr(x), _dtype_code(x), rows, x.stride(0) if rows > 1 else hin * d, hin,
                                n_heads_out, d, _ptr(w), dout, _ptr(out), stride, _stream()), "esa_compress")
+    return out
+
+
+def compress_pack_size(n_heads_in: int, head_dim: int, d_out: int) -> int:
+    """esa_compress_pack_size: bytes of the packed weight, 0 if the packed path does
+    not take the shape."""
+    return load().esa_compress_pack_size(n_heads_in, head_dim, d_out)
+
+
+def compress_pack(w: torch.Tensor, n_heads_in: int, n_heads_out: int, head_dim: int,
+                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """esa_compress_pack: w [Hout*D, d'] f32 -> packed weight (uint8 device tensor)."""
+    if not w.is_cuda or not w.is_contiguous():
+        raise ValueError("libesa takes contiguous CUDA tensors (no CPU path)")
+    dout = w.shape[1]
+    n = compress_pack_size(n_heads_in, head_dim, dout)
+    if n == 0:
+        raise EsaError(ESA_ERR_UNSUPPORTED, "esa_compress_pack", "shape not supported by the packed path")
+    if out is None:
+        out = torch.empty(n, dtype=torch.uint8, device=w.device)
+    _check(load().esa_compress_pack(_ptr(w), n_heads_in, n_heads_out, head_dim, dout, _ptr(out),
+                                    out.numel() * out.element_size(), _stream()), "esa_compress_pack")
+    return out
+
+
+def compress_packed(x: torch.Tensor, packed: torch.Tensor, d_out: int = 128, out: Optional[torch.Tensor] = None,
+                    out_row_stride: Optional[int] = None) -> torch.Tensor:
+    """esa_compress_packed. x: [rows, Hin, D] bf16 (each row contiguous, rows may be
+    strided); packed from compress_pack -> [rows, d_out] f32 (or written into `out`
+    with row stride out_row_stride)."""
+    if not x.is_cuda or not packed.is_cuda:
+        raise ValueError("libesa takes CUDA tensors (no CPU path)")
+    rows, hin, d = x.shape
+    if x.stride(2) != 1 or x.stride(1) != d:
+        raise ValueError("each row of x must be contiguous [Hin, D]")
+    if out is None:
+        out = torch.empty((rows, d_out), dtype=torch.float32, device=x.device)
+        stride = d_out
+    else:
+        stride = out_row_stride or d_out
+    _check(load().esa_compress_packed(_ptr(x), rows, x.stride(0) if rows > 1 else hin * d, hin, d, _ptr(packed),
+                                      d_out, _ptr(out), stride, _stream()), "esa_compress_packed")
     return out
 
 

@@ -19,6 +19,7 @@
 #include "common.cuh"
 #include "compress.cuh"
 #include "compress_tc.cuh"
+#include "compress_pk.cuh"
 #include "moba.cuh"
 #include "score.cuh"
 #include "score_tc.cuh"
@@ -246,6 +247,134 @@ esa_status_t esa_device_status(void* stream) {
   const unsigned code = (unsigned)(v >> 32), site = (unsigned)(v & 0xffffffffu);
   if (code == 5u) return fail(ESA_ERR_CUDA, "kernel site %u found its shared memory misaligned and stopped", site);
   return fail(ESA_ERR_TIMEOUT, "device wait ran out at site %u (status %u)", site, code);
+}
+
+// ------------------------------------------------------- packed-weight compression --
+size_t esa_compress_pack_size(int32_t n_heads_in, int32_t head_dim, int32_t d_out) {
+  if (n_heads_in <= 0 || head_dim <= 0 || d_out != 128) return 0;
+  const int64_t K = (int64_t)n_heads_in * head_dim;
+  if (K % 512 || K > (int64_t)1 << 20) return 0;
+  return (size_t)(2 * 128 * K * 2);
+}
+
+esa_status_t esa_compress_pack(const float* w, int32_t n_heads_in, int32_t n_heads_out, int32_t head_dim,
+                               int32_t d_out, void* packed, size_t packed_bytes, void* stream) {
+  if (!w || !packed) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  if (n_heads_in <= 0 || n_heads_out <= 0 || n_heads_out % n_heads_in)
+    return fail(ESA_ERR_INVALID_ARG, "n_heads_out (%d) must be a positive multiple of n_heads_in (%d)", n_heads_out,
+                n_heads_in);
+  const size_t need = esa_compress_pack_size(n_heads_in, head_dim, d_out);
+  if (need == 0)
+    return fail(ESA_ERR_UNSUPPORTED, "packed compression needs d_out 128 and n_heads_in * head_dim a multiple of 512");
+  if (packed_bytes < need) return fail(ESA_ERR_INVALID_ARG, "packed buffer %zu bytes, need %zu", packed_bytes, need);
+  if (!aligned(packed, 16)) return fail(ESA_ERR_INVALID_ARG, "packed buffer must be 16-byte aligned");
+  const int K = n_heads_in * head_dim;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  esa::compress_pack_kernel<<<dim3(K / 64, 2), 256, 0, s>>>(w, n_heads_in, n_heads_out / n_heads_in, head_dim, K,
+                                                            static_cast<__nv_bfloat16*>(packed));
+  ESA_LAUNCH_CHECK("compress_pack_kernel");
+  return ok();
+}
+
+namespace {
+// 2D bf16 tensor map [outer, inner] (inner contiguous, row pitch in elements), boxes
+// of 128 rows x 64 columns with 128-byte swizzle: K-major MMA operand tiles.
+esa_status_t make_tmap_kmajor_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                                   uint64_t pitch_elems) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode;
+  esa_status_t st = get_encoder(&encode);
+  if (st != ESA_OK) return st;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_elems * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ESA_ERR_CUDA, "cuTensorMapEncodeTiled (k-major) failed (%d)", (int)r);
+  return ESA_OK;
+}
+
+// Cluster size for the packed compression: 16 CTAs when the device can co-schedule
+// them (one CTA per SM, so a whole 16-SM group), else the portable 8.
+esa_status_t pk_cluster_size(int dev, int* cl) {
+  static int cached[64] = {};
+  if (dev < 64 && cached[dev]) {
+    *cl = cached[dev];
+    return ESA_OK;
+  }
+  ESA_CUDA(cudaFuncSetAttribute(esa::compress_pk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                esa::kCpSmemBytes));
+  int best = 8;
+  if (cudaFuncSetAttribute(esa::compress_pk_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+      cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(16, 1, 2);
+    cfg.blockDim = dim3(esa::kCpThreads);
+    cfg.dynamicSmemBytes = esa::kCpSmemBytes;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 16;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, esa::compress_pk_kernel, &cfg) == cudaSuccess && n >= 1) best = 16;
+    cudaGetLastError();   // a refused query is not an error of this call
+  }
+  if (dev < 64) cached[dev] = best;
+  *cl = best;
+  return ESA_OK;
+}
+}  // namespace
+
+esa_status_t esa_compress_packed(const void* x, int64_t rows, int64_t x_row_stride, int32_t n_heads_in,
+                                 int32_t head_dim, const void* packed, int32_t d_out, float* y,
+                                 int64_t y_row_stride, void* stream) {
+  if (rows < 0) return fail(ESA_ERR_INVALID_ARG, "rows must be >= 0");
+  if (rows == 0) return ok();
+  if (!x || !packed || !y) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  if (esa_compress_pack_size(n_heads_in, head_dim, d_out) == 0)
+    return fail(ESA_ERR_UNSUPPORTED, "packed compression needs d_out 128 and n_heads_in * head_dim a multiple of 512");
+  const int K = n_heads_in * head_dim;
+  if (x_row_stride < K || x_row_stride % 8) return fail(ESA_ERR_INVALID_ARG, "x_row_stride must be >= n_heads_in * head_dim and a multiple of 8");
+  if (y_row_stride < 128 || y_row_stride % 4) return fail(ESA_ERR_INVALID_ARG, "y_row_stride must be >= 128 and a multiple of 4");
+  if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(y, 16))
+    return fail(ESA_ERR_INVALID_ARG, "x, packed and y must be 16-byte aligned");
+  int dev = 0;
+  ESA_CUDA(cudaGetDevice(&dev));
+  int cl = 8;
+  esa_status_t st = pk_cluster_size(dev, &cl);
+  if (st != ESA_OK) return st;
+  if (K % (64 * cl)) cl = 8;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  CUtensorMap tw;
+  st = make_tmap_kmajor_bf16(&tw, packed, (uint64_t)K, 256, (uint64_t)K);
+  if (st != ESA_OK) return st;
+  const int64_t max_rows = (int64_t)65535 * esa::kCpRows;
+  for (int64_t r0 = 0; r0 < rows; r0 += max_rows) {
+    const int64_t nr = std::min(rows - r0, max_rows);
+    CUtensorMap tx;
+    st = make_tmap_kmajor_bf16(&tx, static_cast<const __nv_bfloat16*>(x) + r0 * x_row_stride, (uint64_t)K,
+                               (uint64_t)nr, (uint64_t)x_row_stride);
+    if (st != ESA_OK) return st;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cl, (unsigned)cdiv(nr, esa::kCpRows), 2);
+    cfg.blockDim = dim3(esa::kCpThreads);
+    cfg.dynamicSmemBytes = esa::kCpSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)cl;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, esa::compress_pk_kernel, tx, tw, nr, K, y + r0 * y_row_stride, y_row_stride);
+    ESA_LAUNCH_CHECK("compress_pk_kernel");
+  }
+  return ok();
 }
 
 // ------------------------------------------------------------------ esa_compress --

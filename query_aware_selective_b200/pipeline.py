@@ -5,7 +5,8 @@ each chunk's queries select the important middle tokens (all queries of the chun
 count), and in decoding the single current query does. These classes hold the
 caller-side state (compressed key cache, index buffers, workspaces, outputs) and
 issue the C-ABI calls in order on the current stream. They allocate everything up
-front, so a step launches kernels only and can be captured in a CUDA graph.
+front, so a step launches kernels only and can be captured in a CUDA graph
+(``graph_of``), which replays the whole step with one launch.
 """
 from __future__ import annotations
 
@@ -17,8 +18,78 @@ import torch
 from . import _abi
 
 
+def graph_of(fn):
+    """Capture fn() into a CUDA graph. fn runs once eagerly first, on a side stream,
+    so that every one-time host setting (kernel attributes, cluster sizes) is made
+    outside the capture. The graph holds the kernels with the pointers fn used; replay
+    it only while those buffers stay alive and in place."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def _timing_event(external: bool):
+    # external: a record node when captured in a graph (readable after each replay)
+    return torch.cuda.Event(enable_timing=True, external=external) if external else \
+        torch.cuda.Event(enable_timing=True)
+
+
 def _region_lo(c0: int, n_init: int, window: int) -> int:
     return min(c0, max(n_init, c0 - window))
+
+
+class _Compressor:
+    """The two compression maps of a layer (queries: Hq heads in; keys: Hkv heads in,
+    expanded to Hq). With bf16 inputs and a shape the packed path takes, the weights
+    are packed once per pack() call (fold + bf16 high/low split, esa_compress_pack)
+    and every map runs esa_compress_packed; otherwise esa_compress reads the fp32
+    weights directly."""
+
+    def __init__(self, hq: int, hkv: int, head_dim: int, d_c: int, dtype, device):
+        self.hq, self.hkv, self.d, self.d_c = hq, hkv, head_dim, d_c
+        nq = _abi.compress_pack_size(hq, head_dim, d_c) if dtype == torch.bfloat16 else 0
+        nk = _abi.compress_pack_size(hkv, head_dim, d_c) if dtype == torch.bfloat16 else 0
+        self.packed = bool(nq and nk)
+        if self.packed:
+            self.wq_p = torch.empty(nq, dtype=torch.uint8, device=device)
+            self.wk_p = torch.empty(nk, dtype=torch.uint8, device=device)
+        self.key = None
+        self.wq = self.wk = None
+
+    def pack(self, wq, wk):
+        self.wq, self.wk = wq, wk
+        if self.packed:
+            _abi.compress_pack(wq, self.hq, self.hq, self.d, out=self.wq_p)
+            _abi.compress_pack(wk, self.hkv, self.hq, self.d, out=self.wk_p)
+        self.key = (wq.data_ptr(), wq._version, wk.data_ptr(), wk._version)
+
+    def pack_keys(self, wk):
+        """Key map only (filling a cache); the next pack_if_changed packs both."""
+        self.wk = wk
+        if self.packed:
+            _abi.compress_pack(wk, self.hkv, self.hq, self.d, out=self.wk_p)
+        self.key = None
+
+    def pack_if_changed(self, wq, wk):
+        if self.key != (wq.data_ptr(), wq._version, wk.data_ptr(), wk._version):
+            self.pack(wq, wk)
+
+    def queries(self, x, out, out_row_stride=None):
+        if self.packed:
+            return _abi.compress_packed(x, self.wq_p, self.d_c, out=out, out_row_stride=out_row_stride)
+        return _abi.compress(x, self.wq, self.hq, out=out, out_row_stride=out_row_stride)
+
+    def keys(self, x, out, out_row_stride=None):
+        if self.packed:
+            return _abi.compress_packed(x, self.wk_p, self.d_c, out=out, out_row_stride=out_row_stride)
+        return _abi.compress(x, self.wk, self.hq, out=out, out_row_stride=out_row_stride)
 
 
 class EsaPrefill:
@@ -44,15 +115,17 @@ class EsaPrefill:
         self.ws_sel = torch.empty(ws_sel + 256, dtype=torch.uint8, device=device)
         self.ws_att = torch.empty(ws_att + 256, dtype=torch.uint8, device=device) if ws_att else None
         self.out_views = []
+        self.cmp = _Compressor(hq, hkv, head_dim, d_c, dtype, device)
 
     def chunks(self):
         return [(c0, min(self.chunk, self.n_ctx - c0)) for c0 in range(0, self.n_ctx, self.chunk)]
 
     def run_chunk(self, c0: int, lq: int, q, k, v, wq, wk, attn_events=None):
         b = self.batch
+        self.cmp.pack_if_changed(wq, wk)
         for s in range(b):
-            _abi.compress(k[s, c0:c0 + lq], wk, self.hq, out=self.k_c[s, c0:c0 + lq])
-            _abi.compress(q[s, c0:c0 + lq], wq, self.hq, out=self.q_c[s, :lq])
+            self.cmp.keys(k[s, c0:c0 + lq], out=self.k_c[s, c0:c0 + lq])
+            self.cmp.queries(q[s, c0:c0 + lq], out=self.q_c[s, :lq])
         q_c = self.q_c[:, :lq] if lq == self.chunk else self.q_c[:, :lq].contiguous()
         _abi.score_select(q_c, self.k_c, c0, self.p, idx=self.idx, count=self.count, workspace=self.ws_sel)
         qv = q[:, c0:c0 + lq]
@@ -68,14 +141,17 @@ class EsaPrefill:
         if target is not ov:
             ov.copy_(target)
 
-    def run(self, q, k, v, wq, wk, attn_events=None):
+    def run(self, q, k, v, wq, wk, attn_events=None, external_events=False):
         """q [B, N, Hq, D], k, v [B, N, Hkv, D] (device), wq, wk [Hq*D, d'].
         attn_events: optional list that receives one (start, end) CUDA event pair per
-        attention launch. Returns the output [B, N, Hq, D]."""
+        attention launch (external_events: made to be captured in a graph). Returns
+        the output [B, N, Hq, D]. The weights are packed for the tensor-core
+        compression at the start of every run."""
+        self.cmp.pack(wq, wk)
         for c0, lq in self.chunks():
             ev = None
             if attn_events is not None:
-                ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                ev = (_timing_event(external_events), _timing_event(external_events))
                 attn_events.append(ev)
             self.run_chunk(c0, lq, q, k, v, wq, wk, ev)
         return self.out
@@ -100,24 +176,29 @@ class EsaDecode:
                                   dtype=torch.uint8, device=device)
         nb = _abi.sparse_attn_workspace_size(batch, 1, c0, hq, hkv, head_dim, code, p)
         self.ws_att = torch.empty(nb + 256, dtype=torch.uint8, device=device) if nb else None
+        self.cmp = _Compressor(hq, hkv, head_dim, d_c, dtype, device)
 
     def fill_cache(self, k, wk, upto: Optional[int] = None):
         """Compress cached keys [0, upto) of every sequence (prefill state)."""
         upto = self.n_ctx - 1 if upto is None else upto
+        self.cmp.pack_keys(wk)
         step = 1 << 16
         for s in range(self.batch):
             for r0 in range(0, upto, step):
                 r1 = min(upto, r0 + step)
-                _abi.compress(k[s, r0:r1], wk, self.hq, out=self.k_c[s, r0:r1])
+                self.cmp.keys(k[s, r0:r1], out=self.k_c[s, r0:r1])
 
     def step(self, q, k, v, wq, wk, phase_events=None):
-        """q [B, 1, Hq, D]; k, v [B, n_ctx, Hkv, D] with the new token at n_ctx - 1."""
+        """q [B, 1, Hq, D]; k, v [B, n_ctx, Hkv, D] with the new token at n_ctx - 1.
+        The packed weights are reused across steps while wq and wk are the same tensors,
+        unmodified (pointer and version counter); otherwise they are packed again."""
         pos = self.n_ctx - 1
         ev = phase_events
         if ev is not None:
             ev[0].record()
-        _abi.compress(q[:, 0], wq, self.hq, out=self.q_c.view(self.batch, self.d_c))
-        _abi.compress(k[:, pos], wk, self.hq, out=self.k_c[:, pos], out_row_stride=self.n_ctx * self.d_c)
+        self.cmp.pack_if_changed(wq, wk)
+        self.cmp.queries(q[:, 0], out=self.q_c.view(self.batch, self.d_c))
+        self.cmp.keys(k[:, pos], out=self.k_c[:, pos], out_row_stride=self.n_ctx * self.d_c)
         if ev is not None:
             ev[1].record()
         _abi.score_select(self.q_c, self.k_c, pos, self.p, idx=self.idx, count=self.count, workspace=self.ws_sel)

@@ -74,6 +74,31 @@ def test_compress_rejects_bad_arguments(lib):
     assert f(FAKE, 1, 0, xs, 8, 32, 128, FAKE, 128, FAKE, 128, None) == _abi.ESA_OK
 
 
+def test_compress_pack_size_and_rejections(lib):
+    # K = n_heads_in * head_dim must be a multiple of 512 and d_out 128
+    assert lib.esa_compress_pack_size(32, 128, 128) == 2 * 128 * 4096 * 2
+    assert lib.esa_compress_pack_size(8, 128, 128) == 2 * 128 * 1024 * 2
+    assert lib.esa_compress_pack_size(4, 64, 128) == 0          # K = 256
+    assert lib.esa_compress_pack_size(32, 128, 64) == 0         # d_out 64
+    assert lib.esa_compress_pack_size(0, 128, 128) == 0
+    f = lib.esa_compress_pack
+    n = lib.esa_compress_pack_size(8, 128, 128)
+    assert f(None, 8, 32, 128, 128, FAKE, n, None) == _abi.ESA_ERR_INVALID_ARG
+    assert f(FAKE, 8, 30, 128, 128, FAKE, n, None) == _abi.ESA_ERR_INVALID_ARG
+    assert f(FAKE, 4, 4, 64, 128, FAKE, n, None) == _abi.ESA_ERR_UNSUPPORTED
+    assert f(FAKE, 8, 32, 128, 128, FAKE, n - 16, None) == _abi.ESA_ERR_INVALID_ARG
+    assert f(FAKE, 8, 32, 128, 128, FAKE + 8, n, None) == _abi.ESA_ERR_INVALID_ARG
+    g = lib.esa_compress_packed
+    assert g(FAKE, -1, 1024, 8, 128, FAKE, 128, FAKE, 128, None) == _abi.ESA_ERR_INVALID_ARG
+    assert g(FAKE, 0, 1024, 8, 128, FAKE, 128, FAKE, 128, None) == _abi.ESA_OK
+    assert g(None, 4, 1024, 8, 128, FAKE, 128, FAKE, 128, None) == _abi.ESA_ERR_INVALID_ARG
+    assert g(FAKE, 4, 1024, 8, 128, FAKE, 64, FAKE, 128, None) == _abi.ESA_ERR_UNSUPPORTED
+    assert g(FAKE, 4, 1000, 8, 128, FAKE, 128, FAKE, 128, None) == _abi.ESA_ERR_INVALID_ARG
+    assert g(FAKE, 4, 1028, 8, 128, FAKE, 128, FAKE, 128, None) == _abi.ESA_ERR_INVALID_ARG
+    assert g(FAKE, 4, 1024, 8, 128, FAKE, 128, FAKE, 96, None) == _abi.ESA_ERR_INVALID_ARG
+    assert g(FAKE + 2, 4, 1024, 8, 128, FAKE, 128, FAKE, 128, None) == _abi.ESA_ERR_INVALID_ARG
+
+
 def test_score_select_rejects_bad_arguments(lib):
     f = lib.esa_score_select
     good = _abi.params(128, 4096, 2048, 2, 45.25)

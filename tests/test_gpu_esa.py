@@ -72,6 +72,50 @@ def test_compress_writes_into_a_cache_slice():
     assert np.all(got[:10] == 7.0) and np.all(got[30:] == 7.0) and np.all(got[10:30, 32:] == 7.0)
 
 
+@pytest.mark.parametrize("rows,hin,hout", [
+    (512, 32, 32),     # one chunk of queries: K = 4096, 4 row tiles
+    (300, 8, 32),      # keys under GQA (G = 4, K = 1024), ragged last row tile
+    (1, 4, 4),         # K = 512: the smallest reduction the packed path takes
+    (129, 16, 32),     # G = 2, one full tile + one row
+])
+def test_compress_packed_parity(rows, hin, hout):
+    """Packed weight (fold + bf16 hi/lo split, once) then the TMA/tcgen05 map: the
+    oracle's fp64 map within the fp32 bar."""
+    d, dc = 128, 128
+    x = _rand((rows, hin, d), 11, torch.bfloat16)
+    w = _rand((hout * d, dc), 12, torch.float32) / math.sqrt(hout * d)
+    packed = qas.compress_pack(w.to(DEV), hin, hout, d)
+    y = qas.compress_packed(x.to(DEV), packed, dc)
+    ref = oesa.compress(_np(x), _np(w), hout)
+    assert max_abs(_np(y), ref) <= ATOL_F32
+    y2 = qas.compress(x.to(DEV), w.to(DEV), hout)      # the unpacked path: same split, other sum order
+    assert max_abs(_np(y), _np(y2)) <= ATOL_F32
+
+
+def test_compress_packed_strided_rows_of_a_batched_cache():
+    """Decode form: the new key of every sequence (rows n_ctx apart) into that
+    sequence's row of the compressed cache; nothing else is written."""
+    b, n, hkv, hq, d, dc, pos = 5, 40, 8, 32, 128, 128, 37
+    k = _rand((b, n, hkv, d), 15, torch.bfloat16).to(DEV)
+    w = (_rand((hq * d, dc), 16, torch.float32) / math.sqrt(hq * d)).to(DEV)
+    cache = torch.zeros((b, n, dc), device=DEV)
+    packed = qas.compress_pack(w, hkv, hq, d)
+    qas.compress_packed(k[:, pos], packed, dc, out=cache[:, pos], out_row_stride=n * dc)
+    ref = oesa.compress(_np(k[:, pos].cpu()), _np(w.cpu()), hq)
+    got = cache.cpu().numpy()
+    assert max_abs(got[:, pos], ref) <= ATOL_F32
+    assert np.all(np.delete(got, pos, axis=1) == 0.0)
+
+
+def test_compress_packed_is_deterministic():
+    x = _rand((640, 32, 128), 17, torch.bfloat16).to(DEV)
+    w = (_rand((32 * 128, 128), 18, torch.float32) / 64.0).to(DEV)
+    packed = qas.compress_pack(w, 32, 32, 128)
+    a = qas.compress_packed(x, packed)
+    b = qas.compress_packed(x, packed)
+    assert torch.equal(a, b)
+
+
 # ----------------------------------------------------------------------------- selection
 
 def _selection_case(batch, lq, n_cap, c0, dc, p, seed, planted=False):
