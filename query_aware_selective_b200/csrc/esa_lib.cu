@@ -14,6 +14,7 @@
 #include <string>
 
 #include "../../include/esa.h"
+#include "attn_decode.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
@@ -554,6 +555,7 @@ namespace {
 
 struct AttnPlan {
   bool tc;
+  bool dec;          // bulk-copy decode kernel (bf16, head_dim 128, one query)
   int nsplit;
   int64_t keys_per_split;
   size_t ws_bytes;
@@ -571,6 +573,20 @@ AttnPlan plan_attn(int32_t batch, int32_t lq, int64_t c0, int32_t hq, int32_t hk
     return pl;
   }
   const int64_t n_keys_max = r.ni + std::min<int64_t>(p.topk, r.n_mid) + (c0 - r.lo) + lq;
+  pl.dec = dt == ESA_BF16 && head_dim == 128 && lq == 1 && (hkv == 1 || hkv == 2 || hkv == 4 || hkv == 8) &&
+           (g == 1 || g == 2 || g == 4);
+  if (pl.dec) {
+    // one CTA per SM: split each sequence's key list so that batch x nsplit fills the
+    // 148 SMs once, with at least 4 stages per split
+    const int64_t ks = esa::kDecStageBytes / (hkv * head_dim * 2);
+    const int64_t by_sm = std::max<int64_t>(1, 148 / batch);
+    int64_t nsp = std::max<int64_t>(1, std::min(by_sm, cdiv(n_keys_max, 4 * ks)));
+    nsp = std::max(nsp, cdiv(n_keys_max, esa::kDecMaxSplitKeys));   // positions fit in shared memory
+    pl.keys_per_split = cdiv(cdiv(n_keys_max, nsp), ks) * ks;
+    pl.nsplit = (int)cdiv(n_keys_max, pl.keys_per_split);
+    pl.ws_bytes = pl.nsplit > 1 ? up256((size_t)batch * hq * pl.nsplit * (head_dim + 2) * sizeof(float)) : 0;
+    return pl;
+  }
   const int64_t base = (int64_t)batch * lq * hkv;
   const int64_t want_ctas = 4 * 148;
   int64_t per = std::max<int64_t>(256, cdiv(n_keys_max, std::max<int64_t>(1, want_ctas / base)));
@@ -681,6 +697,44 @@ esa_status_t esa_sparse_attn(const void* q, const void* k, const void* v, esa_dt
     esa::attn_tc_kernel<esa::EsaTcProblem><<<grid, esa::kTcThreads, esa::kTcSmemBytes, s>>>(tq, tk, tv, bq, bk, bv,
                                                                                            sk, sv, pr);
     ESA_LAUNCH_CHECK("attn_tc_kernel<esa>");
+    return ok();
+  }
+  if (pl.dec) {
+    static bool dec_attr[64] = {};
+    int dev = 0;
+    ESA_CUDA(cudaGetDevice(&dev));
+    if (dev < 64 && !dec_attr[dev]) {
+      if ((st = set_max_smem(esa::attn_decode_kernel<1>, esa::kDecSmemBytes)) != ESA_OK) return st;
+      if ((st = set_max_smem(esa::attn_decode_kernel<2>, esa::kDecSmemBytes)) != ESA_OK) return st;
+      if ((st = set_max_smem(esa::attn_decode_kernel<4>, esa::kDecSmemBytes)) != ESA_OK) return st;
+      dec_attr[dev] = true;
+    }
+    esa::DecodeAttnArgs d{};
+    d.q = static_cast<const __nv_bfloat16*>(q);
+    d.k = static_cast<const __nv_bfloat16*>(k);
+    d.v = static_cast<const __nv_bfloat16*>(v);
+    d.o = static_cast<__nv_bfloat16*>(o);
+    d.lse = lse;
+    d.part = static_cast<float*>(workspace);
+    d.keys = keys;
+    d.n_cap = n_cap;
+    d.c0 = c0;
+    d.hq = hq;
+    d.hkv = hkv;
+    d.nsplit = pl.nsplit;
+    d.keys_per_split = (int)pl.keys_per_split;
+    d.scale_log2 = sl2;
+    const dim3 grid((unsigned)pl.nsplit, (unsigned)batch);
+    if (g == 1) esa::attn_decode_kernel<1><<<grid, esa::kDecThreads, esa::kDecSmemBytes, s>>>(d);
+    else if (g == 2) esa::attn_decode_kernel<2><<<grid, esa::kDecThreads, esa::kDecSmemBytes, s>>>(d);
+    else esa::attn_decode_kernel<4><<<grid, esa::kDecThreads, esa::kDecSmemBytes, s>>>(d);
+    ESA_LAUNCH_CHECK("attn_decode_kernel");
+    if (pl.nsplit > 1) {
+      const int64_t rows = (int64_t)batch * hq;
+      esa::attn_combine_kernel<__nv_bfloat16, 128><<<dim3((unsigned)cdiv(rows, 8)), 256, 0, s>>>(
+          d.part, rows, pl.nsplit, static_cast<__nv_bfloat16*>(o), lse);
+      ESA_LAUNCH_CHECK("attn_combine_kernel");
+    }
     return ok();
   }
   esa::SimtAttnArgs a{};

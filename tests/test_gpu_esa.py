@@ -208,6 +208,38 @@ def test_sparse_attn_simt_parity(batch, lq, n_cap, c0, hq, hkv, d, dtype, n_init
     assert max_abs(lse.cpu().numpy(), ref_lse) <= 1e-3
 
 
+@pytest.mark.parametrize("batch,n_cap,hq,hkv,n_init,window,topk", [
+    (16, 4000, 32, 8, 128, 1024, 2048),   # 9 key splits per sequence, ragged last stage
+    (150, 200, 8, 2, 16, 64, 50),         # more sequences than SMs: one CTA each, direct output
+    (3, 5000, 8, 4, 32, 512, 777),        # G = 2, two warps per KV head
+    (2, 4000, 8, 2, 16, 300, 500),        # G = 4, four warps per KV head
+    (2, 3000, 1, 1, 8, 200, 300),         # a single head: 128 keys per stage
+    (4, 2500, 8, 8, 0, 100, 1000),        # no initial tokens
+    (2, 300, 32, 8, 128, 4096, 2048),     # the window covers the middle: nothing selected
+])
+def test_sparse_attn_decode_parity(batch, n_cap, hq, hkv, n_init, window, topk):
+    """The bulk-copy decode kernel (bf16, head_dim 128, one query per sequence), with
+    per-sequence selection counts that differ (ragged key lists and splits)."""
+    p = qas.params(n_init, window, topk, 2, 10.0)
+    c0 = n_cap - 1
+    q = _rand((batch, 1, hq, 128), 41, torch.bfloat16)
+    k = _rand((batch, n_cap, hkv, 128), 42, torch.bfloat16)
+    v = _rand((batch, n_cap, hkv, 128), 43, torch.bfloat16)
+    _, (m0, m1), _ = oesa.regions(c0, c0 + 1, n_init, window)
+    idx, cnt = synthetic.random_index_list(batch, m0, m1, topk, seed=44)
+    for b in range(batch):
+        c = max(0, int(cnt[b]) - 37 * b)
+        idx[b, c:] = -1
+        cnt[b] = c
+    o, lse = qas.sparse_attn(q.to(DEV), k.to(DEV), v.to(DEV), c0, idx.to(DEV), cnt.to(DEV), p, want_lse=True)
+    o2, _ = qas.sparse_attn(q.to(DEV), k.to(DEV), v.to(DEV), c0, idx.to(DEV), cnt.to(DEV), p)
+    assert torch.equal(o, o2)                    # no state carried between calls
+    ref_o, ref_lse = oesa.sparse_attn(q.float().numpy(), k.float().numpy(), v.float().numpy(), c0, idx.numpy(),
+                                      cnt.numpy(), n_init, window)
+    assert max_abs(_np(o), ref_o) <= ATOL_BF16
+    assert max_abs(lse.cpu().numpy(), ref_lse) <= 1e-3
+
+
 @pytest.mark.parametrize("batch,lq,n_cap,c0,hq,hkv,n_init,window,topk", [
     (1, 128, 1024, 640, 8, 2, 16, 256, 128),      # 4 row tiles, selection active
     (1, 200, 3000, 2800, 32, 8, 128, 1024, 700),  # ragged chunk (800 rows), 7 row tiles
