@@ -34,26 +34,6 @@ constexpr int kCtPStride = kCtNS + 4;   // padded row of the fp32 partial (sprea
 static_assert(kCtRows * kCtPStride * 4 <= 2 * kCtStage, "partial must fit in the stage buffers");
 constexpr int kCtWq = kCtK * kCtNS / 4 / kCtThreads;    // float4 of one W slice per thread per chunk (8)
 
-__device__ __forceinline__ uint32_t dsmem_map(uint32_t local_addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
 // G = query heads per input head (1 for queries, Hq / Hkv for GQA keys)
 template <int G>
 __global__ void __cluster_dims__(kCtCluster, 1, 1) __launch_bounds__(kCtThreads, 1)

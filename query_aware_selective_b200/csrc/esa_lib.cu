@@ -123,31 +123,53 @@ ScorePath score_path(int32_t batch, int32_t lq, int64_t n_cap, int32_t d_c) {
 }
 
 struct SelWs {
-  float* S;
-  float* s;
-  uint32_t* u;
-  uint32_t* m_key;
-  uint32_t* hist;
-  esa::SelState* st;
-  uint2* tiles;
+  uint32_t* m_key;   // [B, lq] order keys of the per-query maxima (cleared before scoring)
+  float* S;          // [B, lq, n_mid] raw scores (SIMT paths)
+  float* s;          // [B, n_mid] chunk-summed corrected scores (tensor-core path)
+  uint32_t* u;       // [B, n_mid] order keys, when a cluster CTA's range exceeds its shared memory
   size_t bytes;
-  size_t zero_bytes;   // m_key + hist are contiguous and cleared together
 };
 
 SelWs carve_select(void* ws, int32_t batch, int32_t lq, int64_t n_mid, ScorePath path) {
   Carver c{reinterpret_cast<uint8_t*>(ws)};
   SelWs w;
-  const int64_t n_tiles = cdiv(std::max<int64_t>(n_mid, 1), esa::kTkTile);
   w.m_key = c.take<uint32_t>((size_t)batch * lq);
-  w.hist = c.take<uint32_t>((size_t)batch * 3 * esa::kTkBins);
-  w.zero_bytes = c.off;
   w.S = path == ScorePath::TensorCore ? nullptr : c.take<float>((size_t)batch * lq * n_mid);
-  w.s = c.take<float>((size_t)batch * n_mid);
-  w.u = c.take<uint32_t>((size_t)batch * n_mid);
-  w.st = c.take<esa::SelState>((size_t)batch);
-  w.tiles = c.take<uint2>((size_t)batch * n_tiles);
+  w.s = path == ScorePath::TensorCore ? c.take<float>((size_t)batch * n_mid) : nullptr;
+  w.u = c.take<uint32_t>((size_t)batch * (n_mid + 64));   // up to 16 cluster CTAs, each range padded to 4
   w.bytes = c.off;
   return w;
+}
+
+// Cluster size of the selection kernel: 16 CTAs when `batch` such clusters (one per
+// sequence) can be resident at once, else the portable 8. Occupancy is queried once per
+// device.
+int select_cluster_size(int32_t batch) {
+  static int max16[64] = {};   // 0: not queried; -1: 16-CTA clusters unavailable
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return 8;
+  if (!max16[dev]) {
+    max16[dev] = -1;
+    if (cudaFuncSetAttribute(esa::select_cluster_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(16, 1, 1);
+      cfg.blockDim = dim3(esa::kSelThreads);
+      cfg.dynamicSmemBytes = esa::kSelSmemBytes;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = 16;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, esa::select_cluster_kernel<16>, &cfg) == cudaSuccess && n >= 1)
+        max16[dev] = n;
+    }
+    cudaGetLastError();   // a refused query is not an error of this call
+  }
+  return (max16[dev] > 0 && batch <= max16[dev]) ? 16 : 8;
 }
 
 // 2D tensor map over a row-major fp32 matrix [rows, cols], 32 x 128 boxes, 128-byte
@@ -472,6 +494,7 @@ esa_status_t esa_score_select(const float* q_c, const float* k_c, int32_t batch,
   if (!aligned(q_c, 16) || !aligned(k_c, 16)) return fail(ESA_ERR_INVALID_ARG, "q_c and k_c need 16-byte alignment");
   const Regions r = regions(c0, p);
   if (r.n_mid > (int64_t)1 << 30) return fail(ESA_ERR_UNSUPPORTED, "middle longer than 2^30 tokens");
+  if (batch > 65535) return fail(ESA_ERR_UNSUPPORTED, "batch must be <= 65535 (got %d)", batch);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t kk = std::min<int64_t>(p.topk, r.n_mid);
   const bool need_scores = r.n_mid > p.topk || (score_out && r.n_mid > 0);
@@ -481,7 +504,7 @@ esa_status_t esa_score_select(const float* q_c, const float* k_c, int32_t batch,
     if (!workspace || ws_bytes < need.bytes || !aligned(workspace, 256))
       return fail(ESA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need.bytes, ws_bytes);
     const SelWs w = carve_select(workspace, batch, lq, r.n_mid, path);
-    ESA_CUDA(cudaMemsetAsync(w.m_key, 0, w.zero_bytes, s));
+    ESA_CUDA(cudaMemsetAsync(w.m_key, 0, (size_t)batch * lq * sizeof(uint32_t), s));
     if (path == ScorePath::Small) {
       switch (d_c) {
         case 16: launch_score_small<16>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, w.S, w.m_key, s); break;
@@ -518,29 +541,48 @@ esa_status_t esa_score_select(const float* q_c, const float* k_c, int32_t batch,
       ESA_LAUNCH_CHECK("score_tc_kernel<1>");
       esa::score_tc_kernel<2><<<grid, esa::kStThreads, smem, s>>>(tm_k, tm_q, a);
       ESA_LAUNCH_CHECK("score_tc_kernel<2>");
-    } else {
-      esa::clamp_sum_kernel<<<dim3((unsigned)cdiv(r.n_mid, 256), batch), 256, 0, s>>>(w.S, w.m_key, lq, r.n_mid,
-                                                                                      p.clamp_c, w.s);
-      ESA_LAUNCH_CHECK("clamp_sum_kernel");
     }
-    const int n_tiles = (int)cdiv(r.n_mid, esa::kTkTile);
-    const dim3 tgrid(n_tiles, batch);
-    esa::pool_hist_kernel<<<tgrid, esa::kTkThreads, 0, s>>>(w.s, r.n_mid, p.eps, w.u, score_out, w.hist);
-    ESA_LAUNCH_CHECK("pool_hist_kernel");
-    if (r.n_mid > p.topk) {
-      for (int level = 0; level < 3; ++level) {
-        if (level > 0) {
-          esa::radix_hist_kernel<<<tgrid, esa::kTkThreads, 0, s>>>(w.u, r.n_mid, level, w.st, w.hist);
-          ESA_LAUNCH_CHECK("radix_hist_kernel");
-        }
-        esa::radix_select_kernel<<<batch, 1024, 0, s>>>(w.hist, level, (uint32_t)kk, w.st);
-        ESA_LAUNCH_CHECK("radix_select_kernel");
+    if (kk > 0) {
+      esa::SelectArgs sa{};
+      sa.S = path == ScorePath::TensorCore ? nullptr : w.S;
+      sa.m_key = w.m_key;
+      sa.s = w.s;
+      sa.lq = lq;
+      sa.clamp_c = p.clamp_c;
+      sa.n_mid = r.n_mid;
+      sa.mid0 = r.mid0;
+      sa.eps = p.eps;
+      sa.kk = (int)kk;
+      sa.topk = p.topk;
+      sa.u = w.u;
+      sa.s_prime_out = score_out;
+      sa.idx = idx_out;
+      sa.count = count_out;
+      static bool sel_attr[64] = {};
+      int dev = 0;
+      ESA_CUDA(cudaGetDevice(&dev));
+      if (dev < 64 && !sel_attr[dev]) {
+        if ((st = set_max_smem(esa::select_cluster_kernel<8>, esa::kSelSmemBytes)) != ESA_OK) return st;
+        if ((st = set_max_smem(esa::select_cluster_kernel<16>, esa::kSelSmemBytes)) != ESA_OK) return st;
+        sel_attr[dev] = true;
       }
-      esa::compact_count_kernel<<<tgrid, esa::kTkThreads, 0, s>>>(w.u, r.n_mid, w.st, w.tiles, n_tiles);
-      ESA_LAUNCH_CHECK("compact_count_kernel");
-      esa::compact_write_kernel<<<tgrid, esa::kTkThreads, 0, s>>>(w.u, r.n_mid, w.st, w.tiles, n_tiles, r.mid0,
-                                                                  p.topk, idx_out);
-      ESA_LAUNCH_CHECK("compact_write_kernel");
+      const int cl = select_cluster_size(batch);
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)cl, (unsigned)batch, 1);
+      cfg.blockDim = dim3(esa::kSelThreads);
+      cfg.dynamicSmemBytes = esa::kSelSmemBytes;
+      cfg.stream = s;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = (unsigned)cl;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      if (cl == 16) cudaLaunchKernelEx(&cfg, esa::select_cluster_kernel<16>, sa);
+      else cudaLaunchKernelEx(&cfg, esa::select_cluster_kernel<8>, sa);
+      ESA_LAUNCH_CHECK("select_cluster_kernel");
+      return ok();
     }
   }
   const bool all_mid = r.n_mid <= p.topk;
@@ -578,7 +620,7 @@ AttnPlan plan_attn(int32_t batch, int32_t lq, int64_t c0, int32_t hq, int32_t hk
   if (pl.dec) {
     // one CTA per SM: split each sequence's key list so that batch x nsplit fills the
     // 148 SMs once, with at least 4 stages per split
-    const int64_t ks = esa::kDecStageBytes / (hkv * head_dim * 2);
+    const int64_t ks = esa::kDecStageRowsBytes / (hkv * head_dim * 2);
     const int64_t by_sm = std::max<int64_t>(1, 148 / batch);
     int64_t nsp = std::max<int64_t>(1, std::min(by_sm, cdiv(n_keys_max, 4 * ks)));
     nsp = std::max(nsp, cdiv(n_keys_max, esa::kDecMaxSplitKeys));   // positions fit in shared memory

@@ -6,7 +6,9 @@
 //
 //   S_ij = q_c[i] . k_c[mid0 + j]           (fp32)
 //   m_i  = max_j S_ij                       (atomicMax on order keys: order-independent)
+// The kernels here store S and m; the selection kernel (topk.cuh) forms
 //   s_j  = sum_i max(S_ij - m_i, -C)        (fixed order i = 0, 1, ...)
+// as it reads them.
 #pragma once
 #include "common.cuh"
 
@@ -156,25 +158,6 @@ __global__ void __launch_bounds__(256) score_tiled_kernel(const float* __restric
     for (int x = 0; x < 16; ++x) m = fmaxf(m, rmax[tid][x]);
     if (m > -INFINITY) atomicMax(&m_key[b * lq + i0 + tid], order_key(m));
   }
-}
-
-__device__ __forceinline__ float key_to_float(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
-
-// s_j = sum_i max(S_ij - m_i, -C), i in increasing order.
-__global__ void __launch_bounds__(256) clamp_sum_kernel(const float* __restrict__ S, const uint32_t* __restrict__ m_key,
-                                                        int lq, int64_t n_mid, float clamp_c, float* __restrict__ s) {
-  const int b = blockIdx.y;
-  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= n_mid) return;
-  const float lo = -clamp_c;
-  float acc = 0.f;
-  for (int i = 0; i < lq; ++i) {
-    const float m = key_to_float(__ldg(&m_key[b * lq + i]));
-    acc += fmaxf(S[((int64_t)b * lq + i) * n_mid + j] - m, lo);
-  }
-  s[(int64_t)b * n_mid + j] = acc;
 }
 
 }  // namespace esa

@@ -1,219 +1,328 @@
-// topk.cuh - neighbour influence and fixed-count top-k over the middle tokens
-// (ESA write-up: neighbour-influence paragraph - a token's score is lifted by the
-// tokens around it, read as s'_j = max_{|m - j| <= eps, m in middle} s_m; core-steps
-// paragraph - a fixed number k of tokens is kept).
+// topk.cuh - neighbour influence and fixed-count top-k over the middle tokens of each
+// sequence, in one launch (ESA write-up: neighbour-influence paragraph - a token's
+// score is lifted by the tokens around it, read as s'_j = max_{|m - j| <= eps, m in
+// middle} s_m; core-steps paragraph - a fixed number k of tokens is kept;
+// score-correction paragraph - when raw scores come in, s_j = sum_i max(S_ij - m_i, -C)
+// is formed on the fly in query order).
 //
-// Order: s' descending, then position ascending. Exact selection in three radix
-// levels over order-preserving 32-bit keys (11 + 11 + 10 bits): each level builds a
-// histogram of the candidates that still share the threshold's prefix and picks the
-// bin that holds the k-th key. The threshold key T and the number of keys equal to T
-// that are kept (the lowest positions first) then drive an ordered compaction, so
-// the output is ascending by position without a sort. Integer atomics only: the
-// result does not depend on scheduling.
+// One thread-block cluster per sequence (16 CTAs when every sequence's cluster can be
+// resident at once, else 8);
+// CTA r owns a contiguous range of middle positions. Order: s' descending, then
+// position ascending. Exact selection in three radix levels over order-preserving
+// 32-bit keys (11 + 11 + 10 bits). At each level every CTA histograms its keys that
+// still share the threshold's prefix (shared-memory atomics), the cluster merges the
+// histograms through distributed shared memory (reduce-scatter: CTA r sums bin slice r
+// over all CTAs; all-gather: every CTA reads the merged slices), and every CTA finds
+// the same bin holding the want-th largest key. The threshold key T and the number of
+// keys equal to T to keep (lowest positions first) then drive an ordered compaction:
+// the CTAs exchange their (above T, equal to T) counts, and a block scan in position
+// order writes the kept positions ascending, so no sort is needed. Integer atomics
+// only: the result does not depend on scheduling. The keys stay in shared memory when
+// a CTA's range fits (kSelUCap), else in a global scratch array.
 #pragma once
-#include <cub/block/block_reduce.cuh>
 #include <cub/block/block_scan.cuh>
 
 #include "common.cuh"
 
 namespace esa {
 
-constexpr int kTkTile = 1024;      // elements per CTA in the streaming kernels
-constexpr int kTkThreads = 256;    // 4 elements per thread
-constexpr int kTkBins = 2048;
+constexpr int kSelThreads = 512;
+constexpr int kSelBins = 2048;
+constexpr int kSelTile = 4096;       // positions per pooling tile
+constexpr int kSelMaxEps = 64;
+constexpr int kSelUCap = 16384;      // order keys a CTA keeps in shared memory
 
-struct SelState {      // per sequence
-  uint32_t prefix;     // high bits of T fixed so far
-  uint32_t want;       // keys still to take at or below the current prefix
-  uint32_t thresh;     // final T
-  uint32_t pad;
+struct SelectArgs {
+  const float* S;          // [B, lq, n_mid] raw scores, with m_key; or null
+  const uint32_t* m_key;   // [B, lq] order keys of the per-query maxima
+  const float* s;          // [B, n_mid] chunk-summed corrected scores (when S is null)
+  int lq;
+  float clamp_c;
+  int64_t n_mid, mid0;
+  int eps;                 // <= kSelMaxEps
+  int kk;                  // keys to keep: min(topk, n_mid) >= 1
+  int topk;
+  uint32_t* u;             // [B, n_mid] key scratch (used when a CTA's range exceeds kSelUCap)
+  float* s_prime_out;      // [B, n_mid] or null
+  int32_t* idx;            // [B, topk]
+  int32_t* count;          // [B]
 };
 
-__host__ __device__ constexpr int level_shift(int level) { return level == 0 ? 21 : (level == 1 ? 10 : 0); }
-__host__ __device__ constexpr int level_bits(int level) { return level == 2 ? 10 : 11; }
+struct SelSmem {
+  uint32_t hist[kSelBins];   // this CTA's histogram of the current level
+  uint32_t mrg[kSelBins];    // merged counts of the bin slice this CTA owns
+  uint32_t full[kSelBins];   // the merged histogram, gathered from the cluster
+  float sv[kSelTile + 2 * kSelMaxEps + 16];   // + slack: the vector pooling reads 16 values per group
+  uint32_t cnt[2];           // keys above T, keys equal to T (this CTA)
+  uint32_t sel_bin, sel_above;
+  typename cub::BlockScan<uint32_t, kSelThreads>::TempStorage scan;
+  uint32_t ucache[kSelUCap];
+};
+constexpr int kSelSmemBytes = (int)sizeof(SelSmem);
 
-// s' (neighbour max), order keys u, optional s' copy out, and the level-0 histogram.
-__global__ void __launch_bounds__(kTkThreads) pool_hist_kernel(const float* __restrict__ s, int64_t n, int eps,
-                                                              uint32_t* __restrict__ u, float* __restrict__ s_prime_out,
-                                                              uint32_t* __restrict__ hist) {
-  __shared__ float sv[kTkTile + 2 * 64];
-  __shared__ uint32_t h[kTkBins];
-  const int b = blockIdx.y;
-  const int64_t j0 = (int64_t)blockIdx.x * kTkTile;
-  const float* sb = s + (int64_t)b * n;
-  for (int t = threadIdx.x; t < kTkBins; t += kTkThreads) h[t] = 0;
-  for (int t = threadIdx.x; t < kTkTile + 2 * eps; t += kTkThreads) {
-    const int64_t j = j0 - eps + t;
-    sv[t] = (j >= 0 && j < n) ? sb[j] : -INFINITY;
-  }
-  __syncthreads();
-  for (int t = threadIdx.x; t < kTkTile; t += kTkThreads) {
-    const int64_t j = j0 + t;
-    if (j >= n) break;
-    float m = sv[t + eps];
-    for (int o = 1; o <= eps; ++o) m = fmaxf(m, fmaxf(sv[t + eps - o], sv[t + eps + o]));
-    const uint32_t key = order_key(m);
-    u[(int64_t)b * n + j] = key;
-    if (s_prime_out) s_prime_out[(int64_t)b * n + j] = m;
-    atomicAdd(&h[key >> 21], 1u);
-  }
-  __syncthreads();
-  uint32_t* hb = hist + (int64_t)b * 3 * kTkBins;
-  for (int t = threadIdx.x; t < kTkBins; t += kTkThreads)
-    if (h[t]) atomicAdd(&hb[t], h[t]);
-}
+// Raw scores of the tile [g0 - eps, g0 - eps + kSelHaloTile) for this thread's slots
+// (slot e = position tid + e * kSelThreads), or -inf outside the middle.
+constexpr int kSelHaloTile = kSelTile + 2 * kSelMaxEps;
+constexpr int kSelSlots = (kSelHaloTile + kSelThreads - 1) / kSelThreads;
 
-// Histogram of level `level` over keys whose bits above level_shift(level-1)... match.
-__global__ void __launch_bounds__(kTkThreads) radix_hist_kernel(const uint32_t* __restrict__ u, int64_t n, int level,
-                                                               const SelState* __restrict__ st,
-                                                               uint32_t* __restrict__ hist) {
-  __shared__ uint32_t h[kTkBins];
-  const int b = blockIdx.y;
-  const int64_t j0 = (int64_t)blockIdx.x * kTkTile;
-  for (int t = threadIdx.x; t < kTkBins; t += kTkThreads) h[t] = 0;
-  __syncthreads();
-  const uint32_t prefix = st[b].prefix;
-  const int hi_shift = level_shift(level - 1);
-  const int shift = level_shift(level);
-  const uint32_t mask = (1u << level_bits(level)) - 1u;
-  const uint32_t* ub = u + (int64_t)b * n;
-  for (int t = threadIdx.x; t < kTkTile; t += kTkThreads) {
-    const int64_t j = j0 + t;
-    if (j >= n) break;
-    const uint32_t key = ub[j];
-    if ((key >> hi_shift) == prefix) atomicAdd(&h[(key >> shift) & mask], 1u);
-  }
-  __syncthreads();
-  uint32_t* hb = hist + ((int64_t)b * 3 + level) * kTkBins;
-  for (int t = threadIdx.x; t < kTkBins; t += kTkThreads)
-    if (h[t]) atomicAdd(&hb[t], h[t]);
-}
-
-// One CTA per sequence: find the bin holding the want-th largest key of this level.
-// level 0 starts from want = kk (keys to keep).
-__global__ void __launch_bounds__(1024) radix_select_kernel(const uint32_t* __restrict__ hist, int level, uint32_t kk,
-                                                           SelState* __restrict__ st) {
-  using Scan = cub::BlockScan<uint32_t, 1024>;
-  __shared__ typename Scan::TempStorage tmp;
-  __shared__ uint32_t found_bin, found_above;
-  const int b = blockIdx.x;
-  const int nb = 1 << level_bits(level);
-  const uint32_t want = level == 0 ? kk : st[b].want;
-  const uint32_t* hb = hist + ((int64_t)b * 3 + level) * kTkBins;
-  // thread t owns bins in descending order: rank r = 2t, 2t+1 -> bin nb-1-r
-  const int per = nb / 1024;
-  uint32_t c[2] = {0, 0};
-  uint32_t sum = 0;
-  for (int q = 0; q < per; ++q) {
-    c[q] = hb[nb - 1 - (threadIdx.x * per + q)];
-    sum += c[q];
-  }
-  uint32_t before;
-  Scan(tmp).ExclusiveSum(sum, before);
-  uint32_t acc = before;
-  for (int q = 0; q < per; ++q) {
-    if (acc < want && acc + c[q] >= want) {
-      found_bin = nb - 1 - (threadIdx.x * per + q);
-      found_above = acc;
+__device__ __forceinline__ void sel_load_tile(const SelectArgs& a, int b, int64_t g0, int nt, float* v) {
+  const int tid = threadIdx.x;
+  const int64_t n = a.n_mid;
+  const int width = nt + 2 * a.eps;
+  if (!a.S) {
+    const float* sb = a.s + (int64_t)b * n;
+#pragma unroll
+    for (int e = 0; e < kSelSlots; ++e) {
+      const int t = tid + e * kSelThreads;
+      const int64_t j = g0 - a.eps + t;
+      v[e] = (t < width && j >= 0 && j < n) ? __ldcg(sb + j) : -INFINITY;
     }
-    acc += c[q];
+    return;
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const uint32_t prefix = level == 0 ? 0u : st[b].prefix;
-    const uint32_t np = (prefix << level_bits(level)) | found_bin;
-    st[b].prefix = np;
-    st[b].want = want - found_above;
-    if (level == 2) st[b].thresh = np;
+  const float lo = -a.clamp_c;
+#pragma unroll
+  for (int e = 0; e < kSelSlots; ++e) v[e] = 0.f;
+  for (int i = 0; i < a.lq; ++i) {
+    const float m = key_to_float(__ldg(&a.m_key[b * a.lq + i]));
+    const float* Sb = a.S + ((int64_t)b * a.lq + i) * n;
+    float x[kSelSlots];
+#pragma unroll
+    for (int e = 0; e < kSelSlots; ++e) {
+      const int t = tid + e * kSelThreads;
+      const int64_t j = g0 - a.eps + t;
+      x[e] = (t < width && j >= 0 && j < n) ? __ldcg(Sb + j) : 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < kSelSlots; ++e) v[e] += fmaxf(x[e] - m, lo);
+  }
+#pragma unroll
+  for (int e = 0; e < kSelSlots; ++e) {
+    const int t = tid + e * kSelThreads;
+    const int64_t j = g0 - a.eps + t;
+    if (!(t < width && j >= 0 && j < n)) v[e] = -INFINITY;
   }
 }
 
-// Per tile: number of keys above T and equal to T.
-__global__ void __launch_bounds__(kTkThreads) compact_count_kernel(const uint32_t* __restrict__ u, int64_t n,
-                                                                  const SelState* __restrict__ st,
-                                                                  uint2* __restrict__ tile_counts, int n_tiles) {
-  using Red = cub::BlockReduce<uint32_t, kTkThreads>;
-  __shared__ typename Red::TempStorage t1, t2;
+// grid (CL, B), cluster (CL, 1, 1), kSelThreads threads, kSelSmemBytes dynamic shared memory.
+template <int CL>
+__global__ void __launch_bounds__(kSelThreads, 2) select_cluster_kernel(const SelectArgs a) {
+  extern __shared__ __align__(16) uint8_t sel_dsm[];
+  SelSmem& sm = *reinterpret_cast<SelSmem*>(sel_dsm);
+  using Scan = cub::BlockScan<uint32_t, kSelThreads>;
+  const uint32_t rank = cluster_rank();
   const int b = blockIdx.y;
-  const int64_t j0 = (int64_t)blockIdx.x * kTkTile;
-  const uint32_t T = st[b].thresh;
-  const uint32_t* ub = u + (int64_t)b * n;
+  const int tid = threadIdx.x;
+  const int64_t n = a.n_mid;
+  const int64_t per = ((n + CL - 1) / CL + 3) & ~(int64_t)3;   // a multiple of 4: 16-byte key groups
+  const int64_t j0 = min(n, (int64_t)rank * per);
+  const int nloc = (int)(min(n, j0 + per) - j0);
+  // key of position j0 + t at ub[t]; the global scratch gives every CTA `per` slots
+  uint32_t* ub = per <= kSelUCap ? sm.ucache : a.u + ((int64_t)b * CL + rank) * per;
+  const int eps = a.eps;
+
+  // ---- s', order keys and the level-0 histogram; the next tile's scores load while
+  //      this tile is pooled
+  for (int t = tid; t < kSelBins; t += kSelThreads) sm.hist[t] = 0;
+  const int n_tiles = (nloc + kSelTile - 1) / kSelTile;
+  float v[kSelSlots];
+  if (n_tiles > 0) sel_load_tile(a, b, j0, min(nloc, kSelTile), v);
+  for (int tile = 0; tile < n_tiles; ++tile) {
+    const int t0 = tile * kSelTile;
+    const int nt = min(kSelTile, nloc - t0);
+#pragma unroll
+    for (int e = 0; e < kSelSlots; ++e) {
+      const int t = tid + e * kSelThreads;
+      if (t < kSelHaloTile) sm.sv[t] = v[e];
+    }
+    __syncthreads();
+    if (tile + 1 < n_tiles) sel_load_tile(a, b, j0 + t0 + kSelTile, min(kSelTile, nloc - t0 - kSelTile), v);
+    // four consecutive positions per thread; with eps <= 6 the window of all four is one
+    // run of 16 values read as four 16-byte loads
+    for (int t = 4 * tid; t < nt; t += 4 * kSelThreads) {
+      float mq[4];
+      if (eps <= 6) {
+        float w[16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float4 x = *reinterpret_cast<const float4*>(&sm.sv[t + 4 * c]);
+          w[4 * c] = x.x; w[4 * c + 1] = x.y; w[4 * c + 2] = x.z; w[4 * c + 3] = x.w;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          mq[q] = w[q];
+#pragma unroll
+          for (int o = 1; o <= 12; ++o)
+            if (o <= 2 * eps) mq[q] = fmaxf(mq[q], w[q + o]);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float m = sm.sv[t + q];
+          for (int o = 1; o <= 2 * eps; ++o) m = fmaxf(m, sm.sv[t + q + o]);
+          mq[q] = m;
+        }
+      }
+      uint4 k4;
+      k4.x = order_key(mq[0]); k4.y = order_key(mq[1]); k4.z = order_key(mq[2]); k4.w = order_key(mq[3]);
+      *reinterpret_cast<uint4*>(&ub[t0 + t]) = k4;   // slots past nt hold junk that is never read as a key
+      const uint32_t kq[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (t + q < nt) {
+          if (a.s_prime_out) a.s_prime_out[(int64_t)b * n + j0 + t0 + t + q] = mq[q];
+          atomicAdd(&sm.hist[kq[q] >> 21], 1u);
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---- three radix levels, histograms merged across the cluster
+  uint32_t prefix = 0, want = (uint32_t)a.kk;
+  for (int level = 0; level < 3; ++level) {
+    const int bits = level == 2 ? 10 : 11;
+    const int nb = 1 << bits;
+    if (level > 0) {
+      const int shift = level == 1 ? 10 : 0;
+      const int hi_shift = level == 1 ? 21 : 10;
+      for (int t = tid; t < nb; t += kSelThreads) sm.hist[t] = 0;
+      __syncthreads();
+      for (int t = 4 * tid; t < nloc; t += 4 * kSelThreads) {
+        const uint4 k4 = *reinterpret_cast<const uint4*>(&ub[t]);
+        const uint32_t kq[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (t + q < nloc && (kq[q] >> hi_shift) == prefix)
+            atomicAdd(&sm.hist[(kq[q] >> shift) & (uint32_t)(nb - 1)], 1u);
+      }
+    }
+    cluster_sync_all();                    // every CTA's histogram is complete
+    // reduce-scatter: this CTA sums bin slice `rank` over the cluster (all loads first)
+    const int slice = nb / CL;
+    if (tid < slice / 4) {
+      const uint32_t local = smem_u32(&sm.hist[(int)rank * slice + tid * 4]);
+      uint4 acc = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int r0 = 0; r0 < CL; r0 += 8) {   // eight remote loads in flight at a time
+        uint4 x[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) x[r] = ld_dsmem_u4(dsmem_map(local, (uint32_t)(r0 + r)));
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          acc.x += x[r].x;
+          acc.y += x[r].y;
+          acc.z += x[r].z;
+          acc.w += x[r].w;
+        }
+      }
+      *reinterpret_cast<uint4*>(&sm.mrg[(int)rank * slice + tid * 4]) = acc;
+    }
+    cluster_sync_all();                    // every merged slice is complete
+    for (int t = tid * 4; t < nb; t += kSelThreads * 4) {
+      const uint4 x = ld_dsmem_u4(dsmem_map(smem_u32(&sm.mrg[t]), (uint32_t)(t / slice)));
+      *reinterpret_cast<uint4*>(&sm.full[t]) = x;
+    }
+    __syncthreads();
+    // thread tid owns the bins of descending rank tid * per_t + q
+    const int per_t = nb / kSelThreads;
+    uint32_t c[kSelBins / kSelThreads];
+    uint32_t sum = 0;
+#pragma unroll
+    for (int q = 0; q < kSelBins / kSelThreads; ++q) {
+      c[q] = q < per_t ? sm.full[nb - 1 - (tid * per_t + q)] : 0u;
+      sum += c[q];
+    }
+    uint32_t before;
+    Scan(sm.scan).ExclusiveSum(sum, before);
+    uint32_t acc = before;
+#pragma unroll
+    for (int q = 0; q < kSelBins / kSelThreads; ++q) {
+      if (q < per_t && acc < want && acc + c[q] >= want) {
+        sm.sel_bin = (uint32_t)(nb - 1 - (tid * per_t + q));
+        sm.sel_above = acc;
+      }
+      acc += c[q];
+    }
+    __syncthreads();
+    prefix = (prefix << bits) | sm.sel_bin;
+    want -= sm.sel_above;
+    __syncthreads();
+  }
+  const uint32_t T = prefix;
+
+  // ---- ordered compaction: keep key > T, and key == T while fewer than `want` equal
+  //      keys at lower positions were kept. Thread tid owns the contiguous run
+  //      [tid * R, tid * R + R) of this CTA's positions; R is 4 x an odd number, so the
+  //      16-byte loads of a quarter-warp fall in distinct bank groups.
+  const int R = 4 * ((((nloc + kSelThreads - 1) / kSelThreads + 3) / 4) | 1);
+  const int r0 = min(nloc, tid * R), r1 = min(nloc, r0 + R);
   uint32_t gt = 0, eq = 0;
-  for (int t = threadIdx.x; t < kTkTile; t += kTkThreads) {
-    const int64_t j = j0 + t;
-    if (j >= n) break;
-    const uint32_t key = ub[j];
-    gt += key > T;
-    eq += key == T;
+  for (int t = r0; t < r1; t += 4) {
+    const uint4 k4 = *reinterpret_cast<const uint4*>(&ub[t]);
+    const uint32_t kq[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (t + q < r1) {
+        gt += kq[q] > T;
+        eq += kq[q] == T;
+      }
+    }
   }
-  gt = Red(t1).Sum(gt);
-  eq = Red(t2).Sum(eq);
-  if (threadIdx.x == 0) tile_counts[(int64_t)b * n_tiles + blockIdx.x] = make_uint2(gt, eq);
-}
-
-// Ordered compaction: keep key > T, and key == T while fewer than `want` equal keys
-// at lower positions were kept. Writes positions mid0 + j ascending.
-__global__ void __launch_bounds__(kTkThreads) compact_write_kernel(const uint32_t* __restrict__ u, int64_t n,
-                                                                  const SelState* __restrict__ st,
-                                                                  const uint2* __restrict__ tile_counts, int n_tiles,
-                                                                  int64_t mid0, int topk, int32_t* __restrict__ idx) {
-  using Scan = cub::BlockScan<uint32_t, kTkThreads>;
-  __shared__ typename Scan::TempStorage t1, t2;
-  __shared__ uint32_t base_gt, base_eq;
-  const int b = blockIdx.y;
-  const int64_t j0 = (int64_t)blockIdx.x * kTkTile;
-  const uint32_t T = st[b].thresh;
-  const uint32_t want = st[b].want;
-  if (threadIdx.x < 32) {
-    uint32_t g = 0, e = 0;
-    for (int t = threadIdx.x; t < blockIdx.x; t += 32) {
-      const uint2 c = tile_counts[(int64_t)b * n_tiles + t];
-      g += c.x;
-      e += c.y;
+  uint32_t eq_before, eq_total, gt_before, gt_total;
+  Scan(sm.scan).ExclusiveSum(eq, eq_before, eq_total);
+  __syncthreads();
+  Scan(sm.scan).ExclusiveSum(gt, gt_before, gt_total);
+  if (tid == 0) { sm.cnt[0] = gt_total; sm.cnt[1] = eq_total; }
+  cluster_sync_all();                      // every CTA's counts are complete
+  if (tid < 32) {
+    uint32_t bg = 0, be = 0;
+    if ((uint32_t)tid < rank) {
+      bg = ld_dsmem_u32(dsmem_map(smem_u32(&sm.cnt[0]), (uint32_t)tid));
+      be = ld_dsmem_u32(dsmem_map(smem_u32(&sm.cnt[1]), (uint32_t)tid));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      g += __shfl_xor_sync(0xffffffffu, g, o);
-      e += __shfl_xor_sync(0xffffffffu, e, o);
+      bg += __shfl_xor_sync(0xffffffffu, bg, o);
+      be += __shfl_xor_sync(0xffffffffu, be, o);
     }
-    if (threadIdx.x == 0) { base_gt = g; base_eq = e; }
+    if (tid == 0) { sm.sel_bin = bg; sm.sel_above = be; }
   }
-  __syncthreads();
-  // 4 consecutive elements per thread keep index order within the tile
-  uint32_t key[4];
-  uint32_t eq_cnt = 0;
-  const uint32_t* ub = u + (int64_t)b * n;
+  cluster_sync_all();                      // no CTA leaves while another reads its counts
+  const uint32_t base_gt = sm.sel_bin, base_eq = sm.sel_above;
+  uint32_t eq_run = base_eq + eq_before;
+  uint32_t keep_n = 0;
+  for (int t = r0; t < r1; t += 4) {
+    const uint4 k4 = *reinterpret_cast<const uint4*>(&ub[t]);
+    const uint32_t kq[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int64_t j = j0 + threadIdx.x * 4 + q;
-    key[q] = j < n ? ub[j] : 0u;
-    if (j < n && key[q] == T) ++eq_cnt;
-  }
-  uint32_t eq_before;
-  Scan(t1).ExclusiveSum(eq_cnt, eq_before);
-  eq_before += base_eq;
-  bool keep[4];
-  uint32_t keep_cnt = 0;
-  uint32_t eq_run = eq_before;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int64_t j = j0 + threadIdx.x * 4 + q;
-    keep[q] = false;
-    if (j < n) {
-      if (key[q] > T) keep[q] = true;
-      else if (key[q] == T) { keep[q] = eq_run < want; ++eq_run; }
+    for (int q = 0; q < 4; ++q) {
+      if (t + q >= r1) break;
+      if (kq[q] > T) ++keep_n;
+      else if (kq[q] == T) { keep_n += eq_run < want; ++eq_run; }
     }
-    keep_cnt += keep[q];
   }
   uint32_t pos;
-  Scan(t2).ExclusiveSum(keep_cnt, pos);
+  Scan(sm.scan).ExclusiveSum(keep_n, pos);
   pos += base_gt + min(base_eq, want);
+  eq_run = base_eq + eq_before;
+  int32_t* out = a.idx + (int64_t)b * a.topk;
+  for (int t = r0; t < r1; t += 4) {
+    const uint4 k4 = *reinterpret_cast<const uint4*>(&ub[t]);
+    const uint32_t kq[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    if (keep[q]) {
-      if (pos < (uint32_t)topk) idx[(int64_t)b * topk + pos] = (int32_t)(mid0 + j0 + threadIdx.x * 4 + q);
-      ++pos;
+    for (int q = 0; q < 4; ++q) {
+      if (t + q >= r1) break;
+      bool keep = kq[q] > T;
+      if (kq[q] == T) { keep = eq_run < want; ++eq_run; }
+      if (keep) {
+        if (pos < (uint32_t)a.topk) out[pos] = (int32_t)(a.mid0 + j0 + t + q);
+        ++pos;
+      }
     }
+  }
+  if (rank == 0) {
+    for (int t = a.kk + tid; t < a.topk; t += kSelThreads) out[t] = -1;
+    if (tid == 0) a.count[b] = a.kk;
   }
 }
 

@@ -153,6 +153,8 @@ def _selection_case(batch, lq, n_cap, c0, dc, p, seed, planted=False):
     (1, 64, 4096, 4032, 128, 128, 512, 1024, 2, 45.25),    # prefill-like chunk (tiled path)
     (2, 130, 3000, 2870, 48, 16, 300, 200, 3, 8.0),        # ragged chunk, d' = 48
     (1, 512, 9000, 8488, 128, 128, 1024, 2048, 2, 45.25),  # a full 512-query chunk
+    (1, 1, 300000, 299999, 16, 16, 256, 2048, 2, 16.0),    # > 16K positions per cluster CTA: keys in scratch
+    (2, 1, 40, 39, 16, 4, 28, 3, 2, 4.0),                  # 7-token middle: most cluster CTAs own nothing
 ])
 def test_score_select_parity(batch, lq, n_cap, c0, dc, n_init, window, topk, eps, clamp):
     p = qas.params(n_init, window, topk, eps, clamp)
