@@ -20,8 +20,8 @@
 // P is rounded to bf16 for the second product and the row sums add the rounded values.
 // The online softmax runs in base 2 on the S fragments (4 lanes per row); O is rescaled
 // only when a row maximum moves. Warps are merged by log-sum-exp at the end; with
-// several CTAs per sequence (key splits) the partial (o, m, l) rows go to a workspace
-// and attn_combine_kernel merges them.
+// several CTAs per sequence (key splits) each CTA writes its partial (o, m, l) rows to a
+// workspace and counts itself in, and the last CTA of the sequence merges the splits.
 #pragma once
 #include "common.cuh"
 #include "keylist.cuh"
@@ -40,6 +40,7 @@ __host__ __device__ constexpr int dec_operand_bytes(int hkv) {
   return (kDecStageRowsBytes / (hkv * kDecD * 2)) * (hkv * kDecD * 2 + 16);
 }
 constexpr int kDecOperandMax = dec_operand_bytes(1);  // 128 rows of 272 bytes = 34816
+constexpr int kDecPartStride = kDecD + 4;             // partial row: o, m, l, 2 pad (16-byte rows)
 constexpr int kDecSmemBytes = 2 * kDecStages * kDecOperandMax + kDecMaxSplitKeys * 4 + 256;
 
 struct DecodeAttnArgs {
@@ -48,7 +49,8 @@ struct DecodeAttnArgs {
   const __nv_bfloat16* v;
   __nv_bfloat16* o;         // [B, 1, Hq, 128]
   float* lse;               // [B, 1, Hq] or null
-  float* part;              // [B, Hq, nsplit, 130] when nsplit > 1
+  float* part;              // [B, Hq, nsplit, kDecPartStride] when nsplit > 1: o[128], m, l
+  int* arrive;              // [B] zeroed split counters when nsplit > 1
   KeyList keys;
   int64_t n_cap, c0;
   int hq, hkv, nsplit;
@@ -282,8 +284,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const Decod
     }
     return;
   }
-  // per-warp state to shared memory: red[warp][row][0..127 o, 128 m, 129 l]
   float* red = reinterpret_cast<float*>(stage0_ptr);
+  if (hkv == kDecWarps && a.nsplit > 1) {
+    // one warp per KV head: its rows are this CTA's partial rows as they stand
+    if (gid < G) {
+      float* pp = a.part + (((int64_t)b * a.hq + g * G + gid) * a.nsplit + split) * kDecPartStride;
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt)
+        *reinterpret_cast<float2*>(pp + nt * 8 + 2 * tig) = make_float2(acc[nt][0], acc[nt][1]);
+      if (tig == 0) *reinterpret_cast<float2*>(pp + kDecD) = make_float2(m, l);
+    }
+  } else {
+  // per-warp state to shared memory: red[warp][row][0..127 o, 128 m, 129 l]
   if (gid < G) {
     float* r = red + (warp * G + gid) * (kDecD + 2);
 #pragma unroll
@@ -314,11 +326,95 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const Decod
       a.o[row * kDecD + e] = __float2bfloat16_rn(O / L);
       if (e == 0 && a.lse) a.lse[row] = (M + __log2f(L)) * 0.69314718055994531f;
     } else {
-      float* pp = a.part + (row * a.nsplit + split) * (kDecD + 2);
+      float* pp = a.part + (row * a.nsplit + split) * kDecPartStride;
       pp[e] = O;
       if (e == 0) { pp[kDecD] = M; pp[kDecD + 1] = L; }
     }
   }
+  }
+  if (a.nsplit == 1) return;
+
+  // ---- the last CTA of the sequence to finish merges the splits by log-sum-exp
+  __threadfence();                 // this CTA's partial rows are visible before it counts itself in
+  __syncthreads();
+  if (threadIdx.x == 0) sm.done[0] = atomicAdd(&a.arrive[b], 1) == a.nsplit - 1;
+  __syncthreads();
+  if (!sm.done[0]) return;
+  __threadfence();
+  const int ns = a.nsplit;
+  float* coef = red;               // [Hq][nsplit] merge weights 2^(m - M) / L
+  float* lse2 = red + a.hq * ns;   // [Hq] log-sum-exp, base 2
+  float* ml = lse2 + a.hq;         // [Hq][nsplit] (m, l) pairs
+  const float* pb = a.part + (int64_t)b * a.hq * ns * kDecPartStride;
+  for (int i = threadIdx.x; i < a.hq * ns; i += kDecThreads) {
+    const float2 x = __ldcg(reinterpret_cast<const float2*>(pb + (int64_t)i * kDecPartStride + kDecD));
+    ml[2 * i] = x.x;
+    ml[2 * i + 1] = x.y;
+  }
+  __syncthreads();
+  for (int head = threadIdx.x; head < a.hq; head += kDecThreads) {
+    float M = -INFINITY;
+    for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, ml[2 * (head * ns + sp)]);
+    const float Mr = M == -INFINITY ? 0.f : M;
+    float L = 0.f;
+    for (int sp = 0; sp < ns; ++sp) {
+      const float w = fast_exp2(ml[2 * (head * ns + sp)] - Mr);
+      coef[head * ns + sp] = w;
+      L += ml[2 * (head * ns + sp) + 1] * w;
+    }
+    const float inv = 1.f / L;
+    for (int sp = 0; sp < ns; ++sp) coef[head * ns + sp] *= inv;
+    lse2[head] = M + __log2f(L);
+  }
+  __syncthreads();
+  // thread t takes the (head, 4 dims) items t, t + 256, ...: with Hq <= 32 at most four,
+  // whose loads for eight splits are all in flight in each round
+  constexpr int kItems = 32 * (kDecD / 4) / kDecThreads;   // 4
+  const int n_items = a.hq * (kDecD / 4);
+  float4 res[kItems];
+#pragma unroll
+  for (int u = 0; u < kItems; ++u) res[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int sp0 = 0; sp0 < ns; sp0 += 8) {
+    float4 x[kItems][8];
+#pragma unroll
+    for (int u = 0; u < kItems; ++u) {
+      const int it = threadIdx.x + u * kDecThreads;
+      const int head = it / (kDecD / 4), d4 = (it % (kDecD / 4)) * 4;
+      const float* base = pb + (int64_t)head * ns * kDecPartStride + d4;
+#pragma unroll
+      for (int w = 0; w < 8; ++w)
+        x[u][w] = (it < n_items && sp0 + w < ns)
+                      ? __ldcg(reinterpret_cast<const float4*>(base + (int64_t)(sp0 + w) * kDecPartStride))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kItems; ++u) {
+      const int it = threadIdx.x + u * kDecThreads;
+      const int head = it < n_items ? it / (kDecD / 4) : 0;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        const float c = (it < n_items && sp0 + w < ns) ? coef[head * ns + sp0 + w] : 0.f;
+        res[u].x = fmaf(c, x[u][w].x, res[u].x);
+        res[u].y = fmaf(c, x[u][w].y, res[u].y);
+        res[u].z = fmaf(c, x[u][w].z, res[u].z);
+        res[u].w = fmaf(c, x[u][w].w, res[u].w);
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kItems; ++u) {
+    const int it = threadIdx.x + u * kDecThreads;
+    if (it >= n_items) break;
+    const int head = it / (kDecD / 4), d4 = (it % (kDecD / 4)) * 4;
+    const int64_t row = (int64_t)b * a.hq + head;
+    __nv_bfloat162 lo2 = __floats2bfloat162_rn(res[u].x, res[u].y), hi2 = __floats2bfloat162_rn(res[u].z, res[u].w);
+    uint2 packed;
+    packed.x = *reinterpret_cast<uint32_t*>(&lo2);
+    packed.y = *reinterpret_cast<uint32_t*>(&hi2);
+    *reinterpret_cast<uint2*>(a.o + row * kDecD + d4) = packed;
+    if (d4 == 0 && a.lse) a.lse[row] = lse2[head] * 0.69314718055994531f;
+  }
+  if (threadIdx.x == 0) a.arrive[b] = 0;
 }
 
 }  // namespace esa

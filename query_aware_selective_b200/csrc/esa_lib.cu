@@ -240,13 +240,26 @@ esa_status_t make_tmap_f32(CUtensorMap* m, const float* base, uint64_t rows, uin
 template <int DC>
 void launch_score_small(const float* q_c, const float* k_c, int lq, int64_t n_cap, int64_t mid0, int64_t n_mid,
                         int batch, float* S, uint32_t* m_key, cudaStream_t s) {
-  const int64_t keys_per_cta = 512;
-  dim3 grid((unsigned)cdiv(n_mid, keys_per_cta), batch);
+  // one wave of two CTAs per SM over all sequences, each CTA a multiple of a stage
+  constexpr int64_t ks = esa::SmallScoreShape<DC>::KS;
+  const int64_t per_seq = std::max<int64_t>(1, std::min<int64_t>(cdiv(n_mid, ks), (2 * 148) / batch));
+  const int64_t keys_per_cta = cdiv(cdiv(n_mid, per_seq), ks) * ks;
+  const dim3 grid((unsigned)cdiv(n_mid, keys_per_cta), batch);
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev < 64 && !attr_set[dev]) {
+    cudaFuncSetAttribute(esa::score_small_kernel<DC, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         esa::kSsSmemBytes);
+    cudaFuncSetAttribute(esa::score_small_kernel<DC, esa::kScoreSmallLq>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, esa::kSsSmemBytes);
+    attr_set[dev] = true;
+  }
   if (lq == 1)
-    esa::score_small_kernel<DC, 1><<<grid, 256, 0, s>>>(q_c, k_c, lq, n_cap, mid0, n_mid, keys_per_cta, S, m_key);
+    esa::score_small_kernel<DC, 1><<<grid, esa::kSsThreads, esa::kSsSmemBytes, s>>>(q_c, k_c, lq, n_cap, mid0, n_mid,
+                                                                                    keys_per_cta, S, m_key);
   else
-    esa::score_small_kernel<DC, esa::kScoreSmallLq><<<grid, 256, 0, s>>>(q_c, k_c, lq, n_cap, mid0, n_mid,
-                                                                         keys_per_cta, S, m_key);
+    esa::score_small_kernel<DC, esa::kScoreSmallLq><<<grid, esa::kSsThreads, esa::kSsSmemBytes, s>>>(
+        q_c, k_c, lq, n_cap, mid0, n_mid, keys_per_cta, S, m_key);
 }
 
 }  // namespace
@@ -626,7 +639,15 @@ AttnPlan plan_attn(int32_t batch, int32_t lq, int64_t c0, int32_t hq, int32_t hk
     nsp = std::max(nsp, cdiv(n_keys_max, esa::kDecMaxSplitKeys));   // positions fit in shared memory
     pl.keys_per_split = cdiv(cdiv(n_keys_max, nsp), ks) * ks;
     pl.nsplit = (int)cdiv(n_keys_max, pl.keys_per_split);
-    pl.ws_bytes = pl.nsplit > 1 ? up256((size_t)batch * hq * pl.nsplit * (head_dim + 2) * sizeof(float)) : 0;
+    // the last CTA of a sequence merges its splits in the freed stage ring: 3 floats per
+    // (head, split) must fit in it
+    if ((int64_t)hq * pl.nsplit * 3 * 4 > 2 * esa::kDecStages * esa::dec_operand_bytes(8)) pl.dec = false;
+  }
+  if (pl.dec) {
+    // [B] arrival counters, then the split partials
+    pl.ws_bytes = pl.nsplit > 1 ? up256((size_t)batch * sizeof(int)) +
+                                      up256((size_t)batch * hq * pl.nsplit * esa::kDecPartStride * sizeof(float))
+                                : 0;
     return pl;
   }
   const int64_t base = (int64_t)batch * lq * hkv;
@@ -757,7 +778,11 @@ esa_status_t esa_sparse_attn(const void* q, const void* k, const void* v, esa_dt
     d.v = static_cast<const __nv_bfloat16*>(v);
     d.o = static_cast<__nv_bfloat16*>(o);
     d.lse = lse;
-    d.part = static_cast<float*>(workspace);
+    if (pl.nsplit > 1) {
+      d.arrive = static_cast<int*>(workspace);
+      d.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + up256((size_t)batch * sizeof(int)));
+      ESA_CUDA(cudaMemsetAsync(d.arrive, 0, (size_t)batch * sizeof(int), s));
+    }
     d.keys = keys;
     d.n_cap = n_cap;
     d.c0 = c0;
@@ -771,12 +796,6 @@ esa_status_t esa_sparse_attn(const void* q, const void* k, const void* v, esa_dt
     else if (g == 2) esa::attn_decode_kernel<2><<<grid, esa::kDecThreads, esa::kDecSmemBytes, s>>>(d);
     else esa::attn_decode_kernel<4><<<grid, esa::kDecThreads, esa::kDecSmemBytes, s>>>(d);
     ESA_LAUNCH_CHECK("attn_decode_kernel");
-    if (pl.nsplit > 1) {
-      const int64_t rows = (int64_t)batch * hq;
-      esa::attn_combine_kernel<__nv_bfloat16, 128><<<dim3((unsigned)cdiv(rows, 8)), 256, 0, s>>>(
-          d.part, rows, pl.nsplit, static_cast<__nv_bfloat16*>(o), lse);
-      ESA_LAUNCH_CHECK("attn_combine_kernel");
-    }
     return ok();
   }
   esa::SimtAttnArgs a{};

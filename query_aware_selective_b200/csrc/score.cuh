@@ -15,29 +15,84 @@
 namespace esa {
 
 // ------------------------------------------------------------ few queries (decode) --
-// One group of LPK lanes holds one key (VPL floats per lane); a warp covers KPW keys
-// per step and UNR steps per iteration. Lq <= kScoreSmallLq queries live in registers.
+// HBM-bound stream over the compressed keys of the middle. A CTA owns a contiguous run
+// of keys and moves it into shared memory with one bulk copy (cp.async.bulk, mbarrier
+// completion) per stage of kSsStageBytes, through a ring of kSsStages stages; the last
+// of the eight warps to finish a stage issues its refill. In a stage, a group of LPK
+// lanes holds one key (VPL floats per lane, 16-byte shared loads) and a warp covers KPW
+// keys per step. Lq <= kScoreSmallLq queries live in registers.
 constexpr int kScoreSmallLq = 8;
+constexpr int kSsWarps = 8;
+constexpr int kSsThreads = kSsWarps * 32;
+constexpr int kSsStageBytes = 32768;
+constexpr int kSsStages = 3;
+constexpr int kSsSmemBytes = kSsStages * kSsStageBytes + 128 + 64;
 
 template <int DC>
 struct SmallScoreShape {
   static constexpr int VPL = DC >= 128 ? DC / 32 : 4;
   static constexpr int LPK = DC / VPL;
   static constexpr int KPW = 32 / LPK;
+  static constexpr int KS = kSsStageBytes / (DC * 4);     // keys per stage
 };
 
+struct SsSmem {
+  uint64_t full[kSsStages];
+  int done[kSsStages];
+  int abort_flag;
+  int issued;
+};
+
+// grid (ctas per sequence, B); kSsThreads threads; kSsSmemBytes dynamic shared memory.
+// CTA c scores keys [c * keys_per_cta, ...) of the middle (keys_per_cta a multiple of KS).
 template <int DC, int LQ>
-__global__ void __launch_bounds__(256) score_small_kernel(const float* __restrict__ q_c, const float* __restrict__ k_c,
-                                                          int lq, int64_t n_cap, int64_t mid0, int64_t n_mid,
-                                                          int64_t keys_per_cta, float* __restrict__ s_out,
-                                                          uint32_t* __restrict__ m_key) {
+__global__ void __launch_bounds__(kSsThreads, 2) score_small_kernel(const float* __restrict__ q_c,
+                                                                   const float* __restrict__ k_c, int lq,
+                                                                   int64_t n_cap, int64_t mid0, int64_t n_mid,
+                                                                   int64_t keys_per_cta, float* __restrict__ s_out,
+                                                                   uint32_t* __restrict__ m_key) {
   using Sh = SmallScoreShape<DC>;
-  constexpr int VPL = Sh::VPL, LPK = Sh::LPK, KPW = Sh::KPW;
-  constexpr int UNR = 4;
+  constexpr int VPL = Sh::VPL, LPK = Sh::LPK, KPW = Sh::KPW, KS = Sh::KS;
+  constexpr int KEYS_PER_WARP = KS / kSsWarps;             // of a stage
+  extern __shared__ __align__(128) uint8_t ss_dsm[];
+  const uint32_t stage0 = (smem_u32(ss_dsm) + 127u) & ~127u;
+  uint8_t* const stage0_ptr = ss_dsm + (stage0 - smem_u32(ss_dsm));
+  SsSmem& sm = *reinterpret_cast<SsSmem*>(stage0_ptr + kSsStages * kSsStageBytes);
   const int b = blockIdx.y;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int grp = lane / LPK, sub = lane % LPK;
+  const int64_t j_begin = (int64_t)blockIdx.x * keys_per_cta;
+  const int64_t j_end = min(n_mid, j_begin + keys_per_cta);
+  const int nst = j_end > j_begin ? (int)((j_end - j_begin + KS - 1) / KS) : 0;
   const float* kb = k_c + ((int64_t)b * n_cap + mid0) * DC;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSsStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      sm.done[s] = 0;
+    }
+    sm.abort_flag = 0;
+    sm.issued = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  volatile int* abort_flag = &sm.abort_flag;
+  // stage j: keys [j_begin + j KS, ...) as one contiguous copy
+  auto issue = [&](int j) {
+    const int s = j % kSsStages;
+    const int64_t k0 = j_begin + (int64_t)j * KS;
+    const int n_in = (int)(j_end - k0 < KS ? j_end - k0 : KS);
+    const uint32_t bytes = (uint32_t)(n_in * DC * 4);
+    mbar_arrive_expect_tx(&sm.full[s], bytes);
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     stage0 + s * kSsStageBytes),
+                 "l"(kb + k0 * DC), "r"(bytes), "r"(smem_u32(&sm.full[s]))
+                 : "memory");
+    atomicMax(&sm.issued, j + 1);
+  };
+  if (threadIdx.x == 0)
+    for (int j = 0; j < min(nst, kSsStages); ++j) issue(j);
+
   float q[LQ][VPL];
 #pragma unroll
   for (int i = 0; i < LQ; ++i)
@@ -50,42 +105,60 @@ __global__ void __launch_bounds__(256) score_small_kernel(const float* __restric
 #pragma unroll
   for (int i = 0; i < LQ; ++i) mx[i] = -INFINITY;
 
-  const int64_t j_begin = (int64_t)blockIdx.x * keys_per_cta;
-  const int64_t j_end = min(n_mid, j_begin + keys_per_cta);
-  for (int64_t jb = j_begin + (int64_t)warp * KPW * UNR; jb < j_end; jb += (int64_t)nwarp * KPW * UNR) {
-    float kv[UNR][VPL];
+  for (int j = 0; j < nst; ++j) {
+    const int s = j % kSsStages;
+    if (!mbar_wait_warp(&sm.full[s], (j / kSsStages) & 1, abort_flag, 401)) break;
+    const int64_t k0 = j_begin + (int64_t)j * KS;
+    const float* st = reinterpret_cast<const float*>(stage0_ptr + s * kSsStageBytes);
 #pragma unroll
-    for (int u = 0; u < UNR; ++u) {
-      const int64_t j = jb + u * KPW + grp;
-      if (j < j_end) {
+    for (int r = 0; r < KEYS_PER_WARP; r += KPW) {
+      const int kk = warp * KEYS_PER_WARP + r + grp;      // key within the stage
+      const int64_t jj = k0 + kk;
+      float kv[VPL];
 #pragma unroll
-        for (int v = 0; v < VPL; v += 4) {
-          uint4 raw = ld_stream16(kb + j * DC + sub * VPL + v);
-          widen(raw, (const float*)nullptr, &kv[u][v]);
-        }
-      } else {
-#pragma unroll
-        for (int v = 0; v < VPL; ++v) kv[u][v] = 0.f;
+      for (int v = 0; v < VPL; v += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(st + kk * DC + sub * VPL + v);
+        kv[v] = x.x; kv[v + 1] = x.y; kv[v + 2] = x.z; kv[v + 3] = x.w;
       }
-    }
-#pragma unroll
-    for (int u = 0; u < UNR; ++u) {
-      const int64_t j = jb + u * KPW + grp;
 #pragma unroll
       for (int i = 0; i < LQ; ++i) {
         float acc = 0.f;
 #pragma unroll
-        for (int v = 0; v < VPL; ++v) acc = fmaf(q[i][v], kv[u][v], acc);
+        for (int v = 0; v < VPL; ++v) acc = fmaf(q[i][v], kv[v], acc);
 #pragma unroll
         for (int o = LPK / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (j < j_end && i < lq) {
+        if (jj < j_end && i < lq) {
           mx[i] = fmaxf(mx[i], acc);
-          if (sub == 0) s_out[((int64_t)b * lq + i) * n_mid + j] = acc;
+          if (sub == 0) s_out[((int64_t)b * lq + i) * n_mid + jj] = acc;
+        }
+      }
+    }
+    // release the stage; the last warp out refills it
+    __syncwarp();
+    int prev = 0;
+    if (lane == 0) {
+      __threadfence_block();
+      prev = atomicAdd(&sm.done[s], 1);
+      if (prev == kSsWarps - 1) {
+        sm.done[s] = 0;
+        if (j + kSsStages < nst) {
+          fence_proxy_async();
+          issue(j + kSsStages);
         }
       }
     }
   }
-  __shared__ float red[LQ][32];
+  __syncthreads();
+  if (*abort_flag) {
+    // drain the copies that may still be in flight before the CTA's shared memory goes away
+    if (threadIdx.x == 0) {
+      const int issued = sm.issued;
+      for (int j = max(0, issued - kSsStages); j < issued; ++j)
+        mbar_wait(&sm.full[j % kSsStages], (j / kSsStages) & 1, abort_flag, 402, /*respect_abort=*/false);
+    }
+    return;
+  }
+  __shared__ float red[LQ][kSsWarps];
 #pragma unroll
   for (int i = 0; i < LQ; ++i) {
     float v = warp_max(mx[i]);
@@ -94,7 +167,7 @@ __global__ void __launch_bounds__(256) score_small_kernel(const float* __restric
   __syncthreads();
   if (threadIdx.x < lq) {
     float v = -INFINITY;
-    for (int w = 0; w < nwarp; ++w) v = fmaxf(v, red[threadIdx.x][w]);
+    for (int w = 0; w < kSsWarps; ++w) v = fmaxf(v, red[threadIdx.x][w]);
     if (v > -INFINITY) atomicMax(&m_key[b * lq + threadIdx.x], order_key(v));
   }
 }

@@ -10,13 +10,14 @@
 // CTA r owns a contiguous range of middle positions. Order: s' descending, then
 // position ascending. Exact selection in three radix levels over order-preserving
 // 32-bit keys (11 + 11 + 10 bits). At each level every CTA histograms its keys that
-// still share the threshold's prefix (shared-memory atomics), the cluster merges the
-// histograms through distributed shared memory (reduce-scatter: CTA r sums bin slice r
-// over all CTAs; all-gather: every CTA reads the merged slices), and every CTA finds
-// the same bin holding the want-th largest key. The threshold key T and the number of
-// keys equal to T to keep (lowest positions first) then drive an ordered compaction:
-// the CTAs exchange their (above T, equal to T) counts, and a block scan in position
-// order writes the kept positions ascending, so no sort is needed. Integer atomics
+// still share the threshold's prefix (shared-memory atomics) and adds each non-zero bin
+// into the CTA that owns the bin's slice (distributed shared-memory reductions: CTA r
+// owns slice r); after one cluster barrier every CTA reads the merged bins it scans with
+// 16-byte loads from their owners and finds the same bin holding the want-th largest
+// key. The threshold key T and the number of keys equal to T to keep (lowest positions
+// first) then drive an ordered compaction: every CTA pushes its (above T, equal to T)
+// counts to the higher ranks, and a block scan in position order writes the kept
+// positions ascending, so no sort is needed. Integer atomics
 // only: the result does not depend on scheduling. The keys stay in shared memory when
 // a CTA's range fits (kSelUCap), else in a global scratch array.
 #pragma once
@@ -49,11 +50,10 @@ struct SelectArgs {
 };
 
 struct SelSmem {
-  uint32_t hist[kSelBins];   // this CTA's histogram of the current level
-  uint32_t mrg[kSelBins];    // merged counts of the bin slice this CTA owns
-  uint32_t full[kSelBins];   // the merged histogram, gathered from the cluster
+  uint32_t hist[kSelBins];                 // this CTA's histogram of the current level
+  uint32_t merged[2 * kSelBins + 1024];    // per level: the cluster's counts of the bin slice this CTA owns
   float sv[kSelTile + 2 * kSelMaxEps + 16];   // + slack: the vector pooling reads 16 values per group
-  uint32_t cnt[2];           // keys above T, keys equal to T (this CTA)
+  uint32_t cnt_lo[16][2];                  // (above T, equal to T) of each lower-ranked CTA, pushed by it
   uint32_t sel_bin, sel_above;
   typename cub::BlockScan<uint32_t, kSelThreads>::TempStorage scan;
   uint32_t ucache[kSelUCap];
@@ -120,9 +120,15 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_cluster_kernel(const Se
   uint32_t* ub = per <= kSelUCap ? sm.ucache : a.u + ((int64_t)b * CL + rank) * per;
   const int eps = a.eps;
 
+  // every CTA clears its merged slices; the barrier phase this arrival opens is waited
+  // for only after the pooling pass below
+  for (int t = tid; t < 2 * kSelBins + 1024; t += kSelThreads) sm.merged[t] = 0;
+  cluster_arrive();
+
   // ---- s', order keys and the level-0 histogram; the next tile's scores load while
   //      this tile is pooled
   for (int t = tid; t < kSelBins; t += kSelThreads) sm.hist[t] = 0;
+  __syncthreads();
   const int n_tiles = (nloc + kSelTile - 1) / kSelTile;
   float v[kSelSlots];
   if (n_tiles > 0) sel_load_tile(a, b, j0, min(nloc, kSelTile), v);
@@ -140,7 +146,16 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_cluster_kernel(const Se
     // run of 16 values read as four 16-byte loads
     for (int t = 4 * tid; t < nt; t += 4 * kSelThreads) {
       float mq[4];
-      if (eps <= 6) {
+      if (eps == 2) {
+        const float4 x0 = *reinterpret_cast<const float4*>(&sm.sv[t]);
+        const float4 x1 = *reinterpret_cast<const float4*>(&sm.sv[t + 4]);
+        const float m12 = fmaxf(x0.y, x0.z), m23 = fmaxf(x0.z, x0.w), m45 = fmaxf(x1.x, x1.y);
+        const float m34 = fmaxf(x0.w, x1.x), m56 = fmaxf(x1.y, x1.z);
+        mq[0] = fmaxf(fmaxf(x0.x, m12), fmaxf(x0.w, x1.x));
+        mq[1] = fmaxf(fmaxf(m12, m34), x1.y);
+        mq[2] = fmaxf(fmaxf(m23, m45), x1.z);
+        mq[3] = fmaxf(fmaxf(m34, m56), x1.w);
+      } else if (eps <= 6) {
         float w[16];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -177,7 +192,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_cluster_kernel(const Se
     __syncthreads();
   }
 
-  // ---- three radix levels, histograms merged across the cluster
+  // ---- three radix levels, histograms merged slice by slice across the cluster
+  cluster_wait();                          // every CTA's merged slices are cleared
   uint32_t prefix = 0, want = (uint32_t)a.kk;
   for (int level = 0; level < 3; ++level) {
     const int bits = level == 2 ? 10 : 11;
@@ -195,43 +211,34 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_cluster_kernel(const Se
           if (t + q < nloc && (kq[q] >> hi_shift) == prefix)
             atomicAdd(&sm.hist[(kq[q] >> shift) & (uint32_t)(nb - 1)], 1u);
       }
+      __syncthreads();
     }
-    cluster_sync_all();                    // every CTA's histogram is complete
-    // reduce-scatter: this CTA sums bin slice `rank` over the cluster (all loads first)
+    // levels of 2048, 2048 and 1024 bins, one after the other; bin t lives in CTA t / slice
     const int slice = nb / CL;
-    if (tid < slice / 4) {
-      const uint32_t local = smem_u32(&sm.hist[(int)rank * slice + tid * 4]);
-      uint4 acc = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-      for (int r0 = 0; r0 < CL; r0 += 8) {   // eight remote loads in flight at a time
-        uint4 x[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) x[r] = ld_dsmem_u4(dsmem_map(local, (uint32_t)(r0 + r)));
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          acc.x += x[r].x;
-          acc.y += x[r].y;
-          acc.z += x[r].z;
-          acc.w += x[r].w;
-        }
-      }
-      *reinterpret_cast<uint4*>(&sm.mrg[(int)rank * slice + tid * 4]) = acc;
+    const uint32_t merged = smem_u32(&sm.merged[level * kSelBins]);
+    for (int t = tid; t < nb; t += kSelThreads) {
+      const uint32_t c = sm.hist[t];
+      if (c) red_dsmem_add_u32(dsmem_map(merged + 4u * t, (uint32_t)(t / slice)), c);
     }
-    cluster_sync_all();                    // every merged slice is complete
-    for (int t = tid * 4; t < nb; t += kSelThreads * 4) {
-      const uint4 x = ld_dsmem_u4(dsmem_map(smem_u32(&sm.mrg[t]), (uint32_t)(t / slice)));
-      *reinterpret_cast<uint4*>(&sm.full[t]) = x;
-    }
-    __syncthreads();
-    // thread tid owns the bins of descending rank tid * per_t + q
+    cluster_sync_all();                    // every slice holds its merged counts
+    // thread tid owns the bins of descending rank tid * per_t + q, i.e. the per_t
+    // consecutive bins ending at nb - 1 - tid * per_t: one vector load from their owner
     const int per_t = nb / kSelThreads;
     uint32_t c[kSelBins / kSelThreads];
+    {
+      const int lo_bin = nb - per_t * (tid + 1);
+      const uint32_t src = dsmem_map(merged + 4u * lo_bin, (uint32_t)(lo_bin / slice));
+      if (per_t == 4) {
+        const uint4 v4 = ld_dsmem_u4(src);
+        c[0] = v4.w; c[1] = v4.z; c[2] = v4.y; c[3] = v4.x;
+      } else {
+        const uint2 v2 = ld_dsmem_u2(src);
+        c[0] = v2.y; c[1] = v2.x; c[2] = 0u; c[3] = 0u;
+      }
+    }
     uint32_t sum = 0;
 #pragma unroll
-    for (int q = 0; q < kSelBins / kSelThreads; ++q) {
-      c[q] = q < per_t ? sm.full[nb - 1 - (tid * per_t + q)] : 0u;
-      sum += c[q];
-    }
+    for (int q = 0; q < kSelBins / kSelThreads; ++q) sum += c[q];
     uint32_t before;
     Scan(sm.scan).ExclusiveSum(sum, before);
     uint32_t acc = before;
@@ -272,23 +279,19 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_cluster_kernel(const Se
   Scan(sm.scan).ExclusiveSum(eq, eq_before, eq_total);
   __syncthreads();
   Scan(sm.scan).ExclusiveSum(gt, gt_before, gt_total);
-  if (tid == 0) { sm.cnt[0] = gt_total; sm.cnt[1] = eq_total; }
-  cluster_sync_all();                      // every CTA's counts are complete
-  if (tid < 32) {
-    uint32_t bg = 0, be = 0;
-    if ((uint32_t)tid < rank) {
-      bg = ld_dsmem_u32(dsmem_map(smem_u32(&sm.cnt[0]), (uint32_t)tid));
-      be = ld_dsmem_u32(dsmem_map(smem_u32(&sm.cnt[1]), (uint32_t)tid));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      bg += __shfl_xor_sync(0xffffffffu, bg, o);
-      be += __shfl_xor_sync(0xffffffffu, be, o);
-    }
-    if (tid == 0) { sm.sel_bin = bg; sm.sel_above = be; }
+  // push this CTA's totals to every higher rank; after the barrier nothing in the
+  // cluster touches another CTA's shared memory, so each CTA may then finish alone
+  if ((uint32_t)tid > rank && tid < CL) {
+    st_dsmem_u32(dsmem_map(smem_u32(&sm.cnt_lo[rank][0]), (uint32_t)tid), gt_total);
+    st_dsmem_u32(dsmem_map(smem_u32(&sm.cnt_lo[rank][1]), (uint32_t)tid), eq_total);
   }
-  cluster_sync_all();                      // no CTA leaves while another reads its counts
-  const uint32_t base_gt = sm.sel_bin, base_eq = sm.sel_above;
+  cluster_sync_all();
+  uint32_t bg = 0, be = 0;
+  for (uint32_t r = 0; r < rank; ++r) {
+    bg += sm.cnt_lo[r][0];
+    be += sm.cnt_lo[r][1];
+  }
+  const uint32_t base_gt = bg, base_eq = be;
   uint32_t eq_run = base_eq + eq_before;
   uint32_t keep_n = 0;
   for (int t = r0; t < r1; t += 4) {

@@ -177,6 +177,7 @@ class EsaDecode:
         nb = _abi.sparse_attn_workspace_size(batch, 1, c0, hq, hkv, head_dim, code, p)
         self.ws_att = torch.empty(nb + 256, dtype=torch.uint8, device=device) if nb else None
         self.cmp = _Compressor(hq, hkv, head_dim, d_c, dtype, device)
+        self.side = torch.cuda.Stream(device=device)
 
     def fill_cache(self, k, wk, upto: Optional[int] = None):
         """Compress cached keys [0, upto) of every sequence (prefill state)."""
@@ -194,17 +195,23 @@ class EsaDecode:
         unmodified (pointer and version counter); otherwise they are packed again."""
         pos = self.n_ctx - 1
         ev = phase_events
+        cur = torch.cuda.current_stream()
         if ev is not None:
             ev[0].record()
         self.cmp.pack_if_changed(wq, wk)
+        # The new token is in the local window, so this step's scoring never reads its
+        # compressed key: that compression runs beside the query's on a second stream.
+        self.side.wait_stream(cur)
+        with torch.cuda.stream(self.side):
+            self.cmp.keys(k[:, pos], out=self.k_c[:, pos], out_row_stride=self.n_ctx * self.d_c)
         self.cmp.queries(q[:, 0], out=self.q_c.view(self.batch, self.d_c))
-        self.cmp.keys(k[:, pos], out=self.k_c[:, pos], out_row_stride=self.n_ctx * self.d_c)
         if ev is not None:
             ev[1].record()
         _abi.score_select(self.q_c, self.k_c, pos, self.p, idx=self.idx, count=self.count, workspace=self.ws_sel)
         if ev is not None:
             ev[2].record()
         _abi.sparse_attn(q, k, v, pos, self.idx, self.count, self.p, out=self.out, workspace=self.ws_att)
+        cur.wait_stream(self.side)
         if ev is not None:
             ev[3].record()
         return self.out
