@@ -116,15 +116,23 @@ class EsaPrefill:
         self.ws_att = torch.empty(ws_att + 256, dtype=torch.uint8, device=device) if ws_att else None
         self.out_views = []
         self.cmp = _Compressor(hq, hkv, head_dim, d_c, dtype, device)
+        self.side = torch.cuda.Stream(device=device)
 
     def chunks(self):
         return [(c0, min(self.chunk, self.n_ctx - c0)) for c0 in range(0, self.n_ctx, self.chunk)]
 
     def run_chunk(self, c0: int, lq: int, q, k, v, wq, wk, attn_events=None):
         b = self.batch
+        cur = torch.cuda.current_stream()
         self.cmp.pack_if_changed(wq, wk)
+        # The chunk's own keys are local to it (the middle ends `window` tokens before
+        # c0), so its compressed keys are first read by a later chunk's scoring: they
+        # are computed on a second stream beside this chunk's work and joined at the end.
+        self.side.wait_stream(cur)
+        with torch.cuda.stream(self.side):
+            for s in range(b):
+                self.cmp.keys(k[s, c0:c0 + lq], out=self.k_c[s, c0:c0 + lq])
         for s in range(b):
-            self.cmp.keys(k[s, c0:c0 + lq], out=self.k_c[s, c0:c0 + lq])
             self.cmp.queries(q[s, c0:c0 + lq], out=self.q_c[s, :lq])
         q_c = self.q_c[:, :lq] if lq == self.chunk else self.q_c[:, :lq].contiguous()
         _abi.score_select(q_c, self.k_c, c0, self.p, idx=self.idx, count=self.count, workspace=self.ws_sel)
@@ -140,6 +148,7 @@ class EsaPrefill:
             attn_events[1].record()
         if target is not ov:
             ov.copy_(target)
+        cur.wait_stream(self.side)
 
     def run(self, q, k, v, wq, wk, attn_events=None, external_events=False):
         """q [B, N, Hq, D], k, v [B, N, Hkv, D] (device), wq, wk [Hq*D, d'].
