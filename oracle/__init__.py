@@ -13,6 +13,8 @@ can be checked against the pages by eye.
   article, implementation section): compression, importance score, score
   correction, chunk sum, neighbour influence, top-k, attention over
   initial + selected + local tokens.
+* ``oracle.esa_heads`` - the per-head selection variant of ESA (the article's
+  ablation of merged versus per-head importance): one index set per KV head.
 * ``oracle.moba`` - Mixture of Block Attention (MoBA article, sections 1-3):
   block mean pooling, gate, causal top-k, block attention.
 

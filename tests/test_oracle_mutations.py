@@ -10,8 +10,9 @@ import textwrap
 
 import pytest
 
-from oracle import esa, moba
+from oracle import esa, esa_heads, moba
 from tests import test_oracle_esa as pe
+from tests import test_oracle_heads as th
 from tests import test_oracle_moba as pm
 
 MUTATIONS = [
@@ -46,6 +47,14 @@ MUTATIONS = [
      pe.check_attended_count),                                             # window off by one
     (esa, "attended_keys", "np.arange(l0, l1)", "np.arange(l0, l1 - 1)",
      pe.check_full_selection_is_causal_attention),                         # chunk cut short
+    (esa_heads, "compress_heads", "xg = xe[:, g * hpg:(g + 1) * hpg, :].reshape(rows, hpg * d)",
+     "xg = xe[:, :hpg, :].reshape(rows, hpg * d)",
+     th.test_group_maps_equal_the_block_diagonal_merged_map),              # every group reads group 0's heads
+    (esa_heads, "score_select_heads", "cols = slice(g * dg, (g + 1) * dg)",
+     "cols = slice(((g + 1) % n_groups) * dg, ((g + 1) % n_groups + 1) * dg)",
+     th.test_a_needle_seen_by_one_head_is_selected_by_that_head_only),     # another group's slice
+    (esa_heads, "sparse_attn_heads", "idx[b, g], int(count[b, g])", "idx[b, 0], int(count[b, 0])",
+     th.test_each_group_attends_its_own_list),                             # one list for every head
     (moba, "block_means", "k[:, b * block:min((b + 1) * block, s)]", "k[:, b * block:min((b + 1) * block + 1, s)]",
      pm.check_block_means_of_a_ramp),                                      # block boundary
     (moba, "gate", "sc = np.einsum(\"hd,hnd->hn\", q[b, p], kbar[b, :, :cur, :])",
