@@ -48,7 +48,7 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--prefill-ctx", type=int, default=0,
                     help="shorter prefill context (profiling a small case); the line then names that workload")
-    ap.add_argument("--only", choices=["decode", "moba"], default=None,
+    ap.add_argument("--only", choices=["decode", "decode_per_head", "moba"], default=None,
                     help="profiling: run one of the other workloads alone and print its figures")
     ap.add_argument("--decode-batch", type=int, default=0, help="profiling: decode batch (default: the workload's)")
     ap.add_argument("--moba-seq", type=int, default=0, help="profiling: MoBA sequence length (default: the workload's)")
@@ -220,8 +220,10 @@ def run_only(args):
     dev = torch.device("cuda", 0)
     peaks, peak_src = load_peaks()
     flush = make_flush(dev)
-    fn = bench_decode if args.only == "decode" else bench_moba
-    out = fn(args, dev, flush, make_dist_max(), peaks, peak_src, 1)
+    if args.only == "moba":
+        out = bench_moba(args, dev, flush, make_dist_max(), peaks, peak_src, 1)
+    else:
+        out = bench_decode(args, dev, flush, make_dist_max(), peaks, peak_src, 1, per_head=args.only == "decode_per_head")
     print(json.dumps({"only": args.only, **out}), flush=True)
 
 
@@ -329,8 +331,12 @@ def run_ours(args):
     if not args.no_extras:
         del inp, pf, graph
         torch.cuda.empty_cache()
-        line["also"] = {"esa_decode_128k": bench_decode(args, dev, flush, dist_max, peaks, peak_src, world),
-                        "moba_prefill_64k": bench_moba(args, dev, flush, dist_max, peaks, peak_src, world)}
+        line["also"] = {"esa_decode_128k": bench_decode(args, dev, flush, dist_max, peaks, peak_src, world)}
+        torch.cuda.empty_cache()
+        line["also"]["esa_decode_128k_per_head"] = bench_decode(args, dev, flush, dist_max, peaks, peak_src, world,
+                                                                per_head=True)
+        torch.cuda.empty_cache()
+        line["also"]["moba_prefill_64k"] = bench_moba(args, dev, flush, dist_max, peaks, peak_src, world)
     line["clocks"] = sampler.stop()
     line["gpu"] = props.name
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -342,7 +348,9 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
-def bench_decode(args, dev, flush, dist_max, peaks, peak_src, world):
+def bench_decode(args, dev, flush, dist_max, peaks, peak_src, world, per_head=False):
+    """ESA decode at 128K, batch 16. per_head: the per-head selection variant (one
+    index set per KV head, block-diagonal compression maps) on the same inputs."""
     import torch
     import query_aware_selective_b200 as qas
     from query_aware_selective_b200 import cost, pipeline, synthetic
@@ -352,7 +360,10 @@ def bench_decode(args, dev, flush, dist_max, peaks, peak_src, world):
         w = dataclasses.replace(w, batch=args.decode_batch, name=f"esa_decode_llama3_8b_b{args.decode_batch}_ctx{w.n_ctx}")
     p = qas.params(w.n_init, w.window, w.topk, w.eps, w.clamp_c)
     inp = synthetic.make_esa_inputs(w, device=dev)
-    dec = pipeline.EsaDecode(w.batch, w.n_ctx, w.hq, w.hkv, w.head_dim, w.d_c, p, device=dev)
+    if per_head:
+        wq_g, wk_g = synthetic.make_group_maps(w, device=dev)
+        inp["wq"], inp["wk"] = pipeline.block_diagonal(wq_g), pipeline.block_diagonal(wk_g)
+    dec = pipeline.EsaDecode(w.batch, w.n_ctx, w.hq, w.hkv, w.head_dim, w.d_c, p, device=dev, per_head=per_head)
     dec.fill_cache(inp["k"], inp["wk"])
     torch.cuda.synchronize()
     # the headline replays the bare step; the phase split comes from a second graph of the
@@ -372,7 +383,8 @@ def bench_decode(args, dev, flush, dist_max, peaks, peak_src, world):
     step_gbs = by["total"] / (total / steps / 1e3) / 1e9
     sel_gbs = (by["compressed_keys"]) / (sel_ms / 1e3) / 1e9
     att_gbs = (by["kv_rows"]) / (att_ms / 1e3) / 1e9
-    return {"workload": w.name, "value": round(world * w.batch * steps / (total / 1e3), 1), "unit": "tok/s",
+    return {"workload": w.name + ("_per_head" if per_head else ""),
+            "value": round(world * w.batch * steps / (total / 1e3), 1), "unit": "tok/s",
             "ms_per_step": round(total / steps, 4), "steps": steps, "execution": "one CUDA graph per step",
             "roofline": {"bound": "hbm", "achieved": round(step_gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(step_gbs / hbm, 4), "bytes_per_step": by["total"],

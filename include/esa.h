@@ -170,6 +170,49 @@ size_t esa_sparse_attn_workspace_size(int32_t batch, int32_t lq, int64_t c0, int
                                       int32_t hkv, int32_t head_dim, esa_dtype_t dt,
                                       esa_params_t p);
 
+/* esa_score_select_heads - the per-head selection variant (ESA write-up, ablation
+ * after the experiments: ESA merges all heads into one importance score; the
+ * comparison it is tested against chooses tokens per head). Reading: one selection
+ * per group of compressed columns. Group g owns columns [g * d_g, (g + 1) * d_g) of
+ * q_c and k_c (d_g = d_c / n_groups; compress with a block-diagonal map, group g's
+ * block taking the query heads of KV head g), and runs exactly the steps of
+ * esa_score_select on them:
+ *   S^g_ij = q_c[b, i, group g] . k_c[b, j, group g], then correction, clamp, chunk
+ *   sum, neighbour max-pool and top-k per (sequence, group).
+ *   q_c, k_c: as for esa_score_select
+ *   idx_out:   [batch, n_groups, topk] int32, ascending, -1 after count
+ *   count_out: [batch, n_groups] int32
+ *   score_out: NULL, or [batch, n_groups, |middle|] fp32 receiving s'
+ * Requires n_groups in {1, 2, 4, 8} and d_c % n_groups == 0. With lq <= 8 the groups
+ * must split a key's lanes (d_c >= 128, or d_c / 4 divisible by n_groups); with more
+ * queries d_g must be a multiple of 16. n_groups = 1 is esa_score_select. Errors as for
+ * esa_score_select, ESA_ERR_UNSUPPORTED for group shapes outside these. */
+esa_status_t esa_score_select_heads(const float* q_c, const float* k_c, int32_t batch, int32_t lq,
+                                    int64_t n_cap, int64_t c0, int32_t d_c, int32_t n_groups,
+                                    esa_params_t p, int32_t* idx_out, int32_t* count_out,
+                                    float* score_out, void* workspace, size_t ws_bytes,
+                                    void* stream);
+
+size_t esa_score_select_heads_workspace_size(int32_t batch, int32_t lq, int64_t n_cap, int64_t c0,
+                                             int32_t d_c, int32_t n_groups, esa_params_t p);
+
+/* esa_sparse_attn_heads - esa_sparse_attn with one key list per KV head (the attention
+ * of the per-head selection variant): query head h attends initial + the selected
+ * tokens of KV head h / (hq / hkv) + local.
+ *   idx:   [batch, hkv, >= p.topk] int32 per-head selected middle positions, ascending
+ *          (esa_score_select_heads with n_groups = hkv writes them); count: [batch, hkv]
+ * Everything else, requirements and errors as for esa_sparse_attn. */
+esa_status_t esa_sparse_attn_heads(const void* q, const void* k, const void* v, esa_dtype_t dt,
+                                   int32_t batch, int32_t lq, int64_t n_cap, int64_t c0,
+                                   int32_t hq, int32_t hkv, int32_t head_dim,
+                                   const int32_t* idx, const int32_t* count, esa_params_t p,
+                                   float scale, void* o, float* lse,
+                                   void* workspace, size_t ws_bytes, void* stream);
+
+size_t esa_sparse_attn_heads_workspace_size(int32_t batch, int32_t lq, int64_t c0, int32_t hq,
+                                            int32_t hkv, int32_t head_dim, esa_dtype_t dt,
+                                            esa_params_t p);
+
 /* esa_score_select_noalloc - esa_score_select without a workspace argument. The pages
  * have no counterpart of this call: it exists for callers that cannot allocate device
  * memory - a service that plans all its memory at start-up and allows no allocation

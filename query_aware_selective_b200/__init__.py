@@ -6,8 +6,9 @@ benchmark inputs; ``cost`` holds the algorithmic byte and flop counts used for
 rooflines.
 """
 from ._abi import (EsaError, EsaParams, compress, compress_pack, compress_pack_size, compress_packed, device_status,
-                   load, moba_block_attn, moba_block_gate, moba_block_gate_attn, params, score_select, sparse_attn)
+                   load, moba_block_attn, moba_block_gate, moba_block_gate_attn, params, score_select,
+                   score_select_heads, sparse_attn, sparse_attn_heads)
 
 __all__ = ["EsaError", "EsaParams", "compress", "compress_pack", "compress_pack_size", "compress_packed",
            "device_status", "load", "moba_block_attn", "moba_block_gate", "moba_block_gate_attn", "params",
-           "score_select", "sparse_attn"]
+           "score_select", "score_select_heads", "sparse_attn", "sparse_attn_heads"]

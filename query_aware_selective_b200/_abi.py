@@ -56,6 +56,12 @@ SIGNATURES = {
     "esa_score_select_noalloc": (ctypes.c_int, [_vp, _vp, _i32, _i32, _i64, _i64, _i32, EsaParams, _vp, _vp, _vp,
                                                 _vp]),
     "esa_score_select_noalloc_capacity": (_sz, []),
+    "esa_score_select_heads": (ctypes.c_int, [_vp, _vp, _i32, _i32, _i64, _i64, _i32, _i32, EsaParams, _vp, _vp,
+                                              _vp, _vp, _sz, _vp]),
+    "esa_score_select_heads_workspace_size": (_sz, [_i32, _i32, _i64, _i64, _i32, _i32, EsaParams]),
+    "esa_sparse_attn_heads": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i64, _i64, _i32, _i32,
+                                             _i32, _vp, _vp, EsaParams, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "esa_sparse_attn_heads_workspace_size": (_sz, [_i32, _i32, _i64, _i32, _i32, _i32, ctypes.c_int, EsaParams]),
 }
 
 _lib = None
@@ -243,6 +249,61 @@ def score_select_noalloc(q_c: torch.Tensor, k_c: torch.Tensor, c0: int, p: EsaPa
                                            _ptr(count), _ptr(scores) if want_scores else None, _stream()),
            "esa_score_select_noalloc")
     return idx, count, (scores if want_scores else None)
+
+
+def score_select_heads_workspace_size(batch, lq, n_cap, c0, d_c, n_groups, p: EsaParams) -> int:
+    return load().esa_score_select_heads_workspace_size(batch, lq, n_cap, c0, d_c, n_groups, p)
+
+
+def score_select_heads(q_c: torch.Tensor, k_c: torch.Tensor, c0: int, n_groups: int, p: EsaParams,
+                       want_scores: bool = False, idx: Optional[torch.Tensor] = None,
+                       count: Optional[torch.Tensor] = None, scores: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None):
+    """esa_score_select_heads (per-head selection: one per group of compressed columns).
+    Returns (idx [B, G, topk] int32, count [B, G] int32, s' [B, G, n_mid] f32 or None)."""
+    _dev(q_c, k_c)
+    b, lq, dc = q_c.shape
+    n_cap = k_c.shape[1]
+    dev = q_c.device
+    if idx is None:
+        idx = torch.empty((b, n_groups, p.topk), dtype=torch.int32, device=dev)
+    if count is None:
+        count = torch.empty((b, n_groups), dtype=torch.int32, device=dev)
+    if want_scores and scores is None:
+        lo = min(c0, max(p.n_init, c0 - p.window))
+        scores = torch.empty((b, n_groups, max(0, lo - p.n_init)), dtype=torch.float32, device=dev)
+    ws = _workspace(score_select_heads_workspace_size(b, lq, n_cap, c0, dc, n_groups, p), dev, workspace)
+    wp, wn = _ws_ptr(ws)
+    _check(load().esa_score_select_heads(_ptr(q_c), _ptr(k_c), b, lq, n_cap, c0, dc, n_groups, p, _ptr(idx),
+                                         _ptr(count), _ptr(scores) if want_scores else None, wp, wn, _stream()),
+           "esa_score_select_heads")
+    return idx, count, (scores if want_scores else None)
+
+
+def sparse_attn_heads_workspace_size(batch, lq, c0, hq, hkv, d, dtype_code, p: EsaParams) -> int:
+    return load().esa_sparse_attn_heads_workspace_size(batch, lq, c0, hq, hkv, d, dtype_code, p)
+
+
+def sparse_attn_heads(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, c0: int, idx: torch.Tensor,
+                      count: torch.Tensor, p: EsaParams, scale: float = 0.0, want_lse: bool = False,
+                      out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None):
+    """esa_sparse_attn_heads: idx [B, Hkv, >=topk], count [B, Hkv] (one list per KV head).
+    Returns (o [B, Lq, Hq, D], lse [B, Lq, Hq] f32 or None)."""
+    _dev(q, k, v, idx, count)
+    b, lq, hq, d = q.shape
+    n_cap, hkv = k.shape[1], k.shape[2]
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((b, lq, hq), dtype=torch.float32, device=q.device)
+    ws = _workspace(sparse_attn_heads_workspace_size(b, lq, c0, hq, hkv, d, dt, p), q.device, workspace)
+    wp, wn = _ws_ptr(ws)
+    _check(load().esa_sparse_attn_heads(_ptr(q), _ptr(k), _ptr(v), dt, b, lq, n_cap, c0, hq, hkv, d, _ptr(idx),
+                                        _ptr(count), p, scale, _ptr(out), _ptr(lse) if want_lse else None, wp, wn,
+                                        _stream()), "esa_sparse_attn_heads")
+    return out, (lse if want_lse else None)
 
 
 def sparse_attn_workspace_size(batch, lq, c0, hq, hkv, d, dtype_code, p: EsaParams) -> int:

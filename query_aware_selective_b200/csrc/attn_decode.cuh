@@ -53,9 +53,15 @@ struct DecodeAttnArgs {
   int* arrive;              // [B] zeroed split counters when nsplit > 1
   KeyList keys;
   int64_t n_cap, c0;
-  int hq, hkv, nsplit;
+  int hq, hkv, nsplit;       // per (virtual) sequence
   int keys_per_split;       // a multiple of the keys per stage, <= kDecMaxSplitKeys
   float scale_log2;         // softmax scale * log2(e)
+  // Sequence b of the grid is cache sequence b / vheads, KV heads from (b % vheads) * hkv:
+  // 1 normally; with per-head key lists every (sequence, KV head) is a sequence of its
+  // own with hkv = 1. tok_stride: elements from one token's K row to the next (Hkv * 128
+  // of the cache).
+  int vheads;
+  int64_t tok_stride;
 };
 
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -106,13 +112,13 @@ __device__ __forceinline__ void dec_issue(const DecodeAttnArgs& a, DecSmem& sm, 
   const int n_in = (int)(t_end - t0 < ks ? t_end - t0 : ks);
   if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], (uint32_t)(2 * n_in * row_bytes));
   __syncwarp();
-  const int64_t seq = (int64_t)b * a.n_cap * a.hkv * kDecD;
+  const int64_t seq = (int64_t)(b / a.vheads) * a.n_cap * a.tok_stride + (int64_t)(b % a.vheads) * a.hkv * kDecD;
   const uint32_t kdst = stage0 + s * 2 * op_bytes;
   const int rs = row_bytes + 16;
   for (int c = lane; c < 2 * n_in; c += 32) {
     const int kk = c >> 1;
     const int64_t p = pos[j * ks + kk];
-    const __nv_bfloat16* src = ((c & 1) ? a.v : a.k) + seq + p * a.hkv * kDecD;
+    const __nv_bfloat16* src = ((c & 1) ? a.v : a.k) + seq + p * a.tok_stride;
     bulk_g2s(kdst + (c & 1) * op_bytes + kk * rs, src, row_bytes, &sm.full[s]);
   }
   if (lane == 0) atomicMax(&sm.issued, j + 1);

@@ -24,6 +24,7 @@ struct SimtAttnArgs {
   KeyList keys;
   int64_t n_cap, c0;
   int lq, hq, hkv, nsplit;
+  int lists;           // key lists per sequence: 1, or Hkv (one per KV head)
   int64_t keys_per_split;
   float scale_log2;    // scale * log2(e)
 };
@@ -49,7 +50,8 @@ __global__ void __launch_bounds__(kSimtWarps * 32) attn_simt_kernel(SimtAttnArgs
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int grp = lane / LPK, sub = lane % LPK;
 
-  const int cnt = min(max(a.keys.count[b], 0), (int)a.keys.idx_stride);
+  const int list = a.lists > 1 ? b * a.lists + g : b;
+  const int cnt = min(max(a.keys.count[list], 0), (int)a.keys.idx_stride);
   const int64_t n_prior = a.keys.ni + cnt + (a.c0 - a.keys.lo);
   const int64_t n_keys = n_prior + i + 1;                     // causal: keys up to position c0 + i
   const int64_t t_begin = (int64_t)split * a.keys_per_split;
@@ -83,7 +85,7 @@ __global__ void __launch_bounds__(kSimtWarps * 32) attn_simt_kernel(SimtAttnArgs
       const int64_t t = tb + u * KPW + grp;
       ok[u] = t < t_end;
       if (ok[u]) {
-        const int64_t p = a.keys.pos(b, cnt, t);
+        const int64_t p = a.keys.pos(list, cnt, t);
         kr[u] = ld_stream16(kbase + p * row_stride);
         vr[u] = ld_stream16(vbase + p * row_stride);
       }

@@ -462,15 +462,17 @@ struct EsaTcProblem {
   int lq, hq, hkv, G;
   float sl2;
   int staged;            // selected K/V rows were copied to contiguous buffers
+  int lists;             // key lists per sequence: 1, or Hkv (one per KV head)
   // per CTA
-  int b, g, tile, cnt;
+  int b, g, tile, cnt, list;
   int64_t n_prior, nk;
 
   __device__ bool setup() {
     tile = blockIdx.x;
     g = blockIdx.y;
     b = blockIdx.z;
-    cnt = min(max(keys.count[b], 0), (int)keys.idx_stride);
+    list = lists > 1 ? b * lists + g : b;
+    cnt = min(max(keys.count[list], 0), (int)keys.idx_stride);
     n_prior = keys.ni + cnt + (c0 - keys.lo);
     const int rows = lq * G;
     if (tile * kTcRows >= rows) return false;
@@ -485,7 +487,7 @@ struct EsaTcProblem {
     return (int32_t)(((int64_t)b * lq + i) * hq + g * G + hl);
   }
   __device__ int32_t kv_row(int64_t t) const {
-    return (int32_t)(((int64_t)b * n_cap + keys.pos(b, cnt, t)) * hkv + g);
+    return (int32_t)(((int64_t)b * n_cap + keys.pos(list, cnt, t)) * hkv + g);
   }
   // Q tile = 128 / G consecutive queries x the G heads of group g: one box of the
   // [B * lq, hq, 128] map (rows past the chunk belong to no stored output)
@@ -549,22 +551,27 @@ namespace esa {
 // Copy the selected K and V rows of every sequence into contiguous buffers
 // [B, topk, Hkv, D] (all heads of a token are one contiguous row of Hkv * D elements),
 // so that the attention kernel loads selected keys as boxes instead of row gathers.
-// One CTA per (selected entry, sequence); 16-byte pieces.
+// With one list per KV head (lists = Hkv), slot t of head g holds the row of head g
+// of that head's t-th selected token. One CTA per (selected entry, list); 16-byte
+// pieces. row_vec: 16-byte pieces of one token's row (all heads); head_vec: of one head.
 __global__ void __launch_bounds__(256) gather_selected_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                                                               const int32_t* __restrict__ idx,
                                                               const int32_t* __restrict__ count, int64_t n_cap,
-                                                              int topk, int row_vec, uint4* __restrict__ ks,
-                                                              uint4* __restrict__ vs) {
-  const int b = blockIdx.y;
-  const int cnt = min(max(count[b], 0), topk);
+                                                              int topk, int row_vec, int lists, int head_vec,
+                                                              uint4* __restrict__ ks, uint4* __restrict__ vs) {
+  const int list = blockIdx.y;
+  const int b = list / lists, g = list % lists;
+  const int cnt = min(max(count[list], 0), topk);
+  const int width = lists > 1 ? head_vec : row_vec;        // pieces copied per entry
+  const int off = lists > 1 ? g * head_vec : 0;
   for (int t = blockIdx.x; t < cnt; t += gridDim.x) {
-    int64_t p = idx[(int64_t)b * topk + t];
+    int64_t p = idx[(int64_t)list * topk + t];
     p = p < 0 ? 0 : (p >= n_cap ? n_cap - 1 : p);
-    const uint4* ksrc = k + ((int64_t)b * n_cap + p) * row_vec;
-    const uint4* vsrc = v + ((int64_t)b * n_cap + p) * row_vec;
-    uint4* kd = ks + ((int64_t)b * topk + t) * row_vec;
-    uint4* vd = vs + ((int64_t)b * topk + t) * row_vec;
-    for (int e = threadIdx.x; e < row_vec; e += blockDim.x) {
+    const uint4* ksrc = k + ((int64_t)b * n_cap + p) * row_vec + off;
+    const uint4* vsrc = v + ((int64_t)b * n_cap + p) * row_vec + off;
+    uint4* kd = ks + ((int64_t)b * topk + t) * row_vec + off;
+    uint4* vd = vs + ((int64_t)b * topk + t) * row_vec + off;
+    for (int e = threadIdx.x; e < width; e += blockDim.x) {
       kd[e] = ld_stream16(ksrc + e);
       vd[e] = ld_stream16(vsrc + e);
     }

@@ -113,9 +113,14 @@ esa_status_t check_params(const esa_params_t& p) {
 // (two passes, S never stored); anything else -> SIMT tiles (S stored).
 enum class ScorePath { Small, TensorCore, Tiled };
 
-ScorePath score_path(int32_t batch, int32_t lq, int64_t n_cap, int32_t d_c) {
-  if (lq <= esa::kScoreSmallLq && (d_c == 16 || d_c == 32 || d_c == 64 || d_c == 128 || d_c == 256))
+// With ng > 1 groups (per-head selection) there is no tensor-core path, and the small
+// path needs the groups to split a key's lanes (LPK = min(d_c, 128) / 4, 32 from 128 on).
+ScorePath score_path(int32_t batch, int32_t lq, int64_t n_cap, int32_t d_c, int ng = 1) {
+  const int lpk = d_c >= 128 ? 32 : d_c / 4;
+  if (lq <= esa::kScoreSmallLq && (d_c == 16 || d_c == 32 || d_c == 64 || d_c == 128 || d_c == 256) &&
+      lpk % ng == 0)
     return ScorePath::Small;
+  if (ng > 1) return ScorePath::Tiled;
   // TMA row coordinates are 32-bit
   const bool rows_fit = (int64_t)batch * n_cap < ((int64_t)1 << 31) && (int64_t)batch * lq < ((int64_t)1 << 31);
   if (lq >= 16 && rows_fit && (d_c == 32 || d_c == 64 || d_c == 128)) return ScorePath::TensorCore;
@@ -237,9 +242,9 @@ esa_status_t make_tmap_f32(CUtensorMap* m, const float* base, uint64_t rows, uin
   return ESA_OK;
 }
 
-template <int DC>
-void launch_score_small(const float* q_c, const float* k_c, int lq, int64_t n_cap, int64_t mid0, int64_t n_mid,
-                        int batch, float* S, uint32_t* m_key, cudaStream_t s) {
+template <int DC, int NG>
+void launch_score_small_ng(const float* q_c, const float* k_c, int lq, int64_t n_cap, int64_t mid0, int64_t n_mid,
+                           int batch, float* S, uint32_t* m_key, cudaStream_t s) {
   // one wave of two CTAs per SM over all sequences, each CTA a multiple of a stage
   constexpr int64_t ks = esa::SmallScoreShape<DC>::KS;
   const int64_t per_seq = std::max<int64_t>(1, std::min<int64_t>(cdiv(n_mid, ks), (2 * 148) / batch));
@@ -248,18 +253,29 @@ void launch_score_small(const float* q_c, const float* k_c, int lq, int64_t n_ca
   static bool attr_set[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess && dev < 64 && !attr_set[dev]) {
-    cudaFuncSetAttribute(esa::score_small_kernel<DC, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(esa::score_small_kernel<DC, 1, NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          esa::kSsSmemBytes);
-    cudaFuncSetAttribute(esa::score_small_kernel<DC, esa::kScoreSmallLq>,
+    cudaFuncSetAttribute(esa::score_small_kernel<DC, esa::kScoreSmallLq, NG>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, esa::kSsSmemBytes);
     attr_set[dev] = true;
   }
   if (lq == 1)
-    esa::score_small_kernel<DC, 1><<<grid, esa::kSsThreads, esa::kSsSmemBytes, s>>>(q_c, k_c, lq, n_cap, mid0, n_mid,
-                                                                                    keys_per_cta, S, m_key);
-  else
-    esa::score_small_kernel<DC, esa::kScoreSmallLq><<<grid, esa::kSsThreads, esa::kSsSmemBytes, s>>>(
+    esa::score_small_kernel<DC, 1, NG><<<grid, esa::kSsThreads, esa::kSsSmemBytes, s>>>(
         q_c, k_c, lq, n_cap, mid0, n_mid, keys_per_cta, S, m_key);
+  else
+    esa::score_small_kernel<DC, esa::kScoreSmallLq, NG><<<grid, esa::kSsThreads, esa::kSsSmemBytes, s>>>(
+        q_c, k_c, lq, n_cap, mid0, n_mid, keys_per_cta, S, m_key);
+}
+
+// groups must split a key's LPK lanes evenly (checked by score_path)
+template <int DC>
+void launch_score_small(const float* q_c, const float* k_c, int lq, int64_t n_cap, int64_t mid0, int64_t n_mid,
+                        int batch, int ng, float* S, uint32_t* m_key, cudaStream_t s) {
+  constexpr int LPK = esa::SmallScoreShape<DC>::LPK;
+  if (ng == 1) launch_score_small_ng<DC, 1>(q_c, k_c, lq, n_cap, mid0, n_mid, batch, S, m_key, s);
+  else if (ng == 2) launch_score_small_ng<DC, 2>(q_c, k_c, lq, n_cap, mid0, n_mid, batch, S, m_key, s);
+  else if (ng == 4) launch_score_small_ng<DC, 4>(q_c, k_c, lq, n_cap, mid0, n_mid, batch, S, m_key, s);
+  else if constexpr (LPK % 8 == 0) launch_score_small_ng<DC, 8>(q_c, k_c, lq, n_cap, mid0, n_mid, batch, S, m_key, s);
 }
 
 }  // namespace
@@ -485,18 +501,55 @@ esa_status_t esa_compress(const void* x, esa_dtype_t x_dtype, int64_t rows, int6
 }
 
 // ------------------------------------------------------------------ score_select --
+namespace {
+
+size_t score_select_ws(int32_t batch, int32_t lq, int64_t n_cap, int64_t c0, int32_t d_c, int ng,
+                       const esa_params_t& p) {
+  if (batch <= 0 || lq <= 0 || ng <= 0) return 0;
+  const Regions r = regions(c0, p);
+  return carve_select(nullptr, batch * ng, lq, r.n_mid, score_path(batch, lq, n_cap, d_c, ng)).bytes;
+}
+
+esa_status_t score_select_impl(const float* q_c, const float* k_c, int32_t batch, int32_t lq, int64_t n_cap,
+                               int64_t c0, int32_t d_c, int ng, esa_params_t p, int32_t* idx_out,
+                               int32_t* count_out, float* score_out, void* workspace, size_t ws_bytes,
+                               void* stream);
+
+}  // namespace
+
 size_t esa_score_select_workspace_size(int32_t batch, int32_t lq, int64_t n_cap, int64_t c0, int32_t d_c,
                                        esa_params_t p) {
-  (void)n_cap;
-  (void)d_c;
-  if (batch <= 0 || lq <= 0) return 0;
-  const Regions r = regions(c0, p);
-  return carve_select(nullptr, batch, lq, r.n_mid, score_path(batch, lq, n_cap, d_c)).bytes;
+  return score_select_ws(batch, lq, n_cap, c0, d_c, 1, p);
+}
+
+size_t esa_score_select_heads_workspace_size(int32_t batch, int32_t lq, int64_t n_cap, int64_t c0, int32_t d_c,
+                                             int32_t n_groups, esa_params_t p) {
+  return score_select_ws(batch, lq, n_cap, c0, d_c, n_groups, p);
 }
 
 esa_status_t esa_score_select(const float* q_c, const float* k_c, int32_t batch, int32_t lq, int64_t n_cap,
                               int64_t c0, int32_t d_c, esa_params_t p, int32_t* idx_out, int32_t* count_out,
                               float* score_out, void* workspace, size_t ws_bytes, void* stream) {
+  return score_select_impl(q_c, k_c, batch, lq, n_cap, c0, d_c, 1, p, idx_out, count_out, score_out, workspace,
+                           ws_bytes, stream);
+}
+
+esa_status_t esa_score_select_heads(const float* q_c, const float* k_c, int32_t batch, int32_t lq, int64_t n_cap,
+                                    int64_t c0, int32_t d_c, int32_t n_groups, esa_params_t p, int32_t* idx_out,
+                                    int32_t* count_out, float* score_out, void* workspace, size_t ws_bytes,
+                                    void* stream) {
+  if (n_groups != 1 && n_groups != 2 && n_groups != 4 && n_groups != 8)
+    return fail(ESA_ERR_UNSUPPORTED, "n_groups %d (1, 2, 4 or 8)", n_groups);
+  return score_select_impl(q_c, k_c, batch, lq, n_cap, c0, d_c, n_groups, p, idx_out, count_out, score_out,
+                           workspace, ws_bytes, stream);
+}
+
+namespace {
+
+esa_status_t score_select_impl(const float* q_c, const float* k_c, int32_t batch, int32_t lq, int64_t n_cap,
+                               int64_t c0, int32_t d_c, int ng, esa_params_t p, int32_t* idx_out,
+                               int32_t* count_out, float* score_out, void* workspace, size_t ws_bytes,
+                               void* stream) {
   esa_status_t st = check_params(p);
   if (st != ESA_OK) return st;
   if (batch <= 0) return fail(ESA_ERR_INVALID_ARG, "batch must be >= 1");
@@ -507,29 +560,32 @@ esa_status_t esa_score_select(const float* q_c, const float* k_c, int32_t batch,
   if (!aligned(q_c, 16) || !aligned(k_c, 16)) return fail(ESA_ERR_INVALID_ARG, "q_c and k_c need 16-byte alignment");
   const Regions r = regions(c0, p);
   if (r.n_mid > (int64_t)1 << 30) return fail(ESA_ERR_UNSUPPORTED, "middle longer than 2^30 tokens");
-  if (batch > 65535) return fail(ESA_ERR_UNSUPPORTED, "batch must be <= 65535 (got %d)", batch);
+  if (d_c % ng || (ng > 1 && (d_c / ng) % 16 && score_path(batch, lq, n_cap, d_c, ng) != ScorePath::Small))
+    return fail(ESA_ERR_UNSUPPORTED, "d_c %d in %d groups: each group needs a multiple of 16 columns here", d_c, ng);
+  const int64_t vb = (int64_t)batch * ng;   // independent selections: sequence x group
+  if (vb > 65535) return fail(ESA_ERR_UNSUPPORTED, "batch x groups must be <= 65535 (got %lld)", (long long)vb);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t kk = std::min<int64_t>(p.topk, r.n_mid);
   const bool need_scores = r.n_mid > p.topk || (score_out && r.n_mid > 0);
   if (need_scores) {
-    const ScorePath path = score_path(batch, lq, n_cap, d_c);
-    const SelWs need = carve_select(nullptr, batch, lq, r.n_mid, path);
+    const ScorePath path = score_path(batch, lq, n_cap, d_c, ng);
+    const SelWs need = carve_select(nullptr, (int32_t)vb, lq, r.n_mid, path);
     if (!workspace || ws_bytes < need.bytes || !aligned(workspace, 256))
       return fail(ESA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need.bytes, ws_bytes);
-    const SelWs w = carve_select(workspace, batch, lq, r.n_mid, path);
-    ESA_CUDA(cudaMemsetAsync(w.m_key, 0, (size_t)batch * lq * sizeof(uint32_t), s));
+    const SelWs w = carve_select(workspace, (int32_t)vb, lq, r.n_mid, path);
+    ESA_CUDA(cudaMemsetAsync(w.m_key, 0, (size_t)vb * lq * sizeof(uint32_t), s));
     if (path == ScorePath::Small) {
       switch (d_c) {
-        case 16: launch_score_small<16>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, w.S, w.m_key, s); break;
-        case 32: launch_score_small<32>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, w.S, w.m_key, s); break;
-        case 64: launch_score_small<64>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, w.S, w.m_key, s); break;
-        case 128: launch_score_small<128>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, w.S, w.m_key, s); break;
-        default: launch_score_small<256>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, w.S, w.m_key, s); break;
+        case 16: launch_score_small<16>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, s); break;
+        case 32: launch_score_small<32>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, s); break;
+        case 64: launch_score_small<64>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, s); break;
+        case 128: launch_score_small<128>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, s); break;
+        default: launch_score_small<256>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, s); break;
       }
       ESA_LAUNCH_CHECK("score_small_kernel");
     } else if (path == ScorePath::Tiled) {
-      dim3 grid((unsigned)cdiv(r.n_mid, esa::kScT), (unsigned)cdiv(lq, esa::kScT), batch);
-      esa::score_tiled_kernel<<<grid, 256, 0, s>>>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, d_c, w.S, w.m_key);
+      dim3 grid((unsigned)cdiv(r.n_mid, esa::kScT), (unsigned)cdiv(lq, esa::kScT), (unsigned)vb);
+      esa::score_tiled_kernel<<<grid, 256, 0, s>>>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, d_c, ng, w.S, w.m_key);
       ESA_LAUNCH_CHECK("score_tiled_kernel");
     }
     if (path == ScorePath::TensorCore) {
@@ -579,9 +635,9 @@ esa_status_t esa_score_select(const float* q_c, const float* k_c, int32_t batch,
         if ((st = set_max_smem(esa::select_cluster_kernel<16>, esa::kSelSmemBytes)) != ESA_OK) return st;
         sel_attr[dev] = true;
       }
-      const int cl = select_cluster_size(batch);
+      const int cl = select_cluster_size((int32_t)vb);
       cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3((unsigned)cl, (unsigned)batch, 1);
+      cfg.gridDim = dim3((unsigned)cl, (unsigned)vb, 1);
       cfg.blockDim = dim3(esa::kSelThreads);
       cfg.dynamicSmemBytes = esa::kSelSmemBytes;
       cfg.stream = s;
@@ -599,11 +655,13 @@ esa_status_t esa_score_select(const float* q_c, const float* k_c, int32_t batch,
     }
   }
   const bool all_mid = r.n_mid <= p.topk;
-  esa::fill_selection_kernel<<<dim3((unsigned)std::max<int64_t>(1, cdiv(p.topk, 256)), batch), 256, 0, s>>>(
+  esa::fill_selection_kernel<<<dim3((unsigned)std::max<int64_t>(1, cdiv(p.topk, 256)), (unsigned)vb), 256, 0, s>>>(
       idx_out, count_out, p.topk, (int)kk, r.mid0, all_mid ? 1 : 0);
   ESA_LAUNCH_CHECK("fill_selection_kernel");
   return ok();
 }
+
+}  // namespace
 
 // ------------------------------------------------------------------ sparse_attn --
 namespace {
@@ -679,16 +737,64 @@ bool dispatch_simt_g(const esa::SimtAttnArgs& a, int g, int batch, cudaStream_t 
 
 }  // namespace
 
+namespace {
+
+// With one key list per KV head (lists > 1), a one-query bf16 call runs the bulk-copy
+// decode kernel over batch x Hkv virtual sequences of one KV head each.
+bool heads_as_sequences(int lists, esa_dtype_t dt, int32_t lq, int32_t hq, int32_t hkv, int32_t head_dim) {
+  const int g = hq / hkv;
+  return lists > 1 && dt == ESA_BF16 && head_dim == 128 && lq == 1 && (g == 1 || g == 2 || g == 4);
+}
+
+size_t sparse_attn_ws(int32_t batch, int32_t lq, int64_t c0, int32_t hq, int32_t hkv, int32_t head_dim,
+                      esa_dtype_t dt, const esa_params_t& p, int lists) {
+  if (batch <= 0 || lq <= 0 || hkv <= 0 || hq <= 0 || hq % hkv) return 0;
+  if (heads_as_sequences(lists, dt, lq, hq, hkv, head_dim))
+    return plan_attn(batch * hkv, lq, c0, hq / hkv, 1, head_dim, dt, p).ws_bytes;
+  return plan_attn(batch, lq, c0, hq, hkv, head_dim, dt, p).ws_bytes;
+}
+
+esa_status_t sparse_attn_impl(const void* q, const void* k, const void* v, esa_dtype_t dt, int32_t batch,
+                              int32_t lq, int64_t n_cap, int64_t c0, int32_t hq, int32_t hkv, int32_t head_dim,
+                              const int32_t* idx, const int32_t* count, esa_params_t p, float scale, void* o,
+                              float* lse, void* workspace, size_t ws_bytes, void* stream, int lists);
+
+}  // namespace
+
 size_t esa_sparse_attn_workspace_size(int32_t batch, int32_t lq, int64_t c0, int32_t hq, int32_t hkv,
                                       int32_t head_dim, esa_dtype_t dt, esa_params_t p) {
-  if (batch <= 0 || lq <= 0 || hkv <= 0 || hq <= 0 || hq % hkv) return 0;
-  return plan_attn(batch, lq, c0, hq, hkv, head_dim, dt, p).ws_bytes;
+  return sparse_attn_ws(batch, lq, c0, hq, hkv, head_dim, dt, p, 1);
+}
+
+size_t esa_sparse_attn_heads_workspace_size(int32_t batch, int32_t lq, int64_t c0, int32_t hq, int32_t hkv,
+                                            int32_t head_dim, esa_dtype_t dt, esa_params_t p) {
+  return sparse_attn_ws(batch, lq, c0, hq, hkv, head_dim, dt, p, hkv);
 }
 
 esa_status_t esa_sparse_attn(const void* q, const void* k, const void* v, esa_dtype_t dt, int32_t batch, int32_t lq,
                              int64_t n_cap, int64_t c0, int32_t hq, int32_t hkv, int32_t head_dim,
                              const int32_t* idx, const int32_t* count, esa_params_t p, float scale, void* o,
                              float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  return sparse_attn_impl(q, k, v, dt, batch, lq, n_cap, c0, hq, hkv, head_dim, idx, count, p, scale, o, lse,
+                          workspace, ws_bytes, stream, 1);
+}
+
+esa_status_t esa_sparse_attn_heads(const void* q, const void* k, const void* v, esa_dtype_t dt, int32_t batch,
+                                   int32_t lq, int64_t n_cap, int64_t c0, int32_t hq, int32_t hkv, int32_t head_dim,
+                                   const int32_t* idx, const int32_t* count, esa_params_t p, float scale, void* o,
+                                   float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  if (hkv <= 0) return fail(ESA_ERR_INVALID_ARG, "hkv must be >= 1");
+  return sparse_attn_impl(q, k, v, dt, batch, lq, n_cap, c0, hq, hkv, head_dim, idx, count, p, scale, o, lse,
+                          workspace, ws_bytes, stream, hkv);
+}
+
+namespace {
+
+
+esa_status_t sparse_attn_impl(const void* q, const void* k, const void* v, esa_dtype_t dt, int32_t batch,
+                              int32_t lq, int64_t n_cap, int64_t c0, int32_t hq, int32_t hkv, int32_t head_dim,
+                              const int32_t* idx, const int32_t* count, esa_params_t p, float scale, void* o,
+                              float* lse, void* workspace, size_t ws_bytes, void* stream, int lists) {
   esa_status_t st = check_params(p);
   if (st != ESA_OK) return st;
   if (dt != ESA_F32 && dt != ESA_BF16) return fail(ESA_ERR_INVALID_ARG, "bad dtype %d", (int)dt);
@@ -703,7 +809,9 @@ esa_status_t esa_sparse_attn(const void* q, const void* k, const void* v, esa_dt
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16))
     return fail(ESA_ERR_INVALID_ARG, "q, k, v, o need 16-byte alignment");
   const Regions r = regions(c0, p);
-  const AttnPlan pl = plan_attn(batch, lq, c0, hq, hkv, head_dim, dt, p);
+  const bool vseq = heads_as_sequences(lists, dt, lq, hq, hkv, head_dim);
+  const AttnPlan pl = vseq ? plan_attn(batch * hkv, lq, c0, hq / hkv, 1, head_dim, dt, p)
+                           : plan_attn(batch, lq, c0, hq, hkv, head_dim, dt, p);
   if (pl.ws_bytes && (!workspace || ws_bytes < pl.ws_bytes || !aligned(workspace, 256)))
     return fail(ESA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", pl.ws_bytes, ws_bytes);
   if (scale <= 0.f) scale = 1.f / std::sqrt((float)head_dim);
@@ -733,6 +841,7 @@ esa_status_t esa_sparse_attn(const void* q, const void* k, const void* v, esa_dt
     pr.hkv = hkv;
     pr.G = g;
     pr.sl2 = sl2;
+    pr.lists = lists;
     if ((int64_t)batch * n_cap * hkv >= ((int64_t)1 << 31) || (int64_t)batch * lq * hq >= ((int64_t)1 << 31))
       return fail(ESA_ERR_UNSUPPORTED, "more than 2^31 K/V or Q rows");
     uint8_t* ks = static_cast<uint8_t*>(workspace);
@@ -741,10 +850,10 @@ esa_status_t esa_sparse_attn(const void* q, const void* k, const void* v, esa_dt
     const int64_t max_sel = std::min<int64_t>(p.topk, r.n_mid);
     pr.staged = max_sel > 0 ? 1 : 0;
     if (max_sel > 0) {
-      const dim3 ggrid((unsigned)std::min<int64_t>(max_sel, 4096), batch);
+      const dim3 ggrid((unsigned)std::min<int64_t>(max_sel, 4096), (unsigned)(batch * lists));
       esa::gather_selected_kernel<<<ggrid, 128, 0, s>>>(
-          static_cast<const uint4*>(k), static_cast<const uint4*>(v), idx, count, n_cap, p.topk, row_vec,
-          reinterpret_cast<uint4*>(ks), reinterpret_cast<uint4*>(vs));
+          static_cast<const uint4*>(k), static_cast<const uint4*>(v), idx, count, n_cap, p.topk, row_vec, lists,
+          head_dim * 2 / 16, reinterpret_cast<uint4*>(ks), reinterpret_cast<uint4*>(vs));
       ESA_LAUNCH_CHECK("gather_selected_kernel");
     }
     CUtensorMap tq, tk, tv, bq, bk, bv, sk, sv;
@@ -779,19 +888,22 @@ esa_status_t esa_sparse_attn(const void* q, const void* k, const void* v, esa_dt
     d.o = static_cast<__nv_bfloat16*>(o);
     d.lse = lse;
     if (pl.nsplit > 1) {
+      const size_t nseq = (size_t)(vseq ? batch * hkv : batch);
       d.arrive = static_cast<int*>(workspace);
-      d.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + up256((size_t)batch * sizeof(int)));
-      ESA_CUDA(cudaMemsetAsync(d.arrive, 0, (size_t)batch * sizeof(int), s));
+      d.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + up256(nseq * sizeof(int)));
+      ESA_CUDA(cudaMemsetAsync(d.arrive, 0, nseq * sizeof(int), s));
     }
     d.keys = keys;
     d.n_cap = n_cap;
     d.c0 = c0;
-    d.hq = hq;
-    d.hkv = hkv;
+    d.hq = vseq ? hq / hkv : hq;
+    d.hkv = vseq ? 1 : hkv;
+    d.vheads = vseq ? hkv : 1;
+    d.tok_stride = (int64_t)hkv * head_dim;
     d.nsplit = pl.nsplit;
     d.keys_per_split = (int)pl.keys_per_split;
     d.scale_log2 = sl2;
-    const dim3 grid((unsigned)pl.nsplit, (unsigned)batch);
+    const dim3 grid((unsigned)pl.nsplit, (unsigned)(vseq ? batch * hkv : batch));
     if (g == 1) esa::attn_decode_kernel<1><<<grid, esa::kDecThreads, esa::kDecSmemBytes, s>>>(d);
     else if (g == 2) esa::attn_decode_kernel<2><<<grid, esa::kDecThreads, esa::kDecSmemBytes, s>>>(d);
     else esa::attn_decode_kernel<4><<<grid, esa::kDecThreads, esa::kDecSmemBytes, s>>>(d);
@@ -812,6 +924,7 @@ esa_status_t esa_sparse_attn(const void* q, const void* k, const void* v, esa_dt
   a.hq = hq;
   a.hkv = hkv;
   a.nsplit = pl.nsplit;
+  a.lists = lists;
   a.keys_per_split = pl.keys_per_split;
   a.scale_log2 = sl2;
   bool launched;
@@ -844,6 +957,8 @@ esa_status_t esa_sparse_attn(const void* q, const void* k, const void* v, esa_dt
   }
   return ok();
 }
+
+}  // namespace
 
 // ------------------------------------------------------------------ MoBA --
 namespace {

@@ -21,6 +21,11 @@ namespace esa {
 // of the eight warps to finish a stage issues its refill. In a stage, a group of LPK
 // lanes holds one key (VPL floats per lane, 16-byte shared loads) and a warp covers KPW
 // keys per step. Lq <= kScoreSmallLq queries live in registers.
+//
+// With NG > 1 groups (the per-head variant: group g owns compressed columns
+// [g d_g, (g + 1) d_g)) the LPK lanes of a key split into NG runs of LPK / NG lanes,
+// each reduced on its own: S is written as [B, NG, Lq, n_mid] and the maxima as
+// [B, NG, Lq], i.e. B * NG independent selections.
 constexpr int kScoreSmallLq = 8;
 constexpr int kSsWarps = 8;
 constexpr int kSsThreads = kSsWarps * 32;
@@ -45,7 +50,7 @@ struct SsSmem {
 
 // grid (ctas per sequence, B); kSsThreads threads; kSsSmemBytes dynamic shared memory.
 // CTA c scores keys [c * keys_per_cta, ...) of the middle (keys_per_cta a multiple of KS).
-template <int DC, int LQ>
+template <int DC, int LQ, int NG>
 __global__ void __launch_bounds__(kSsThreads, 2) score_small_kernel(const float* __restrict__ q_c,
                                                                    const float* __restrict__ k_c, int lq,
                                                                    int64_t n_cap, int64_t mid0, int64_t n_mid,
@@ -54,6 +59,8 @@ __global__ void __launch_bounds__(kSsThreads, 2) score_small_kernel(const float*
   using Sh = SmallScoreShape<DC>;
   constexpr int VPL = Sh::VPL, LPK = Sh::LPK, KPW = Sh::KPW, KS = Sh::KS;
   constexpr int KEYS_PER_WARP = KS / kSsWarps;             // of a stage
+  constexpr int LPG = LPK / NG;                            // lanes per group of a key
+  static_assert(LPK % NG == 0, "groups split a key's lanes evenly");
   extern __shared__ __align__(128) uint8_t ss_dsm[];
   const uint32_t stage0 = (smem_u32(ss_dsm) + 127u) & ~127u;
   uint8_t* const stage0_ptr = ss_dsm + (stage0 - smem_u32(ss_dsm));
@@ -61,6 +68,7 @@ __global__ void __launch_bounds__(kSsThreads, 2) score_small_kernel(const float*
   const int b = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int grp = lane / LPK, sub = lane % LPK;
+  const int hg = sub / LPG;                                // this lane's group
   const int64_t j_begin = (int64_t)blockIdx.x * keys_per_cta;
   const int64_t j_end = min(n_mid, j_begin + keys_per_cta);
   const int nst = j_end > j_begin ? (int)((j_end - j_begin + KS - 1) / KS) : 0;
@@ -126,10 +134,10 @@ __global__ void __launch_bounds__(kSsThreads, 2) score_small_kernel(const float*
 #pragma unroll
         for (int v = 0; v < VPL; ++v) acc = fmaf(q[i][v], kv[v], acc);
 #pragma unroll
-        for (int o = LPK / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        for (int o = LPG / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
         if (jj < j_end && i < lq) {
           mx[i] = fmaxf(mx[i], acc);
-          if (sub == 0) s_out[((int64_t)b * lq + i) * n_mid + jj] = acc;
+          if (sub % LPG == 0) s_out[(((int64_t)b * NG + hg) * lq + i) * n_mid + jj] = acc;
         }
       }
     }
@@ -158,17 +166,32 @@ __global__ void __launch_bounds__(kSsThreads, 2) score_small_kernel(const float*
     }
     return;
   }
-  __shared__ float red[LQ][kSsWarps];
+  if (NG == 1) {
+    __shared__ float red[LQ][kSsWarps];
 #pragma unroll
-  for (int i = 0; i < LQ; ++i) {
-    float v = warp_max(mx[i]);
-    if (lane == 0) red[i][warp] = v;
-  }
-  __syncthreads();
-  if (threadIdx.x < lq) {
-    float v = -INFINITY;
-    for (int w = 0; w < kSsWarps; ++w) v = fmaxf(v, red[threadIdx.x][w]);
-    if (v > -INFINITY) atomicMax(&m_key[b * lq + threadIdx.x], order_key(v));
+    for (int i = 0; i < LQ; ++i) {
+      float v = warp_max(mx[i]);
+      if (lane == 0) red[i][warp] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < lq) {
+      float v = -INFINITY;
+      for (int w = 0; w < kSsWarps; ++w) v = fmaxf(v, red[threadIdx.x][w]);
+      if (v > -INFINITY) atomicMax(&m_key[b * lq + threadIdx.x], order_key(v));
+    }
+  } else {
+    // per (query, group): shared-memory order-key maxima, then one global atomic each
+    __shared__ uint32_t redk[LQ][NG];
+    for (int t = threadIdx.x; t < LQ * NG; t += kSsThreads) (&redk[0][0])[t] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < LQ; ++i)
+      if (i < lq && sub % LPG == 0 && mx[i] > -INFINITY) atomicMax(&redk[i][hg], order_key(mx[i]));
+    __syncthreads();
+    for (int t = threadIdx.x; t < lq * NG; t += kSsThreads) {
+      const int i = t / NG, g = t % NG;
+      if (redk[i][g]) atomicMax(&m_key[((int64_t)b * NG + g) * lq + i], redk[i][g]);
+    }
   }
 }
 
@@ -178,13 +201,17 @@ __global__ void __launch_bounds__(kSsThreads, 2) score_small_kernel(const float*
 constexpr int kScT = 64;
 constexpr int kScK = 16;
 
+// grid (key tiles, query tiles, B * ng); sequence b, group g = blockIdx.z / ng, % ng
+// reduces over the compressed columns [g dg, (g + 1) dg) of rows of dc floats.
 __global__ void __launch_bounds__(256) score_tiled_kernel(const float* __restrict__ q_c, const float* __restrict__ k_c,
                                                           int lq, int64_t n_cap, int64_t mid0, int64_t n_mid, int dc,
-                                                          float* __restrict__ s_out, uint32_t* __restrict__ m_key) {
+                                                          int ng, float* __restrict__ s_out,
+                                                          uint32_t* __restrict__ m_key) {
   __shared__ float qs[kScK][kScT + 4];
   __shared__ float ks[kScK][kScT + 4];
   __shared__ float rmax[kScT][17];
-  const int b = blockIdx.z;
+  const int bg = blockIdx.z;                     // sequence * ng + group
+  const int b = bg / ng, col0 = (bg % ng) * (dc / ng), dg = dc / ng;
   const int i0 = blockIdx.y * kScT;
   const int64_t j0 = (int64_t)blockIdx.x * kScT;
   const int tid = threadIdx.x;
@@ -192,7 +219,7 @@ __global__ void __launch_bounds__(256) score_tiled_kernel(const float* __restric
   float acc[4][4] = {};
   const float* qb = q_c + (int64_t)b * lq * dc;
   const float* kb = k_c + ((int64_t)b * n_cap + mid0) * dc;
-  for (int d0 = 0; d0 < dc; d0 += kScK) {
+  for (int d0 = col0; d0 < col0 + dg; d0 += kScK) {
     for (int t = tid; t < kScT * kScK; t += 256) {
       const int r = t / kScK, c = t % kScK;
       qs[c][r] = (i0 + r < lq) ? qb[(int64_t)(i0 + r) * dc + d0 + c] : 0.f;
@@ -219,7 +246,7 @@ __global__ void __launch_bounds__(256) score_tiled_kernel(const float* __restric
     for (int v = 0; v < 4; ++v) {
       const int64_t j = j0 + tx * 4 + v;
       if (i < lq && j < n_mid) {
-        s_out[((int64_t)b * lq + i) * n_mid + j] = acc[u][v];
+        s_out[((int64_t)bg * lq + i) * n_mid + j] = acc[u][v];
         m = fmaxf(m, acc[u][v]);
       }
     }
@@ -229,7 +256,7 @@ __global__ void __launch_bounds__(256) score_tiled_kernel(const float* __restric
   if (tid < kScT && i0 + tid < lq) {
     float m = -INFINITY;
     for (int x = 0; x < 16; ++x) m = fmaxf(m, rmax[tid][x]);
-    if (m > -INFINITY) atomicMax(&m_key[b * lq + i0 + tid], order_key(m));
+    if (m > -INFINITY) atomicMax(&m_key[(int64_t)bg * lq + i0 + tid], order_key(m));
   }
 }
 

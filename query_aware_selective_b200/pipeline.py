@@ -45,6 +45,13 @@ def _region_lo(c0: int, n_init: int, window: int) -> int:
     return min(c0, max(n_init, c0 - window))
 
 
+def block_diagonal(w_groups: torch.Tensor) -> torch.Tensor:
+    """Per-head selection: the groups' maps [G, gin, d_g] stacked into the one
+    [G * gin, G * d_g] map the compression calls take (zero off the diagonal
+    blocks), so that group g's compressed columns see group g's heads only."""
+    return torch.block_diag(*w_groups.unbind(0)).contiguous()
+
+
 class _Compressor:
     """The two compression maps of a layer (queries: Hq heads in; keys: Hkv heads in,
     expanded to Hq). With bf16 inputs and a shape the packed path takes, the weights
@@ -98,20 +105,30 @@ class EsaPrefill:
     select middle tokens, attend over initial + selected + local."""
 
     def __init__(self, batch: int, n_ctx: int, chunk: int, hq: int, hkv: int, head_dim: int, d_c: int,
-                 p: _abi.EsaParams, dtype=torch.bfloat16, device="cuda"):
+                 p: _abi.EsaParams, dtype=torch.bfloat16, device="cuda", per_head: bool = False):
         self.batch, self.n_ctx, self.chunk = batch, n_ctx, chunk
         self.hq, self.hkv, self.d, self.d_c, self.p = hq, hkv, head_dim, d_c, p
+        self.per_head = per_head      # one selection per KV head (block-diagonal maps)
+        lists = (batch, hkv) if per_head else (batch,)
         self.device = torch.device(device)
         self.k_c = torch.zeros((batch, n_ctx, d_c), dtype=torch.float32, device=device)
         self.q_c = torch.empty((batch, chunk, d_c), dtype=torch.float32, device=device)
-        self.idx = torch.empty((batch, p.topk), dtype=torch.int32, device=device)
-        self.count = torch.empty((batch,), dtype=torch.int32, device=device)
+        self.idx = torch.empty((*lists, p.topk), dtype=torch.int32, device=device)
+        self.count = torch.empty(lists, dtype=torch.int32, device=device)
         self.out = torch.empty((batch, n_ctx, hq, head_dim), dtype=dtype, device=device)
         code = _abi.ESA_BF16 if dtype == torch.bfloat16 else _abi.ESA_F32
-        ws_sel = max(_abi.score_select_workspace_size(batch, min(chunk, n_ctx - c0), n_ctx, c0, d_c, p)
-                     for c0 in range(0, n_ctx, chunk))
-        ws_att = max(_abi.sparse_attn_workspace_size(batch, min(chunk, n_ctx - c0), c0, hq, hkv, head_dim, code, p)
-                     for c0 in range(0, n_ctx, chunk))
+        if per_head:
+            ws_sel = max(_abi.score_select_heads_workspace_size(batch, min(chunk, n_ctx - c0), n_ctx, c0, d_c, hkv, p)
+                         for c0 in range(0, n_ctx, chunk))
+            ws_att = max(_abi.sparse_attn_heads_workspace_size(batch, min(chunk, n_ctx - c0), c0, hq, hkv, head_dim,
+                                                               code, p)
+                         for c0 in range(0, n_ctx, chunk))
+        else:
+            ws_sel = max(_abi.score_select_workspace_size(batch, min(chunk, n_ctx - c0), n_ctx, c0, d_c, p)
+                         for c0 in range(0, n_ctx, chunk))
+            ws_att = max(_abi.sparse_attn_workspace_size(batch, min(chunk, n_ctx - c0), c0, hq, hkv, head_dim, code,
+                                                         p)
+                         for c0 in range(0, n_ctx, chunk))
         self.ws_sel = torch.empty(ws_sel + 256, dtype=torch.uint8, device=device)
         self.ws_att = torch.empty(ws_att + 256, dtype=torch.uint8, device=device) if ws_att else None
         self.out_views = []
@@ -135,7 +152,11 @@ class EsaPrefill:
         for s in range(b):
             self.cmp.queries(q[s, c0:c0 + lq], out=self.q_c[s, :lq])
         q_c = self.q_c[:, :lq] if lq == self.chunk else self.q_c[:, :lq].contiguous()
-        _abi.score_select(q_c, self.k_c, c0, self.p, idx=self.idx, count=self.count, workspace=self.ws_sel)
+        if self.per_head:
+            _abi.score_select_heads(q_c, self.k_c, c0, self.hkv, self.p, idx=self.idx, count=self.count,
+                                    workspace=self.ws_sel)
+        else:
+            _abi.score_select(q_c, self.k_c, c0, self.p, idx=self.idx, count=self.count, workspace=self.ws_sel)
         qv = q[:, c0:c0 + lq]
         if not qv.is_contiguous():
             qv = qv.contiguous()
@@ -143,7 +164,8 @@ class EsaPrefill:
         target = ov if ov.is_contiguous() else torch.empty_like(ov)
         if attn_events is not None:
             attn_events[0].record()
-        _abi.sparse_attn(qv, k, v, c0, self.idx, self.count, self.p, out=target, workspace=self.ws_att)
+        attn = _abi.sparse_attn_heads if self.per_head else _abi.sparse_attn
+        attn(qv, k, v, c0, self.idx, self.count, self.p, out=target, workspace=self.ws_att)
         if attn_events is not None:
             attn_events[1].record()
         if target is not ov:
@@ -172,18 +194,26 @@ class EsaDecode:
     n_ctx tokens; the query sits at position n_ctx - 1."""
 
     def __init__(self, batch: int, n_ctx: int, hq: int, hkv: int, head_dim: int, d_c: int, p: _abi.EsaParams,
-                 dtype=torch.bfloat16, device="cuda"):
+                 dtype=torch.bfloat16, device="cuda", per_head: bool = False):
         self.batch, self.n_ctx, self.hq, self.hkv, self.d, self.d_c, self.p = batch, n_ctx, hq, hkv, head_dim, d_c, p
+        # per_head: one selection per KV head (the compression maps given to step() are
+        # then block-diagonal, see block_diagonal)
+        self.per_head = per_head
+        lists = (batch, hkv) if per_head else (batch,)
         self.k_c = torch.zeros((batch, n_ctx, d_c), dtype=torch.float32, device=device)
         self.q_c = torch.empty((batch, 1, d_c), dtype=torch.float32, device=device)
-        self.idx = torch.empty((batch, p.topk), dtype=torch.int32, device=device)
-        self.count = torch.empty((batch,), dtype=torch.int32, device=device)
+        self.idx = torch.empty((*lists, p.topk), dtype=torch.int32, device=device)
+        self.count = torch.empty(lists, dtype=torch.int32, device=device)
         self.out = torch.empty((batch, 1, hq, head_dim), dtype=dtype, device=device)
         code = _abi.ESA_BF16 if dtype == torch.bfloat16 else _abi.ESA_F32
         c0 = n_ctx - 1
-        self.ws_sel = torch.empty(_abi.score_select_workspace_size(batch, 1, n_ctx, c0, d_c, p) + 256,
-                                  dtype=torch.uint8, device=device)
-        nb = _abi.sparse_attn_workspace_size(batch, 1, c0, hq, hkv, head_dim, code, p)
+        if per_head:
+            n_sel = _abi.score_select_heads_workspace_size(batch, 1, n_ctx, c0, d_c, hkv, p)
+            nb = _abi.sparse_attn_heads_workspace_size(batch, 1, c0, hq, hkv, head_dim, code, p)
+        else:
+            n_sel = _abi.score_select_workspace_size(batch, 1, n_ctx, c0, d_c, p)
+            nb = _abi.sparse_attn_workspace_size(batch, 1, c0, hq, hkv, head_dim, code, p)
+        self.ws_sel = torch.empty(n_sel + 256, dtype=torch.uint8, device=device)
         self.ws_att = torch.empty(nb + 256, dtype=torch.uint8, device=device) if nb else None
         self.cmp = _Compressor(hq, hkv, head_dim, d_c, dtype, device)
         self.side = torch.cuda.Stream(device=device)
@@ -216,10 +246,16 @@ class EsaDecode:
         self.cmp.queries(q[:, 0], out=self.q_c.view(self.batch, self.d_c))
         if ev is not None:
             ev[1].record()
-        _abi.score_select(self.q_c, self.k_c, pos, self.p, idx=self.idx, count=self.count, workspace=self.ws_sel)
+        if self.per_head:
+            _abi.score_select_heads(self.q_c, self.k_c, pos, self.hkv, self.p, idx=self.idx, count=self.count,
+                                    workspace=self.ws_sel)
+        else:
+            _abi.score_select(self.q_c, self.k_c, pos, self.p, idx=self.idx, count=self.count,
+                              workspace=self.ws_sel)
         if ev is not None:
             ev[2].record()
-        _abi.sparse_attn(q, k, v, pos, self.idx, self.count, self.p, out=self.out, workspace=self.ws_att)
+        attn = _abi.sparse_attn_heads if self.per_head else _abi.sparse_attn
+        attn(q, k, v, pos, self.idx, self.count, self.p, out=self.out, workspace=self.ws_att)
         cur.wait_stream(self.side)
         if ev is not None:
             ev[3].record()

@@ -139,6 +139,21 @@ def make_esa_inputs(w: EsaWorkload, device="cpu", n_ctx: Optional[int] = None,
     return out
 
 
+def make_group_maps(w: EsaWorkload, device="cpu") -> tuple:
+    """Per-head selection: the groups' one-layer maps for queries and keys, each
+    [Hkv, G * D, d' / Hkv] ~ N(0, 1 / (G * D)), from their own generator (seed
+    w.seed + 1000) so that the workload's Q, K, V stay those of the merged form.
+    Returns (wq_groups, wk_groups), fp32."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed + 1000)
+    g = w.hq // w.hkv
+    gin, dg = g * w.head_dim, w.d_c // w.hkv
+    std = 1.0 / math.sqrt(gin)
+    wq = torch.randn((w.hkv, gin, dg), generator=gen, device=device, dtype=torch.float32) * std
+    wk = torch.randn((w.hkv, gin, dg), generator=gen, device=device, dtype=torch.float32) * std
+    return wq, wk
+
+
 def needle_positions(w: EsaWorkload, n_ctx: int, gen: torch.Generator) -> torch.Tensor:
     """Needle positions per sequence: one per equal segment of the middle,
     at least eps from either edge of the segment (hence >= 2*eps+1 apart)."""
