@@ -113,8 +113,11 @@ class EsaPrefill:
         self.device = torch.device(device)
         self.k_c = torch.zeros((batch, n_ctx, d_c), dtype=torch.float32, device=device)
         self.q_c = torch.empty((batch, chunk, d_c), dtype=torch.float32, device=device)
-        self.idx = torch.empty((*lists, p.topk), dtype=torch.int32, device=device)
-        self.count = torch.empty(lists, dtype=torch.int32, device=device)
+        # one index list (set) per chunk: chunk j + 1's selection may run while chunk j
+        # attends, and a chunk's selection stays readable after run()
+        n_chunks = (n_ctx + chunk - 1) // chunk
+        self.idx_all = torch.empty((n_chunks, *lists, p.topk), dtype=torch.int32, device=device)
+        self.count_all = torch.empty((n_chunks, *lists), dtype=torch.int32, device=device)
         self.out = torch.empty((batch, n_ctx, hq, head_dim), dtype=dtype, device=device)
         code = _abi.ESA_BF16 if dtype == torch.bfloat16 else _abi.ESA_F32
         if per_head:
@@ -138,25 +141,25 @@ class EsaPrefill:
     def chunks(self):
         return [(c0, min(self.chunk, self.n_ctx - c0)) for c0 in range(0, self.n_ctx, self.chunk)]
 
-    def run_chunk(self, c0: int, lq: int, q, k, v, wq, wk, attn_events=None):
+    def front(self, ci: int, c0: int, lq: int, q, k):
+        """Everything of chunk ci before its attention, on the current stream: compress
+        the chunk's keys into the compressed cache (first read by a later chunk: the
+        middle ends `window` tokens before c0) and its queries, select into the
+        chunk's index list."""
         b = self.batch
-        cur = torch.cuda.current_stream()
-        self.cmp.pack_if_changed(wq, wk)
-        # The chunk's own keys are local to it (the middle ends `window` tokens before
-        # c0), so its compressed keys are first read by a later chunk's scoring: they
-        # are computed on a second stream beside this chunk's work and joined at the end.
-        self.side.wait_stream(cur)
-        with torch.cuda.stream(self.side):
-            for s in range(b):
-                self.cmp.keys(k[s, c0:c0 + lq], out=self.k_c[s, c0:c0 + lq])
         for s in range(b):
+            self.cmp.keys(k[s, c0:c0 + lq], out=self.k_c[s, c0:c0 + lq])
             self.cmp.queries(q[s, c0:c0 + lq], out=self.q_c[s, :lq])
         q_c = self.q_c[:, :lq] if lq == self.chunk else self.q_c[:, :lq].contiguous()
         if self.per_head:
-            _abi.score_select_heads(q_c, self.k_c, c0, self.hkv, self.p, idx=self.idx, count=self.count,
-                                    workspace=self.ws_sel)
+            _abi.score_select_heads(q_c, self.k_c, c0, self.hkv, self.p, idx=self.idx_all[ci],
+                                    count=self.count_all[ci], workspace=self.ws_sel)
         else:
-            _abi.score_select(q_c, self.k_c, c0, self.p, idx=self.idx, count=self.count, workspace=self.ws_sel)
+            _abi.score_select(q_c, self.k_c, c0, self.p, idx=self.idx_all[ci], count=self.count_all[ci],
+                              workspace=self.ws_sel)
+
+    def attend(self, ci: int, c0: int, lq: int, q, k, v, attn_events=None):
+        """Chunk ci's attention over initial + its selected + local tokens."""
         qv = q[:, c0:c0 + lq]
         if not qv.is_contiguous():
             qv = qv.contiguous()
@@ -165,26 +168,44 @@ class EsaPrefill:
         if attn_events is not None:
             attn_events[0].record()
         attn = _abi.sparse_attn_heads if self.per_head else _abi.sparse_attn
-        attn(qv, k, v, c0, self.idx, self.count, self.p, out=target, workspace=self.ws_att)
+        attn(qv, k, v, c0, self.idx_all[ci], self.count_all[ci], self.p, out=target, workspace=self.ws_att)
         if attn_events is not None:
             attn_events[1].record()
         if target is not ov:
             ov.copy_(target)
-        cur.wait_stream(self.side)
+
+    def run_chunk(self, c0: int, lq: int, q, k, v, wq, wk, attn_events=None):
+        """One chunk, in order on the current stream (the chunks must come in order)."""
+        self.cmp.pack_if_changed(wq, wk)
+        ci = c0 // self.chunk
+        self.front(ci, c0, lq, q, k)
+        self.attend(ci, c0, lq, q, k, v, attn_events)
 
     def run(self, q, k, v, wq, wk, attn_events=None, external_events=False):
         """q [B, N, Hq, D], k, v [B, N, Hkv, D] (device), wq, wk [Hq*D, d'].
         attn_events: optional list that receives one (start, end) CUDA event pair per
         attention launch (external_events: made to be captured in a graph). Returns
         the output [B, N, Hq, D]. The weights are packed for the tensor-core
-        compression at the start of every run."""
+        compression at the start of every run.
+
+        Two streams: the chunks' front work (compression and selection) runs in order
+        on a second stream, each chunk's attention on the current stream once its
+        selection is done, so chunk j + 1's selection overlaps chunk j's attention."""
+        main = torch.cuda.current_stream()
         self.cmp.pack(wq, wk)
-        for c0, lq in self.chunks():
+        self.side.wait_stream(main)
+        for ci, (c0, lq) in enumerate(self.chunks()):
+            done = torch.cuda.Event()
+            with torch.cuda.stream(self.side):
+                self.front(ci, c0, lq, q, k)
+                done.record()
+            main.wait_event(done)
             ev = None
             if attn_events is not None:
                 ev = (_timing_event(external_events), _timing_event(external_events))
                 attn_events.append(ev)
-            self.run_chunk(c0, lq, q, k, v, wq, wk, ev)
+            self.attend(ci, c0, lq, q, k, v, ev)
+        main.wait_stream(self.side)
         return self.out
 
 
