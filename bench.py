@@ -48,7 +48,7 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--prefill-ctx", type=int, default=0,
                     help="shorter prefill context (profiling a small case); the line then names that workload")
-    ap.add_argument("--only", choices=["decode", "decode_per_head", "moba"], default=None,
+    ap.add_argument("--only", choices=["decode", "decode_per_head", "moba", "moba_decode"], default=None,
                     help="profiling: run one of the other workloads alone and print its figures")
     ap.add_argument("--decode-batch", type=int, default=0, help="profiling: decode batch (default: the workload's)")
     ap.add_argument("--moba-seq", type=int, default=0, help="profiling: MoBA sequence length (default: the workload's)")
@@ -222,6 +222,8 @@ def run_only(args):
     flush = make_flush(dev)
     if args.only == "moba":
         out = bench_moba(args, dev, flush, make_dist_max(), peaks, peak_src, 1)
+    elif args.only == "moba_decode":
+        out = bench_moba_decode(args, dev, flush, make_dist_max(), peaks, peak_src, 1)
     else:
         out = bench_decode(args, dev, flush, make_dist_max(), peaks, peak_src, 1, per_head=args.only == "decode_per_head")
     print(json.dumps({"only": args.only, **out}), flush=True)
@@ -337,6 +339,8 @@ def run_ours(args):
                                                                 per_head=True)
         torch.cuda.empty_cache()
         line["also"]["moba_prefill_64k"] = bench_moba(args, dev, flush, dist_max, peaks, peak_src, world)
+        torch.cuda.empty_cache()
+        line["also"]["moba_decode_64k"] = bench_moba_decode(args, dev, flush, dist_max, peaks, peak_src, world)
     line["clocks"] = sampler.stop()
     line["gpu"] = props.name
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -391,6 +395,28 @@ def bench_decode(args, dev, flush, dist_max, peaks, peak_src, world, per_head=Fa
                          "peak_source": f"{peak_src} HBM copy"},
             "phases": {"score_select_ms": round(sel_ms, 4), "score_select_gbs": round(sel_gbs, 1),
                        "sparse_attn_ms": round(att_ms, 4), "sparse_attn_gbs": round(att_gbs, 1)}}
+
+
+def bench_moba_decode(args, dev, flush, dist_max, peaks, peak_src, world):
+    """MoBA decode: batch 16, 32 heads, one query at position 65535, top-3 past blocks."""
+    import torch
+    from query_aware_selective_b200 import cost, pipeline, synthetic
+    w = synthetic.MOBA_DECODE_64K
+    inp = synthetic.make_moba_decode_inputs(w, device=dev)
+    dec = pipeline.MobaDecode(w.batch, w.seq, w.heads, w.head_dim, w.block, w.topk, device=dev)
+    dec.fill(inp["k"])
+    torch.cuda.synchronize()
+    graph = pipeline.graph_of(lambda: dec.step(inp["q"], inp["k"], inp["v"]))
+    steps = max(args.steps, 20)
+    ms, total = time_steps(graph.replay, steps, args.warmup, flush, dist_max)
+    by = cost.moba_decode_bytes(w.batch, w.seq, w.heads, w.head_dim, w.block, w.topk)
+    gbs = by["total"] / (total / steps / 1e3) / 1e9
+    hbm = peaks["hbm_gbs"]
+    return {"workload": w.name, "value": round(world * w.batch * steps / (total / 1e3), 1), "unit": "tok/s",
+            "ms_per_step": round(total / steps, 4), "steps": steps, "execution": "one CUDA graph per step",
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "bytes_per_step": by["total"],
+                         "peak_source": f"{peak_src} HBM copy"}}
 
 
 def bench_moba(args, dev, flush, dist_max, peaks, peak_src, world):

@@ -282,6 +282,36 @@ esa_status_t moba_block_gate_attn(const void* q, const void* k, const void* v, e
 size_t moba_workspace_size(int32_t which, int32_t batch, int64_t seq, int32_t heads,
                            int32_t head_dim, int32_t block, int32_t topk);
 
+/* moba_block_means - the block means of a key cache (MoBA article, section 2: a block
+ * is represented by the mean of its keys), for blocks [blk_begin, blk_end) of
+ * kbar [batch, heads, ceil(n_cap / block), head_dim] fp32 (caller-owned). k: [batch,
+ * n_cap, heads, head_dim] bf16. A decode loop computes the means of the complete
+ * blocks once and one more each time a block fills. Requires head_dim 128, block a
+ * multiple of 16 (<= 1024 blocks). */
+esa_status_t moba_block_means(const void* k, esa_dtype_t dt, int32_t batch, int64_t n_cap, int32_t heads,
+                              int32_t head_dim, int32_t block, int32_t blk_begin, int32_t blk_end,
+                              float* kbar, void* stream);
+
+/* moba_decode_attn - one MoBA decode step (MoBA article, sections 2-3, for a single
+ * query): per (sequence, head) the gate scores the query at position pos against the
+ * means of the past blocks (blocks < pos / block), keeps the top min(topk, past) by
+ * (score desc, block asc), and the attention runs over the kept blocks plus the
+ * current block up to pos (one softmax).
+ *   q:    [batch, 1, heads, head_dim] bf16;  k, v: [batch, n_cap, heads, head_dim] bf16
+ *   kbar: [batch, heads, ceil(n_cap / block), head_dim] fp32 with every past block's
+ *         mean (moba_block_means)
+ *   o:    [batch, 1, heads, head_dim];  lse: NULL or [batch, 1, heads] fp32
+ *   blocks_out: NULL or [batch, heads, topk + 1] int16: kept blocks ascending, the
+ *         current block, -1 padding
+ * Requires 1 <= topk <= 15, 0 <= pos < n_cap, head_dim 128. */
+esa_status_t moba_decode_attn(const void* q, const void* k, const void* v, esa_dtype_t dt, int32_t batch,
+                              int64_t n_cap, int64_t pos, int32_t heads, int32_t head_dim, int32_t block,
+                              int32_t topk, const float* kbar, float scale, void* o, float* lse,
+                              int16_t* blocks_out, void* workspace, size_t ws_bytes, void* stream);
+
+size_t moba_decode_workspace_size(int32_t batch, int64_t n_cap, int64_t pos, int32_t heads, int32_t head_dim,
+                                  int32_t block, int32_t topk);
+
 /* ------------------------------------------------------------------- status -- */
 
 /* Message for the last non-OK status returned on this thread ("" if none). */

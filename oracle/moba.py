@@ -112,3 +112,16 @@ def moba(q, k, v, block, topk, scale=None, positions=None):
     blocks = gate(q, kbar, block, topk, positions)
     o, lse = attend(q, k, v, blocks, block, scale, positions)
     return dict(kbar=kbar, blocks=blocks, o=o, lse=lse)
+
+
+def decode_step(q1, k, v, block, topk, scale=None):
+    """MoBA for one query per sequence at the last cached position (decode): the same
+    gate and attention as the prefill, evaluated at position S - 1 only.
+    q1: [B, 1, H, D]; k, v: [B, S, H, D]. Returns dict(blocks [B, 1, H, topk+1],
+    o [B, 1, H, D], lse [B, 1, H])."""
+    bsz, s, h, d = np.shape(k)
+    q = np.zeros((bsz, s, h, d))
+    q[:, s - 1] = np.asarray(q1, dtype=np.float64)[:, 0]
+    out = moba(q, k, v, block, topk, scale, positions=[s - 1])
+    return dict(blocks=out["blocks"], o=out["o"], lse=out["lse"])
+

@@ -6,9 +6,11 @@ benchmark inputs; ``cost`` holds the algorithmic byte and flop counts used for
 rooflines.
 """
 from ._abi import (EsaError, EsaParams, compress, compress_pack, compress_pack_size, compress_packed, device_status,
-                   load, moba_block_attn, moba_block_gate, moba_block_gate_attn, params, score_select,
+                   load, moba_block_attn, moba_block_gate, moba_block_gate_attn, moba_block_means,
+                   moba_decode_attn, params, score_select,
                    score_select_heads, sparse_attn, sparse_attn_heads)
 
 __all__ = ["EsaError", "EsaParams", "compress", "compress_pack", "compress_pack_size", "compress_packed",
-           "device_status", "load", "moba_block_attn", "moba_block_gate", "moba_block_gate_attn", "params",
+           "device_status", "load", "moba_block_attn", "moba_block_gate", "moba_block_gate_attn", "moba_block_means",
+           "moba_decode_attn", "params",
            "score_select", "score_select_heads", "sparse_attn", "sparse_attn_heads"]

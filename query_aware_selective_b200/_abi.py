@@ -56,6 +56,10 @@ SIGNATURES = {
     "esa_score_select_noalloc": (ctypes.c_int, [_vp, _vp, _i32, _i32, _i64, _i64, _i32, EsaParams, _vp, _vp, _vp,
                                                 _vp]),
     "esa_score_select_noalloc_capacity": (_sz, []),
+    "moba_block_means": (ctypes.c_int, [_vp, ctypes.c_int, _i32, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
+    "moba_decode_attn": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i64, _i64, _i32, _i32, _i32, _i32, _vp,
+                                        _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moba_decode_workspace_size": (_sz, [_i32, _i64, _i64, _i32, _i32, _i32, _i32]),
     "esa_score_select_heads": (ctypes.c_int, [_vp, _vp, _i32, _i32, _i64, _i64, _i32, _i32, EsaParams, _vp, _vp,
                                               _vp, _vp, _sz, _vp]),
     "esa_score_select_heads_workspace_size": (_sz, [_i32, _i32, _i64, _i64, _i32, _i32, EsaParams]),
@@ -330,6 +334,48 @@ def sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, c0: int, idx:
                                   _ptr(count), p, scale, _ptr(out), _ptr(lse) if want_lse else None, wp, wn,
                                   _stream()), "esa_sparse_attn")
     return out, (lse if want_lse else None)
+
+
+def moba_block_means(k: torch.Tensor, block: int, blk_begin: int = 0, blk_end: Optional[int] = None,
+                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """moba_block_means: means of blocks [blk_begin, blk_end) of k [B, n_cap, H, D] bf16
+    into kbar [B, H, ceil(n_cap / block), D] fp32 (allocated when out is None)."""
+    _dev(k)
+    b, n_cap, h, d = k.shape
+    nb = (n_cap + block - 1) // block
+    if out is None:
+        out = torch.zeros((b, h, nb, d), dtype=torch.float32, device=k.device)
+    end = nb if blk_end is None else blk_end
+    _check(load().moba_block_means(_ptr(k), _dtype_code(k), b, n_cap, h, d, block, blk_begin, end, _ptr(out),
+                                   _stream()), "moba_block_means")
+    return out
+
+
+def moba_decode_workspace_size(batch, n_cap, pos, heads, d, block, topk) -> int:
+    return load().moba_decode_workspace_size(batch, n_cap, pos, heads, d, block, topk)
+
+
+def moba_decode_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pos: int, kbar: torch.Tensor, block: int,
+                     topk: int, scale: float = 0.0, want_lse: bool = False, want_blocks: bool = False,
+                     out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                     blocks: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None):
+    """moba_decode_attn: one decode step for the query q [B, 1, H, D] at position pos.
+    Returns (o [B, 1, H, D], lse [B, 1, H] or None, blocks [B, H, topk+1] int16 or None)."""
+    _dev(q, k, v, kbar)
+    b, _, h, d = q.shape
+    n_cap = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((b, 1, h), dtype=torch.float32, device=q.device)
+    if want_blocks and blocks is None:
+        blocks = torch.empty((b, h, topk + 1), dtype=torch.int16, device=q.device)
+    ws = _workspace(moba_decode_workspace_size(b, n_cap, pos, h, d, block, topk), q.device, workspace)
+    wp, wn = _ws_ptr(ws)
+    _check(load().moba_decode_attn(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), b, n_cap, pos, h, d, block, topk,
+                                   _ptr(kbar), scale, _ptr(out), _ptr(lse) if want_lse else None,
+                                   _ptr(blocks) if want_blocks else None, wp, wn, _stream()), "moba_decode_attn")
+    return out, (lse if want_lse else None), (blocks if want_blocks else None)
 
 
 def moba_workspace_size(which, batch, seq, heads, d, block, topk) -> int:

@@ -108,3 +108,15 @@ def moba_flops(seq: int, heads: int, d: int, block: int, topk: int) -> dict:
         gate += n_q * c * d * 2                     # <q, mean> against every past block
     att = 4 * d * heads * keys
     return dict(attention=att, gate=gate * heads, total=att + gate * heads)
+
+
+def moba_decode_bytes(batch: int, n_ctx: int, heads: int, d: int, block: int, topk: int,
+                      kv_bytes: int = 2) -> dict:
+    """Compulsory HBM bytes of one MoBA decode step (query at n_ctx - 1): the past
+    blocks' means (fp32, read by the gate) and the K and V rows of the kept blocks and
+    of the current block up to the query, for every (sequence, head)."""
+    cur = (n_ctx - 1) // block
+    means = batch * heads * cur * d * 4
+    keys = min(topk, cur) * block + (n_ctx - cur * block)
+    rows = batch * heads * keys * d * kv_bytes * 2
+    return dict(block_means=means, kv_rows=rows, total=means + rows)

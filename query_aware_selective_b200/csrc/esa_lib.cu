@@ -1031,7 +1031,7 @@ esa_status_t moba_gate_launch(const MobaWs& w, const void* q, const void* k, int
                               int32_t block, int32_t topk, int16_t* blocks_out, cudaStream_t s) {
   const int nb = (int)cdiv(seq, block);
   esa::moba_mean_kernel<__nv_bfloat16><<<dim3(nb, heads, batch), 256, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(k), seq, heads, 128, block, w.kbar);
+      static_cast<const __nv_bfloat16*>(k), seq, heads, 128, block, 0, nb, w.kbar);
   ESA_LAUNCH_CHECK("moba_mean_kernel");
   esa::moba_gate_kernel<__nv_bfloat16, 128><<<dim3((unsigned)cdiv(seq, 128), heads, batch), 128, 0, s>>>(
       static_cast<const __nv_bfloat16*>(q), w.kbar, seq, heads, block, nb, topk, blocks_out);
@@ -1173,6 +1173,81 @@ esa_status_t moba_block_gate_attn(const void* q, const void* k, const void* v, e
   if (st != ESA_OK) return st;
   st = moba_attn_launch(w, q, k, v, batch, seq, heads, block, topk, blocks, scale, o, lse, s);
   return st == ESA_OK ? ok() : st;
+}
+
+// ------------------------------------------------------------------ MoBA decode --
+esa_status_t moba_block_means(const void* k, esa_dtype_t dt, int32_t batch, int64_t n_cap, int32_t heads,
+                              int32_t head_dim, int32_t block, int32_t blk_begin, int32_t blk_end, float* kbar,
+                              void* stream) {
+  esa_status_t st = moba_check(k, k, dt, batch, n_cap, heads, head_dim, block, 0);
+  if (st != ESA_OK) return st;
+  if (!kbar) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  const int nb = (int)cdiv(n_cap, block);
+  blk_begin = std::max(0, blk_begin);
+  blk_end = std::min(nb, blk_end);
+  if (blk_end <= blk_begin) return ok();
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  esa::moba_mean_kernel<__nv_bfloat16><<<dim3(blk_end - blk_begin, heads, batch), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(k), n_cap, heads, 128, block, blk_begin, nb, kbar);
+  ESA_LAUNCH_CHECK("moba_mean_kernel");
+  return ok();
+}
+
+namespace {
+
+// the attention half of a MoBA decode step, as esa_sparse_attn_heads sees it: no
+// initial tokens, the kept blocks' positions as the selected middle, and the current
+// block up to the query as the local part
+esa_params_t moba_decode_params(int64_t pos, int32_t block, int32_t topk) {
+  esa_params_t p{};
+  p.n_init = 0;
+  p.window = (int32_t)(pos - (pos / block) * block);
+  p.topk = topk * block;
+  p.eps = 0;
+  p.clamp_c = INFINITY;
+  return p;
+}
+
+}  // namespace
+
+size_t moba_decode_workspace_size(int32_t batch, int64_t n_cap, int64_t pos, int32_t heads, int32_t head_dim,
+                                  int32_t block, int32_t topk) {
+  if (batch <= 0 || heads <= 0 || block <= 0 || topk <= 0) return 0;
+  const int64_t lists = (int64_t)batch * heads;
+  const esa_params_t p = moba_decode_params(pos, block, topk);
+  (void)n_cap;
+  return up256((size_t)lists * topk * block * sizeof(int32_t)) + up256((size_t)lists * sizeof(int32_t)) +
+         sparse_attn_ws(batch, 1, pos, heads, heads, head_dim, ESA_BF16, p, heads);
+}
+
+esa_status_t moba_decode_attn(const void* q, const void* k, const void* v, esa_dtype_t dt, int32_t batch,
+                              int64_t n_cap, int64_t pos, int32_t heads, int32_t head_dim, int32_t block,
+                              int32_t topk, const float* kbar, float scale, void* o, float* lse,
+                              int16_t* blocks_out, void* workspace, size_t ws_bytes, void* stream) {
+  esa_status_t st = moba_check(q, k, dt, batch, n_cap, heads, head_dim, block, topk);
+  if (st != ESA_OK) return st;
+  if (topk < 1) return fail(ESA_ERR_INVALID_ARG, "topk must be >= 1");
+  if (pos < 0 || pos >= n_cap) return fail(ESA_ERR_INVALID_ARG, "need 0 <= pos < n_cap");
+  if (!v || !o || !kbar) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(v, 16) || !aligned(o, 16) || !aligned(kbar, 16))
+    return fail(ESA_ERR_INVALID_ARG, "16-byte alignment required");
+  const size_t need = moba_decode_workspace_size(batch, n_cap, pos, heads, head_dim, block, topk);
+  if (!workspace || ws_bytes < need || !aligned(workspace, 256))
+    return fail(ESA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need, ws_bytes);
+  const int64_t lists = (int64_t)batch * heads;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws);
+  ws += up256((size_t)lists * topk * block * sizeof(int32_t));
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws);
+  ws += up256((size_t)lists * sizeof(int32_t));
+  const size_t ws_att = ws_bytes - (size_t)(ws - static_cast<uint8_t*>(workspace));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int nb = (int)cdiv(n_cap, block);
+  esa::moba_decode_gate_kernel<__nv_bfloat16, 128><<<(unsigned)cdiv(lists, 4), 128, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(q), kbar, batch, heads, nb, block, pos, topk, idx, cnt, blocks_out);
+  ESA_LAUNCH_CHECK("moba_decode_gate_kernel");
+  return sparse_attn_impl(q, k, v, dt, batch, 1, n_cap, pos, heads, heads, head_dim, idx, cnt,
+                          moba_decode_params(pos, block, topk), scale, o, lse, ws, ws_att, stream, heads);
 }
 
 

@@ -25,10 +25,11 @@ constexpr int kMobaMaxTopk = 15;
 // ------------------------------------------------------------------ block means --
 // grid (n_blocks, H, B), 256 threads: thread = (d pair, row phase); fixed order sums.
 template <typename T>
+// Blocks [blk0, blk0 + gridDim.x) of kbar [B, H, nb_total, D].
 __global__ void __launch_bounds__(256) moba_mean_kernel(const T* __restrict__ k, int64_t seq, int heads, int d,
-                                                        int block, float* __restrict__ kbar) {
+                                                        int block, int blk0, int nb_total, float* __restrict__ kbar) {
   __shared__ float part[256][2];
-  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int blk = blk0 + (int)blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int pairs = d / 2;
   const int dp = threadIdx.x % pairs;
   const int ph = threadIdx.x / pairs;
@@ -51,7 +52,7 @@ __global__ void __launch_bounds__(256) moba_mean_kernel(const T* __restrict__ k,
       s1 += part[q * pairs + threadIdx.x][1];
     }
     const float inv = 1.f / (float)(r1 - r0);
-    float* o = kbar + (((int64_t)b * heads + h) * gridDim.x + blk) * d + 2 * threadIdx.x;
+    float* o = kbar + (((int64_t)b * heads + h) * nb_total + blk) * d + 2 * threadIdx.x;
     o[0] = s0 * inv;
     o[1] = s1 * inv;
   }
@@ -352,6 +353,76 @@ __global__ void __launch_bounds__(256) moba_combine_kernel(const float* __restri
 #pragma unroll
   for (int e = 0; e < D / 32; ++e) o[row * D + lane + 32 * e] = __float2bfloat16_rn(acc[e] * inv);
   if (lane == 0 && lse) lse[row] = M + __logf(L);
+}
+
+// ------------------------------------------------------------------ decode gate --
+// One query per (sequence, head) at position pos (decode; MoBA article, section 2: the
+// gate of one query over the means of the past blocks). One warp per (sequence, head):
+// the query row is spread over the lanes (D / 32 values each), every past block's mean
+// is one warp dot product, and the kept list is the prefill gate's (ties to the lower
+// block). The kept blocks, ascending, are expanded into positions: idx[list, j * block
+// + t] = blk_j * block + t, count[list] = kept * block, so that the attention can take
+// them as a per-head list of selected middle positions (the current block is the local
+// part [cur * block, pos]). blocks_out (optional): kept blocks then the current block.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) moba_decode_gate_kernel(const T* __restrict__ q, const float* __restrict__ kbar,
+                                                               int batch, int heads, int nb, int block, int64_t pos,
+                                                               int topk, int32_t* __restrict__ idx,
+                                                               int32_t* __restrict__ count,
+                                                               int16_t* __restrict__ blocks_out) {
+  constexpr int VPL = D / 32;
+  const int list = blockIdx.x * 4 + (threadIdx.x >> 5);     // sequence * heads + head
+  const int lane = threadIdx.x & 31;
+  if (list >= batch * heads) return;
+  const int cur = (int)(pos / block);
+  float qv[VPL];
+  load_vec(q + (int64_t)list * D + lane * VPL, qv);
+  if (VPL == 8) load_vec(q + (int64_t)list * D + lane * VPL + 4, qv + 4);
+  float vals[kMobaMaxTopk];
+  int ids[kMobaMaxTopk];
+#pragma unroll
+  for (int i = 0; i < kMobaMaxTopk; ++i) { vals[i] = -INFINITY; ids[i] = -1; }
+  const float* kb = kbar + (int64_t)list * nb * D;
+  for (int blk = 0; blk < cur; ++blk) {
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < VPL; ++e) acc = fmaf(qv[e], __ldg(kb + (int64_t)blk * D + lane * VPL + e), acc);
+    acc = warp_sum(acc);
+    // insert (acc, blk) into the descending list; equal values stay ahead (lower block)
+    float v = acc;
+    int id = blk;
+#pragma unroll
+    for (int i = 0; i < kMobaMaxTopk; ++i) {
+      if (i < topk && v > vals[i]) {
+        const float tv = vals[i];
+        const int ti = ids[i];
+        vals[i] = v; ids[i] = id;
+        v = tv; id = ti;
+      }
+    }
+  }
+  // kept blocks in ascending order (selection sort over at most kMobaMaxTopk entries)
+  const int kept = min(topk, cur);
+  int asc[kMobaMaxTopk];
+#pragma unroll
+  for (int i = 0; i < kMobaMaxTopk; ++i) asc[i] = i < kept ? ids[i] : 0x7fffffff;
+#pragma unroll
+  for (int i = 0; i < kMobaMaxTopk; ++i)
+#pragma unroll
+    for (int j = i + 1; j < kMobaMaxTopk; ++j)
+      if (asc[j] < asc[i]) { const int t = asc[i]; asc[i] = asc[j]; asc[j] = t; }
+  const int64_t stride = (int64_t)topk * block;
+  int32_t* out = idx + (int64_t)list * stride;
+  for (int i = 0; i < kept; ++i)
+    for (int t = lane; t < block; t += 32) out[(int64_t)i * block + t] = asc[i] * block + t;
+  for (int64_t t = (int64_t)kept * block + lane; t < stride; t += 32) out[t] = -1;
+  if (lane == 0) {
+    count[list] = kept * block;
+    if (blocks_out) {
+      int16_t* bo = blocks_out + (int64_t)list * (topk + 1);
+      for (int i = 0; i <= topk; ++i) bo[i] = (int16_t)(i < kept ? asc[i] : (i == kept ? cur : -1));
+    }
+  }
 }
 
 }  // namespace esa

@@ -298,3 +298,30 @@ class MobaPrefill:
         _abi.moba_block_gate_attn(q, k, v, self.block, self.topk, out=self.out, blocks=self.blocks,
                                   want_blocks=True, workspace=self.ws)
         return self.out
+
+
+class MobaDecode:
+    """MoBA decode for a batch at position n_ctx - 1: the block means of the cache's
+    complete blocks are computed once by fill() (a decode loop adds one block's mean
+    each time a block fills), every step gates over them and attends."""
+
+    def __init__(self, batch: int, n_ctx: int, heads: int, head_dim: int, block: int, topk: int,
+                 dtype=torch.bfloat16, device="cuda"):
+        self.batch, self.n_ctx, self.heads, self.d, self.block, self.topk = batch, n_ctx, heads, head_dim, block, topk
+        nb = (n_ctx + block - 1) // block
+        self.kbar = torch.zeros((batch, heads, nb, head_dim), dtype=torch.float32, device=device)
+        self.out = torch.empty((batch, 1, heads, head_dim), dtype=dtype, device=device)
+        self.blocks = torch.empty((batch, heads, topk + 1), dtype=torch.int16, device=device)
+        pos = n_ctx - 1
+        self.ws = torch.empty(_abi.moba_decode_workspace_size(batch, n_ctx, pos, heads, head_dim, block, topk) + 256,
+                              dtype=torch.uint8, device=device)
+
+    def fill(self, k):
+        """Means of the blocks before the query's block."""
+        _abi.moba_block_means(k, self.block, 0, (self.n_ctx - 1) // self.block, out=self.kbar)
+
+    def step(self, q, k, v):
+        _abi.moba_decode_attn(q, k, v, self.n_ctx - 1, self.kbar, self.block, self.topk, out=self.out,
+                              blocks=self.blocks, want_blocks=True, workspace=self.ws)
+        return self.out
+

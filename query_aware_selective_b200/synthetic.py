@@ -95,7 +95,12 @@ MOBA_64K = MobaWorkload("moba_prefill_h32_seq65536_block1024_top3", 1, 32, 128, 
 DECODE_1M = EsaWorkload("esa_decode_mistral_7b_b4_ctx1048576", 4, 32, 8, 128, 1048576, 1,
                         128, 128, 4096, 2048, 2, default_clamp(128), 16, "bf16", 4, "decode")
 
-WORKLOADS = {w.name: w for w in (TINY_DECODE, PREFILL_32K, DECODE_128K, MOBA_64K, DECODE_1M)}
+# MoBA decode (a next row past the five configurations): batch 16 of the MoBA layer,
+# one query at position 65535 of a 65536-token cache, top-3 past blocks + current
+MOBA_DECODE_64K = MobaWorkload("moba_decode_h32_b16_ctx65536_block1024_top3", 16, 32, 128, 65536, 1024, 3,
+                               "bf16", 5)
+
+WORKLOADS = {w.name: w for w in (TINY_DECODE, PREFILL_32K, DECODE_128K, MOBA_64K, DECODE_1M, MOBA_DECODE_64K)}
 
 
 def local_start(c0: int, n_init: int, window: int) -> int:
@@ -204,6 +209,21 @@ def make_moba_inputs(w: MobaWorkload, device="cpu", seq: Optional[int] = None,
     q = _randn((b, s, h, w.head_dim), dt, gen, device)
     k = _randn((b, s, h, w.head_dim), dt, gen, device)
     v = _randn((b, s, h, w.head_dim), dt, gen, device)
+    return dict(q=q, k=k, v=v)
+
+
+def make_moba_decode_inputs(w: MobaWorkload, device="cpu", seq: Optional[int] = None,
+                            batch: Optional[int] = None) -> dict:
+    """Draw the decode query q [B, 1, H, D] (position seq - 1), then K, V [B, S, H, D],
+    standard normal in the workload dtype, from the workload's seed."""
+    s = seq or w.seq
+    b = batch or w.batch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed)
+    dt = w.torch_dtype
+    q = _randn((b, 1, w.heads, w.head_dim), dt, gen, device)
+    k = _randn((b, s, w.heads, w.head_dim), dt, gen, device)
+    v = _randn((b, s, w.heads, w.head_dim), dt, gen, device)
     return dict(q=q, k=k, v=v)
 
 

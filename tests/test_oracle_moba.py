@@ -127,3 +127,18 @@ def test_sparsity_matches_the_article():
     assert attended == pages["attended"]
     sparsity = 100.0 * (1.0 - attended / pages["blocks"])
     assert abs(sparsity - pages["value"]) <= pages["tol"]
+
+
+def test_decode_step_pins():
+    # all past blocks kept: the last row of full causal attention; none kept (topk 0):
+    # attention over the current block only; otherwise the prefill's last row
+    s, block, h, d = 43, 8, 3, 8
+    q1, k, v = _rand((2, 1, h, d), 11), _rand((2, s, h, d), 12), _rand((2, s, h, d), 13)
+    qfull = np.concatenate([np.zeros((2, s - 1, h, d)), q1], axis=1)
+    full = _sdpa(qfull, k, v, torch.tril(torch.ones(s, s, dtype=torch.bool)))[:, -1:]
+    np.testing.assert_allclose(moba.decode_step(q1, k, v, block, 64)["o"], full, atol=1e-12, rtol=0)
+    cur0 = (s - 1) // block * block
+    local = _sdpa(q1, k[:, cur0:], v[:, cur0:], None)
+    np.testing.assert_allclose(moba.decode_step(q1, k, v, block, 0)["o"], local, atol=1e-12, rtol=0)
+    r = moba.decode_step(q1, k, v, block, 2)
+    assert (r["blocks"][:, 0, :, -1] == (s - 1) // block).all()
