@@ -904,6 +904,21 @@ esa_status_t sparse_attn_impl(const void* q, const void* k, const void* v, esa_d
     d.keys_per_split = (int)pl.keys_per_split;
     d.scale_log2 = sl2;
     const dim3 grid((unsigned)pl.nsplit, (unsigned)(vseq ? batch * hkv : batch));
+    if (d.hkv == 1) {
+      // one KV head per sequence: per-warp row streams instead of per-row bulk copies
+      static bool row_attr[64] = {};
+      if (dev < 64 && !row_attr[dev]) {
+        if ((st = set_max_smem(esa::attn_decode_rows_kernel<1>, esa::kRowSmemBytes)) != ESA_OK) return st;
+        if ((st = set_max_smem(esa::attn_decode_rows_kernel<2>, esa::kRowSmemBytes)) != ESA_OK) return st;
+        if ((st = set_max_smem(esa::attn_decode_rows_kernel<4>, esa::kRowSmemBytes)) != ESA_OK) return st;
+        row_attr[dev] = true;
+      }
+      if (g == 1) esa::attn_decode_rows_kernel<1><<<grid, esa::kDecThreads, esa::kRowSmemBytes, s>>>(d);
+      else if (g == 2) esa::attn_decode_rows_kernel<2><<<grid, esa::kDecThreads, esa::kRowSmemBytes, s>>>(d);
+      else esa::attn_decode_rows_kernel<4><<<grid, esa::kDecThreads, esa::kRowSmemBytes, s>>>(d);
+      ESA_LAUNCH_CHECK("attn_decode_rows_kernel");
+      return ok();
+    }
     if (g == 1) esa::attn_decode_kernel<1><<<grid, esa::kDecThreads, esa::kDecSmemBytes, s>>>(d);
     else if (g == 2) esa::attn_decode_kernel<2><<<grid, esa::kDecThreads, esa::kDecSmemBytes, s>>>(d);
     else esa::attn_decode_kernel<4><<<grid, esa::kDecThreads, esa::kDecSmemBytes, s>>>(d);
