@@ -30,9 +30,17 @@ def graph_of(fn):
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
+    # captured on a high-priority stream: the work fn issues on the current stream (the
+    # attention of a pipelined prefill) goes ahead of what it forks to low-priority
+    # side streams (see _side_stream) when both wait for free SMs
+    with torch.cuda.graph(g, stream=torch.cuda.Stream(priority=torch.cuda.Stream.priority_range()[1])):
         fn()
     return g
+
+
+def _side_stream(device) -> torch.cuda.Stream:
+    """A lowest-priority stream for work that runs beside the main stream's."""
+    return torch.cuda.Stream(device=device, priority=torch.cuda.Stream.priority_range()[0])
 
 
 def _timing_event(external: bool):
@@ -105,8 +113,10 @@ class EsaPrefill:
     select middle tokens, attend over initial + selected + local."""
 
     def __init__(self, batch: int, n_ctx: int, chunk: int, hq: int, hkv: int, head_dim: int, d_c: int,
-                 p: _abi.EsaParams, dtype=torch.bfloat16, device="cuda", per_head: bool = False):
+                 p: _abi.EsaParams, dtype=torch.bfloat16, device="cuda", per_head: bool = False,
+                 key_chunks: int = 2):
         self.batch, self.n_ctx, self.chunk = batch, n_ctx, chunk
+        self.key_chunks = key_chunks      # chunks whose keys run() compresses in one launch
         self.hq, self.hkv, self.d, self.d_c, self.p = hq, hkv, head_dim, d_c, p
         self.per_head = per_head      # one selection per KV head (block-diagonal maps)
         lists = (batch, hkv) if per_head else (batch,)
@@ -136,19 +146,26 @@ class EsaPrefill:
         self.ws_att = torch.empty(ws_att + 256, dtype=torch.uint8, device=device) if ws_att else None
         self.out_views = []
         self.cmp = _Compressor(hq, hkv, head_dim, d_c, dtype, device)
-        self.side = torch.cuda.Stream(device=device)
+        self.side = _side_stream(device)
+        self.kside = _side_stream(device)
 
     def chunks(self):
         return [(c0, min(self.chunk, self.n_ctx - c0)) for c0 in range(0, self.n_ctx, self.chunk)]
 
-    def front(self, ci: int, c0: int, lq: int, q, k):
-        """Everything of chunk ci before its attention, on the current stream: compress
-        the chunk's keys into the compressed cache (first read by a later chunk: the
-        middle ends `window` tokens before c0) and its queries, select into the
-        chunk's index list."""
-        b = self.batch
-        for s in range(b):
+    def compress_keys(self, c0: int, lq: int, k):
+        """Chunk [c0, c0 + lq)'s keys into the compressed cache. A chunk's scoring reads
+        only positions before c0 (the middle ends at most at c0), so these rows are
+        first needed by a later chunk."""
+        for s in range(self.batch):
             self.cmp.keys(k[s, c0:c0 + lq], out=self.k_c[s, c0:c0 + lq])
+
+    def front(self, ci: int, c0: int, lq: int, q, k=None):
+        """Chunk ci's work before its attention, on the current stream: (its keys, if k
+        is given,) its queries, and the selection into the chunk's index list."""
+        b = self.batch
+        if k is not None:
+            self.compress_keys(c0, lq, k)
+        for s in range(b):
             self.cmp.queries(q[s, c0:c0 + lq], out=self.q_c[s, :lq])
         q_c = self.q_c[:, :lq] if lq == self.chunk else self.q_c[:, :lq].contiguous()
         if self.per_head:
@@ -188,16 +205,46 @@ class EsaPrefill:
         the output [B, N, Hq, D]. The weights are packed for the tensor-core
         compression at the start of every run.
 
-        Two streams: the chunks' front work (compression and selection) runs in order
-        on a second stream, each chunk's attention on the current stream once its
-        selection is done, so chunk j + 1's selection overlaps chunk j's attention."""
+        Three streams: the chunks' key compressions run in order on one, their query
+        compression and selection in order on another (chunk j's selection waiting for
+        the keys of chunks < j only), and each chunk's attention on the current stream
+        once its selection is done, so chunk j + 1's selection overlaps chunk j's
+        attention and no chunk's selection waits for its own keys."""
         main = torch.cuda.current_stream()
         self.cmp.pack(wq, wk)
         self.side.wait_stream(main)
-        for ci, (c0, lq) in enumerate(self.chunks()):
+        self.kside.wait_stream(main)
+        chunks = self.chunks()
+        # keys are compressed in batches of up to kbatch chunks (fewer, larger launches
+        # beside the attention); chunk j's selection waits for the batch holding the
+        # last chunk its middle reads (positions < lo <= c0)
+        kbatch = max(1, self.key_chunks)
+        n_batches = (len(chunks) + kbatch - 1) // kbatch
+        issued = 0                                  # batches issued so far, in order
+        last_done = None                            # event after the last issued batch
+
+        def issue_batches(upto):                    # batches [issued, upto] on the key stream
+            nonlocal issued, last_done
+            while issued <= upto:
+                b0, b1 = issued * kbatch, min(len(chunks), (issued + 1) * kbatch)
+                with torch.cuda.stream(self.kside):
+                    self.compress_keys(chunks[b0][0], chunks[b1 - 1][0] + chunks[b1 - 1][1] - chunks[b0][0], k)
+                    last_done = torch.cuda.Event()
+                    last_done.record()
+                issued += 1
+
+        for ci, (c0, lq) in enumerate(chunks):
+            lo = _region_lo(c0, self.p.n_init, self.p.window)
+            needed = (lo - 1) // self.chunk if lo > self.p.n_init else -1   # last chunk the middle reads
+            wait = None
+            if needed >= 0:
+                issue_batches(needed // kbatch)
+                wait = last_done
             done = torch.cuda.Event()
             with torch.cuda.stream(self.side):
-                self.front(ci, c0, lq, q, k)
+                if wait is not None:
+                    self.side.wait_event(wait)
+                self.front(ci, c0, lq, q)
                 done.record()
             main.wait_event(done)
             ev = None
@@ -205,7 +252,9 @@ class EsaPrefill:
                 ev = (_timing_event(external_events), _timing_event(external_events))
                 attn_events.append(ev)
             self.attend(ci, c0, lq, q, k, v, ev)
+        issue_batches(n_batches - 1)               # the rest complete the compressed cache
         main.wait_stream(self.side)
+        main.wait_stream(self.kside)
         return self.out
 
 
@@ -237,7 +286,7 @@ class EsaDecode:
         self.ws_sel = torch.empty(n_sel + 256, dtype=torch.uint8, device=device)
         self.ws_att = torch.empty(nb + 256, dtype=torch.uint8, device=device) if nb else None
         self.cmp = _Compressor(hq, hkv, head_dim, d_c, dtype, device)
-        self.side = torch.cuda.Stream(device=device)
+        self.side = _side_stream(device)
 
     def fill_cache(self, k, wk, upto: Optional[int] = None):
         """Compress cached keys [0, upto) of every sequence (prefill state)."""
