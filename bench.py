@@ -402,6 +402,10 @@ def bench_moba_decode(args, dev, flush, dist_max, peaks, peak_src, world):
     import torch
     from query_aware_selective_b200 import cost, pipeline, synthetic
     w = synthetic.MOBA_DECODE_64K
+    if args.decode_batch:
+        import dataclasses
+        w = dataclasses.replace(w, batch=args.decode_batch,
+                                name=f"moba_decode_h{w.heads}_b{args.decode_batch}_ctx{w.seq}_block{w.block}_top{w.topk}")
     inp = synthetic.make_moba_decode_inputs(w, device=dev)
     dec = pipeline.MobaDecode(w.batch, w.seq, w.heads, w.head_dim, w.block, w.topk, device=dev)
     dec.fill(inp["k"])

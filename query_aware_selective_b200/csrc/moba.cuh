@@ -383,21 +383,32 @@ __global__ void __launch_bounds__(128) moba_decode_gate_kernel(const T* __restri
 #pragma unroll
   for (int i = 0; i < kMobaMaxTopk; ++i) { vals[i] = -INFINITY; ids[i] = -1; }
   const float* kb = kbar + (int64_t)list * nb * D;
-  for (int blk = 0; blk < cur; ++blk) {
-    float acc = 0.f;
+  constexpr int UNR = 8;                   // block means in flight per round
+  for (int blk0 = 0; blk0 < cur; blk0 += UNR) {
+    float kv[UNR][VPL];
 #pragma unroll
-    for (int e = 0; e < VPL; ++e) acc = fmaf(qv[e], __ldg(kb + (int64_t)blk * D + lane * VPL + e), acc);
-    acc = warp_sum(acc);
-    // insert (acc, blk) into the descending list; equal values stay ahead (lower block)
-    float v = acc;
-    int id = blk;
+    for (int u = 0; u < UNR; ++u)
 #pragma unroll
-    for (int i = 0; i < kMobaMaxTopk; ++i) {
-      if (i < topk && v > vals[i]) {
-        const float tv = vals[i];
-        const int ti = ids[i];
-        vals[i] = v; ids[i] = id;
-        v = tv; id = ti;
+      for (int e = 0; e < VPL; ++e)
+        kv[u][e] = blk0 + u < cur ? __ldg(kb + (int64_t)(blk0 + u) * D + lane * VPL + e) : 0.f;
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      if (blk0 + u >= cur) break;
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < VPL; ++e) acc = fmaf(qv[e], kv[u][e], acc);
+      acc = warp_sum(acc);
+      // insert (acc, blk) into the descending list; equal values stay ahead (lower block)
+      float v = acc;
+      int id = blk0 + u;
+#pragma unroll
+      for (int i = 0; i < kMobaMaxTopk; ++i) {
+        if (i < topk && v > vals[i]) {
+          const float tv = vals[i];
+          const int ti = ids[i];
+          vals[i] = v; ids[i] = id;
+          v = tv; id = ti;
+        }
       }
     }
   }
