@@ -1079,13 +1079,16 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
   if ((st = make_tmap_box_bf16(&bk, k, heads, (uint64_t)batch * seq, 1, esa::kTcKeys)) != ESA_OK) return st;
   if ((st = make_tmap_box_bf16(&bv, v, heads, (uint64_t)batch * seq, 1, esa::kTcKeys)) != ESA_OK) return st;
   ESA_CUDA(cudaMemsetAsync(w.cnt, 0, w.zero_bytes, s));
-  const dim3 lgrid((unsigned)cdiv(seq * heads, 256), batch);
+  const dim3 lgrid((unsigned)nb, heads, batch);
+  const size_t lsmem = 2 * (size_t)nb * sizeof(uint32_t);
   if (topk > 0 && w.pairs > 0) {
-    esa::moba_list_kernel<<<lgrid, 256, 0, s>>>(blocks, seq, heads, block, nb, topk, 0, w.cnt, w.off, w.fill, w.list);
+    esa::moba_list_kernel<<<lgrid, esa::kMobaListThreads, lsmem, s>>>(blocks, seq, heads, block, nb, topk, 0, w.cnt,
+                                                                      w.off, w.fill, w.list);
     ESA_LAUNCH_CHECK("moba_list_kernel(count)");
     esa::moba_scan_kernel<<<1, 1024, 0, s>>>(w.cnt, w.n_lists, w.off, w.tile_off, w.totals);
     ESA_LAUNCH_CHECK("moba_scan_kernel");
-    esa::moba_list_kernel<<<lgrid, 256, 0, s>>>(blocks, seq, heads, block, nb, topk, 1, w.cnt, w.off, w.fill, w.list);
+    esa::moba_list_kernel<<<lgrid, esa::kMobaListThreads, lsmem, s>>>(blocks, seq, heads, block, nb, topk, 1, w.cnt,
+                                                                      w.off, w.fill, w.list);
     ESA_LAUNCH_CHECK("moba_list_kernel(fill)");
     esa::MobaPastProblem pp{};
     pp.q = static_cast<const __nv_bfloat16*>(q);

@@ -142,26 +142,52 @@ __global__ void __launch_bounds__(128) moba_gate_kernel(const T* __restrict__ q,
 // entries), count (pass 0) or append (pass 1) the pair (p, slot) to the list of
 // (b, h, block). The order inside a list is not fixed, but every pair owns its own
 // output slot, so the results do not depend on it.
-__global__ void moba_list_kernel(const int16_t* __restrict__ blocks, int64_t seq, int heads, int block,
-                                 int n_blocks, int topk, int pass, uint32_t* __restrict__ cnt,
-                                 const uint32_t* __restrict__ off, uint32_t* __restrict__ fill,
-                                 uint32_t* __restrict__ list) {
-  const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // (p, h) of sequence b
-  const int b = blockIdx.y;
-  if (row >= seq * heads) return;
-  const int64_t p = row / heads;
-  const int h = (int)(row % heads);
-  const int n_past = min(topk, (int)(p / block));
-  const int16_t* lst = blocks + ((int64_t)b * seq * heads + row) * (topk + 1);
-  for (int s = 0; s < n_past; ++s) {
-    const int blk = lst[s];
-    if (blk < 0 || blk >= n_blocks) break;
-    const int64_t li = ((int64_t)b * heads + h) * n_blocks + blk;
-    if (pass == 0) {
-      atomicAdd(&cnt[li], 1u);
-    } else {
-      const uint32_t at = atomicAdd(&fill[li], 1u);
-      list[off[li] + at] = ((uint32_t)p << 4) | (uint32_t)s;
+//
+// grid (query blocks, H, B): a CTA takes the queries of one query block c for one head.
+// They all choose among the same past blocks (< c), so their entries are counted in
+// shared memory first and each past block costs one global atomic per CTA (pass 0: add
+// the count; pass 1: reserve the CTA's range of the list) instead of one per entry.
+constexpr int kMobaListThreads = 256;
+
+__global__ void __launch_bounds__(kMobaListThreads) moba_list_kernel(const int16_t* __restrict__ blocks, int64_t seq,
+                                                                     int heads, int block, int n_blocks, int topk,
+                                                                     int pass, uint32_t* __restrict__ cnt,
+                                                                     const uint32_t* __restrict__ off,
+                                                                     uint32_t* __restrict__ fill,
+                                                                     uint32_t* __restrict__ list) {
+  extern __shared__ uint32_t lsm[];        // [n_blocks] counts, then [n_blocks] bases / cursors
+  uint32_t* c_s = lsm;
+  uint32_t* base_s = lsm + n_blocks;
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int64_t p0 = (int64_t)c * block, p1 = min(seq, p0 + block);
+  for (int i = threadIdx.x; i < c; i += kMobaListThreads) c_s[i] = 0;
+  __syncthreads();
+  const int n_past = min(topk, c);         // the same for every query of the block
+  for (int64_t p = p0 + threadIdx.x; p < p1; p += kMobaListThreads) {
+    const int16_t* lst = blocks + (((int64_t)b * seq + p) * heads + h) * (topk + 1);
+    for (int s2 = 0; s2 < n_past; ++s2) {
+      const int blk = lst[s2];
+      if (blk < 0 || blk >= c) break;
+      atomicAdd(&c_s[blk], 1u);
+    }
+  }
+  __syncthreads();
+  const int64_t lbase = ((int64_t)b * heads + h) * n_blocks;
+  if (pass == 0) {
+    for (int i = threadIdx.x; i < c; i += kMobaListThreads)
+      if (c_s[i]) atomicAdd(&cnt[lbase + i], c_s[i]);
+    return;
+  }
+  for (int i = threadIdx.x; i < c; i += kMobaListThreads)
+    base_s[i] = c_s[i] ? off[lbase + i] + atomicAdd(&fill[lbase + i], c_s[i]) : 0u;
+  __syncthreads();
+  for (int64_t p = p0 + threadIdx.x; p < p1; p += kMobaListThreads) {
+    const int16_t* lst = blocks + (((int64_t)b * seq + p) * heads + h) * (topk + 1);
+    for (int s2 = 0; s2 < n_past; ++s2) {
+      const int blk = lst[s2];
+      if (blk < 0 || blk >= c) break;
+      const uint32_t at = atomicAdd(&base_s[blk], 1u);
+      list[at] = ((uint32_t)p << 4) | (uint32_t)s2;
     }
   }
 }
