@@ -174,6 +174,8 @@ int select_cluster_size(int32_t batch) {
     }
     cudaGetLastError();   // a refused query is not an error of this call
   }
+  // (smaller clusters for many selections were measured slower: a CTA then sweeps tens
+  // of thousands of keys through the global scratch)
   return (max16[dev] > 0 && batch <= max16[dev]) ? 16 : 8;
 }
 

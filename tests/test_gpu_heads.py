@@ -29,6 +29,9 @@ def _rand(shape, seed, dtype=torch.float32):
     (2, 1, 4000, 128, 2, 32, 300, 500, 3, math.inf),   # 2 groups, no clamp
     (1, 64, 4096, 128, 8, 128, 512, 1024, 2, 45.25),   # a chunk (tiled path per group)
     (2, 130, 3000, 128, 8, 16, 300, 200, 2, 8.0),      # ragged chunk
+    (5, 1, 5000, 128, 8, 32, 300, 400, 2, 45.25),      # 40 selections in flight
+    (10, 1, 3000, 128, 8, 32, 300, 200, 2, 45.25),     # 80 selections
+    (40, 1, 2000, 128, 8, 32, 200, 100, 2, 45.25),     # 320 selections (more clusters than fit at once)
 ])
 def test_score_select_heads_parity(batch, lq, n_cap, dc, ng, n_init, window, topk, eps, clamp):
     p = qas.params(n_init, window, topk, eps, clamp)
