@@ -15,6 +15,8 @@ can be checked against the pages by eye.
   initial + selected + local tokens.
 * ``oracle.esa_heads`` - the per-head selection variant of ESA (the article's
   ablation of merged versus per-head importance): one index set per KV head.
+* ``oracle.esa_varlen`` - ESA decode over a batch of sequences of different
+  lengths: each sequence runs the one-sequence step at its own position.
 * ``oracle.moba`` - Mixture of Block Attention (MoBA article, sections 1-3):
   block mean pooling, gate, causal top-k, block attention.
 

@@ -10,10 +10,11 @@ import textwrap
 
 import pytest
 
-from oracle import esa, esa_heads, moba
+from oracle import esa, esa_heads, esa_varlen, moba
 from tests import test_oracle_esa as pe
 from tests import test_oracle_heads as th
 from tests import test_oracle_moba as pm
+from tests import test_oracle_varlen as tv
 
 MUTATIONS = [
     # (module, function, snippet, replacement, pin)
@@ -65,6 +66,12 @@ MUTATIONS = [
      pm.check_all_blocks_is_full_attention),                               # current block not causal
     (moba, "attend", "scale = 1.0 / math.sqrt(d)", "scale = 1.0",
      pm.check_no_past_block_is_block_local),                               # missing scale
+    (esa_varlen, "score_select_varlen", "c0 = n - 1", "c0 = n - 2",
+     tv.check_short_sequences_attend_everything),                          # query position off by one
+    (esa_varlen, "sparse_attn_varlen", "c0 = n - 1", "c0 = n - 2",
+     tv.check_short_sequences_attend_everything),                          # attention stops one row short
+    (esa_varlen, "sparse_attn_varlen", "if lists == 1:", "if True:",
+     tv.check_per_head_lists_per_sequence),                                # first list for every head
 ]
 
 
