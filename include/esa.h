@@ -312,6 +312,61 @@ esa_status_t moba_decode_attn(const void* q, const void* k, const void* v, esa_d
 size_t moba_decode_workspace_size(int32_t batch, int64_t n_cap, int64_t pos, int32_t heads, int32_t head_dim,
                                   int32_t block, int32_t topk);
 
+/* ----------------------------------------------- variable-length decode batches -- */
+
+/* A decode batch whose sequences hold different numbers of cached tokens (ESA write-up,
+ * problem statement: decode over each sequence's own KV cache; the pages batch nothing,
+ * so this is the plain reading: every sequence runs the one-query step on its own).
+ *   seq_len: device int64 [batch], caller-owned. Sequence b holds seq_len[b] tokens:
+ *            rows [0, seq_len[b]) of its K/V and compressed caches; its one query sits
+ *            at position seq_len[b] - 1, and the region rule (initial, middle, local)
+ *            applies with c0 = seq_len[b] - 1. Rows past seq_len[b] are never read.
+ *            The lengths stay on the device (a captured decode graph can replay with
+ *            new lengths); a length outside [1, n_cap] is clamped into it and recorded
+ *            in the device status word, which esa_device_status() then reports as
+ *            ESA_ERR_INVALID_ARG.
+ * Caches are laid out as for the equal-length calls with n_cap rows per sequence. */
+
+/* esa_compress_packed_varlen - esa_compress_packed of one new key row per sequence,
+ * written to that sequence's last token: x row b (bf16 [n_heads_in, head_dim] at
+ * x + b * x_row_stride) -> k_c[b * n_cap + seq_len[b] - 1] (fp32 [batch, n_cap, d_out],
+ * rows of d_out floats). Requirements and errors as for esa_compress_packed. */
+esa_status_t esa_compress_packed_varlen(const void* x, int32_t batch, int64_t x_row_stride, int32_t n_heads_in,
+                                        int32_t head_dim, const void* packed, int32_t d_out, float* k_c,
+                                        int64_t n_cap, const int64_t* seq_len, void* stream);
+
+/* esa_score_select_varlen - esa_score_select (n_groups 1) or esa_score_select_heads
+ * (n_groups 2, 4, 8) for one query per sequence at its own position.
+ *   q_c:       [batch, 1, d_c] fp32 (16-byte aligned); k_c: [batch, n_cap, d_c] fp32
+ *   idx_out:   [batch, n_groups, topk] int32, ascending, -1 past count;
+ *   count_out: [batch, n_groups] int32 = min(topk, that sequence's middle length)
+ *   score_out: NULL or [batch, n_groups, n_mid_max] fp32 s', n_mid_max the middle
+ *              length of a query at n_cap - 1; entries past a sequence's own middle
+ *              are left unwritten.
+ * Requires d_c in {16, 32, 64, 128, 256} with d_c / 4 (32 from 128 on) lanes per key
+ * divisible by n_groups; else ESA_ERR_UNSUPPORTED. Workspace: ..._workspace_size
+ * bytes (256-byte aligned), which covers every length up to n_cap. */
+esa_status_t esa_score_select_varlen(const float* q_c, const float* k_c, int32_t batch, int64_t n_cap,
+                                     const int64_t* seq_len, int32_t d_c, int32_t n_groups, esa_params_t p,
+                                     int32_t* idx_out, int32_t* count_out, float* score_out, void* workspace,
+                                     size_t ws_bytes, void* stream);
+size_t esa_score_select_varlen_workspace_size(int32_t batch, int64_t n_cap, int32_t d_c, int32_t n_groups,
+                                              esa_params_t p);
+
+/* esa_sparse_attn_varlen - esa_sparse_attn (lists 1) or esa_sparse_attn_heads (lists
+ * == hkv) for one query per sequence at position seq_len[b] - 1: it attends initial +
+ * idx[:count] + local [lo, seq_len[b]) of its own sequence.
+ *   q: [batch, 1, hq, head_dim]; k, v: [batch, n_cap, hkv, head_dim]; o like q;
+ *   lse: NULL or [batch, 1, hq]; idx/count as esa_score_select_varlen writes them.
+ * Dtypes, head dims, GQA groups, scale and errors as for esa_sparse_attn. */
+esa_status_t esa_sparse_attn_varlen(const void* q, const void* k, const void* v, esa_dtype_t dt, int32_t batch,
+                                    int64_t n_cap, const int64_t* seq_len, int32_t hq, int32_t hkv,
+                                    int32_t head_dim, const int32_t* idx, const int32_t* count, int32_t lists,
+                                    esa_params_t p, float scale, void* o, float* lse, void* workspace,
+                                    size_t ws_bytes, void* stream);
+size_t esa_sparse_attn_varlen_workspace_size(int32_t batch, int64_t n_cap, int32_t hq, int32_t hkv,
+                                             int32_t head_dim, esa_dtype_t dt, int32_t lists, esa_params_t p);
+
 /* ------------------------------------------------------------------- status -- */
 
 /* Message for the last non-OK status returned on this thread ("" if none). */
@@ -319,8 +374,9 @@ const char* esa_last_error(void);
 
 /* Waits for `stream`, then reads and clears the device status word of the current
  * device. Returns ESA_OK, ESA_ERR_TIMEOUT if a kernel's bounded wait ran out since the
- * last read (the message names the kernel and the wait), or ESA_ERR_CUDA if a kernel
- * stopped early on a launch-environment check (e.g. misaligned shared memory). */
+ * last read (the message names the kernel and the wait), ESA_ERR_CUDA if a kernel
+ * stopped early on a launch-environment check (e.g. misaligned shared memory), or
+ * ESA_ERR_INVALID_ARG if a variable-length call read a length outside [1, n_cap]. */
 esa_status_t esa_device_status(void* stream);
 
 /* Number of kernels this library has launched in this process, all devices and

@@ -66,6 +66,13 @@ SIGNATURES = {
     "esa_sparse_attn_heads": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i64, _i64, _i32, _i32,
                                              _i32, _vp, _vp, EsaParams, _f32, _vp, _vp, _vp, _sz, _vp]),
     "esa_sparse_attn_heads_workspace_size": (_sz, [_i32, _i32, _i64, _i32, _i32, _i32, ctypes.c_int, EsaParams]),
+    "esa_compress_packed_varlen": (ctypes.c_int, [_vp, _i32, _i64, _i32, _i32, _vp, _i32, _vp, _i64, _vp, _vp]),
+    "esa_score_select_varlen": (ctypes.c_int, [_vp, _vp, _i32, _i64, _vp, _i32, _i32, EsaParams, _vp, _vp, _vp,
+                                               _vp, _sz, _vp]),
+    "esa_score_select_varlen_workspace_size": (_sz, [_i32, _i64, _i32, _i32, EsaParams]),
+    "esa_sparse_attn_varlen": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i64, _vp, _i32, _i32, _i32, _vp,
+                                              _vp, _i32, EsaParams, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "esa_sparse_attn_varlen_workspace_size": (_sz, [_i32, _i64, _i32, _i32, _i32, ctypes.c_int, _i32, EsaParams]),
 }
 
 _lib = None
@@ -333,6 +340,91 @@ def sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, c0: int, idx:
     _check(load().esa_sparse_attn(_ptr(q), _ptr(k), _ptr(v), dt, b, lq, n_cap, c0, hq, hkv, d, _ptr(idx),
                                   _ptr(count), p, scale, _ptr(out), _ptr(lse) if want_lse else None, wp, wn,
                                   _stream()), "esa_sparse_attn")
+    return out, (lse if want_lse else None)
+
+
+def _seq_len(seq_len: torch.Tensor, batch: int) -> torch.Tensor:
+    if not seq_len.is_cuda or seq_len.dtype != torch.int64 or seq_len.shape != (batch,) or not seq_len.is_contiguous():
+        raise ValueError("seq_len must be a contiguous CUDA int64 tensor of shape [batch]")
+    return seq_len
+
+
+def compress_packed_varlen(x: torch.Tensor, packed: torch.Tensor, k_c: torch.Tensor, seq_len: torch.Tensor) -> None:
+    """esa_compress_packed_varlen: x [B, Hin, D] bf16 (one new key row per sequence, each
+    row contiguous) -> k_c[b, seq_len[b] - 1] of k_c [B, n_cap, d_out] f32."""
+    if not x.is_cuda or not packed.is_cuda or not k_c.is_cuda:
+        raise ValueError("libesa takes CUDA tensors (no CPU path)")
+    b, hin, d = x.shape
+    if x.stride(2) != 1 or x.stride(1) != d:
+        raise ValueError("each row of x must be contiguous [Hin, D]")
+    if not k_c.is_contiguous():
+        raise ValueError("k_c must be contiguous")
+    _check(load().esa_compress_packed_varlen(_ptr(x), b, x.stride(0) if b > 1 else hin * d, hin, d, _ptr(packed),
+                                             k_c.shape[2], _ptr(k_c), k_c.shape[1], _ptr(_seq_len(seq_len, b)),
+                                             _stream()), "esa_compress_packed_varlen")
+
+
+def score_select_varlen_workspace_size(batch, n_cap, d_c, n_groups, p: EsaParams) -> int:
+    return load().esa_score_select_varlen_workspace_size(batch, n_cap, d_c, n_groups, p)
+
+
+def score_select_varlen(q_c: torch.Tensor, k_c: torch.Tensor, seq_len: torch.Tensor, p: EsaParams, n_groups: int = 1,
+                        want_scores: bool = False, idx: Optional[torch.Tensor] = None,
+                        count: Optional[torch.Tensor] = None, scores: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None):
+    """esa_score_select_varlen: one query per sequence at position seq_len[b] - 1.
+    q_c [B, 1, d_c], k_c [B, n_cap, d_c] f32. Returns (idx [B, G, topk] int32,
+    count [B, G] int32, s' [B, G, n_mid_max] f32 or None); G = n_groups."""
+    _dev(q_c, k_c)
+    b, lq, dc = q_c.shape
+    if lq != 1:
+        raise ValueError("one query per sequence")
+    n_cap = k_c.shape[1]
+    dev = q_c.device
+    if idx is None:
+        idx = torch.empty((b, n_groups, p.topk), dtype=torch.int32, device=dev)
+    if count is None:
+        count = torch.empty((b, n_groups), dtype=torch.int32, device=dev)
+    if want_scores and scores is None:
+        c0 = n_cap - 1
+        lo = min(c0, max(p.n_init, c0 - p.window))
+        scores = torch.full((b, n_groups, max(0, lo - p.n_init)), float("nan"), dtype=torch.float32, device=dev)
+    ws = _workspace(score_select_varlen_workspace_size(b, n_cap, dc, n_groups, p), dev, workspace)
+    wp, wn = _ws_ptr(ws)
+    _check(load().esa_score_select_varlen(_ptr(q_c), _ptr(k_c), b, n_cap, _ptr(_seq_len(seq_len, b)), dc, n_groups,
+                                          p, _ptr(idx), _ptr(count), _ptr(scores) if want_scores else None, wp, wn,
+                                          _stream()), "esa_score_select_varlen")
+    return idx, count, (scores if want_scores else None)
+
+
+def sparse_attn_varlen_workspace_size(batch, n_cap, hq, hkv, d, dtype_code, lists, p: EsaParams) -> int:
+    return load().esa_sparse_attn_varlen_workspace_size(batch, n_cap, hq, hkv, d, dtype_code, lists, p)
+
+
+def sparse_attn_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_len: torch.Tensor, idx: torch.Tensor,
+                       count: torch.Tensor, p: EsaParams, scale: float = 0.0, want_lse: bool = False,
+                       out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None):
+    """esa_sparse_attn_varlen: q [B, 1, Hq, D]; k, v [B, n_cap, Hkv, D]; idx [B, L, >=topk],
+    count [B, L] with L = 1 (shared list) or Hkv (one per KV head), or idx [B, topk] and
+    count [B]. Returns (o [B, 1, Hq, D], lse [B, 1, Hq] f32 or None)."""
+    _dev(q, k, v, idx, count)
+    b, lq, hq, d = q.shape
+    if lq != 1:
+        raise ValueError("one query per sequence")
+    n_cap, hkv = k.shape[1], k.shape[2]
+    lists = count.shape[1] if count.dim() == 2 else 1
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((b, lq, hq), dtype=torch.float32, device=q.device)
+    ws = _workspace(sparse_attn_varlen_workspace_size(b, n_cap, hq, hkv, d, dt, lists, p), q.device, workspace)
+    wp, wn = _ws_ptr(ws)
+    _check(load().esa_sparse_attn_varlen(_ptr(q), _ptr(k), _ptr(v), dt, b, n_cap, _ptr(_seq_len(seq_len, b)), hq,
+                                         hkv, d, _ptr(idx), _ptr(count), lists, p, scale, _ptr(out),
+                                         _ptr(lse) if want_lse else None, wp, wn, _stream()),
+           "esa_sparse_attn_varlen")
     return out, (lse if want_lse else None)
 
 

@@ -286,8 +286,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const Decod
   int32_t* pos = reinterpret_cast<int32_t*>(stage0_ptr + 2 * kDecStages * op_bytes);   // this split's keys
   DecSmem& sm = *reinterpret_cast<DecSmem*>(pos + kDecMaxSplitKeys);
 
-  const int cnt = min(max(a.keys.count[b], 0), (int)a.keys.idx_stride);
-  const int64_t n_keys = a.keys.ni + cnt + (a.c0 - a.keys.lo) + 1;
+  KeyList kl = a.keys;
+  const int64_t c0 = kl.vl.len ? kl.resolve(b, 701) : a.c0;
+  const int cnt = min(max(kl.count[b], 0), (int)kl.idx_stride);
+  const int64_t n_keys = kl.ni + cnt + (c0 - kl.lo) + 1;
   const int64_t t_begin = (int64_t)split * a.keys_per_split;
   const int64_t t_end = min(n_keys, t_begin + a.keys_per_split);
   const int nst = t_end > t_begin ? (int)((t_end - t_begin + ks - 1) / ks) : 0;
@@ -301,7 +303,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const Decod
     sm.issued = 0;
     fence_barrier_init();
   }
-  for (int64_t t = t_begin + threadIdx.x; t < t_end; t += kDecThreads) pos[t - t_begin] = (int32_t)a.keys.pos(b, cnt, t);
+  for (int64_t t = t_begin + threadIdx.x; t < t_end; t += kDecThreads) pos[t - t_begin] = (int32_t)kl.pos(b, cnt, t);
   if (nst > 0) {
     // V rows past the end of the last stage are multiplied by P = 0: make sure they hold
     // finite values (zeros) if that ring slot is never filled by an earlier stage
@@ -460,8 +462,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_rows_kernel(const 
   const int split = blockIdx.x, b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int ks = kDecWarps * kDecKeysPerWarp;                  // 128 keys per stage
-  const int cnt = min(max(a.keys.count[b], 0), (int)a.keys.idx_stride);
-  const int64_t n_keys = a.keys.ni + cnt + (a.c0 - a.keys.lo) + 1;
+  KeyList kl = a.keys;
+  const int64_t c0 = kl.vl.len ? kl.resolve(b, 702) : a.c0;
+  const int cnt = min(max(kl.count[b], 0), (int)kl.idx_stride);
+  const int64_t n_keys = kl.ni + cnt + (c0 - kl.lo) + 1;
   const int64_t t_begin = (int64_t)split * a.keys_per_split;
   const int64_t t_end = min(n_keys, t_begin + a.keys_per_split);
   const int nst = t_end > t_begin ? (int)((t_end - t_begin + ks - 1) / ks) : 0;
@@ -473,7 +477,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_rows_kernel(const 
   auto issue = [&](int j) {
     if (j < nst) {
       const int64_t t0 = t_begin + (int64_t)j * ks + warp * kDecKeysPerWarp;
-      const int my_pos = (lane < kDecKeysPerWarp && t0 + lane < t_end) ? (int)a.keys.pos(b, cnt, t0 + lane) : -1;
+      const int my_pos = (lane < kDecKeysPerWarp && t0 + lane < t_end) ? (int)kl.pos(b, cnt, t0 + lane) : -1;
       const int op = lane >> 4, pc = lane & 15;
       const __nv_bfloat16* src = (op ? a.v : a.k) + seq + pc * 8;
       const uint32_t dst = wring + (j % kRowStages) * kRowWarpSlot + op * kDecKeysPerWarp * kRowStride + pc * 16;

@@ -51,8 +51,10 @@ __global__ void __launch_bounds__(kSimtWarps * 32) attn_simt_kernel(SimtAttnArgs
   const int grp = lane / LPK, sub = lane % LPK;
 
   const int list = a.lists > 1 ? b * a.lists + g : b;
-  const int cnt = min(max(a.keys.count[list], 0), (int)a.keys.idx_stride);
-  const int64_t n_prior = a.keys.ni + cnt + (a.c0 - a.keys.lo);
+  KeyList kl = a.keys;
+  const int64_t c0 = kl.vl.len ? kl.resolve(b, 703) : a.c0;
+  const int cnt = min(max(kl.count[list], 0), (int)kl.idx_stride);
+  const int64_t n_prior = kl.ni + cnt + (c0 - kl.lo);
   const int64_t n_keys = n_prior + i + 1;                     // causal: keys up to position c0 + i
   const int64_t t_begin = (int64_t)split * a.keys_per_split;
   const int64_t t_end = min(n_keys, t_begin + a.keys_per_split);
@@ -85,7 +87,7 @@ __global__ void __launch_bounds__(kSimtWarps * 32) attn_simt_kernel(SimtAttnArgs
       const int64_t t = tb + u * KPW + grp;
       ok[u] = t < t_end;
       if (ok[u]) {
-        const int64_t p = a.keys.pos(list, cnt, t);
+        const int64_t p = kl.pos(list, cnt, t);
         kr[u] = ld_stream16(kbase + p * row_stride);
         vr[u] = ld_stream16(vbase + p * row_stride);
       }

@@ -44,6 +44,37 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (x & 0x80000000u) ? ~x : (x | 0x80000000u);
 }
 
+// ------------------------------------------------------- variable-length decode --
+// A decode batch whose sequences hold different numbers of cached tokens: sequence s
+// holds len[s] tokens and its one query sits at position len[s] - 1 (ESA write-up,
+// problem statement: decode over each sequence's own KV cache). The region rule then
+// applies per sequence. A length outside [1, n_cap] is clamped into it and recorded in
+// the status word (code 1).
+struct VarLen {
+  const int64_t* len;   // [sequences] device lengths, or null: every sequence as the call's c0
+  int64_t n_cap;
+  int32_t n_init, window;
+  int32_t div;          // grid sequence b reads len[b / div]
+  __device__ __forceinline__ int64_t c0(int b, unsigned site) const {
+    int64_t n = len[b / div];
+    if (n < 1 || n > n_cap) {
+      record_status(1u, site);
+      n = n < 1 ? 1 : n_cap;
+    }
+    return n - 1;
+  }
+  // first local position of the query at c0: min(c0, max(n_init, c0 - window))
+  __device__ __forceinline__ int64_t lo(int64_t c0) const {
+    const int64_t a = c0 - window > (int64_t)n_init ? c0 - window : (int64_t)n_init;
+    return a < c0 ? a : c0;
+  }
+  // middle [n_init, lo) length of sequence b
+  __device__ __forceinline__ int64_t n_mid(int b, unsigned site) const {
+    const int64_t m = lo(c0(b, site)) - n_init;
+    return m > 0 ? m : 0;
+  }
+};
+
 // Inverse of order_key.
 __device__ __forceinline__ float key_to_float(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);

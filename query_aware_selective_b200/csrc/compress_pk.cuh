@@ -60,9 +60,11 @@ __global__ void __launch_bounds__(256) compress_pack_kernel(const float* __restr
 }
 
 // grid (cl, row tiles, 2 halves), cluster (cl, 1, 1); cl in {8, 16}; K % (64 cl) == 0.
+// Row r of x goes to row r of y; with yl.len (one new key per sequence of a
+// variable-length batch) to row r * yl.n_cap + yl.len[r] - 1, its sequence's last token.
 __global__ void __launch_bounds__(kCpThreads, 1)
     compress_pk_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw, int64_t rows,
-                       int K, float* __restrict__ y, int64_t ystride) {
+                       int K, float* __restrict__ y, int64_t ystride, const VarLen yl) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   const uint32_t s0 = smem_u32(smem);
@@ -178,7 +180,10 @@ __global__ void __launch_bounds__(kCpThreads, 1)
         acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
       }
       const int64_t row = r0 + rl;
-      if (fin && row < rows) *reinterpret_cast<float4*>(y + row * ystride + h * 64 + c4) = acc;
+      if (fin && row < rows) {
+        const int64_t yrow = yl.len ? row * yl.n_cap + yl.c0((int)row, 321) : row;
+        *reinterpret_cast<float4*>(y + yrow * ystride + h * 64 + c4) = acc;
+      }
     }
   }
   cluster_sync_all();

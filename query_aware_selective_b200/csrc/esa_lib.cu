@@ -246,10 +246,13 @@ esa_status_t make_tmap_f32(CUtensorMap* m, const float* base, uint64_t rows, uin
 
 template <int DC, int NG>
 void launch_score_small_ng(const float* q_c, const float* k_c, int lq, int64_t n_cap, int64_t mid0, int64_t n_mid,
-                           int batch, float* S, uint32_t* m_key, cudaStream_t s) {
-  // one wave of two CTAs per SM over all sequences, each CTA a multiple of a stage
+                           int batch, float* S, uint32_t* m_key, const esa::VarLen& vl, cudaStream_t s) {
+  // one wave of two CTAs per SM over all sequences, each CTA a multiple of a stage; with
+  // variable lengths four such waves for the longest possible middles, so that the CTAs
+  // of short sequences end at once and the block scheduler spreads the rest
   constexpr int64_t ks = esa::SmallScoreShape<DC>::KS;
-  const int64_t per_seq = std::max<int64_t>(1, std::min<int64_t>(cdiv(n_mid, ks), (2 * 148) / batch));
+  const int64_t waves = vl.len ? 4 : 1;
+  const int64_t per_seq = std::max<int64_t>(1, std::min<int64_t>(cdiv(n_mid, ks), waves * (2 * 148) / batch));
   const int64_t keys_per_cta = cdiv(cdiv(n_mid, per_seq), ks) * ks;
   const dim3 grid((unsigned)cdiv(n_mid, keys_per_cta), batch);
   static bool attr_set[64] = {};
@@ -263,21 +266,22 @@ void launch_score_small_ng(const float* q_c, const float* k_c, int lq, int64_t n
   }
   if (lq == 1)
     esa::score_small_kernel<DC, 1, NG><<<grid, esa::kSsThreads, esa::kSsSmemBytes, s>>>(
-        q_c, k_c, lq, n_cap, mid0, n_mid, keys_per_cta, S, m_key);
+        q_c, k_c, lq, n_cap, mid0, n_mid, keys_per_cta, S, m_key, vl);
   else
     esa::score_small_kernel<DC, esa::kScoreSmallLq, NG><<<grid, esa::kSsThreads, esa::kSsSmemBytes, s>>>(
-        q_c, k_c, lq, n_cap, mid0, n_mid, keys_per_cta, S, m_key);
+        q_c, k_c, lq, n_cap, mid0, n_mid, keys_per_cta, S, m_key, vl);
 }
 
 // groups must split a key's LPK lanes evenly (checked by score_path)
 template <int DC>
 void launch_score_small(const float* q_c, const float* k_c, int lq, int64_t n_cap, int64_t mid0, int64_t n_mid,
-                        int batch, int ng, float* S, uint32_t* m_key, cudaStream_t s) {
+                        int batch, int ng, float* S, uint32_t* m_key, const esa::VarLen& vl, cudaStream_t s) {
   constexpr int LPK = esa::SmallScoreShape<DC>::LPK;
-  if (ng == 1) launch_score_small_ng<DC, 1>(q_c, k_c, lq, n_cap, mid0, n_mid, batch, S, m_key, s);
-  else if (ng == 2) launch_score_small_ng<DC, 2>(q_c, k_c, lq, n_cap, mid0, n_mid, batch, S, m_key, s);
-  else if (ng == 4) launch_score_small_ng<DC, 4>(q_c, k_c, lq, n_cap, mid0, n_mid, batch, S, m_key, s);
-  else if constexpr (LPK % 8 == 0) launch_score_small_ng<DC, 8>(q_c, k_c, lq, n_cap, mid0, n_mid, batch, S, m_key, s);
+  if (ng == 1) launch_score_small_ng<DC, 1>(q_c, k_c, lq, n_cap, mid0, n_mid, batch, S, m_key, vl, s);
+  else if (ng == 2) launch_score_small_ng<DC, 2>(q_c, k_c, lq, n_cap, mid0, n_mid, batch, S, m_key, vl, s);
+  else if (ng == 4) launch_score_small_ng<DC, 4>(q_c, k_c, lq, n_cap, mid0, n_mid, batch, S, m_key, vl, s);
+  else if constexpr (LPK % 8 == 0)
+    launch_score_small_ng<DC, 8>(q_c, k_c, lq, n_cap, mid0, n_mid, batch, S, m_key, vl, s);
 }
 
 }  // namespace
@@ -300,6 +304,8 @@ esa_status_t esa_device_status(void* stream) {
   ESA_CUDA(cudaMemcpyToSymbol(esa::g_status, &zero, sizeof(zero)));
   const unsigned code = (unsigned)(v >> 32), site = (unsigned)(v & 0xffffffffu);
   if (code == 5u) return fail(ESA_ERR_CUDA, "kernel site %u found its shared memory misaligned and stopped", site);
+  if (code == 1u)
+    return fail(ESA_ERR_INVALID_ARG, "kernel site %u read a sequence length outside [1, n_cap] (clamped)", site);
   return fail(ESA_ERR_TIMEOUT, "device wait ran out at site %u (status %u)", site, code);
 }
 
@@ -383,9 +389,32 @@ esa_status_t pk_cluster_size(int dev, int* cl) {
 }
 }  // namespace
 
+namespace {
+esa_status_t compress_packed_impl(const void* x, int64_t rows, int64_t x_row_stride, int32_t n_heads_in,
+                                  int32_t head_dim, const void* packed, int32_t d_out, float* y, int64_t y_row_stride,
+                                  const esa::VarLen& yl, void* stream);
+}  // namespace
+
 esa_status_t esa_compress_packed(const void* x, int64_t rows, int64_t x_row_stride, int32_t n_heads_in,
                                  int32_t head_dim, const void* packed, int32_t d_out, float* y,
                                  int64_t y_row_stride, void* stream) {
+  return compress_packed_impl(x, rows, x_row_stride, n_heads_in, head_dim, packed, d_out, y, y_row_stride,
+                              esa::VarLen{}, stream);
+}
+
+esa_status_t esa_compress_packed_varlen(const void* x, int32_t batch, int64_t x_row_stride, int32_t n_heads_in,
+                                        int32_t head_dim, const void* packed, int32_t d_out, float* k_c,
+                                        int64_t n_cap, const int64_t* seq_len, void* stream) {
+  if (!seq_len) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  if (n_cap < 1) return fail(ESA_ERR_INVALID_ARG, "n_cap must be >= 1");
+  return compress_packed_impl(x, batch, x_row_stride, n_heads_in, head_dim, packed, d_out, k_c, d_out,
+                              esa::VarLen{seq_len, n_cap, 0, 0, 1}, stream);
+}
+
+namespace {
+esa_status_t compress_packed_impl(const void* x, int64_t rows, int64_t x_row_stride, int32_t n_heads_in,
+                                  int32_t head_dim, const void* packed, int32_t d_out, float* y, int64_t y_row_stride,
+                                  const esa::VarLen& yl, void* stream) {
   if (rows < 0) return fail(ESA_ERR_INVALID_ARG, "rows must be >= 0");
   if (rows == 0) return ok();
   if (!x || !packed || !y) return fail(ESA_ERR_INVALID_ARG, "null pointer");
@@ -425,11 +454,13 @@ esa_status_t esa_compress_packed(const void* x, int64_t rows, int64_t x_row_stri
     at[0].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, esa::compress_pk_kernel, tx, tw, nr, K, y + r0 * y_row_stride, y_row_stride);
+    if (yl.len && r0 > 0) return fail(ESA_ERR_UNSUPPORTED, "too many sequences");
+    cudaLaunchKernelEx(&cfg, esa::compress_pk_kernel, tx, tw, nr, K, y + r0 * y_row_stride, y_row_stride, yl);
     ESA_LAUNCH_CHECK("compress_pk_kernel");
   }
   return ok();
 }
+}  // namespace
 
 // ------------------------------------------------------------------ esa_compress --
 esa_status_t esa_compress(const void* x, esa_dtype_t x_dtype, int64_t rows, int64_t x_row_stride,
@@ -515,7 +546,7 @@ size_t score_select_ws(int32_t batch, int32_t lq, int64_t n_cap, int64_t c0, int
 esa_status_t score_select_impl(const float* q_c, const float* k_c, int32_t batch, int32_t lq, int64_t n_cap,
                                int64_t c0, int32_t d_c, int ng, esa_params_t p, int32_t* idx_out,
                                int32_t* count_out, float* score_out, void* workspace, size_t ws_bytes,
-                               void* stream);
+                               void* stream, const int64_t* seq_len = nullptr);
 
 }  // namespace
 
@@ -546,12 +577,30 @@ esa_status_t esa_score_select_heads(const float* q_c, const float* k_c, int32_t 
                            workspace, ws_bytes, stream);
 }
 
+size_t esa_score_select_varlen_workspace_size(int32_t batch, int64_t n_cap, int32_t d_c, int32_t n_groups,
+                                              esa_params_t p) {
+  if (n_cap < 1) return 0;
+  return score_select_ws(batch, 1, n_cap, n_cap - 1, d_c, n_groups, p);
+}
+
+esa_status_t esa_score_select_varlen(const float* q_c, const float* k_c, int32_t batch, int64_t n_cap,
+                                     const int64_t* seq_len, int32_t d_c, int32_t n_groups, esa_params_t p,
+                                     int32_t* idx_out, int32_t* count_out, float* score_out, void* workspace,
+                                     size_t ws_bytes, void* stream) {
+  if (n_groups != 1 && n_groups != 2 && n_groups != 4 && n_groups != 8)
+    return fail(ESA_ERR_UNSUPPORTED, "n_groups %d (1, 2, 4 or 8)", n_groups);
+  if (!seq_len) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  if (n_cap < 1) return fail(ESA_ERR_INVALID_ARG, "n_cap must be >= 1");
+  return score_select_impl(q_c, k_c, batch, 1, n_cap, n_cap - 1, d_c, n_groups, p, idx_out, count_out, score_out,
+                           workspace, ws_bytes, stream, seq_len);
+}
+
 namespace {
 
 esa_status_t score_select_impl(const float* q_c, const float* k_c, int32_t batch, int32_t lq, int64_t n_cap,
                                int64_t c0, int32_t d_c, int ng, esa_params_t p, int32_t* idx_out,
                                int32_t* count_out, float* score_out, void* workspace, size_t ws_bytes,
-                               void* stream) {
+                               void* stream, const int64_t* seq_len) {
   esa_status_t st = check_params(p);
   if (st != ESA_OK) return st;
   if (batch <= 0) return fail(ESA_ERR_INVALID_ARG, "batch must be >= 1");
@@ -567,10 +616,16 @@ esa_status_t score_select_impl(const float* q_c, const float* k_c, int32_t batch
   const int64_t vb = (int64_t)batch * ng;   // independent selections: sequence x group
   if (vb > 65535) return fail(ESA_ERR_UNSUPPORTED, "batch x groups must be <= 65535 (got %lld)", (long long)vb);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // a variable-length batch (c0 = n_cap - 1 here: the longest middle) selects per sequence
+  // in the selection kernel, so it always scores
+  const esa::VarLen vl_score{seq_len, n_cap, p.n_init, p.window, 1};
+  const esa::VarLen vl_sel{seq_len, n_cap, p.n_init, p.window, ng};
   const int64_t kk = std::min<int64_t>(p.topk, r.n_mid);
-  const bool need_scores = r.n_mid > p.topk || (score_out && r.n_mid > 0);
+  const bool need_scores = r.n_mid > p.topk || ((score_out || seq_len) && r.n_mid > 0);
   if (need_scores) {
     const ScorePath path = score_path(batch, lq, n_cap, d_c, ng);
+    if (seq_len && path != ScorePath::Small)
+      return fail(ESA_ERR_UNSUPPORTED, "variable lengths need one query and d_c in {16, 32, 64, 128, 256}");
     const SelWs need = carve_select(nullptr, (int32_t)vb, lq, r.n_mid, path);
     if (!workspace || ws_bytes < need.bytes || !aligned(workspace, 256))
       return fail(ESA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need.bytes, ws_bytes);
@@ -578,11 +633,11 @@ esa_status_t score_select_impl(const float* q_c, const float* k_c, int32_t batch
     ESA_CUDA(cudaMemsetAsync(w.m_key, 0, (size_t)vb * lq * sizeof(uint32_t), s));
     if (path == ScorePath::Small) {
       switch (d_c) {
-        case 16: launch_score_small<16>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, s); break;
-        case 32: launch_score_small<32>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, s); break;
-        case 64: launch_score_small<64>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, s); break;
-        case 128: launch_score_small<128>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, s); break;
-        default: launch_score_small<256>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, s); break;
+        case 16: launch_score_small<16>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, vl_score, s); break;
+        case 32: launch_score_small<32>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, vl_score, s); break;
+        case 64: launch_score_small<64>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, vl_score, s); break;
+        case 128: launch_score_small<128>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, vl_score, s); break;
+        default: launch_score_small<256>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, vl_score, s); break;
       }
       ESA_LAUNCH_CHECK("score_small_kernel");
     } else if (path == ScorePath::Tiled) {
@@ -625,6 +680,7 @@ esa_status_t score_select_impl(const float* q_c, const float* k_c, int32_t batch
       sa.eps = p.eps;
       sa.kk = (int)kk;
       sa.topk = p.topk;
+      sa.vl = vl_sel;
       sa.u = w.u;
       sa.s_prime_out = score_out;
       sa.idx = idx_out;
@@ -759,7 +815,8 @@ size_t sparse_attn_ws(int32_t batch, int32_t lq, int64_t c0, int32_t hq, int32_t
 esa_status_t sparse_attn_impl(const void* q, const void* k, const void* v, esa_dtype_t dt, int32_t batch,
                               int32_t lq, int64_t n_cap, int64_t c0, int32_t hq, int32_t hkv, int32_t head_dim,
                               const int32_t* idx, const int32_t* count, esa_params_t p, float scale, void* o,
-                              float* lse, void* workspace, size_t ws_bytes, void* stream, int lists);
+                              float* lse, void* workspace, size_t ws_bytes, void* stream, int lists,
+                              const int64_t* seq_len = nullptr);
 
 }  // namespace
 
@@ -790,13 +847,33 @@ esa_status_t esa_sparse_attn_heads(const void* q, const void* k, const void* v, 
                           workspace, ws_bytes, stream, hkv);
 }
 
+size_t esa_sparse_attn_varlen_workspace_size(int32_t batch, int64_t n_cap, int32_t hq, int32_t hkv, int32_t head_dim,
+                                             esa_dtype_t dt, int32_t lists, esa_params_t p) {
+  if (n_cap < 1) return 0;
+  return sparse_attn_ws(batch, 1, n_cap - 1, hq, hkv, head_dim, dt, p, lists);
+}
+
+esa_status_t esa_sparse_attn_varlen(const void* q, const void* k, const void* v, esa_dtype_t dt, int32_t batch,
+                                    int64_t n_cap, const int64_t* seq_len, int32_t hq, int32_t hkv,
+                                    int32_t head_dim, const int32_t* idx, const int32_t* count, int32_t lists,
+                                    esa_params_t p, float scale, void* o, float* lse, void* workspace,
+                                    size_t ws_bytes, void* stream) {
+  if (hkv <= 0) return fail(ESA_ERR_INVALID_ARG, "hkv must be >= 1");
+  if (lists != 1 && lists != hkv) return fail(ESA_ERR_INVALID_ARG, "lists must be 1 or hkv (got %d)", lists);
+  if (!seq_len) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  if (n_cap < 1) return fail(ESA_ERR_INVALID_ARG, "n_cap must be >= 1");
+  return sparse_attn_impl(q, k, v, dt, batch, 1, n_cap, n_cap - 1, hq, hkv, head_dim, idx, count, p, scale, o, lse,
+                          workspace, ws_bytes, stream, lists, seq_len);
+}
+
 namespace {
 
 
 esa_status_t sparse_attn_impl(const void* q, const void* k, const void* v, esa_dtype_t dt, int32_t batch,
                               int32_t lq, int64_t n_cap, int64_t c0, int32_t hq, int32_t hkv, int32_t head_dim,
                               const int32_t* idx, const int32_t* count, esa_params_t p, float scale, void* o,
-                              float* lse, void* workspace, size_t ws_bytes, void* stream, int lists) {
+                              float* lse, void* workspace, size_t ws_bytes, void* stream, int lists,
+                              const int64_t* seq_len) {
   esa_status_t st = check_params(p);
   if (st != ESA_OK) return st;
   if (dt != ESA_F32 && dt != ESA_BF16) return fail(ESA_ERR_INVALID_ARG, "bad dtype %d", (int)dt);
@@ -820,6 +897,11 @@ esa_status_t sparse_attn_impl(const void* q, const void* k, const void* v, esa_d
   const float sl2 = scale * 1.4426950408889634f;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   esa::KeyList keys{idx, p.topk, r.ni, r.lo, n_cap, count};
+  if (seq_len) {
+    // a variable-length decode batch (c0 = n_cap - 1 here: the plan covers the longest key list)
+    if (lq != 1 || pl.tc) return fail(ESA_ERR_UNSUPPORTED, "variable lengths need one query per sequence");
+    keys.vl = esa::VarLen{seq_len, n_cap, p.n_init, p.window, vseq ? hkv : 1};
+  }
   if (pl.tc) {
     static bool attr_set[64] = {};
     int dev = 0;

@@ -49,13 +49,14 @@ struct SsSmem {
 };
 
 // grid (ctas per sequence, B); kSsThreads threads; kSsSmemBytes dynamic shared memory.
-// CTA c scores keys [c * keys_per_cta, ...) of the middle (keys_per_cta a multiple of KS).
+// CTA c scores keys [c * keys_per_cta, ...) of the middle (keys_per_cta a multiple of KS);
+// in a variable-length batch (vl.len) CTAs past their sequence's middle have nothing to do.
 template <int DC, int LQ, int NG>
 __global__ void __launch_bounds__(kSsThreads, 2) score_small_kernel(const float* __restrict__ q_c,
                                                                    const float* __restrict__ k_c, int lq,
                                                                    int64_t n_cap, int64_t mid0, int64_t n_mid,
                                                                    int64_t keys_per_cta, float* __restrict__ s_out,
-                                                                   uint32_t* __restrict__ m_key) {
+                                                                   uint32_t* __restrict__ m_key, const VarLen vl) {
   using Sh = SmallScoreShape<DC>;
   constexpr int VPL = Sh::VPL, LPK = Sh::LPK, KPW = Sh::KPW, KS = Sh::KS;
   constexpr int KEYS_PER_WARP = KS / kSsWarps;             // of a stage
@@ -70,7 +71,8 @@ __global__ void __launch_bounds__(kSsThreads, 2) score_small_kernel(const float*
   const int grp = lane / LPK, sub = lane % LPK;
   const int hg = sub / LPG;                                // this lane's group
   const int64_t j_begin = (int64_t)blockIdx.x * keys_per_cta;
-  const int64_t j_end = min(n_mid, j_begin + keys_per_cta);
+  // n_mid is the row stride of S; a variable-length batch scores each sequence's own middle
+  const int64_t j_end = min(vl.len ? vl.n_mid(b, 801) : n_mid, j_begin + keys_per_cta);
   const int nst = j_end > j_begin ? (int)((j_end - j_begin + KS - 1) / KS) : 0;
   const float* kb = k_c + ((int64_t)b * n_cap + mid0) * DC;
 

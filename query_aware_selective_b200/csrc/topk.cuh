@@ -43,6 +43,8 @@ struct SelectArgs {
   int eps;                 // <= kSelMaxEps
   int kk;                  // keys to keep: min(topk, n_mid) >= 1
   int topk;
+  VarLen vl;               // vl.len: a variable-length decode batch; n_mid is then the longest
+                           // possible middle (the row stride of S, s, s_prime_out) and kk == topk
   uint32_t* u;             // [B, n_mid] key scratch (used when a CTA's range exceeds kSelUCap)
   float* s_prime_out;      // [B, n_mid] or null
   int32_t* idx;            // [B, topk]
@@ -65,12 +67,11 @@ constexpr int kSelSmemBytes = (int)sizeof(SelSmem);
 constexpr int kSelHaloTile = kSelTile + 2 * kSelMaxEps;
 constexpr int kSelSlots = (kSelHaloTile + kSelThreads - 1) / kSelThreads;
 
-__device__ __forceinline__ void sel_load_tile(const SelectArgs& a, int b, int64_t g0, int nt, float* v) {
+__device__ __forceinline__ void sel_load_tile(const SelectArgs& a, int b, int64_t n, int64_t g0, int nt, float* v) {
   const int tid = threadIdx.x;
-  const int64_t n = a.n_mid;
   const int width = nt + 2 * a.eps;
   if (!a.S) {
-    const float* sb = a.s + (int64_t)b * n;
+    const float* sb = a.s + (int64_t)b * a.n_mid;
 #pragma unroll
     for (int e = 0; e < kSelSlots; ++e) {
       const int t = tid + e * kSelThreads;
@@ -84,7 +85,7 @@ __device__ __forceinline__ void sel_load_tile(const SelectArgs& a, int b, int64_
   for (int e = 0; e < kSelSlots; ++e) v[e] = 0.f;
   for (int i = 0; i < a.lq; ++i) {
     const float m = key_to_float(__ldg(&a.m_key[b * a.lq + i]));
-    const float* Sb = a.S + ((int64_t)b * a.lq + i) * n;
+    const float* Sb = a.S + ((int64_t)b * a.lq + i) * a.n_mid;
     float x[kSelSlots];
 #pragma unroll
     for (int e = 0; e < kSelSlots; ++e) {
@@ -112,12 +113,22 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_cluster_kernel(const Se
   const uint32_t rank = cluster_rank();
   const int b = blockIdx.y;
   const int tid = threadIdx.x;
-  const int64_t n = a.n_mid;
+  // this selection's middle length and keep count (a variable-length batch: its own)
+  const int64_t n = a.vl.len ? a.vl.n_mid(b, 901) : a.n_mid;
+  const int kk = (int)min((int64_t)a.kk, n);
+  if (kk == 0) {                           // empty middle: nothing kept (before any cluster step)
+    if (rank == 0) {
+      for (int t = tid; t < a.topk; t += kSelThreads) a.idx[(int64_t)b * a.topk + t] = -1;
+      if (tid == 0) a.count[b] = 0;
+    }
+    return;
+  }
   const int64_t per = ((n + CL - 1) / CL + 3) & ~(int64_t)3;   // a multiple of 4: 16-byte key groups
+  const int64_t per_stride = ((a.n_mid + CL - 1) / CL + 3) & ~(int64_t)3;
   const int64_t j0 = min(n, (int64_t)rank * per);
   const int nloc = (int)(min(n, j0 + per) - j0);
-  // key of position j0 + t at ub[t]; the global scratch gives every CTA `per` slots
-  uint32_t* ub = per <= kSelUCap ? sm.ucache : a.u + ((int64_t)b * CL + rank) * per;
+  // key of position j0 + t at ub[t]; the global scratch gives every CTA per_stride slots
+  uint32_t* ub = per <= kSelUCap ? sm.ucache : a.u + ((int64_t)b * CL + rank) * per_stride;
   const int eps = a.eps;
 
   // every CTA clears its merged slices; the barrier phase this arrival opens is waited
@@ -131,7 +142,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_cluster_kernel(const Se
   __syncthreads();
   const int n_tiles = (nloc + kSelTile - 1) / kSelTile;
   float v[kSelSlots];
-  if (n_tiles > 0) sel_load_tile(a, b, j0, min(nloc, kSelTile), v);
+  if (n_tiles > 0) sel_load_tile(a, b, n, j0, min(nloc, kSelTile), v);
   for (int tile = 0; tile < n_tiles; ++tile) {
     const int t0 = tile * kSelTile;
     const int nt = min(kSelTile, nloc - t0);
@@ -141,7 +152,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_cluster_kernel(const Se
       if (t < kSelHaloTile) sm.sv[t] = v[e];
     }
     __syncthreads();
-    if (tile + 1 < n_tiles) sel_load_tile(a, b, j0 + t0 + kSelTile, min(kSelTile, nloc - t0 - kSelTile), v);
+    if (tile + 1 < n_tiles) sel_load_tile(a, b, n, j0 + t0 + kSelTile, min(kSelTile, nloc - t0 - kSelTile), v);
     // four consecutive positions per thread; with eps <= 6 the window of all four is one
     // run of 16 values read as four 16-byte loads
     for (int t = 4 * tid; t < nt; t += 4 * kSelThreads) {
@@ -184,7 +195,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_cluster_kernel(const Se
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         if (t + q < nt) {
-          if (a.s_prime_out) a.s_prime_out[(int64_t)b * n + j0 + t0 + t + q] = mq[q];
+          if (a.s_prime_out) a.s_prime_out[(int64_t)b * a.n_mid + j0 + t0 + t + q] = mq[q];
           atomicAdd(&sm.hist[kq[q] >> 21], 1u);
         }
       }
@@ -194,7 +205,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_cluster_kernel(const Se
 
   // ---- three radix levels, histograms merged slice by slice across the cluster
   cluster_wait();                          // every CTA's merged slices are cleared
-  uint32_t prefix = 0, want = (uint32_t)a.kk;
+  uint32_t prefix = 0, want = (uint32_t)kk;
   for (int level = 0; level < 3; ++level) {
     const int bits = level == 2 ? 10 : 11;
     const int nb = 1 << bits;
@@ -324,8 +335,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_cluster_kernel(const Se
     }
   }
   if (rank == 0) {
-    for (int t = a.kk + tid; t < a.topk; t += kSelThreads) out[t] = -1;
-    if (tid == 0) a.count[b] = a.kk;
+    for (int t = kk + tid; t < a.topk; t += kSelThreads) out[t] = -1;
+    if (tid == 0) a.count[b] = kk;
   }
 }
 

@@ -332,6 +332,63 @@ class EsaDecode:
         return self.out
 
 
+class EsaDecodeVarlen:
+    """One decode step for a batch of sequences of different lengths. Sequence b holds
+    seq_len[b] tokens (a device int64 tensor, so a captured step replays with new
+    lengths) in caches of n_cap rows, its query at position seq_len[b] - 1; its new
+    key row (already appended to the KV cache by the caller) is compressed into row
+    seq_len[b] - 1 of the compressed cache. Needs the packed compression path (bf16,
+    d_c 128)."""
+
+    def __init__(self, batch: int, n_cap: int, hq: int, hkv: int, head_dim: int, d_c: int, p: _abi.EsaParams,
+                 dtype=torch.bfloat16, device="cuda", per_head: bool = False):
+        self.batch, self.n_cap, self.hq, self.hkv, self.d, self.d_c, self.p = batch, n_cap, hq, hkv, head_dim, d_c, p
+        self.per_head = per_head
+        self.ng = hkv if per_head else 1
+        self.cmp = _Compressor(hq, hkv, head_dim, d_c, dtype, device)
+        if not self.cmp.packed:
+            raise ValueError("variable-length decode needs the packed compression path (bf16, d_c 128)")
+        self.k_c = torch.zeros((batch, n_cap, d_c), dtype=torch.float32, device=device)
+        self.q_c = torch.empty((batch, 1, d_c), dtype=torch.float32, device=device)
+        self.idx = torch.empty((batch, self.ng, p.topk), dtype=torch.int32, device=device)
+        self.count = torch.empty((batch, self.ng), dtype=torch.int32, device=device)
+        self.out = torch.empty((batch, 1, hq, head_dim), dtype=dtype, device=device)
+        code = _abi.ESA_BF16 if dtype == torch.bfloat16 else _abi.ESA_F32
+        n_sel = _abi.score_select_varlen_workspace_size(batch, n_cap, d_c, self.ng, p)
+        nb = _abi.sparse_attn_varlen_workspace_size(batch, n_cap, hq, hkv, head_dim, code, self.ng, p)
+        self.ws_sel = torch.empty(n_sel + 256, dtype=torch.uint8, device=device)
+        self.ws_att = torch.empty(nb + 256, dtype=torch.uint8, device=device) if nb else None
+        self.side = _side_stream(device)
+
+    def fill_cache(self, k, wk, lengths):
+        """Compress cached keys [0, lengths[b] - 1) of every sequence (prefill state);
+        lengths: host integers."""
+        self.cmp.pack_keys(wk)
+        step = 1 << 16
+        for s in range(self.batch):
+            upto = int(lengths[s]) - 1
+            for r0 in range(0, upto, step):
+                r1 = min(upto, r0 + step)
+                self.cmp.keys(k[s, r0:r1], out=self.k_c[s, r0:r1])
+
+    def step(self, q, k_new, k, v, wq, wk, seq_len):
+        """q [B, 1, Hq, D]; k_new [B, Hkv, D] the new key rows (also at row seq_len[b] - 1
+        of k); k, v [B, n_cap, Hkv, D]; seq_len [B] int64 on the device."""
+        cur = torch.cuda.current_stream()
+        self.cmp.pack_if_changed(wq, wk)
+        # the new token is local to its own query: its compressed key is not read this step
+        self.side.wait_stream(cur)
+        with torch.cuda.stream(self.side):
+            _abi.compress_packed_varlen(k_new, self.cmp.wk_p, self.k_c, seq_len)
+        self.cmp.queries(q[:, 0], out=self.q_c.view(self.batch, self.d_c))
+        _abi.score_select_varlen(self.q_c, self.k_c, seq_len, self.p, n_groups=self.ng, idx=self.idx,
+                                 count=self.count, workspace=self.ws_sel)
+        _abi.sparse_attn_varlen(q, k, v, seq_len, self.idx, self.count, self.p, out=self.out,
+                                workspace=self.ws_att)
+        cur.wait_stream(self.side)
+        return self.out
+
+
 class MobaPrefill:
     """MoBA causal prefill of one layer: gate, then block attention."""
 

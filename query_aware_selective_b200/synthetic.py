@@ -227,6 +227,16 @@ def make_moba_decode_inputs(w: MobaWorkload, device="cpu", seq: Optional[int] = 
     return dict(q=q, k=k, v=v)
 
 
+def varlen_lengths(batch: int, n_max: int, n_min: int, seed: int) -> torch.Tensor:
+    """Lengths of a variable-length decode batch: sequence 0 holds n_max tokens, the
+    others a seeded uniform draw from [n_min, n_max]. Returns int64 [batch] (host)."""
+    gen = torch.Generator()
+    gen.manual_seed(seed)
+    lens = torch.randint(n_min, n_max + 1, (batch,), generator=gen, dtype=torch.int64)
+    lens[0] = n_max
+    return lens
+
+
 def random_index_list(batch: int, mid0: int, mid1: int, topk: int, seed: int) -> tuple:
     """A valid selection result drawn at random: per sequence, min(topk, |mid|)
     distinct middle positions, ascending, padded with -1. Used to test the
