@@ -48,7 +48,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--prefill-ctx", type=int, default=0,
                     help="shorter prefill context (profiling a small case); the line then names that workload")
-    ap.add_argument("--only", choices=["decode", "decode_per_head", "moba", "moba_decode"], default=None,
+    ap.add_argument("--only", choices=["decode", "decode_per_head", "decode_varlen", "moba", "moba_decode"],
+                    default=None,
                     help="profiling: run one of the other workloads alone and print its figures")
     ap.add_argument("--decode-batch", type=int, default=0, help="profiling: decode batch (default: the workload's)")
     ap.add_argument("--moba-seq", type=int, default=0, help="profiling: MoBA sequence length (default: the workload's)")
@@ -224,6 +225,8 @@ def run_only(args):
         out = bench_moba(args, dev, flush, make_dist_max(), peaks, peak_src, 1)
     elif args.only == "moba_decode":
         out = bench_moba_decode(args, dev, flush, make_dist_max(), peaks, peak_src, 1)
+    elif args.only == "decode_varlen":
+        out = bench_decode_varlen(args, dev, flush, make_dist_max(), peaks, peak_src, 1)
     else:
         out = bench_decode(args, dev, flush, make_dist_max(), peaks, peak_src, 1, per_head=args.only == "decode_per_head")
     print(json.dumps({"only": args.only, **out}), flush=True)
@@ -338,6 +341,9 @@ def run_ours(args):
         line["also"]["esa_decode_128k_per_head"] = bench_decode(args, dev, flush, dist_max, peaks, peak_src, world,
                                                                 per_head=True)
         torch.cuda.empty_cache()
+        line["also"]["esa_decode_128k_varlen"] = bench_decode_varlen(args, dev, flush, dist_max, peaks, peak_src,
+                                                                     world)
+        torch.cuda.empty_cache()
         line["also"]["moba_prefill_64k"] = bench_moba(args, dev, flush, dist_max, peaks, peak_src, world)
         torch.cuda.empty_cache()
         line["also"]["moba_decode_64k"] = bench_moba_decode(args, dev, flush, dist_max, peaks, peak_src, world)
@@ -395,6 +401,35 @@ def bench_decode(args, dev, flush, dist_max, peaks, peak_src, world, per_head=Fa
                          "peak_source": f"{peak_src} HBM copy"},
             "phases": {"score_select_ms": round(sel_ms, 4), "score_select_gbs": round(sel_gbs, 1),
                        "sparse_attn_ms": round(att_ms, 4), "sparse_attn_gbs": round(att_gbs, 1)}}
+
+
+def bench_decode_varlen(args, dev, flush, dist_max, peaks, peak_src, world):
+    """ESA decode, batch 16, caches of 128K rows holding a seeded mix of lengths
+    (sequence 0 at 131072, the rest uniform in [8192, 131072]), lengths on the device."""
+    import torch
+    import query_aware_selective_b200 as qas
+    from query_aware_selective_b200 import cost, pipeline, synthetic
+    w = synthetic.DECODE_128K
+    p = qas.params(w.n_init, w.window, w.topk, w.eps, w.clamp_c)
+    lens = synthetic.varlen_lengths(w.batch, w.n_ctx, 8192, seed=w.seed + 2000)
+    inp = synthetic.make_esa_inputs(w, device=dev)
+    dec = pipeline.EsaDecodeVarlen(w.batch, w.n_ctx, w.hq, w.hkv, w.head_dim, w.d_c, p, device=dev)
+    dec.fill_cache(inp["k"], inp["wk"], lens.tolist())
+    seq_len = lens.to(dev)
+    k_new = inp["k"][torch.arange(w.batch, device=dev), seq_len - 1].contiguous()
+    torch.cuda.synchronize()
+    graph = pipeline.graph_of(lambda: dec.step(inp["q"], k_new, inp["k"], inp["v"], inp["wq"], inp["wk"], seq_len))
+    steps = max(args.steps, 20)
+    ms, total = time_steps(graph.replay, steps, args.warmup, flush, dist_max)
+    by = cost.decode_varlen_bytes(lens.tolist(), w.hq, w.hkv, w.head_dim, w.d_c, w.n_init, w.window, w.topk)
+    gbs = by["total"] / (total / steps / 1e3) / 1e9
+    hbm = peaks["hbm_gbs"]
+    return {"workload": f"esa_decode_llama3_8b_b{w.batch}_varlen8192to131072",
+            "lengths": lens.tolist(), "value": round(world * w.batch * steps / (total / 1e3), 1), "unit": "tok/s",
+            "ms_per_step": round(total / steps, 4), "steps": steps, "execution": "one CUDA graph per step",
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "bytes_per_step": by["total"],
+                         "peak_source": f"{peak_src} HBM copy"}}
 
 
 def bench_moba_decode(args, dev, flush, dist_max, peaks, peak_src, world):

@@ -81,6 +81,18 @@ def decode_bytes(batch: int, n_ctx: int, hq: int, hkv: int, d: int, d_c: int, n_
                 n_mid=n_mid, attended=n_att)
 
 
+def decode_varlen_bytes(lengths, hq: int, hkv: int, d: int, d_c: int, n_init: int, window: int, topk: int,
+                        kv_bytes: int = 2) -> dict:
+    """One decode step of a batch whose sequence b holds lengths[b] tokens (its query at
+    lengths[b] - 1): the per-sequence bytes summed, the weights read once."""
+    parts = [decode_bytes(1, int(n), hq, hkv, d, d_c, n_init, window, topk, kv_bytes) for n in lengths]
+    kc = sum(x["compressed_keys"] for x in parts)
+    kv = sum(x["kv_rows"] for x in parts)
+    io = sum(x["io"] for x in parts)
+    weights = parts[0]["weights"]
+    return dict(compressed_keys=kc, kv_rows=kv, weights=weights, io=io, total=kc + kv + weights + io)
+
+
 def full_decode_bytes(batch: int, n_ctx: int, hkv: int, d: int, kv_bytes: int = 2) -> int:
     return batch * n_ctx * hkv * d * kv_bytes * 2
 

@@ -90,11 +90,6 @@ __device__ __forceinline__ void mma_bf16_rows8(float* d, uint32_t a0, uint32_t a
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
 struct DecSmem {
   uint64_t full[kDecStages];
   int done[kDecStages];   // warps finished with the stage's current fill

@@ -1071,7 +1071,7 @@ struct MobaWs {
   uint32_t* tile_off;
   uint32_t* totals;
   uint32_t* list;
-  float* part_o;
+  __nv_bfloat16* part_o;   // past partials: [B, seq, H, topk, D] bf16, lse [B, seq, H, topk]
   float* part_lse;
   size_t zero_bytes;
   size_t bytes;
@@ -1105,8 +1105,8 @@ MobaWs carve_moba(void* ws, int which, int32_t batch, int64_t seq, int32_t heads
     w.tile_off = c.take<uint32_t>(w.n_lists + 1);
     w.totals = c.take<uint32_t>(2);
     w.list = c.take<uint32_t>(std::max<int64_t>(1, w.pairs));
-    w.part_o = c.take<float>((size_t)batch * seq * heads * (topk + 1) * d);
-    w.part_lse = c.take<float>((size_t)batch * seq * heads * (topk + 1));
+    w.part_o = c.take<__nv_bfloat16>((size_t)batch * seq * heads * topk * d);
+    w.part_lse = c.take<float>((size_t)batch * seq * heads * topk);
   }
   w.bytes = c.off;
   return w;
@@ -1201,6 +1201,8 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
   cp.v = static_cast<const __nv_bfloat16*>(v);
   cp.part_o = w.part_o;
   cp.part_lse = w.part_lse;
+  cp.o = static_cast<__nv_bfloat16*>(o);
+  cp.lse = lse;
   cp.seq = seq;
   cp.heads = heads;
   cp.n_blocks = nb;
@@ -1212,10 +1214,6 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
       <<<dim3(cp.tiles_per_block * nb, heads, batch), esa::kTcThreads, esa::kTcSmemBytes, s>>>(tq, tk, tv, bq, bk, bv,
                                                                                             bk, bv, cp);
   ESA_LAUNCH_CHECK("attn_tc_kernel<moba current>");
-  const int64_t rows = (int64_t)batch * seq * heads;
-  esa::moba_combine_kernel<128><<<(unsigned)cdiv(rows, 8), 256, 0, s>>>(
-      w.part_o, w.part_lse, seq, heads, block, topk, rows, static_cast<__nv_bfloat16*>(o), lse);
-  ESA_LAUNCH_CHECK("moba_combine_kernel");
   return ESA_OK;
 }
 

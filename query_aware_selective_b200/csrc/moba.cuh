@@ -8,10 +8,12 @@
 // The attention is grouped by key block instead of by query: for every (sequence,
 // head, past block) the queries that chose that block form a list, and one tensor-core
 // CTA attends 128 listed queries to the block's contiguous keys. Each (query, head)
-// thereby gets one partial (o, lse) per attended block, written to its slot (the
-// block's rank in the query's list); the current block is one more partial, and a
-// final kernel merges the partials by log-sum-exp. The work is exactly the selected
-// (query, block) pairs, so no key is attended that the gate did not keep.
+// thereby gets one partial per attended past block, written to its slot (the block's
+// rank in the query's list) as a normalised bf16 row and a base-2 log-sum-exp. The
+// CTA that attends a query tile to its own (current) block, causally, runs after them
+// and merges the tile's past partials into its result by log-sum-exp in its epilogue,
+// writing the output. The work is exactly the selected (query, block) pairs, so no
+// key is attended that the gate did not keep.
 #pragma once
 #include <cub/block/block_scan.cuh>
 
@@ -224,12 +226,13 @@ __global__ void __launch_bounds__(1024) moba_scan_kernel(const uint32_t* __restr
 }
 
 // ------------------------------------------------------------------ TC problems --
-// Partials: part_o [B, seq, H, topk+1, D] fp32 (normalised), part_lse [B, seq, H, topk+1].
+// Past partials: part_o [B, seq, H, topk, D] bf16 (normalised), part_lse [B, seq, H,
+// topk] fp32, base 2; slot s of (b, p, h) is the s-th kept past block of that query.
 struct MobaPastProblem {
   const __nv_bfloat16* q;
   const __nv_bfloat16* k;
   const __nv_bfloat16* v;
-  float* part_o;
+  __nv_bfloat16* part_o;
   float* part_lse;
   const uint32_t* tile_off;   // [n_lists + 1]
   const uint32_t* off;        // [n_lists]
@@ -282,13 +285,19 @@ struct MobaPastProblem {
     const uint32_t e = list[e0 + r];
     const int64_t p = e >> 4;
     const int slot = e & 15;
-    const int64_t row = (((int64_t)b * seq + p) * heads + h) * (topk + 1) + slot;
+    const int64_t row = (((int64_t)b * seq + p) * heads + h) * topk + slot;
     const float inv = 1.f / l;
-    float4* dst = reinterpret_cast<float4*>(part_o + row * kTcD + col0);
+    uint4* dst = reinterpret_cast<uint4*>(part_o + row * kTcD + col0);
 #pragma unroll
-    for (int c = 0; c < kTcD / kTcSplit / 4; ++c)
-      dst[c] = make_float4(acc[4 * c] * inv, acc[4 * c + 1] * inv, acc[4 * c + 2] * inv, acc[4 * c + 3] * inv);
-    if (col0 == 0) part_lse[row] = (m2 + __log2f(l)) * 0.69314718055994531f;
+    for (int c = 0; c < kTcD / kTcSplit / 8; ++c) {
+      uint4 u;
+      u.x = bf16x2_rn(acc[8 * c] * inv, acc[8 * c + 1] * inv);
+      u.y = bf16x2_rn(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
+      u.z = bf16x2_rn(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv);
+      u.w = bf16x2_rn(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
+      dst[c] = u;
+    }
+    if (col0 == 0) part_lse[row] = m2 + __log2f(l);
   }
 };
 
@@ -298,8 +307,10 @@ struct MobaCurrentProblem {
   const __nv_bfloat16* q;
   const __nv_bfloat16* k;
   const __nv_bfloat16* v;
-  float* part_o;
-  float* part_lse;
+  const __nv_bfloat16* part_o;   // the past partials (MobaPastProblem), complete before this kernel
+  const float* part_lse;
+  __nv_bfloat16* o;              // [B, seq, H, D]
+  float* lse;                    // [B, seq, H] or null
   int64_t seq;
   int heads, n_blocks, block, topk, tiles_per_block;
   float sl2;
@@ -336,50 +347,53 @@ struct MobaCurrentProblem {
   }
   __device__ int64_t limit(int r) const { return p0 + min((int64_t)r, nrows - 1) - kb0; }
   __device__ float scale_log2() const { return sl2; }
+  // this part of the row merged with the query's min(topk, blk) past partials by
+  // log-sum-exp (base 2), then written as the output
   __device__ void store(int r, int col0, const float* acc, float m2, float l) {
+    constexpr int HC = kTcD / kTcSplit;
     if (r >= nrows) return;
-    const int64_t p = p0 + r;
-    const int slot = min(topk, blk);
-    const int64_t row = (((int64_t)b * seq + p) * heads + h) * (topk + 1) + slot;
-    const float inv = 1.f / l;
-    float4* dst = reinterpret_cast<float4*>(part_o + row * kTcD + col0);
+    const int64_t row = ((int64_t)b * seq + p0 + r) * heads + h;
+    const int ns = min(topk, blk);
+    const float* pl = part_lse + row * topk;
+    const float lc = m2 + __log2f(l);
+    float M = lc;
+    for (int s = 0; s < ns; ++s) M = fmaxf(M, __ldg(pl + s));
+    const float wc = exp2f(lc - M);
+    float L = wc;
+    float out[HC];
+    const float cw = wc / l;
 #pragma unroll
-    for (int c = 0; c < kTcD / kTcSplit / 4; ++c)
-      dst[c] = make_float4(acc[4 * c] * inv, acc[4 * c + 1] * inv, acc[4 * c + 2] * inv, acc[4 * c + 3] * inv);
-    if (col0 == 0) part_lse[row] = (m2 + __log2f(l)) * 0.69314718055994531f;
+    for (int c = 0; c < HC; ++c) out[c] = acc[c] * cw;
+    for (int s = 0; s < ns; ++s) {
+      const float w = exp2f(__ldg(pl + s) - M);
+      L += w;
+      const uint4* src = reinterpret_cast<const uint4*>(part_o + (row * topk + s) * kTcD + col0);
+#pragma unroll
+      for (int c = 0; c < HC / 8; ++c) {
+        const uint4 u = __ldg(src + c);
+        const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = bf16x2_to_float2(wd[e]);
+          out[8 * c + 2 * e] = fmaf(w, f.x, out[8 * c + 2 * e]);
+          out[8 * c + 2 * e + 1] = fmaf(w, f.y, out[8 * c + 2 * e + 1]);
+        }
+      }
+    }
+    const float inv = 1.f / L;
+    uint4* dst = reinterpret_cast<uint4*>(o + row * kTcD + col0);
+#pragma unroll
+    for (int c = 0; c < HC / 8; ++c) {
+      uint4 u;
+      u.x = bf16x2_rn(out[8 * c] * inv, out[8 * c + 1] * inv);
+      u.y = bf16x2_rn(out[8 * c + 2] * inv, out[8 * c + 3] * inv);
+      u.z = bf16x2_rn(out[8 * c + 4] * inv, out[8 * c + 5] * inv);
+      u.w = bf16x2_rn(out[8 * c + 6] * inv, out[8 * c + 7] * inv);
+      dst[c] = u;
+    }
+    if (col0 == 0 && lse) lse[row] = (M + __log2f(L)) * 0.69314718055994531f;
   }
 };
-
-// Merge the min(topk, cur) + 1 partials of each (b, p, h). One warp per row.
-template <int D>
-__global__ void __launch_bounds__(256) moba_combine_kernel(const float* __restrict__ part_o,
-                                                           const float* __restrict__ part_lse, int64_t seq, int heads,
-                                                           int block, int topk, int64_t n_rows,
-                                                           __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
-  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);   // (b, p, h) flattened
-  const int lane = threadIdx.x & 31;
-  if (row >= n_rows) return;
-  const int64_t p = (row / heads) % seq;
-  const int ns = min(topk, (int)(p / block)) + 1;
-  const float* lr = part_lse + row * (topk + 1);
-  float M = -INFINITY;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, lr[s]);
-  float L = 0.f;
-  float acc[D / 32];
-#pragma unroll
-  for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
-  for (int s = 0; s < ns; ++s) {
-    const float w = __expf(lr[s] - M);
-    L += w;
-    const float* po = part_o + (row * (topk + 1) + s) * D;
-#pragma unroll
-    for (int e = 0; e < D / 32; ++e) acc[e] = fmaf(w, po[lane + 32 * e], acc[e]);
-  }
-  const float inv = 1.f / L;
-#pragma unroll
-  for (int e = 0; e < D / 32; ++e) o[row * D + lane + 32 * e] = __float2bfloat16_rn(acc[e] * inv);
-  if (lane == 0 && lse) lse[row] = M + __logf(L);
-}
 
 // ------------------------------------------------------------------ decode gate --
 // One query per (sequence, head) at position pos (decode; MoBA article, section 2: the

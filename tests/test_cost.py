@@ -45,3 +45,14 @@ def test_moba_flops_limits():
     s, h, d, blk = 4096, 2, 64, 256
     assert cost.moba_flops(s, h, d, blk, 10**6)["attention"] == cost.full_causal_attn_flops(s, h, d)
     assert cost.moba_flops(s, h, d, blk, 0)["attention"] == (s // blk) * cost.full_causal_attn_flops(blk, h, d)
+
+
+def test_varlen_bytes_reduce_to_the_equal_length_batch():
+    a = cost.decode_varlen_bytes([131072] * 16, 32, 8, 128, 128, 128, 4096, 2048)
+    b = cost.decode_bytes(16, 131072, 32, 8, 128, 128, 128, 4096, 2048)
+    assert a["total"] == b["total"]
+    # a short sequence reads no compressed keys (empty middle) and only its own rows
+    c = cost.decode_varlen_bytes([131072, 100], 32, 8, 128, 128, 128, 4096, 2048)
+    d = cost.decode_bytes(1, 131072, 32, 8, 128, 128, 128, 4096, 2048)
+    assert c["compressed_keys"] == d["compressed_keys"]
+    assert c["kv_rows"] == d["kv_rows"] + 100 * 8 * 128 * 2 * 2
