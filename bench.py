@@ -40,7 +40,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true", help="time the headline workload only")
@@ -48,7 +48,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--prefill-ctx", type=int, default=0,
                     help="shorter prefill context (profiling a small case); the line then names that workload")
-    ap.add_argument("--only", choices=["decode", "decode_per_head", "decode_varlen", "moba", "moba_decode"],
+    ap.add_argument("--only", choices=["decode", "decode_per_head", "decode_varlen", "decode_1m", "moba",
+                                       "moba_decode"],
                     default=None,
                     help="profiling: run one of the other workloads alone and print its figures")
     ap.add_argument("--decode-batch", type=int, default=0, help="profiling: decode batch (default: the workload's)")
@@ -87,7 +88,7 @@ def traffic_for(kernel: str, sources):
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples every 200 ms while running (clocks, power, throttle reasons)."""
+    """nvidia-smi samples every 100 ms while running (clocks, power, throttle reasons)."""
 
     FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "utilization.gpu", "clocks_event_reasons.active",
               "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
@@ -99,7 +100,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -227,6 +228,9 @@ def run_only(args):
         out = bench_moba_decode(args, dev, flush, make_dist_max(), peaks, peak_src, 1)
     elif args.only == "decode_varlen":
         out = bench_decode_varlen(args, dev, flush, make_dist_max(), peaks, peak_src, 1)
+    elif args.only == "decode_1m":
+        from query_aware_selective_b200 import synthetic
+        out = bench_decode(args, dev, flush, make_dist_max(), peaks, peak_src, 1, workload=synthetic.DECODE_1M)
     else:
         out = bench_decode(args, dev, flush, make_dist_max(), peaks, peak_src, 1, per_head=args.only == "decode_per_head")
     print(json.dumps({"only": args.only, **out}), flush=True)
@@ -344,13 +348,16 @@ def run_ours(args):
         line["also"]["esa_decode_128k_varlen"] = bench_decode_varlen(args, dev, flush, dist_max, peaks, peak_src,
                                                                      world)
         torch.cuda.empty_cache()
+        line["also"]["esa_decode_1m"] = bench_decode(args, dev, flush, dist_max, peaks, peak_src, world,
+                                                     workload=synthetic.DECODE_1M)
+        torch.cuda.empty_cache()
         line["also"]["moba_prefill_64k"] = bench_moba(args, dev, flush, dist_max, peaks, peak_src, world)
         torch.cuda.empty_cache()
         line["also"]["moba_decode_64k"] = bench_moba_decode(args, dev, flush, dist_max, peaks, peak_src, world)
     line["clocks"] = sampler.stop()
     line["gpu"] = props.name
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_prefill(seconds_hint=10.0)
+        line["cpu_baseline"] = cpu_baseline_prefill()
     if _dist is not None:
         _dist.barrier()
         _dist.destroy_process_group()
@@ -358,13 +365,14 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
-def bench_decode(args, dev, flush, dist_max, peaks, peak_src, world, per_head=False):
-    """ESA decode at 128K, batch 16. per_head: the per-head selection variant (one
-    index set per KV head, block-diagonal compression maps) on the same inputs."""
+def bench_decode(args, dev, flush, dist_max, peaks, peak_src, world, per_head=False, workload=None):
+    """ESA decode at 128K, batch 16 (or `workload`, e.g. the 1M-token stress case).
+    per_head: the per-head selection variant (one index set per KV head,
+    block-diagonal compression maps) on the same inputs."""
     import torch
     import query_aware_selective_b200 as qas
     from query_aware_selective_b200 import cost, pipeline, synthetic
-    w = synthetic.DECODE_128K
+    w = workload or synthetic.DECODE_128K
     if args.decode_batch:
         import dataclasses
         w = dataclasses.replace(w, batch=args.decode_batch, name=f"esa_decode_llama3_8b_b{args.decode_batch}_ctx{w.n_ctx}")
@@ -504,17 +512,20 @@ def oracle_prefill_sample(w, inp_np, c0, rows):
     return t_sel + t_att, 1.0 / per_token
 
 
-def oracle_setup(device="cpu"):
+def oracle_setup(device="cpu", n_chunks=1):
+    """The prefill workload's inputs on the host for the oracle, with the compressed
+    cache filled up to c0 = 16384 (untimed) and the queries of n_chunks chunks from c0."""
     import numpy as np
     from oracle import esa as oesa
     from query_aware_selective_b200 import synthetic
     w = synthetic.PREFILL_32K
     inp = synthetic.make_esa_inputs(w, device=device)
     c0 = (w.n_ctx // 2 // w.chunk) * w.chunk                     # the middle chunk (c0 = 16384)
-    inp_np = {"q": inp["q"][:, c0:c0 + w.chunk].float().cpu().numpy(), "k": inp["k"].float().cpu().numpy(),
+    c1 = c0 + n_chunks * w.chunk
+    inp_np = {"q": inp["q"][:, c0:c1].float().cpu().numpy(), "k": inp["k"].float().cpu().numpy(),
               "v": inp["v"].float().cpu().numpy(), "wq": inp["wq"].cpu().numpy(), "wk": inp["wk"].cpu().numpy()}
-    # queries outside the sampled chunk are not needed: re-index so the chunk sits at c0
-    q_full = np.zeros((1, c0 + w.chunk) + inp_np["q"].shape[2:], dtype=np.float32)
+    # queries outside the sampled chunks are not needed: re-index so they sit at c0
+    q_full = np.zeros((1, c1) + inp_np["q"].shape[2:], dtype=np.float32)
     q_full[:, c0:] = inp_np["q"]
     inp_np["q"] = q_full
     inp_np["k_c"] = np.zeros((1, w.n_ctx, w.d_c))
@@ -531,14 +542,24 @@ def blas_threads():
         return os.cpu_count()
 
 
-def cpu_baseline_prefill(seconds_hint=10.0):
-    w, inp_np, c0 = oracle_setup()
+def cpu_baseline_prefill(seconds_hint=12.0, max_chunks=16):
+    """The oracle on consecutive chunks of the prefill from c0 = 16384 until about
+    seconds_hint of CPU work (at most max_chunks chunks)."""
+    w, inp_np, c0 = oracle_setup(n_chunks=max_chunks)
     rows = 16
-    secs, tps = oracle_prefill_sample(w, inp_np, c0, rows)
-    return {"value": round(tps, 3), "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"one 512-token chunk at c0={c0} of the 32768-token prefill: compress its keys and queries, "
-                      f"select over its {c0 - w.window - w.n_init}-token middle, attend {rows} of its query rows; "
-                      f"tok/s = 1 / (select time / 512 + attention time / {rows}); {secs:.1f} s of CPU work"}
+    secs, per_tok, n = 0.0, [], 0
+    while n < max_chunks and secs < seconds_hint:
+        s, tps = oracle_prefill_sample(w, inp_np, c0 + n * w.chunk, rows)
+        secs += s
+        per_tok.append(1.0 / tps)
+        n += 1
+    value = 1.0 / (sum(per_tok) / len(per_tok))
+    return {"value": round(value, 3), "unit": "tok/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} consecutive 512-token chunks of the 32768-token prefill from c0={c0}: per chunk, "
+                      f"compress its keys and queries, select over its middle "
+                      f"({c0 - w.window - w.n_init} tokens and up), attend {rows} of its query rows; "
+                      f"tok/s = 1 / mean over chunks of (select time / 512 + attention time / {rows}); "
+                      f"{secs:.1f} s of CPU work"}
 
 
 def run_reference(args):
