@@ -198,13 +198,15 @@ def dist_barrier():
         _dist.barrier()
 
 
-def make_dist_max():
+def make_dist_max(device="cuda"):
+    """x -> the max of x over the ranks (identity without a process group). The
+    reduction tensor lives on `device`: the rank's GPU under NCCL, the CPU under gloo."""
     import torch
     if _dist is None:
         return lambda x: x
 
     def f(x):
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        t = torch.tensor([x], dtype=torch.float64, device=device)
         _dist.all_reduce(t, op=_dist.ReduceOp.MAX)
         return float(t.item())
     return f
