@@ -169,3 +169,39 @@ def test_rejected_calls_launch_nothing(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError, match="not built"):
         _abi.load(str(tmp_path / "libesa.so"))
+
+
+def test_varlen_calls_reject_bad_arguments(lib):
+    p = _abi.params(128, 4096, 2048, 2, 45.25)
+    sel = lambda seq_len=FAKE, n_cap=131072, dc=128, ng=1, ws=FAKE, wsn=1 << 40: lib.esa_score_select_varlen(
+        FAKE, FAKE, 16, n_cap, seq_len, dc, ng, p, FAKE, FAKE, None, ws, wsn, None)
+    assert sel(seq_len=None) == _abi.ESA_ERR_INVALID_ARG
+    assert sel(n_cap=0) == _abi.ESA_ERR_INVALID_ARG
+    assert sel(ng=3) == _abi.ESA_ERR_UNSUPPORTED
+    assert sel(dc=96) == _abi.ESA_ERR_UNSUPPORTED            # no one-query scoring path for d_c 96
+    assert sel(wsn=16) == _abi.ESA_ERR_WORKSPACE
+    att = lambda seq_len=FAKE, lists=1, n_cap=131072: lib.esa_sparse_attn_varlen(
+        FAKE, FAKE, FAKE, 1, 16, n_cap, seq_len, 32, 8, 128, FAKE, FAKE, lists, p, 0.0, FAKE, None, FAKE, 1 << 40,
+        None)
+    assert att(seq_len=None) == _abi.ESA_ERR_INVALID_ARG
+    assert att(lists=3) == _abi.ESA_ERR_INVALID_ARG           # 1 or hkv lists
+    assert att(n_cap=0) == _abi.ESA_ERR_INVALID_ARG
+    cmp = lambda seq_len=FAKE, n_cap=131072, d_out=128: lib.esa_compress_packed_varlen(
+        FAKE, 16, 1024, 8, 128, FAKE, d_out, FAKE, n_cap, seq_len, None)
+    assert cmp(seq_len=None) == _abi.ESA_ERR_INVALID_ARG
+    assert cmp(n_cap=0) == _abi.ESA_ERR_INVALID_ARG
+    assert cmp(d_out=64) == _abi.ESA_ERR_UNSUPPORTED
+
+
+def test_varlen_workspaces_cover_the_longest_sequence(lib):
+    # sized for a query at n_cap - 1: the equal-length call's workspace at that position
+    p = _abi.params(128, 4096, 2048, 2, 45.25)
+    assert _abi.score_select_varlen_workspace_size(16, 131072, 128, 1, p) == \
+        _abi.score_select_workspace_size(16, 1, 131072, 131071, 128, p)
+    assert _abi.score_select_varlen_workspace_size(16, 131072, 128, 8, p) == \
+        _abi.score_select_heads_workspace_size(16, 1, 131072, 131071, 128, 8, p)
+    assert _abi.sparse_attn_varlen_workspace_size(16, 131072, 32, 8, 128, 1, 1, p) == \
+        _abi.sparse_attn_workspace_size(16, 1, 131071, 32, 8, 128, 1, p)
+    assert _abi.sparse_attn_varlen_workspace_size(16, 131072, 32, 8, 128, 1, 8, p) == \
+        _abi.sparse_attn_heads_workspace_size(16, 1, 131071, 32, 8, 128, 1, p)
+    assert _abi.score_select_varlen_workspace_size(16, 0, 128, 1, p) == 0
