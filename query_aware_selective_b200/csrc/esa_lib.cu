@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <mutex>
 #include <string>
+#include <type_traits>
 
 #include "../../include/esa.h"
 #include "attn_decode.cuh"
@@ -632,12 +633,16 @@ esa_status_t score_select_impl(const float* q_c, const float* k_c, int32_t batch
     const SelWs w = carve_select(workspace, (int32_t)vb, lq, r.n_mid, path);
     ESA_CUDA(cudaMemsetAsync(w.m_key, 0, (size_t)vb * lq * sizeof(uint32_t), s));
     if (path == ScorePath::Small) {
+      auto launch = [&](auto dc) {
+        launch_score_small<decltype(dc)::value>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key,
+                                                vl_score, s);
+      };
       switch (d_c) {
-        case 16: launch_score_small<16>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, vl_score, s); break;
-        case 32: launch_score_small<32>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, vl_score, s); break;
-        case 64: launch_score_small<64>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, vl_score, s); break;
-        case 128: launch_score_small<128>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, vl_score, s); break;
-        default: launch_score_small<256>(q_c, k_c, lq, n_cap, r.mid0, r.n_mid, batch, ng, w.S, w.m_key, vl_score, s); break;
+        case 16: launch(std::integral_constant<int, 16>{}); break;
+        case 32: launch(std::integral_constant<int, 32>{}); break;
+        case 64: launch(std::integral_constant<int, 64>{}); break;
+        case 128: launch(std::integral_constant<int, 128>{}); break;
+        default: launch(std::integral_constant<int, 256>{}); break;
       }
       ESA_LAUNCH_CHECK("score_small_kernel");
     } else if (path == ScorePath::Tiled) {
