@@ -17,6 +17,8 @@ can be checked against the pages by eye.
   ablation of merged versus per-head importance): one index set per KV head.
 * ``oracle.esa_varlen`` - ESA decode over a batch of sequences of different
   lengths: each sequence runs the one-sequence step at its own position.
+* ``oracle.esa_fit`` - the offline least-squares fit of ESA's two compression maps
+  from calibration queries and keys.
 * ``oracle.moba`` - Mixture of Block Attention (MoBA article, sections 1-3):
   block mean pooling, gate, causal top-k, block attention.
 

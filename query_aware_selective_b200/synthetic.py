@@ -227,6 +227,24 @@ def make_moba_decode_inputs(w: MobaWorkload, device="cpu", seq: Optional[int] = 
     return dict(q=q, k=k, v=v)
 
 
+def make_calibration(hq: int, hkv: int, d: int, n_tokens: int, rank: int, seed: int, noise: float = 0.1) -> tuple:
+    """Calibration queries and keys for the offline fit of the compression maps (they
+    stand in for the model's own queries and keys on a calibration text, which are not
+    available here). Each token's query is a rank-`rank` latent times fixed loadings
+    plus N(0, noise^2) noise, and so is each key, with their own latents and loadings:
+    the merged scores then have a dominant low-rank part, as attention scores do.
+    Returns (q [n, hq, d], k [n, hkv, d]) float32 on the host."""
+    gen = torch.Generator()
+    gen.manual_seed(seed)
+    a_q = torch.randn((rank, hq * d), generator=gen) / math.sqrt(rank)
+    a_k = torch.randn((rank, hkv * d), generator=gen) / math.sqrt(rank)
+    z_q = torch.randn((n_tokens, rank), generator=gen)
+    z_k = torch.randn((n_tokens, rank), generator=gen)
+    q = z_q @ a_q + noise * torch.randn((n_tokens, hq * d), generator=gen)
+    k = z_k @ a_k + noise * torch.randn((n_tokens, hkv * d), generator=gen)
+    return q.reshape(n_tokens, hq, d), k.reshape(n_tokens, hkv, d)
+
+
 def varlen_lengths(batch: int, n_max: int, n_min: int, seed: int) -> torch.Tensor:
     """Lengths of a variable-length decode batch: sequence 0 holds n_max tokens, the
     others a seeded uniform draw from [n_min, n_max]. Returns int64 [batch] (host)."""

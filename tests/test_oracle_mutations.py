@@ -10,8 +10,9 @@ import textwrap
 
 import pytest
 
-from oracle import esa, esa_heads, esa_varlen, moba
+from oracle import esa, esa_fit, esa_heads, esa_varlen, moba
 from tests import test_oracle_esa as pe
+from tests import test_oracle_fit as tf
 from tests import test_oracle_heads as th
 from tests import test_oracle_moba as pm
 from tests import test_oracle_varlen as tv
@@ -72,6 +73,16 @@ MUTATIONS = [
      tv.check_short_sequences_attend_everything),                          # attention stops one row short
     (esa_varlen, "sparse_attn_varlen", "if lists == 1:", "if True:",
      tv.check_per_head_lists_per_sequence),                                # first list for every head
+    (esa_fit, "expansion", "kv = h // g", "kv = h % hkv",
+     tf.check_full_rank_fit_is_exact),                                     # GQA order in the fit
+    (esa_fit, "fit_maps", "w_k = e @ b / g", "w_k = e @ b",
+     tf.check_full_rank_fit_is_exact),                                     # expanded key map not divided
+    (esa_fit, "fit_maps", "u[:, :d_c] * root", "u[:, -d_c:] * root",
+     tf.check_matches_alternating_least_squares),                          # trailing singular vectors
+    (esa_fit, "_upper_cholesky", "return np.linalg.cholesky(gram).T", "return np.linalg.cholesky(gram)",
+     tf.check_matches_alternating_least_squares),                          # lower factor for the upper one
+    (esa_fit, "scores_full", "np.repeat(k, g, axis=1)", "np.tile(k, (1, g, 1))",
+     tf.check_full_rank_fit_is_exact),                                     # target scores with the wrong heads
 ]
 
 
