@@ -19,6 +19,8 @@ can be checked against the pages by eye.
   lengths: each sequence runs the one-sequence step at its own position.
 * ``oracle.esa_fit`` - the offline least-squares fit of ESA's two compression maps
   from calibration queries and keys.
+* ``oracle.cca`` - CCA-style attention: core tokens pooled per group of g tokens by
+  the group's last query, plus a group-aligned local window, in one softmax.
 * ``oracle.moba`` - Mixture of Block Attention (MoBA article, sections 1-3):
   block mean pooling, gate, causal top-k, block attention.
 

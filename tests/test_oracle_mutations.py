@@ -10,7 +10,8 @@ import textwrap
 
 import pytest
 
-from oracle import esa, esa_fit, esa_heads, esa_varlen, moba
+from oracle import cca, esa, esa_fit, esa_heads, esa_varlen, moba
+from tests import test_oracle_cca as tc
 from tests import test_oracle_esa as pe
 from tests import test_oracle_fit as tf
 from tests import test_oracle_heads as th
@@ -83,6 +84,16 @@ MUTATIONS = [
      tf.check_matches_alternating_least_squares),                          # lower factor for the upper one
     (esa_fit, "scores_full", "np.repeat(k, g, axis=1)", "np.tile(k, (1, g, 1))",
      tf.check_full_rank_fit_is_exact),                                     # target scores with the wrong heads
+    (cca, "window_start", "return max(0, g * (i // g) - w)", "return max(0, i - w)",
+     tc.check_counts_and_tiling),                                          # window not on a group boundary
+    (cca, "attend", "n_core = lo // g", "n_core = lo // g + 1",
+     tc.check_counts_and_tiling),                                          # core of the window's first group too
+    (cca, "core_tokens", "x = scale * (k[b, t0:t1, kv] @ q[b, t1 - 1, h])",
+     "x = scale * (k[b, t0:t1, kv] @ q[b, t0, h])", tc.check_dominant_key_is_the_core_token),  # first query pools
+    (cca, "attend", "kv = h // gq", "kv = h % hkv",
+     tc.check_groups_of_one_are_full_attention),                           # GQA order
+    (cca, "attend", "x = scale * (keys @ q[b, i, h])", "x = keys @ q[b, i, h]",
+     tc.check_window_over_everything_is_full_attention),                   # missing scale
 ]
 
 
