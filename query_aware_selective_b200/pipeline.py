@@ -53,6 +53,16 @@ def _region_lo(c0: int, n_init: int, window: int) -> int:
     return min(c0, max(n_init, c0 - window))
 
 
+def key_batch_needed(c0: int, chunk: int, n_init: int, window: int, kbatch: int) -> int:
+    """The last batch of kbatch consecutive chunks whose compressed keys the selection of
+    the chunk starting at c0 reads (its middle is [n_init, lo), lo <= c0), or -1 when
+    its middle is empty."""
+    lo = _region_lo(c0, n_init, window)
+    if lo <= n_init:
+        return -1
+    return ((lo - 1) // chunk) // kbatch
+
+
 def block_diagonal(w_groups: torch.Tensor) -> torch.Tensor:
     """Per-head selection: the groups' maps [G, gin, d_g] stacked into the one
     [G * gin, G * d_g] map the compression calls take (zero off the diagonal
@@ -234,11 +244,10 @@ class EsaPrefill:
                 issued += 1
 
         for ci, (c0, lq) in enumerate(chunks):
-            lo = _region_lo(c0, self.p.n_init, self.p.window)
-            needed = (lo - 1) // self.chunk if lo > self.p.n_init else -1   # last chunk the middle reads
+            needed = key_batch_needed(c0, self.chunk, self.p.n_init, self.p.window, kbatch)
             wait = None
             if needed >= 0:
-                issue_batches(needed // kbatch)
+                issue_batches(needed)
                 wait = last_done
             done = torch.cuda.Event()
             with torch.cuda.stream(self.side):
