@@ -52,6 +52,17 @@ def test_decode_1m_batch4():
     _decode_full(synthetic.DECODE_1M, seqs=(0,))
 
 
+def test_decode_varlen_128k_batch16():
+    # the variable-length decode workload bench.py times (the 128K inputs, the same
+    # seeded length mix); the longest and the shortest sequence against the oracle
+    from tests.test_gpu_varlen import _decode
+    w = synthetic.DECODE_128K
+    lens = synthetic.varlen_lengths(w.batch, w.n_ctx, 8192, seed=w.seed + 2000).tolist()
+    shortest = min(range(len(lens)), key=lambda i: lens[i])
+    _decode(False, w.n_ctx, lens, seqs=(0, shortest))
+    torch.cuda.empty_cache()
+
+
 def test_prefill_32k_sampled_chunks():
     w = synthetic.PREFILL_32K
     p = qas.params(w.n_init, w.window, w.topk, w.eps, w.clamp_c)
