@@ -52,6 +52,13 @@ def test_decode_1m_batch4():
     _decode_full(synthetic.DECODE_1M, seqs=(0,))
 
 
+def test_decode_per_head_128k_batch16():
+    # the per-head selection variant on the decode workload bench.py times
+    from tests.test_gpu_heads import _decode_heads
+    _decode_heads(synthetic.DECODE_128K, None, synthetic.DECODE_128K.batch, seqs=(0, 15))
+    torch.cuda.empty_cache()
+
+
 def test_decode_varlen_128k_batch16():
     # the variable-length decode workload bench.py times (the 128K inputs, the same
     # seeded length mix); the longest and the shortest sequence against the oracle
