@@ -168,6 +168,7 @@ def test_score_select_ties_follow_position_order():
 
 @pytest.mark.parametrize("topk,c0,window", [
     (500, 520, 8),     # |mid| = 504 > topk by 4
+    (503, 520, 8),     # |mid| = topk + 1: one position dropped
     (504, 520, 8),     # |mid| == topk: everything
     (600, 520, 8),     # |mid| < topk: everything, -1 padding
     (10, 300, 292),    # empty middle
