@@ -132,3 +132,39 @@ def moba_decode_bytes(batch: int, n_ctx: int, heads: int, d: int, block: int, to
     keys = min(topk, cur) * block + (n_ctx - cur * block)
     rows = batch * heads * keys * d * kv_bytes * 2
     return dict(block_means=means, kv_rows=rows, total=means + rows)
+
+
+# ----------------------------------------------------------------------------- CCA-style attention
+
+def cca_keys(i: int, g: int, w: int) -> int:
+    """Keys query i attends: the core tokens of the groups that end before its window
+    [max(0, g * (i // g) - w), i], then the window's tokens."""
+    lo = max(0, g * (i // g) - w)
+    return lo // g + (i - lo + 1)
+
+
+def cca_flops(seq: int, hq: int, d: int, g: int, w: int) -> dict:
+    """Causal prefill of one layer: pooling (per complete group and query head: the
+    last query's g scores and the weighted sums of g keys and g values) and the fused
+    attention (4 * D flops per (query, head, attended key))."""
+    keys = sum(cca_keys(i, g, w) for i in range(seq))
+    att = 4 * d * hq * keys
+    pool = (seq // g) * hq * g * 6 * d
+    return dict(attention=att, pooling=pool, total=att + pool)
+
+
+# ----------------------------------------------------------------------------- offline fit
+
+def fit_flops(n_q: int, n_k: int, hq: int, hkv: int, d: int, d_c: int) -> dict:
+    """The least-squares fit of the two maps: the Gram matrices of the calibration
+    queries (n_q x Hq*D) and keys (n_k x Hkv*D), their Cholesky factorisations, the
+    coupled matrix Rq E Rk^T and its leading d' singular triples (counted as one dense
+    SVD of that matrix), and the two triangular solves."""
+    dq, dk = hq * d, hkv * d
+    gram = 2 * n_q * dq * dq + 2 * n_k * dk * dk
+    chol = (dq ** 3 + dk ** 3) // 3
+    couple = 2 * dq * dk * dk
+    svd = 4 * dq * dk * dk + 8 * dk ** 3
+    solve = dq * dq * d_c + dk * dk * d_c
+    return dict(gram=gram, cholesky=chol, couple=couple, svd=svd, solve=solve,
+                total=gram + chol + couple + svd + solve)

@@ -56,3 +56,29 @@ def test_varlen_bytes_reduce_to_the_equal_length_batch():
     d = cost.decode_bytes(1, 131072, 32, 8, 128, 128, 128, 4096, 2048)
     assert c["compressed_keys"] == d["compressed_keys"]
     assert c["kv_rows"] == d["kv_rows"] + 100 * 8 * 128 * 2 * 2
+
+
+def test_cca_keys_match_the_oracle():
+    # zero keys make every attended key equally likely: the oracle's lse is log(#keys)
+    import math
+    import numpy as np
+    from oracle import cca
+    s, g, w = 45, 5, 10
+    q = np.random.default_rng(0).standard_normal((1, s, 2, 4))
+    k = np.zeros((1, s, 1, 4))
+    v = np.zeros((1, s, 1, 4))
+    _, lse = cca.attend(q, k, v, g, w)
+    for i in range(s):
+        assert cost.cca_keys(i, g, w) == round(math.exp(lse[0, i, 0]))
+
+
+def test_cca_flops_reduce_to_full_attention():
+    # groups of one token or a window over everything: every earlier token once
+    assert cost.cca_flops(300, 32, 128, 1, 7)["attention"] == cost.full_causal_attn_flops(300, 32, 128)
+    assert cost.cca_flops(300, 32, 128, 4, 400)["attention"] == cost.full_causal_attn_flops(300, 32, 128)
+
+
+def test_fit_flops_gram_dominates_for_long_calibration():
+    f = cost.fit_flops(65536, 65536, 32, 8, 128, 128)
+    assert f["gram"] == 2 * 65536 * 4096 ** 2 + 2 * 65536 * 1024 ** 2
+    assert f["gram"] > 0.5 * f["total"]
