@@ -400,6 +400,13 @@ const char* esa_last_error(void);
  * ESA_ERR_INVALID_ARG if a variable-length call read a length outside [1, n_cap]. */
 esa_status_t esa_device_status(void* stream);
 
+/* esa_wait_selftest - runs the bounded-wait path on demand: one CTA waits on a barrier
+ * that nothing arrives at; after limit_ns (1 us .. 2 s) the wait gives up, records
+ * ESA_ERR_TIMEOUT at site 9901 in the device status word and the kernel returns, with
+ * no fault and no hang. The next esa_device_status() reports it. ESA_ERR_INVALID_ARG for
+ * a limit out of range. For tests of the failure path. */
+esa_status_t esa_wait_selftest(uint64_t limit_ns, void* stream);
+
 /* Number of kernels this library has launched in this process, all devices and
  * threads together (accounting only). */
 uint64_t esa_launch_count(void);

@@ -66,6 +66,7 @@ SIGNATURES = {
     "esa_sparse_attn_heads": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i64, _i64, _i32, _i32,
                                              _i32, _vp, _vp, EsaParams, _f32, _vp, _vp, _vp, _sz, _vp]),
     "esa_sparse_attn_heads_workspace_size": (_sz, [_i32, _i32, _i64, _i32, _i32, _i32, ctypes.c_int, EsaParams]),
+    "esa_wait_selftest": (ctypes.c_int, [ctypes.c_uint64, _vp]),
     "cca_attn": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i64, _i32, _i32, _i32, _i32, _i32, _f32, _vp,
                                 _vp, _vp, _sz, _vp]),
     "cca_workspace_size": (_sz, [_i32, _i64, _i32, _i32, _i32]),
@@ -553,6 +554,12 @@ def moba_block_gate_attn(q, k, v, block: int, topk: int, scale: float = 0.0, wan
 def launch_count() -> int:
     """Kernels libesa has launched in this process."""
     return int(load().esa_launch_count())
+
+
+def wait_selftest(limit_ns: int) -> None:
+    """esa_wait_selftest: a kernel whose bounded wait runs out after limit_ns and
+    records a timeout (read back by device_status)."""
+    _check(load().esa_wait_selftest(int(limit_ns), _stream()), "esa_wait_selftest")
 
 
 def device_status() -> None:

@@ -297,6 +297,14 @@ const char* esa_last_error(void) { return g_err.c_str(); }
 
 uint64_t esa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+esa_status_t esa_wait_selftest(uint64_t limit_ns, void* stream) {
+  if (limit_ns < 1000 || limit_ns > ESA_WAIT_LIMIT_NS)
+    return fail(ESA_ERR_INVALID_ARG, "limit_ns must be in [1 us, %llu ns]", (unsigned long long)ESA_WAIT_LIMIT_NS);
+  esa::wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns);
+  ESA_LAUNCH_CHECK("wait_selftest_kernel");
+  return ok();
+}
+
 esa_status_t esa_device_status(void* stream) {
   ESA_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
   unsigned long long v = 0;

@@ -222,3 +222,8 @@ def test_cca_rejects_bad_arguments(lib):
     assert f(FAKE, FAKE, FAKE, 1, 1, 65536, 32, 8, 128, 128, 1024, 0.0, FAKE, None, FAKE, 16, None) == \
         _abi.ESA_ERR_WORKSPACE
     assert _abi.cca_workspace_size(1, 65536, 32, 128, 128) > _abi.cca_workspace_size(1, 65536, 32, 128, 256) > 0
+
+
+def test_wait_selftest_rejects_out_of_range_limits(lib):
+    assert lib.esa_wait_selftest(10, None) == _abi.ESA_ERR_INVALID_ARG
+    assert lib.esa_wait_selftest(10 ** 12, None) == _abi.ESA_ERR_INVALID_ARG
