@@ -49,7 +49,7 @@ def parse_args():
     ap.add_argument("--prefill-ctx", type=int, default=0,
                     help="shorter prefill context (profiling a small case); the line then names that workload")
     ap.add_argument("--only", choices=["decode", "decode_per_head", "decode_varlen", "decode_1m", "moba",
-                                       "moba_decode"],
+                                       "moba_decode", "cca"],
                     default=None,
                     help="profiling: run one of the other workloads alone and print its figures")
     ap.add_argument("--decode-batch", type=int, default=0, help="profiling: decode batch (default: the workload's)")
@@ -228,6 +228,8 @@ def run_only(args):
         out = bench_moba(args, dev, flush, make_dist_max(), peaks, peak_src, 1)
     elif args.only == "moba_decode":
         out = bench_moba_decode(args, dev, flush, make_dist_max(), peaks, peak_src, 1)
+    elif args.only == "cca":
+        out = bench_cca(args, dev, flush, make_dist_max(), peaks, peak_src, 1)
     elif args.only == "decode_varlen":
         out = bench_decode_varlen(args, dev, flush, make_dist_max(), peaks, peak_src, 1)
     elif args.only == "decode_1m":
@@ -356,6 +358,8 @@ def run_ours(args):
         line["also"]["moba_prefill_64k"] = bench_moba(args, dev, flush, dist_max, peaks, peak_src, world)
         torch.cuda.empty_cache()
         line["also"]["moba_decode_64k"] = bench_moba_decode(args, dev, flush, dist_max, peaks, peak_src, world)
+        torch.cuda.empty_cache()
+        line["also"]["cca_prefill_64k"] = bench_cca(args, dev, flush, dist_max, peaks, peak_src, world)
     line["clocks"] = sampler.stop()
     line["gpu"] = props.name
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -440,6 +444,31 @@ def bench_decode_varlen(args, dev, flush, dist_max, peaks, peak_src, world):
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4), "bytes_per_step": by["total"],
                          "peak_source": f"{peak_src} HBM copy"}}
+
+
+def bench_cca(args, dev, flush, dist_max, peaks, peak_src, world):
+    """CCA-style causal prefill: 65536 tokens, 32 / 8 heads, groups of 128, window 1024."""
+    import torch
+    import query_aware_selective_b200 as qas
+    from query_aware_selective_b200 import cost, pipeline, synthetic
+    w = synthetic.CCA_64K
+    inp = synthetic.make_cca_inputs(w, device=dev)
+    out = torch.empty_like(inp["q"])
+    ws = torch.empty(qas._abi.cca_workspace_size(w.batch, w.seq, w.hq, w.head_dim, w.group) + 256,
+                     dtype=torch.uint8, device=dev)
+    graph = pipeline.graph_of(lambda: qas.cca_attn(inp["q"], inp["k"], inp["v"], w.group, w.window, out=out,
+                                                   workspace=ws))
+    steps = max(3, args.steps // 2)
+    ms, total = time_steps(graph.replay, steps, args.warmup, flush, dist_max)
+    fl = cost.cca_flops(w.seq, w.hq, w.head_dim, w.group, w.window)
+    ach = fl["total"] * w.batch / (total / steps / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    return {"workload": w.name, "value": round(world * w.batch * w.seq * steps / (total / 1e3), 1),
+            "unit": "tok/s", "ms_per_step": round(total / steps, 3), "steps": steps,
+            "execution": "one CUDA graph per step",
+            "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(ach / peak, 4), "flops_per_step": fl["total"] * w.batch,
+                         "peak_source": f"{peak_src} bf16 sustained"}}
 
 
 def bench_moba_decode(args, dev, flush, dist_max, peaks, peak_src, world):

@@ -312,6 +312,27 @@ esa_status_t moba_decode_attn(const void* q, const void* k, const void* v, esa_d
 size_t moba_decode_workspace_size(int32_t batch, int64_t n_cap, int64_t pos, int32_t heads, int32_t head_dim,
                                   int32_t block, int32_t topk);
 
+/* ------------------------------------------------------- CCA-style attention -- */
+
+/* cca_attn - causal prefill of one layer with CCA-style attention (CCA-Attention
+ * article: global-aware pooling, locality-preserving module, and their fusion). The
+ * sequence is cut into groups of `group` tokens; a complete group's core key and value
+ * are its keys and values weighted by the softmax (scale as below) of the group's last
+ * query against the group's keys, per query head. Query i attends, in one softmax, the
+ * core tokens of the groups that end before its window and the window's tokens
+ * [max(0, group * floor(i / group) - window), i].
+ *   q: [batch, seq, hq, head_dim]; k, v: [batch, seq, hkv, head_dim]; o like q;
+ *   lse: NULL or [batch, seq, hq] fp32 (natural log).
+ *   scale: softmax scale; <= 0 means 1/sqrt(head_dim).
+ * Requires bf16, head_dim 128, hq / hkv in {1, 2, 4, 8}, group a multiple of 128,
+ * window a multiple of group. Workspace: cca_workspace_size bytes, 256-byte aligned
+ * (core keys and values bf16, the core pass's bf16 partials and fp32 LSE). Errors as
+ * for esa_sparse_attn. */
+esa_status_t cca_attn(const void* q, const void* k, const void* v, esa_dtype_t dt, int32_t batch, int64_t seq,
+                      int32_t hq, int32_t hkv, int32_t head_dim, int32_t group, int32_t window, float scale,
+                      void* o, float* lse, void* workspace, size_t ws_bytes, void* stream);
+size_t cca_workspace_size(int32_t batch, int64_t seq, int32_t hq, int32_t head_dim, int32_t group);
+
 /* ----------------------------------------------- variable-length decode batches -- */
 
 /* A decode batch whose sequences hold different numbers of cached tokens (ESA write-up,
@@ -378,6 +399,13 @@ const char* esa_last_error(void);
  * stopped early on a launch-environment check (e.g. misaligned shared memory), or
  * ESA_ERR_INVALID_ARG if a variable-length call read a length outside [1, n_cap]. */
 esa_status_t esa_device_status(void* stream);
+
+/* esa_wait_selftest - runs the bounded-wait path on demand: one CTA waits on a barrier
+ * that nothing arrives at; after limit_ns (1 us .. 2 s) the wait gives up, records
+ * ESA_ERR_TIMEOUT at site 9901 in the device status word and the kernel returns, with
+ * no fault and no hang. The next esa_device_status() reports it. ESA_ERR_INVALID_ARG for
+ * a limit out of range. For tests of the failure path. */
+esa_status_t esa_wait_selftest(uint64_t limit_ns, void* stream);
 
 /* Number of kernels this library has launched in this process, all devices and
  * threads together (accounting only). */

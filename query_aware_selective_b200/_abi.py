@@ -66,6 +66,10 @@ SIGNATURES = {
     "esa_sparse_attn_heads": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i64, _i64, _i32, _i32,
                                              _i32, _vp, _vp, EsaParams, _f32, _vp, _vp, _vp, _sz, _vp]),
     "esa_sparse_attn_heads_workspace_size": (_sz, [_i32, _i32, _i64, _i32, _i32, _i32, ctypes.c_int, EsaParams]),
+    "esa_wait_selftest": (ctypes.c_int, [ctypes.c_uint64, _vp]),
+    "cca_attn": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i64, _i32, _i32, _i32, _i32, _i32, _f32, _vp,
+                                _vp, _vp, _sz, _vp]),
+    "cca_workspace_size": (_sz, [_i32, _i64, _i32, _i32, _i32]),
     "esa_compress_packed_varlen": (ctypes.c_int, [_vp, _i32, _i64, _i32, _i32, _vp, _i32, _vp, _i64, _vp, _vp]),
     "esa_score_select_varlen": (ctypes.c_int, [_vp, _vp, _i32, _i64, _vp, _i32, _i32, EsaParams, _vp, _vp, _vp,
                                                _vp, _sz, _vp]),
@@ -428,6 +432,29 @@ def sparse_attn_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_le
     return out, (lse if want_lse else None)
 
 
+def cca_workspace_size(batch, seq, hq, d, group) -> int:
+    return load().cca_workspace_size(batch, seq, hq, d, group)
+
+
+def cca_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, group: int, window: int, scale: float = 0.0,
+             want_lse: bool = False, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+             workspace: Optional[torch.Tensor] = None):
+    """cca_attn: CCA-style causal attention. q [B, S, Hq, D], k, v [B, S, Hkv, D] bf16.
+    Returns (o [B, S, Hq, D], lse [B, S, Hq] f32 or None)."""
+    _dev(q, k, v)
+    b, s, hq, d = q.shape
+    hkv = k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((b, s, hq), dtype=torch.float32, device=q.device)
+    ws = _workspace(cca_workspace_size(b, s, hq, d, group), q.device, workspace)
+    wp, wn = _ws_ptr(ws)
+    _check(load().cca_attn(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), b, s, hq, hkv, d, group, window, scale,
+                           _ptr(out), _ptr(lse) if want_lse else None, wp, wn, _stream()), "cca_attn")
+    return out, (lse if want_lse else None)
+
+
 def moba_block_means(k: torch.Tensor, block: int, blk_begin: int = 0, blk_end: Optional[int] = None,
                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """moba_block_means: means of blocks [blk_begin, blk_end) of k [B, n_cap, H, D] bf16
@@ -527,6 +554,12 @@ def moba_block_gate_attn(q, k, v, block: int, topk: int, scale: float = 0.0, wan
 def launch_count() -> int:
     """Kernels libesa has launched in this process."""
     return int(load().esa_launch_count())
+
+
+def wait_selftest(limit_ns: int) -> None:
+    """esa_wait_selftest: a kernel whose bounded wait runs out after limit_ns and
+    records a timeout (read back by device_status)."""
+    _check(load().esa_wait_selftest(int(limit_ns), _stream()), "esa_wait_selftest")
 
 
 def device_status() -> None:

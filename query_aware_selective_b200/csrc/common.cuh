@@ -196,18 +196,34 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // With respect_abort = false the wait keeps going after an abort (used to drain work
 // already in flight before releasing resources), still bounded by the time limit.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned site, bool respect_abort = true) {
+                                          unsigned site, bool respect_abort = true,
+                                          uint64_t limit_ns = ESA_WAIT_LIMIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
     if (respect_abort && *abort_flag) return false;
-    if (globaltimer_ns() - t0 > ESA_WAIT_LIMIT_NS) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       record_status(4u, site);
       return false;
     }
   }
+}
+
+// The bounded-wait path on demand: one thread waits on a barrier that nothing ever
+// arrives at, with a limit of limit_ns; the wait runs out, records a timeout at site
+// 9901 and the kernel returns (no fault, no hang). Launched with one CTA of 32 threads.
+__global__ void wait_selftest_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, 9901, true, limit_ns);
 }
 
 // Warp-uniform version: every lane of the warp gets the same answer, so that the

@@ -18,6 +18,7 @@
 #include "attn_decode.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
+#include "cca.cuh"
 #include "common.cuh"
 #include "compress.cuh"
 #include "compress_tc.cuh"
@@ -295,6 +296,14 @@ const char* esa_version(void) { return "libesa 0.1 (sm_100a)"; }
 const char* esa_last_error(void) { return g_err.c_str(); }
 
 uint64_t esa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+esa_status_t esa_wait_selftest(uint64_t limit_ns, void* stream) {
+  if (limit_ns < 1000 || limit_ns > ESA_WAIT_LIMIT_NS)
+    return fail(ESA_ERR_INVALID_ARG, "limit_ns must be in [1 us, %llu ns]", (unsigned long long)ESA_WAIT_LIMIT_NS);
+  esa::wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns);
+  ESA_LAUNCH_CHECK("wait_selftest_kernel");
+  return ok();
+}
 
 esa_status_t esa_device_status(void* stream) {
   ESA_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
@@ -1278,6 +1287,135 @@ esa_status_t moba_block_gate_attn(const void* q, const void* k, const void* v, e
   if (st != ESA_OK) return st;
   st = moba_attn_launch(w, q, k, v, batch, seq, heads, block, topk, blocks, scale, o, lse, s);
   return st == ESA_OK ? ok() : st;
+}
+
+// ------------------------------------------------------------------ CCA-style attention --
+namespace {
+
+struct CcaWs {
+  __nv_bfloat16* kc;        // [B, m, Hq, D] core keys
+  __nv_bfloat16* vc;        // [B, m, Hq, D] core values
+  __nv_bfloat16* part_o;    // [B, S, Hq, D] core-pass partials
+  float* part_lse;          // [B, S, Hq]
+  size_t bytes;
+};
+
+CcaWs carve_cca(void* ws, int32_t batch, int64_t seq, int32_t hq, int32_t head_dim, int32_t group) {
+  Carver c{reinterpret_cast<uint8_t*>(ws)};
+  CcaWs w{};
+  const int64_t m = seq / group;
+  w.kc = c.take<__nv_bfloat16>((size_t)std::max<int64_t>(1, batch * m * hq) * head_dim);
+  w.vc = c.take<__nv_bfloat16>((size_t)std::max<int64_t>(1, batch * m * hq) * head_dim);
+  w.part_o = c.take<__nv_bfloat16>((size_t)batch * seq * hq * head_dim);
+  w.part_lse = c.take<float>((size_t)batch * seq * hq);
+  w.bytes = c.off;
+  return w;
+}
+
+esa_status_t cca_check(const void* q, const void* k, const void* v, const void* o, esa_dtype_t dt, int32_t batch,
+                       int64_t seq, int32_t hq, int32_t hkv, int32_t head_dim, int32_t group, int32_t window) {
+  if (dt != ESA_BF16) return fail(ESA_ERR_UNSUPPORTED, "CCA attention takes bf16 tensors");
+  if (batch <= 0 || seq <= 0) return fail(ESA_ERR_INVALID_ARG, "batch and seq must be >= 1");
+  if (hq <= 0 || hkv <= 0 || hq % hkv) return fail(ESA_ERR_INVALID_ARG, "hq must be a positive multiple of hkv");
+  const int g = hq / hkv;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return fail(ESA_ERR_UNSUPPORTED, "GQA group %d (1, 2, 4 or 8)", g);
+  if (head_dim != 128) return fail(ESA_ERR_UNSUPPORTED, "head_dim %d (128)", head_dim);
+  if (group < 128 || group % 128) return fail(ESA_ERR_UNSUPPORTED, "group %d (a multiple of 128)", group);
+  if (window < 0 || window % group) return fail(ESA_ERR_INVALID_ARG, "window must be a multiple of the group (>= 0)");
+  if ((int64_t)batch * seq * hq >= ((int64_t)1 << 31)) return fail(ESA_ERR_UNSUPPORTED, "more than 2^31 query rows");
+  if (!q || !k || !v || !o) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16))
+    return fail(ESA_ERR_INVALID_ARG, "q, k, v, o need 16-byte alignment");
+  return ESA_OK;
+}
+
+template <int G>
+void launch_cca_pool(const void* q, const void* k, const void* v, int32_t batch, int64_t seq, int32_t hkv,
+                     int32_t group, float sl2, const CcaWs& w, cudaStream_t s) {
+  const int64_t m = seq / group;
+  const int64_t items = (int64_t)batch * m * hkv;
+  esa::cca_pool_kernel<G><<<(unsigned)cdiv(items, esa::kCcaPoolWarps), esa::kCcaPoolWarps * 32, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+      static_cast<const __nv_bfloat16*>(v), batch, seq, hkv, group, m, sl2, w.kc, w.vc);
+}
+
+}  // namespace
+
+size_t cca_workspace_size(int32_t batch, int64_t seq, int32_t hq, int32_t head_dim, int32_t group) {
+  if (batch <= 0 || seq <= 0 || hq <= 0 || head_dim <= 0 || group <= 0) return 0;
+  return carve_cca(nullptr, batch, seq, hq, head_dim, group).bytes;
+}
+
+esa_status_t cca_attn(const void* q, const void* k, const void* v, esa_dtype_t dt, int32_t batch, int64_t seq,
+                      int32_t hq, int32_t hkv, int32_t head_dim, int32_t group, int32_t window, float scale, void* o,
+                      float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  esa_status_t st = cca_check(q, k, v, o, dt, batch, seq, hq, hkv, head_dim, group, window);
+  if (st != ESA_OK) return st;
+  const size_t need = carve_cca(nullptr, batch, seq, hq, head_dim, group).bytes;
+  if (!workspace || ws_bytes < need || !aligned(workspace, 256))
+    return fail(ESA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need, ws_bytes);
+  const CcaWs w = carve_cca(workspace, batch, seq, hq, head_dim, group);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (scale <= 0.f) scale = 1.f / std::sqrt((float)head_dim);
+  const float sl2 = scale * 1.4426950408889634f;
+  const int g = hq / hkv;
+  const int64_t m = seq / group;
+  if (m > 0) {
+    if (g == 1) launch_cca_pool<1>(q, k, v, batch, seq, hkv, group, sl2, w, s);
+    else if (g == 2) launch_cca_pool<2>(q, k, v, batch, seq, hkv, group, sl2, w, s);
+    else if (g == 4) launch_cca_pool<4>(q, k, v, batch, seq, hkv, group, sl2, w, s);
+    else launch_cca_pool<8>(q, k, v, batch, seq, hkv, group, sl2, w, s);
+    ESA_LAUNCH_CHECK("cca_pool_kernel");
+  }
+  static bool attr_set[64] = {};
+  int dev = 0;
+  ESA_CUDA(cudaGetDevice(&dev));
+  if (dev < 64 && !attr_set[dev]) {
+    if ((st = set_max_smem(esa::attn_tc_kernel<esa::CcaCoreProblem>, esa::kTcSmemBytes)) != ESA_OK) return st;
+    if ((st = set_max_smem(esa::attn_tc_kernel<esa::CcaWindowProblem>, esa::kTcSmemBytes)) != ESA_OK) return st;
+    attr_set[dev] = true;
+  }
+  CUtensorMap tq, tk, tv, bq, bk, bv, sk, sv;
+  const uint64_t rows_q = (uint64_t)batch * seq * hq, rows_kv = (uint64_t)batch * seq * hkv;
+  if ((st = make_tmap_rows_bf16(&tq, q, rows_q)) != ESA_OK) return st;
+  if ((st = make_tmap_rows_bf16(&tk, k, rows_kv)) != ESA_OK) return st;
+  if ((st = make_tmap_rows_bf16(&tv, v, rows_kv)) != ESA_OK) return st;
+  if ((st = make_tmap_box_bf16(&bq, q, hq, (uint64_t)batch * seq, 1, esa::kTcRows)) != ESA_OK) return st;
+  if ((st = make_tmap_box_bf16(&bk, k, hkv, (uint64_t)batch * seq, 1, esa::kTcKeys)) != ESA_OK) return st;
+  if ((st = make_tmap_box_bf16(&bv, v, hkv, (uint64_t)batch * seq, 1, esa::kTcKeys)) != ESA_OK) return st;
+  const uint64_t core_tokens = (uint64_t)std::max<int64_t>(1, (int64_t)batch * m);
+  if ((st = make_tmap_box_bf16(&sk, w.kc, hq, core_tokens, 1, esa::kTcKeys)) != ESA_OK) return st;
+  if ((st = make_tmap_box_bf16(&sv, w.vc, hq, core_tokens, 1, esa::kTcKeys)) != ESA_OK) return st;
+  const dim3 grid((unsigned)cdiv(seq, esa::kTcRows), (unsigned)hq, (unsigned)batch);
+  auto tile = [&](esa::CcaTile& t) {
+    t.seq = seq;
+    t.m = m;
+    t.hq = hq;
+    t.hkv = hkv;
+    t.G = g;
+    t.group = group;
+    t.window = window;
+    t.sl2 = sl2;
+  };
+  if (m > 0) {
+    esa::CcaCoreProblem cp{};
+    tile(cp);
+    cp.part_o = w.part_o;
+    cp.part_lse = w.part_lse;
+    esa::attn_tc_kernel<esa::CcaCoreProblem><<<grid, esa::kTcThreads, esa::kTcSmemBytes, s>>>(tq, tk, tv, bq, bk, bv,
+                                                                                           sk, sv, cp);
+    ESA_LAUNCH_CHECK("attn_tc_kernel<cca core>");
+  }
+  esa::CcaWindowProblem wp{};
+  tile(wp);
+  wp.part_o = w.part_o;
+  wp.part_lse = w.part_lse;
+  wp.o = static_cast<__nv_bfloat16*>(o);
+  wp.lse = lse;
+  esa::attn_tc_kernel<esa::CcaWindowProblem><<<grid, esa::kTcThreads, esa::kTcSmemBytes, s>>>(tq, tk, tv, bq, bk, bv,
+                                                                                           sk, sv, wp);
+  ESA_LAUNCH_CHECK("attn_tc_kernel<cca window>");
+  return ok();
 }
 
 // ------------------------------------------------------------------ MoBA decode --

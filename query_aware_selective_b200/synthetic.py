@@ -197,6 +197,37 @@ def plant_needles(w: EsaWorkload, q, k, wq, wk, gen) -> torch.Tensor:
     return pos
 
 
+@dataclasses.dataclass(frozen=True)
+class CcaWorkload:
+    """Shape and parameters of one CCA-style causal prefill workload (random inputs;
+    the article's group size and window are not on the pages: g = 128, w = 1024)."""
+
+    name: str
+    batch: int
+    hq: int
+    hkv: int
+    head_dim: int
+    seq: int
+    group: int
+    window: int
+    seed: int
+
+
+CCA_64K = CcaWorkload("cca_prefill_llama3_8b_seq65536_group128_window1024", 1, 32, 8, 128, 65536, 128, 1024, 6)
+
+
+def make_cca_inputs(w: CcaWorkload, device="cpu", seq: Optional[int] = None, batch: Optional[int] = None) -> dict:
+    """Draw Q [B, S, Hq, D] and K, V [B, S, Hkv, D] ~ N(0, 1), bf16, for a CCA workload."""
+    s = seq or w.seq
+    b = batch or w.batch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed)
+    q = _randn((b, s, w.hq, w.head_dim), torch.bfloat16, gen, device)
+    k = _randn((b, s, w.hkv, w.head_dim), torch.bfloat16, gen, device)
+    v = _randn((b, s, w.hkv, w.head_dim), torch.bfloat16, gen, device)
+    return dict(q=q, k=k, v=v)
+
+
 def make_moba_inputs(w: MobaWorkload, device="cpu", seq: Optional[int] = None,
                      heads: Optional[int] = None, batch: Optional[int] = None) -> dict:
     """Draw Q, K, V ([B, S, H, D]) for a MoBA workload."""

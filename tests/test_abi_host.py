@@ -205,3 +205,25 @@ def test_varlen_workspaces_cover_the_longest_sequence(lib):
     assert _abi.sparse_attn_varlen_workspace_size(16, 131072, 32, 8, 128, 1, 8, p) == \
         _abi.sparse_attn_heads_workspace_size(16, 1, 131071, 32, 8, 128, 1, p)
     assert _abi.score_select_varlen_workspace_size(16, 0, 128, 1, p) == 0
+
+
+def test_cca_rejects_bad_arguments(lib):
+    a = lambda dt=1, hq=32, hkv=8, d=128, group=128, window=1024, q=FAKE: lib.cca_attn(
+        q, FAKE, FAKE, dt, 1, 65536, hq, hkv, d, group, window, 0.0, FAKE, None, FAKE, 1 << 40, None)
+    assert a(dt=0) == _abi.ESA_ERR_UNSUPPORTED                 # fp32
+    assert a(hq=24) == _abi.ESA_ERR_UNSUPPORTED                # GQA group 3
+    assert a(hq=30) == _abi.ESA_ERR_INVALID_ARG
+    assert a(d=64) == _abi.ESA_ERR_UNSUPPORTED
+    assert a(group=64) == _abi.ESA_ERR_UNSUPPORTED             # not a multiple of the 128-row tile
+    assert a(window=1000) == _abi.ESA_ERR_INVALID_ARG          # not a multiple of the group
+    assert a(q=None) == _abi.ESA_ERR_INVALID_ARG
+    assert a(q=FAKE + 2) == _abi.ESA_ERR_INVALID_ARG
+    f = lib.cca_attn
+    assert f(FAKE, FAKE, FAKE, 1, 1, 65536, 32, 8, 128, 128, 1024, 0.0, FAKE, None, FAKE, 16, None) == \
+        _abi.ESA_ERR_WORKSPACE
+    assert _abi.cca_workspace_size(1, 65536, 32, 128, 128) > _abi.cca_workspace_size(1, 65536, 32, 128, 256) > 0
+
+
+def test_wait_selftest_rejects_out_of_range_limits(lib):
+    assert lib.esa_wait_selftest(10, None) == _abi.ESA_ERR_INVALID_ARG
+    assert lib.esa_wait_selftest(10 ** 12, None) == _abi.ESA_ERR_INVALID_ARG
