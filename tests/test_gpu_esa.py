@@ -332,6 +332,12 @@ def test_small_chunked_prefill_end_to_end():
         _, (m0, _), _ = oesa.regions(c0, c0 + chunk, p.n_init, p.window)
         check_selection(idx[0].cpu().numpy(), cnt[0].item(), ref["idx"][0], ref["count"][0], ref["s_prime"][0], m0,
                         p.topk)
+        # the output over the GPU's own selection, always (a band swap changes the key
+        # set but not the rule), and against the oracle's end-to-end output when the
+        # two selections agree
+        own_o, _ = oesa.sparse_attn(_np(q[:, c0:c0 + chunk]), _np(k), _np(v), c0, idx.cpu().numpy(),
+                                    cnt.cpu().numpy(), p.n_init, p.window)
+        assert max_abs(_np(o), own_o) <= ATOL_BF16
         if set(idx[0, :cnt[0]].tolist()) == set(ref["idx"][0, :ref["count"][0]].tolist()):
             assert max_abs(_np(o), ref["o"]) <= ATOL_BF16
     qas.device_status()

@@ -40,6 +40,8 @@ def _decode_full(w, seqs):
         for pos in inp["needles"][b].tolist():
             assert all(j in chosen for j in range(pos - w.eps, pos + w.eps + 1)), pos
         assert max_abs(_f64(o[b:b + 1]), ref["o"]) <= ATOL_BF16
+        own_o, _ = oesa.sparse_attn(qb, kb, vb, w.n_ctx - 1, idx[b:b + 1], cnt[b:b + 1], w.n_init, w.window)
+        assert max_abs(_f64(o[b:b + 1]), own_o) <= ATOL_BF16      # over the GPU's own selection
     del inp, dec
     torch.cuda.empty_cache()
 
@@ -94,6 +96,11 @@ def test_prefill_32k_sampled_chunks():
         check_selection(idx[0], cnt[0], ref["idx"][0], ref["count"][0], ref["s_prime"][0], m0, w.topk)
         got = _f64(out[:, c0:c0 + w.chunk])
         assert max_abs(got[:, rows], ref["o"][:, rows]) <= ATOL_BF16
+        # the same rows over the GPU's own selection (equal to the above unless a band
+        # swap changed a key)
+        own_o, _ = oesa.sparse_attn(qn[:, c0:c0 + w.chunk], kn, vn, c0, idx, cnt, w.n_init, w.window,
+                                    rows=[(0, i) for i in rows])
+        assert max_abs(got[:, rows], own_o[:, rows]) <= ATOL_BF16
 
 
 def test_moba_64k_sampled_positions():
@@ -123,3 +130,6 @@ def test_moba_64k_sampled_positions():
     ref_o, _ = omoba.attend(qn, kn, vn, ref_blocks, w.block, positions=pos)
     got = _f64(out[:, pos])
     assert max_abs(got[same], ref_o[same]) <= ATOL_BF16
+    # every sampled row, swapped gates included: attention over the GPU's own blocks
+    own_o, _ = omoba.attend(qn, kn, vn, got_blocks, w.block, positions=pos)
+    assert max_abs(got, own_o) <= ATOL_BF16

@@ -104,8 +104,15 @@ def test_gate_attn_end_to_end():
                                               want_lse=True)
     same = _gate_check(q, k, block, topk, blocks)
     ref = omoba.moba(_np(q), _np(k), _np(v), block, topk)
-    got = _np(o)
+    got, got_lse = _np(o), lse.cpu().numpy()
     assert same.mean() > 0.99
+    # rows whose gate agrees with the oracle's: the oracle's end-to-end output
     assert max_abs(got[same], ref["o"][same]) <= ATOL_BF16
-    assert max_abs(lse.cpu().numpy()[same], ref["lse"][same]) <= 2e-2
+    assert max_abs(got_lse[same], ref["lse"][same]) <= 2e-2
+    # every row, those whose gate swapped a block inside the tie band included: the
+    # oracle's attention over the GPU's own block lists (the article's
+    # Softmax(q K[I]^T) V[I] over the set the gate chose)
+    own_o, own_lse = omoba.attend(_np(q), _np(k), _np(v), blocks.cpu().numpy().astype(np.int64), block)
+    assert max_abs(got, own_o) <= ATOL_BF16
+    assert max_abs(got_lse, own_lse) <= 2e-2
     qas.device_status()

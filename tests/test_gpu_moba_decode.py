@@ -16,7 +16,8 @@ DEV = "cuda:0"
 def _check(q, k, v, block, topk, seqs=None):
     """Run one decode step on the GPU and compare sequences `seqs` with the oracle:
     kept blocks exactly (a differing block only inside the 1e-3 score band), outputs
-    within the bf16 bar where the kept blocks agree."""
+    within the bf16 bar against the oracle's where the kept blocks agree, and for every
+    head against the oracle's attention over the GPU's own blocks."""
     b, s, h, d = k.shape
     dec = pipeline.MobaDecode(b, s, h, d, block, topk, device=DEV)
     dec.fill(k)
@@ -39,9 +40,16 @@ def _check(q, k, v, block, topk, seqs=None):
             kth = np.sort(sc)[::-1][min(topk, cur) - 1]
             for blk in set(got.tolist()) ^ set(want.tolist()):
                 assert abs(sc[blk] - kth) <= 1e-3 * abs(kth) + 1e-6, (bi, hh, got, want)
+        got_o = o[bi, 0].float().cpu().numpy()                     # [H, D]
         if agree.any():
-            got_o = o[bi, 0].float().cpu().numpy()[agree]          # [heads that agree, D]
-            assert max_abs(got_o, ref["o"][0, 0][agree]) <= ATOL_BF16
+            assert max_abs(got_o[agree], ref["o"][0, 0][agree]) <= ATOL_BF16
+        # every head, swapped gates included: attention over the GPU's own blocks
+        # the oracle reads the query at position s - 1 only; a broadcast view stands in
+        # for the rest of the rows
+        q_at = np.broadcast_to(q[bi:bi + 1].float().cpu().numpy().astype(np.float64), (1, s, h, d))
+        own_o, _ = omoba.attend(q_at, kb, v[bi:bi + 1].float().cpu().numpy(), blocks[bi][None, None], block,
+                                positions=[s - 1])
+        assert max_abs(got_o, own_o[0, 0]) <= ATOL_BF16
 
 
 @pytest.mark.parametrize("batch,seq,heads,block,topk", [

@@ -6,7 +6,8 @@ allocator, a latency-critical loop that may not stall on an allocation. For them
 library keeps a fixed scratch array in device memory and offers this entry point,
 which takes no workspace. These tests call it through the C ABI and compare it, on
 two calls in a row (the array keeps the previous call's contents), with
-esa_score_select, which takes a caller-allocated workspace. This file runs last so
+esa_score_select, which takes a caller-allocated workspace, and with the oracle's
+selection. This file runs last so
 that a failure here cannot hide the rest of the suite.
 """
 import math
@@ -15,7 +16,9 @@ import numpy as np
 import pytest
 import torch
 
+from oracle import esa as oesa
 from query_aware_selective_b200 import _abi
+from tests.parity import check_selection
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -45,6 +48,13 @@ def test_noalloc_matches_the_workspace_entry_point(batch, lq, n_cap, dc, n_init,
         assert torch.equal(idx.cpu(), ref_idx.cpu()), call        # index work: bit-exact
         scale = max(1.0, float(ref_s.abs().max()))
         assert float((sc - ref_s).abs().max()) <= 1e-4 * scale, call
+        # and against the oracle itself: the same selection rule as every other
+        # selection test (exact outside the 1e-3 tie band around the k-th value)
+        o_idx, o_cnt, o_sp = oesa.score_select(q_c.double().cpu().numpy(), k_c.double().cpu().numpy(), c0, n_init,
+                                               window, topk, eps, clamp)
+        _, (m0, _), _ = oesa.regions(c0, c0 + lq, n_init, window)
+        for b in range(batch):
+            check_selection(idx[b].cpu().numpy(), int(cnt[b]), o_idx[b], o_cnt[b], o_sp[b], m0, topk)
     _abi.device_status()
 
 
