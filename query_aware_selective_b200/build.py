@@ -1,6 +1,7 @@
 """Build libesa.so in-tree for sm_100a with nvcc (one translation unit)."""
 from __future__ import annotations
 
+import hashlib
 import os
 import shutil
 import subprocess
@@ -27,17 +28,35 @@ def sources():
         [os.path.join(os.path.dirname(HERE), "include", "esa.h")]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(OUT):
+STAMP = OUT + ".sha256"
+
+
+def source_hash(extra_flags=()) -> str:
+    """SHA-256 over every source the library is built from (names and contents) and
+    the compiler flags: the binary is reused only when this matches the hash recorded
+    beside it at its build, whatever the files' modification times."""
+    h = hashlib.sha256()
+    for f in sources():
+        h.update(os.path.basename(f).encode() + b"\0")
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+        h.update(b"\0")
+    h.update(" ".join([*NVCC_FLAGS, *extra_flags]).encode())
+    return h.hexdigest()
+
+
+def up_to_date(extra_flags=()) -> bool:
+    if not (os.path.exists(OUT) and os.path.exists(STAMP)):
         return False
-    t = os.path.getmtime(OUT)
-    return all(os.path.getmtime(s) <= t for s in sources())
+    with open(STAMP) as fh:
+        return fh.read().strip() == source_hash(extra_flags)
 
 
 def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     """Compile csrc/esa_lib.cu into libesa.so next to this file. Returns its path."""
-    if not force and up_to_date():
+    if not force and up_to_date(extra_flags):
         return OUT
+    digest = source_hash(extra_flags)
     cmd = [nvcc_path(), *NVCC_FLAGS, *extra_flags, "-o", OUT + ".tmp", SRC]
     if verbose:
         print(" ".join(cmd))
@@ -46,6 +65,8 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
         sys.stderr.write(r.stdout + r.stderr)
         raise RuntimeError("nvcc failed building libesa")
     os.replace(OUT + ".tmp", OUT)
+    with open(STAMP, "w") as fh:
+        fh.write(digest + "\n")
     return OUT
 
 
