@@ -225,9 +225,10 @@ size_t esa_sparse_attn_heads_workspace_size(int32_t batch, int32_t lq, int64_t c
  *   - Arguments and results are those of esa_score_select.
  *   - A selection whose scratch (esa_score_select_workspace_size) exceeds the array
  *     returns ESA_ERR_WORKSPACE without launching anything.
- *   - The first call on a device looks up the array's device address with that device
- *     current (a one-time host call per device); make that first call before any
- *     stream capture.
+ *   - The first call in each CUDA context (the device's primary context, or one the
+ *     caller made current) looks up the array's device address there (a one-time host
+ *     call per context, remembered under the context's unique id); make that first
+ *     call before any stream capture.
  *   - All calls share the one array, and it keeps the previous call's contents; the
  *     call clears what must start at zero itself. Calls whose GPU work overlaps (on
  *     different streams or threads, for the same device) race on the array and give

@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <map>
 #include <mutex>
 #include <string>
 #include <type_traits>
@@ -102,6 +103,87 @@ esa_status_t set_max_smem(K kernel, int bytes) {
   return ESA_OK;
 }
 
+// ------------------------------------------------------ set-up once per CUDA context --
+// Kernel attributes (dynamic shared memory, cluster sizes), occupancy answers and the
+// no-alloc scratch address belong to the CUDA context they were made in, which is not
+// always the device's primary context (a plugin inside another runtime may make its own
+// current). Each is made once per context and remembered under the context's id
+// (cuCtxGetId: unique for the life of the process, never reused), so a context created
+// after another was destroyed never inherits its set-up. One mutex guards the table:
+// calls from several host threads neither race on it nor repeat the set-up.
+struct CtxFns {
+  PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  PFN_cuCtxGetId_v12000 get_id = nullptr;
+};
+
+const CtxFns& ctx_fns() {
+  static const CtxFns fns = [] {
+    CtxFns f;
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(fn);
+    cudaGetLastError();
+    return f;
+  }();
+  return fns;
+}
+
+// The id of the context the runtime uses for this thread's calls (the device's primary
+// context, initialised here, when none is current).
+esa_status_t current_context_id(unsigned long long* id) {
+  const CtxFns& f = ctx_fns();
+  if (!f.get_current || !f.get_id) return fail(ESA_ERR_CUDA, "cuCtxGetCurrent / cuCtxGetId not available");
+  CUcontext ctx = nullptr;
+  if (f.get_current(&ctx) != CUDA_SUCCESS) return fail(ESA_ERR_CUDA, "cuCtxGetCurrent failed");
+  if (!ctx) {
+    ESA_CUDA(cudaFree(nullptr));     // no allocation: makes the runtime's context current
+    if (f.get_current(&ctx) != CUDA_SUCCESS || !ctx) return fail(ESA_ERR_CUDA, "no current CUDA context");
+  }
+  if (f.get_id(ctx, id) != CUDA_SUCCESS) return fail(ESA_ERR_CUDA, "cuCtxGetId failed");
+  return ESA_OK;
+}
+
+std::mutex g_setup_mu;
+std::map<std::pair<const void*, unsigned long long>, intptr_t> g_setup;   // (what, context id) -> value
+
+// The value `make` produced for `what` in the current context, making it on the first
+// call there (make returns ESA_OK and writes *value; a failure is not remembered).
+template <class F>
+esa_status_t per_context(const void* what, intptr_t* value, F&& make) {
+  unsigned long long id = 0;
+  const esa_status_t st = current_context_id(&id);
+  if (st != ESA_OK) return st;
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  const auto key = std::make_pair(what, id);
+  const auto it = g_setup.find(key);
+  if (it != g_setup.end()) {
+    *value = it->second;
+    return ESA_OK;
+  }
+  intptr_t v = 0;
+  const esa_status_t made = make(&v);
+  if (made != ESA_OK) return made;
+  g_setup.emplace(key, v);
+  *value = v;
+  return ESA_OK;
+}
+
+// Runs `set` (kernel attributes) once per context; `what` names the group of kernels.
+template <class F>
+esa_status_t once_per_context(const void* what, F&& set) {
+  intptr_t unused = 0;
+  return per_context(what, &unused, [&](intptr_t* v) {
+    *v = 1;
+    return set();
+  });
+}
+
 esa_status_t check_params(const esa_params_t& p) {
   if (p.n_init < 0 || p.window < 0) return fail(ESA_ERR_INVALID_ARG, "n_init and window must be >= 0");
   if (p.topk < 1) return fail(ESA_ERR_INVALID_ARG, "topk must be >= 1 (got %d)", p.topk);
@@ -152,11 +234,10 @@ SelWs carve_select(void* ws, int32_t batch, int32_t lq, int64_t n_mid, ScorePath
 // sequence) can be resident at once, else the portable 8. Occupancy is queried once per
 // device.
 int select_cluster_size(int32_t batch) {
-  static int max16[64] = {};   // 0: not queried; -1: 16-CTA clusters unavailable
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return 8;
-  if (!max16[dev]) {
-    max16[dev] = -1;
+  static const char what = 0;
+  intptr_t max16 = -1;          // -1: 16-CTA clusters unavailable
+  const esa_status_t st = per_context(&what, &max16, [](intptr_t* v) {
+    *v = -1;
     if (cudaFuncSetAttribute(esa::select_cluster_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
         cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
@@ -171,27 +252,31 @@ int select_cluster_size(int32_t batch) {
       cfg.attrs = at;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, esa::select_cluster_kernel<16>, &cfg) == cudaSuccess && n >= 1)
-        max16[dev] = n;
+      if (cudaOccupancyMaxActiveClusters(&n, esa::select_cluster_kernel<16>, &cfg) == cudaSuccess && n >= 1) *v = n;
     }
     cudaGetLastError();   // a refused query is not an error of this call
-  }
+    return ESA_OK;
+  });
   // (smaller clusters for many selections were measured slower: a CTA then sweeps tens
   // of thousands of keys through the global scratch)
-  return (max16[dev] > 0 && batch <= max16[dev]) ? 16 : 8;
+  return (st == ESA_OK && max16 > 0 && batch <= max16) ? 16 : 8;
 }
 
 // 2D tensor map over a row-major fp32 matrix [rows, cols], 32 x 128 boxes, 128-byte
 // swizzle (the shared-memory layout the tf32 MMA descriptors expect).
 esa_status_t get_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
-  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-  if (!encode) {
+  // looked up once (a thread-safe static initialisation); the driver's entry point is
+  // the same for every context
+  static const PFN_cuTensorMapEncodeTiled_v12000 encode = [] {
     cudaDriverEntryPointQueryResult q;
     void* fn = nullptr;
-    ESA_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
-    if (q != cudaDriverEntryPointSuccess || !fn) return fail(ESA_ERR_CUDA, "cuTensorMapEncodeTiled not available");
-    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  }
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      fn = nullptr;
+    cudaGetLastError();
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }();
+  if (!encode) return fail(ESA_ERR_CUDA, "cuTensorMapEncodeTiled not available");
   *out = encode;
   return ESA_OK;
 }
@@ -257,15 +342,13 @@ void launch_score_small_ng(const float* q_c, const float* k_c, int lq, int64_t n
   const int64_t per_seq = std::max<int64_t>(1, std::min<int64_t>(cdiv(n_mid, ks), waves * (2 * 148) / batch));
   const int64_t keys_per_cta = cdiv(cdiv(n_mid, per_seq), ks) * ks;
   const dim3 grid((unsigned)cdiv(n_mid, keys_per_cta), batch);
-  static bool attr_set[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess && dev < 64 && !attr_set[dev]) {
-    cudaFuncSetAttribute(esa::score_small_kernel<DC, 1, NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         esa::kSsSmemBytes);
-    cudaFuncSetAttribute(esa::score_small_kernel<DC, esa::kScoreSmallLq, NG>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, esa::kSsSmemBytes);
-    attr_set[dev] = true;
-  }
+  static const char what = 0;   // one per instantiation
+  // a failure here shows as the launch's error, which the caller checks
+  once_per_context(&what, [] {
+    esa_status_t st = set_max_smem(esa::score_small_kernel<DC, 1, NG>, esa::kSsSmemBytes);
+    if (st == ESA_OK) st = set_max_smem(esa::score_small_kernel<DC, esa::kScoreSmallLq, NG>, esa::kSsSmemBytes);
+    return st;
+  });
   if (lq == 1)
     esa::score_small_kernel<DC, 1, NG><<<grid, esa::kSsThreads, esa::kSsSmemBytes, s>>>(
         q_c, k_c, lq, n_cap, mid0, n_mid, keys_per_cta, S, m_key, vl);
@@ -367,34 +450,34 @@ esa_status_t make_tmap_kmajor_bf16(CUtensorMap* m, const void* base, uint64_t in
 
 // Cluster size for the packed compression: 16 CTAs when the device can co-schedule
 // them (one CTA per SM, so a whole 16-SM group), else the portable 8.
-esa_status_t pk_cluster_size(int dev, int* cl) {
-  static int cached[64] = {};
-  if (dev < 64 && cached[dev]) {
-    *cl = cached[dev];
+esa_status_t pk_cluster_size(int* cl) {
+  static const char what = 0;
+  intptr_t best = 8;
+  const esa_status_t st = per_context(&what, &best, [](intptr_t* v) {
+    *v = 8;
+    ESA_CUDA(cudaFuncSetAttribute(esa::compress_pk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  esa::kCpSmemBytes));
+    if (cudaFuncSetAttribute(esa::compress_pk_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(16, 1, 2);
+      cfg.blockDim = dim3(esa::kCpThreads);
+      cfg.dynamicSmemBytes = esa::kCpSmemBytes;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = 16;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, esa::compress_pk_kernel, &cfg) == cudaSuccess && n >= 1) *v = 16;
+      cudaGetLastError();   // a refused query is not an error of this call
+    }
     return ESA_OK;
-  }
-  ESA_CUDA(cudaFuncSetAttribute(esa::compress_pk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                esa::kCpSmemBytes));
-  int best = 8;
-  if (cudaFuncSetAttribute(esa::compress_pk_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-      cudaSuccess) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(16, 1, 2);
-    cfg.blockDim = dim3(esa::kCpThreads);
-    cfg.dynamicSmemBytes = esa::kCpSmemBytes;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = 16;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, esa::compress_pk_kernel, &cfg) == cudaSuccess && n >= 1) best = 16;
-    cudaGetLastError();   // a refused query is not an error of this call
-  }
-  if (dev < 64) cached[dev] = best;
-  *cl = best;
+  });
+  if (st != ESA_OK) return st;
+  *cl = (int)best;
   return ESA_OK;
 }
 }  // namespace
@@ -435,10 +518,8 @@ esa_status_t compress_packed_impl(const void* x, int64_t rows, int64_t x_row_str
   if (y_row_stride < 128 || y_row_stride % 4) return fail(ESA_ERR_INVALID_ARG, "y_row_stride must be >= 128 and a multiple of 4");
   if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(y, 16))
     return fail(ESA_ERR_INVALID_ARG, "x, packed and y must be 16-byte aligned");
-  int dev = 0;
-  ESA_CUDA(cudaGetDevice(&dev));
   int cl = 8;
-  esa_status_t st = pk_cluster_size(dev, &cl);
+  esa_status_t st = pk_cluster_size(&cl);
   if (st != ESA_OK) return st;
   if (K % (64 * cl)) cl = 8;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -492,16 +573,14 @@ esa_status_t esa_compress(const void* x, esa_dtype_t x_dtype, int64_t rows, int6
   const int g = n_heads_out / n_heads_in;
   if (x_dtype == ESA_BF16 && d_out == esa::kCtN && (g == 1 || g == 2 || g == 4)) {
     // tensor-core path: 8-CTA clusters split the reduction, 128 rows x 64 columns per CTA
-    static bool attr_set[64] = {};
-    int dev = 0;
-    ESA_CUDA(cudaGetDevice(&dev));
-    if (dev < 64 && !attr_set[dev]) {
+    static const char what = 0;
+    const esa_status_t sa = once_per_context(&what, [] {
       esa_status_t st = set_max_smem(esa::compress_tc_kernel<1>, esa::kCtSmemBytes);
       if (st == ESA_OK) st = set_max_smem(esa::compress_tc_kernel<2>, esa::kCtSmemBytes);
       if (st == ESA_OK) st = set_max_smem(esa::compress_tc_kernel<4>, esa::kCtSmemBytes);
-      if (st != ESA_OK) return st;
-      attr_set[dev] = true;
-    }
+      return st;
+    });
+    if (sa != ESA_OK) return sa;
     const int64_t max_rows = (int64_t)65535 * esa::kCtRows;
     for (int64_t r0 = 0; r0 < rows; r0 += max_rows) {
       const int64_t nr = std::min(rows - r0, max_rows);
@@ -667,15 +746,14 @@ esa_status_t score_select_impl(const float* q_c, const float* k_c, int32_t batch
       if (st != ESA_OK) return st;
       esa::ScoreTcArgs a{lq, d_c, n_cap, r.mid0, r.n_mid, w.m_key, w.s, p.clamp_c};
       const int smem = 1024 + 3 * esa::kStRows * d_c * 4 + 256 + lq * 4;
-      static bool attr_set[64] = {};
-      int dev = 0;
-      ESA_CUDA(cudaGetDevice(&dev));
-      if (dev < 64 && !attr_set[dev]) {
+      static const char what = 0;
+      st = once_per_context(&what, [] {
         const int max_smem = 1024 + 3 * esa::kStRows * 128 * 4 + 256 + 4096 * 4;
-        if ((st = set_max_smem(esa::score_tc_kernel<1>, max_smem)) != ESA_OK) return st;
-        if ((st = set_max_smem(esa::score_tc_kernel<2>, max_smem)) != ESA_OK) return st;
-        attr_set[dev] = true;
-      }
+        esa_status_t sa = set_max_smem(esa::score_tc_kernel<1>, max_smem);
+        if (sa == ESA_OK) sa = set_max_smem(esa::score_tc_kernel<2>, max_smem);
+        return sa;
+      });
+      if (st != ESA_OK) return st;
       const dim3 grid((unsigned)cdiv(r.n_mid, esa::kStRows), batch);
       esa::score_tc_kernel<1><<<grid, esa::kStThreads, smem, s>>>(tm_k, tm_q, a);
       ESA_LAUNCH_CHECK("score_tc_kernel<1>");
@@ -699,14 +777,13 @@ esa_status_t score_select_impl(const float* q_c, const float* k_c, int32_t batch
       sa.s_prime_out = score_out;
       sa.idx = idx_out;
       sa.count = count_out;
-      static bool sel_attr[64] = {};
-      int dev = 0;
-      ESA_CUDA(cudaGetDevice(&dev));
-      if (dev < 64 && !sel_attr[dev]) {
-        if ((st = set_max_smem(esa::select_cluster_kernel<8>, esa::kSelSmemBytes)) != ESA_OK) return st;
-        if ((st = set_max_smem(esa::select_cluster_kernel<16>, esa::kSelSmemBytes)) != ESA_OK) return st;
-        sel_attr[dev] = true;
-      }
+      static const char what = 0;
+      st = once_per_context(&what, [] {
+        esa_status_t sa = set_max_smem(esa::select_cluster_kernel<8>, esa::kSelSmemBytes);
+        if (sa == ESA_OK) sa = set_max_smem(esa::select_cluster_kernel<16>, esa::kSelSmemBytes);
+        return sa;
+      });
+      if (st != ESA_OK) return st;
       const int cl = select_cluster_size((int32_t)vb);
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3((unsigned)cl, (unsigned)vb, 1);
@@ -917,14 +994,9 @@ esa_status_t sparse_attn_impl(const void* q, const void* k, const void* v, esa_d
     keys.vl = esa::VarLen{seq_len, n_cap, p.n_init, p.window, vseq ? hkv : 1};
   }
   if (pl.tc) {
-    static bool attr_set[64] = {};
-    int dev = 0;
-    ESA_CUDA(cudaGetDevice(&dev));
-    if (dev < 64 && !attr_set[dev]) {
-      st = set_max_smem(esa::attn_tc_kernel<esa::EsaTcProblem>, esa::kTcSmemBytes);
-      if (st != ESA_OK) return st;
-      attr_set[dev] = true;
-    }
+    static const char what = 0;
+    st = once_per_context(&what, [] { return set_max_smem(esa::attn_tc_kernel<esa::EsaTcProblem>, esa::kTcSmemBytes); });
+    if (st != ESA_OK) return st;
     esa::EsaTcProblem pr{};
     pr.q = static_cast<const __nv_bfloat16*>(q);
     pr.k = static_cast<const __nv_bfloat16*>(k);
@@ -970,15 +1042,14 @@ esa_status_t sparse_attn_impl(const void* q, const void* k, const void* v, esa_d
     return ok();
   }
   if (pl.dec) {
-    static bool dec_attr[64] = {};
-    int dev = 0;
-    ESA_CUDA(cudaGetDevice(&dev));
-    if (dev < 64 && !dec_attr[dev]) {
-      if ((st = set_max_smem(esa::attn_decode_kernel<1>, esa::kDecSmemBytes)) != ESA_OK) return st;
-      if ((st = set_max_smem(esa::attn_decode_kernel<2>, esa::kDecSmemBytes)) != ESA_OK) return st;
-      if ((st = set_max_smem(esa::attn_decode_kernel<4>, esa::kDecSmemBytes)) != ESA_OK) return st;
-      dec_attr[dev] = true;
-    }
+    static const char what_dec = 0;
+    st = once_per_context(&what_dec, [] {
+      esa_status_t sa = set_max_smem(esa::attn_decode_kernel<1>, esa::kDecSmemBytes);
+      if (sa == ESA_OK) sa = set_max_smem(esa::attn_decode_kernel<2>, esa::kDecSmemBytes);
+      if (sa == ESA_OK) sa = set_max_smem(esa::attn_decode_kernel<4>, esa::kDecSmemBytes);
+      return sa;
+    });
+    if (st != ESA_OK) return st;
     esa::DecodeAttnArgs d{};
     d.q = static_cast<const __nv_bfloat16*>(q);
     d.k = static_cast<const __nv_bfloat16*>(k);
@@ -1004,13 +1075,14 @@ esa_status_t sparse_attn_impl(const void* q, const void* k, const void* v, esa_d
     const dim3 grid((unsigned)pl.nsplit, (unsigned)(vseq ? batch * hkv : batch));
     if (d.hkv == 1) {
       // one KV head per sequence: per-warp row streams instead of per-row bulk copies
-      static bool row_attr[64] = {};
-      if (dev < 64 && !row_attr[dev]) {
-        if ((st = set_max_smem(esa::attn_decode_rows_kernel<1>, esa::kRowSmemBytes)) != ESA_OK) return st;
-        if ((st = set_max_smem(esa::attn_decode_rows_kernel<2>, esa::kRowSmemBytes)) != ESA_OK) return st;
-        if ((st = set_max_smem(esa::attn_decode_rows_kernel<4>, esa::kRowSmemBytes)) != ESA_OK) return st;
-        row_attr[dev] = true;
-      }
+      static const char what_rows = 0;
+      st = once_per_context(&what_rows, [] {
+        esa_status_t sa = set_max_smem(esa::attn_decode_rows_kernel<1>, esa::kRowSmemBytes);
+        if (sa == ESA_OK) sa = set_max_smem(esa::attn_decode_rows_kernel<2>, esa::kRowSmemBytes);
+        if (sa == ESA_OK) sa = set_max_smem(esa::attn_decode_rows_kernel<4>, esa::kRowSmemBytes);
+        return sa;
+      });
+      if (st != ESA_OK) return st;
       if (g == 1) esa::attn_decode_rows_kernel<1><<<grid, esa::kDecThreads, esa::kRowSmemBytes, s>>>(d);
       else if (g == 2) esa::attn_decode_rows_kernel<2><<<grid, esa::kDecThreads, esa::kRowSmemBytes, s>>>(d);
       else esa::attn_decode_rows_kernel<4><<<grid, esa::kDecThreads, esa::kRowSmemBytes, s>>>(d);
@@ -1158,16 +1230,13 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
   const int nb = (int)cdiv(seq, block);
   if (scale <= 0.f) scale = 1.f / std::sqrt(128.f);
   const float sl2 = scale * 1.4426950408889634f;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  ESA_CUDA(cudaGetDevice(&dev));
-  if (dev < 64 && !attr_set[dev]) {
-    esa_status_t sa = set_max_smem(esa::attn_tc_kernel<esa::MobaPastProblem>, esa::kTcSmemBytes);
-    if (sa != ESA_OK) return sa;
-    sa = set_max_smem(esa::attn_tc_kernel<esa::MobaCurrentProblem>, esa::kTcSmemBytes);
-    if (sa != ESA_OK) return sa;
-    attr_set[dev] = true;
-  }
+  static const char what = 0;
+  const esa_status_t sa = once_per_context(&what, [] {
+    esa_status_t st = set_max_smem(esa::attn_tc_kernel<esa::MobaPastProblem>, esa::kTcSmemBytes);
+    if (st == ESA_OK) st = set_max_smem(esa::attn_tc_kernel<esa::MobaCurrentProblem>, esa::kTcSmemBytes);
+    return st;
+  });
+  if (sa != ESA_OK) return sa;
   CUtensorMap tq, tk, tv, bq, bk, bv;
   esa_status_t st;
   if ((st = make_tmap_rows_bf16(&tq, q, (uint64_t)batch * seq * heads)) != ESA_OK) return st;
@@ -1367,14 +1436,13 @@ esa_status_t cca_attn(const void* q, const void* k, const void* v, esa_dtype_t d
     else launch_cca_pool<8>(q, k, v, batch, seq, hkv, group, sl2, w, s);
     ESA_LAUNCH_CHECK("cca_pool_kernel");
   }
-  static bool attr_set[64] = {};
-  int dev = 0;
-  ESA_CUDA(cudaGetDevice(&dev));
-  if (dev < 64 && !attr_set[dev]) {
-    if ((st = set_max_smem(esa::attn_tc_kernel<esa::CcaCoreProblem>, esa::kTcSmemBytes)) != ESA_OK) return st;
-    if ((st = set_max_smem(esa::attn_tc_kernel<esa::CcaWindowProblem>, esa::kTcSmemBytes)) != ESA_OK) return st;
-    attr_set[dev] = true;
-  }
+  static const char what = 0;
+  st = once_per_context(&what, [] {
+    esa_status_t sa = set_max_smem(esa::attn_tc_kernel<esa::CcaCoreProblem>, esa::kTcSmemBytes);
+    if (sa == ESA_OK) sa = set_max_smem(esa::attn_tc_kernel<esa::CcaWindowProblem>, esa::kTcSmemBytes);
+    return sa;
+  });
+  if (st != ESA_OK) return st;
   CUtensorMap tq, tk, tv, bq, bk, bv, sk, sv;
   const uint64_t rows_q = (uint64_t)batch * seq * hq, rows_kv = (uint64_t)batch * seq * hkv;
   if ((st = make_tmap_rows_bf16(&tq, q, rows_q)) != ESA_OK) return st;
@@ -1497,26 +1565,26 @@ esa_status_t moba_decode_attn(const void* q, const void* k, const void* v, esa_d
 // ------------------------------------------------------------------ no-alloc selection --
 // Scratch for esa_score_select_noalloc: a fixed array in device memory that every GPU
 // loading this library holds until the process exits. Host code may not use the name
-// as a device address; the address comes from cudaGetSymbolAddress, once per device.
+// as a device address; the address comes from cudaGetSymbolAddress, once per context.
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;     // 8 MiB
 __device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchBytes];
 
-std::mutex g_scratch_mu;
-void* g_scratch_addr[64] = {};
-
-esa_status_t scratch_for_current_device(void** out) {
-  int dev = 0;
-  ESA_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64) return fail(ESA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+// The array's device address in the current context, looked up with
+// cudaGetSymbolAddress on the first call in each context and remembered under the
+// context's unique id (a context made after another was destroyed gets its own lookup).
+esa_status_t scratch_for_current_context(void** out) {
+  static const char what = 0;
+  intptr_t addr = 0;
+  const esa_status_t st = per_context(&what, &addr, [](intptr_t* v) {
     void* p = nullptr;
     ESA_CUDA(cudaGetSymbolAddress(&p, g_select_scratch));
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+    *v = reinterpret_cast<intptr_t>(p);
+    return ESA_OK;
+  });
+  if (st != ESA_OK) return st;
+  *out = reinterpret_cast<void*>(addr);
   return ESA_OK;
 }
 
@@ -1533,7 +1601,7 @@ esa_status_t esa_score_select_noalloc(const float* q_c, const float* k_c, int32_
                 "with a workspace)",
                 need, kNoAllocScratchBytes);
   void* scratch = nullptr;
-  const esa_status_t st = scratch_for_current_device(&scratch);
+  const esa_status_t st = scratch_for_current_context(&scratch);
   if (st != ESA_OK) return st;
   return esa_score_select(q_c, k_c, batch, lq, n_cap, c0, d_c, p, idx_out, count_out, score_out, scratch,
                           kNoAllocScratchBytes, stream);
