@@ -49,7 +49,7 @@ def parse_args():
     ap.add_argument("--prefill-ctx", type=int, default=0,
                     help="shorter prefill context (profiling a small case); the line then names that workload")
     ap.add_argument("--only", choices=["decode", "decode_per_head", "decode_varlen", "decode_1m", "moba",
-                                       "moba_decode", "cca"],
+                                       "moba_decode", "cca", "tiny_decode"],
                     default=None,
                     help="profiling: run one of the other workloads alone and print its figures")
     ap.add_argument("--decode-batch", type=int, default=0, help="profiling: decode batch (default: the workload's)")
@@ -83,6 +83,42 @@ def traffic_for(kernel: str, sources):
     if not e or e.get("source_hash") != source_hash(*sources):
         return None
     return e.get("dram_bytes_per_launch")
+
+
+def choose_tensor_peak(clocks, peaks, peak_src):
+    """The dense bf16 peak a tensor-core kernel of this run is held against, chosen from
+    the run's own clock record: the burst figure (measured at full clock) when the SM
+    clock under load stayed at its maximum and no power cap was sampled, else the
+    sustained one (measured under the power cap at a lower clock). Returns (peak, regime,
+    source text)."""
+    burst, sustained = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
+    if clocks and clocks.get("sm_mhz") and clocks.get("sm_max_mhz"):
+        at_max = clocks["sm_mhz"] >= 0.97 * clocks["sm_max_mhz"]
+        capped = "sw_power_cap" in (clocks.get("reasons") or [])
+        if at_max and not capped:
+            return burst, "burst", (f"{peak_src} bf16 burst: SM clock under load {clocks['sm_mhz']:.0f} of "
+                                    f"{clocks['sm_max_mhz']:.0f} MHz, no power cap sampled")
+        return sustained, "sustained", (f"{peak_src} bf16 sustained: SM clock under load {clocks['sm_mhz']:.0f} of "
+                                        f"{clocks['sm_max_mhz']:.0f} MHz, reasons {clocks.get('reasons') or []}")
+    return burst, "burst", f"{peak_src} bf16 burst (no clock record: the higher peak, so the lower fraction)"
+
+
+def finish_tensor_roofline(r, clocks, peaks, peak_src):
+    """Fill peak and fraction of a tensor-bound roofline entry whose 'achieved' is set."""
+    peak, regime, src = choose_tensor_peak(clocks, peaks, peak_src)
+    r["peak"] = peak
+    r["frac"] = round(r["achieved"] / peak, 4)
+    r["frac_of_burst"] = round(r["achieved"] / peaks["bf16_tflops"], 4)
+    r["frac_of_sustained"] = round(r["achieved"] / peaks["bf16_tflops_sustained"], 4)
+    r["peak_regime"] = regime
+    r["peak_source"] = src
+
+
+def finish_rooflines(line, clocks, peaks, peak_src):
+    entries = [line.get("roofline")] + [e.get("roofline") for e in (line.get("also") or {}).values()]
+    for r in entries:
+        if r and r.get("bound") == "tensor":
+            finish_tensor_roofline(r, clocks, peaks, peak_src)
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -224,6 +260,7 @@ def run_only(args):
     dev = torch.device("cuda", 0)
     peaks, peak_src = load_peaks()
     flush = make_flush(dev)
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)).start()
     if args.only == "moba":
         out = bench_moba(args, dev, flush, make_dist_max(), peaks, peak_src, 1)
     elif args.only == "moba_decode":
@@ -235,8 +272,13 @@ def run_only(args):
     elif args.only == "decode_1m":
         from query_aware_selective_b200 import synthetic
         out = bench_decode(args, dev, flush, make_dist_max(), peaks, peak_src, 1, workload=synthetic.DECODE_1M)
+    elif args.only == "tiny_decode":
+        out = bench_tiny_decode(args, dev, flush, make_dist_max(), world=1)
     else:
         out = bench_decode(args, dev, flush, make_dist_max(), peaks, peak_src, 1, per_head=args.only == "decode_per_head")
+    out["clocks"] = sampler.stop()
+    if out.get("roofline", {}).get("bound") == "tensor":
+        finish_tensor_roofline(out["roofline"], out["clocks"], peaks, peak_src)
     print(json.dumps({"only": args.only, **out}), flush=True)
 
 
@@ -249,8 +291,8 @@ def run_ours(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.gpus > 1 and world == 1:
-        raise SystemExit("--gpus N > 1 runs under torch.distributed.run (one process per GPU)")
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
     torch.cuda.set_device(local)
     if world > 1:
         import datetime
@@ -301,11 +343,10 @@ def run_ours(args):
     n_attn = len(attn_ms)
     attn_time_s = sum(attn_ms) / 1e3
     achieved = fl["attention"] * args.steps / attn_time_s / 1e12
-    peak = peaks["bf16_tflops_sustained"]
+    # peak and frac are filled in from this run's clock record (finish_rooflines)
     roofline = {"bound": "tensor", "kernel": "attn_tc_kernel<EsaTcProblem>", "achieved": round(achieved, 1),
-                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak": None, "unit": "TFLOP/s", "frac": None,
                 "traffic": traffic_for("attn_tc_kernel<EsaTcProblem>", ["attn_tc.cuh", "common.cuh", "keylist.cuh"]),
-                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
                 "flops_per_launch": fl["attention"] // (n_attn // args.steps),
                 "launches": n_attn, "avg_launch_us": round(1e3 * sum(attn_ms) / n_attn, 2),
                 "share_of_step": round(sum(attn_ms) / sum(ms), 3)}
@@ -346,6 +387,9 @@ def run_ours(args):
         torch.cuda.empty_cache()
         line["also"] = {"esa_decode_128k": bench_decode(args, dev, flush, dist_max, peaks, peak_src, world)}
         torch.cuda.empty_cache()
+        line["also"]["esa_tiny_decode"] = bench_tiny_decode(args, dev, flush, dist_max, world,
+                                                            oracle=rank == 0 and world == 1)
+        torch.cuda.empty_cache()
         line["also"]["esa_decode_128k_per_head"] = bench_decode(args, dev, flush, dist_max, peaks, peak_src, world,
                                                                 per_head=True)
         torch.cuda.empty_cache()
@@ -361,6 +405,7 @@ def run_ours(args):
         torch.cuda.empty_cache()
         line["also"]["cca_prefill_64k"] = bench_cca(args, dev, flush, dist_max, peaks, peak_src, world)
     line["clocks"] = sampler.stop()
+    finish_rooflines(line, line["clocks"], peaks, peak_src)
     line["gpu"] = props.name
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_prefill()
@@ -417,6 +462,46 @@ def bench_decode(args, dev, flush, dist_max, peaks, peak_src, world, per_head=Fa
                        "sparse_attn_ms": round(att_ms, 4), "sparse_attn_gbs": round(att_gbs, 1)}}
 
 
+def bench_tiny_decode(args, dev, flush, dist_max, world, oracle=True):
+    """The tiny fp32 ESA decode step (one sequence of 2048 cached tokens, 4 heads of 64,
+    map 256 -> 16, top-128): a latency case, reported in microseconds per step, with the
+    oracle's time for the same whole step beside it (host cores, float64)."""
+    import torch
+    import query_aware_selective_b200 as qas
+    from query_aware_selective_b200 import pipeline, synthetic
+    w = synthetic.TINY_DECODE
+    p = qas.params(w.n_init, w.window, w.topk, w.eps, w.clamp_c)
+    inp = synthetic.make_esa_inputs(w)
+    dinp = {n: t.to(dev) for n, t in inp.items() if torch.is_tensor(t)}
+    dec = pipeline.EsaDecode(w.batch, w.n_ctx, w.hq, w.hkv, w.head_dim, w.d_c, p, dtype=torch.float32, device=dev)
+    dec.fill_cache(dinp["k"], dinp["wk"])
+    torch.cuda.synchronize()
+    graph = pipeline.graph_of(lambda: dec.step(dinp["q"], dinp["k"], dinp["v"], dinp["wq"], dinp["wk"]))
+    steps = max(args.steps, 50)
+    launches0 = qas._abi.launch_count()
+    dec.step(dinp["q"], dinp["k"], dinp["v"], dinp["wq"], dinp["wk"])
+    torch.cuda.synchronize()
+    launches = qas._abi.launch_count() - launches0
+    ms, total = time_steps(graph.replay, steps, args.warmup, flush, dist_max)
+    us = 1e3 * total / steps
+    out = {"workload": w.name, "value": round(world * w.batch * steps / (total / 1e3), 1), "unit": "tok/s",
+           "us_per_step": round(us, 2), "steps": steps, "dtype": "f32", "kernels_per_step": launches,
+           "execution": "one CUDA graph per step (query and key compression, selection, attention)",
+           "bound": "latency (0.9 MB per step: launch and dependency latency, not bandwidth)"}
+    if oracle:
+        from oracle import esa as oesa
+        args_np = [inp[n].numpy() for n in ("q", "k", "v", "wq", "wk")]
+        reps, t0 = 0, time.perf_counter()
+        while reps < 3 or time.perf_counter() - t0 < 2.0:
+            oesa.decode_step(*args_np, w.n_init, w.window, w.topk, w.eps, w.clamp_c)
+            reps += 1
+        o_us = 1e6 * (time.perf_counter() - t0) / reps
+        out["oracle"] = {"us_per_step": round(o_us, 1), "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"the whole step (compress the 2048 keys and the query, select, attend), "
+                                   f"{reps} runs"}
+    return out
+
+
 def bench_decode_varlen(args, dev, flush, dist_max, peaks, peak_src, world):
     """ESA decode, batch 16, caches of 128K rows holding a seeded mix of lengths
     (sequence 0 at 131072, the rest uniform in [8192, 131072]), lengths on the device."""
@@ -462,13 +547,11 @@ def bench_cca(args, dev, flush, dist_max, peaks, peak_src, world):
     ms, total = time_steps(graph.replay, steps, args.warmup, flush, dist_max)
     fl = cost.cca_flops(w.seq, w.hq, w.head_dim, w.group, w.window)
     ach = fl["total"] * w.batch / (total / steps / 1e3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
     return {"workload": w.name, "value": round(world * w.batch * w.seq * steps / (total / 1e3), 1),
             "unit": "tok/s", "ms_per_step": round(total / steps, 3), "steps": steps,
             "execution": "one CUDA graph per step",
-            "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
-                         "frac": round(ach / peak, 4), "flops_per_step": fl["total"] * w.batch,
-                         "peak_source": f"{peak_src} bf16 sustained"}}
+            "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": None, "unit": "TFLOP/s",
+                         "frac": None, "flops_per_step": fl["total"] * w.batch}}
 
 
 def bench_moba_decode(args, dev, flush, dist_max, peaks, peak_src, world):
@@ -511,13 +594,11 @@ def bench_moba(args, dev, flush, dist_max, peaks, peak_src, world):
     ms, total = time_steps(graph.replay, steps, args.warmup, flush, dist_max)
     fl = cost.moba_flops(w.seq, w.heads, w.head_dim, w.block, w.topk)
     ach = fl["total"] / (total / steps / 1e3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
     return {"workload": w.name, "value": round(world * w.batch * w.seq * steps / (total / 1e3), 1),
             "unit": "tok/s", "ms_per_step": round(total / steps, 3), "steps": steps,
             "execution": "one CUDA graph per step",
-            "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
-                         "frac": round(ach / peak, 4), "flops_per_step": fl["total"],
-                         "peak_source": f"{peak_src} bf16 sustained"}}
+            "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": None, "unit": "TFLOP/s",
+                         "frac": None, "flops_per_step": fl["total"]}}
 
 
 # ----------------------------------------------------------------------------- oracle arm
@@ -620,8 +701,27 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def spawn_command(argv, n, port):
+    """The torch.distributed.run command that runs this script as n ranks on one node
+    (one process per GPU), with the same arguments."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+
+
+def self_spawn(n, argv):
+    """`bench.py --gpus N` started as a single process: start the N ranks here and pass
+    their exit status on (rank 0 prints the line)."""
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    return subprocess.call(spawn_command(argv, n, port))
+
+
 def main():
     args = parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ and not args.only:
+        sys.exit(self_spawn(args.gpus, sys.argv[1:]))
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":

@@ -73,3 +73,23 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     monkeypatch.setattr(bench, "oracle_setup", lambda *a, **k: pytest.fail("rank 1 must not run the oracle"))
     assert bench.run_reference(bench.argparse.Namespace(steps=1, warmup=0)) is None
     assert capsys.readouterr().out == ""
+
+
+def test_bench_started_as_one_process_spawns_its_ranks():
+    # `bench.py --gpus 2` without torch.distributed.run around it starts the two ranks
+    # itself (torch.distributed.run, one process per GPU); here the oracle arm, which
+    # needs no GPU: rank 0 alone prints the line, rank 1 exits 0 without work
+    import json
+    import subprocess
+    import bench
+    cmd = bench.spawn_command(["--impl", "reference", "--gpus", "2"], 2, 29999)
+    assert cmd[1:3] == ["-m", "torch.distributed.run"] and "--nproc-per-node=2" in cmd
+    assert "--master-addr=127.0.0.1" in cmd and cmd[-2:] == ["--gpus", "2"]
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    env["OMP_NUM_THREADS"] = "2"
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "0"], capture_output=True, text=True, env=env, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(ln) for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
