@@ -71,7 +71,12 @@ struct TcSmem {
   uint64_t q_full;
   uint64_t k_full[kTcKStages], k_empty[kTcKStages], v_full[kTcVStages], v_empty[kTcVStages];
   uint64_t s_full[kTcSBufs], p_full[kTcSBufs];
-  uint64_t pv_full[2];
+  // PV_j completes pv_full[j % 3]. The softmax waits on it only now and then (a
+  // rescale, the epilogue), and a parity wait is sound only if the slot's previous
+  // phase has completed. Once S_j is seen complete, PV_{j-3} is (S_j was issued after
+  // it, and a commit covers every earlier MMA), so three slots make every such wait
+  // safe; with two, the epilogue's wait could pass on PV_{j-2}'s phase still open.
+  uint64_t pv_full[3];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -179,7 +184,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.p_full[s], 4 * kTcSplit);        // one arrival per softmax warp
     }
-    for (int s = 0; s < 2; ++s) mbar_init(&sm.pv_full[s], 1);
+    for (int s = 0; s < 3; ++s) mbar_init(&sm.pv_full[s], 1);
     mbar_init(&sm.mma_done, 1);
     sm.abort_flag = 0;
     fence_barrier_init();
@@ -261,7 +266,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           // B = V (MN-major: 8-key row groups of 1024 bytes, d blocks 16 KB apart)
           umma_f16_ts2(tmem + kTmemO, pa + kk * 8, vb + kk * 128, v_hi, idesc_pv, kk > 0 ? 1u : acc0);
         }
-        umma_commit(&sm.pv_full[j & 1]);
+        umma_commit(&sm.pv_full[j % 3]);
         umma_commit(&sm.v_empty[vs]);
       }
       // every MMA issued so far has completed before TMEM is released
@@ -330,7 +335,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const float m_new = fmaxf(m, mx);        // > m + 2^8 for the whole row group
       if (m != -INFINITY) {
         const float alpha = fast_exp2(m - m_new);
-        const bool done = mbar_wait_warp(&sm.pv_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, 110);
+        const bool done = mbar_wait_warp(&sm.pv_full[(j - 1) % 3], ((j - 1) / 3) & 1, abort_flag, 110);
         if (!(ok = bar_all(row_bar, kGroup, done))) return false;
         tc_fence_after();
         float ov[32];
@@ -427,7 +432,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
     bool fin = ok;
-    if (ok && nt > 0) fin = mbar_wait_warp(&sm.pv_full[(nt - 1) & 1], ((nt - 1) >> 1) & 1, abort_flag, 113);
+    if (ok && nt > 0) fin = mbar_wait_warp(&sm.pv_full[(nt - 1) % 3], ((nt - 1) / 3) & 1, abort_flag, 113);
     ok = bar_all(row_bar, kGroup, fin);        // every warp of the row group gets here
     sm.red[part][r] = l;
     asm volatile("bar.sync %0, %1;" ::"r"(row_bar), "r"(kGroup) : "memory");
