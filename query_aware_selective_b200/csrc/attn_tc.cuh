@@ -45,6 +45,9 @@
 #pragma once
 #include <cuda.h>
 
+#include <type_traits>
+#include <utility>
+
 #include "common.cuh"
 #include "keylist.cuh"
 
@@ -146,6 +149,13 @@ __device__ __forceinline__ void stream_kv(const Problem& prob, const CUtensorMap
     }
   }
 }
+
+// Optional hook: a policy with `void prefetch(int r, int col0)` has it called by each
+// softmax thread before the key loop, to start loads its store() will need.
+template <class P, class = void>
+struct HasPrefetch : std::false_type {};
+template <class P>
+struct HasPrefetch<P, std::void_t<decltype(std::declval<P&>().prefetch(0, 0))>> : std::true_type {};
 
 template <class Problem>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -284,6 +294,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t o_addr = lane_base + kTmemO + part * HC;
     const uint32_t row_bar = 1 + quad;         // named barrier of the kTcSplit warps of this quadrant
+    if constexpr (HasPrefetch<Problem>::value) prob.prefetch(r, part * (kTcD / kTcSplit));
     const int64_t lim = prob.limit(r);
     const float sl2 = prob.scale_log2();
     constexpr float kRescale = 8.0f;           // log2 units: rescale when the max grows by > 2^8

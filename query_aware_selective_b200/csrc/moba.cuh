@@ -347,6 +347,16 @@ struct MobaCurrentProblem {
   }
   __device__ int64_t limit(int r) const { return p0 + min((int64_t)r, nrows - 1) - kb0; }
   __device__ float scale_log2() const { return sl2; }
+  // The epilogue reads the query's past partials (a scattered 64-byte piece of each
+  // partial row per thread, and its LSE): prefetched into L2 when the CTA starts, so
+  // the loads in store() do not wait on DRAM after the last tile.
+  __device__ void prefetch(int r, int col0) const {
+    if (r >= nrows) return;
+    const int64_t row = ((int64_t)b * seq + p0 + r) * heads + h;
+    const int ns = min(topk, blk);
+    for (int s = 0; s < ns; ++s) prefetch_l2(part_o + (row * topk + s) * kTcD + col0);
+    if (col0 == 0 && ns > 0) prefetch_l2(part_lse + row * topk);
+  }
   // this part of the row merged with the query's min(topk, blk) past partials by
   // log-sum-exp (base 2), then written as the output
   __device__ void store(int r, int col0, const float* acc, float m2, float l) {
