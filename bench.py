@@ -49,7 +49,7 @@ def parse_args():
     ap.add_argument("--prefill-ctx", type=int, default=0,
                     help="shorter prefill context (profiling a small case); the line then names that workload")
     ap.add_argument("--only", choices=["decode", "decode_per_head", "decode_varlen", "decode_1m", "moba",
-                                       "moba_decode", "cca", "tiny_decode"],
+                                       "moba_decode", "cca", "tiny_decode", "fit"],
                     default=None,
                     help="profiling: run one of the other workloads alone and print its figures")
     ap.add_argument("--decode-batch", type=int, default=0, help="profiling: decode batch (default: the workload's)")
@@ -274,6 +274,8 @@ def run_only(args):
         out = bench_decode(args, dev, flush, make_dist_max(), peaks, peak_src, 1, workload=synthetic.DECODE_1M)
     elif args.only == "tiny_decode":
         out = bench_tiny_decode(args, dev, flush, make_dist_max(), world=1)
+    elif args.only == "fit":
+        out = bench_fit(args, dev, flush, make_dist_max(), peaks, peak_src, 1)
     else:
         out = bench_decode(args, dev, flush, make_dist_max(), peaks, peak_src, 1, per_head=args.only == "decode_per_head")
     out["clocks"] = sampler.stop()
@@ -404,6 +406,8 @@ def run_ours(args):
         line["also"]["moba_decode_64k"] = bench_moba_decode(args, dev, flush, dist_max, peaks, peak_src, world)
         torch.cuda.empty_cache()
         line["also"]["cca_prefill_64k"] = bench_cca(args, dev, flush, dist_max, peaks, peak_src, world)
+        torch.cuda.empty_cache()
+        line["also"]["esa_fit_64k"] = bench_fit(args, dev, flush, dist_max, peaks, peak_src, world)
     line["clocks"] = sampler.stop()
     finish_rooflines(line, line["clocks"], peaks, peak_src)
     line["gpu"] = props.name
@@ -500,6 +504,40 @@ def bench_tiny_decode(args, dev, flush, dist_max, world, oracle=True):
                          "sample": f"the whole step (compress the 2048 keys and the query, select, attend), "
                                    f"{reps} runs"}
     return out
+
+
+def bench_fit(args, dev, flush, dist_max, peaks, peak_src, world):
+    """Offline fit of the compression maps (4096 -> 128) from 65536 calibration tokens of
+    the Llama-3-8B layer shape: Gram matrices on the tensor cores, fp64 factorisations and
+    the subspace iteration, timed as one CUDA graph; the query Gram product (the tensor
+    work) is also timed alone for its roofline."""
+    import torch
+    import query_aware_selective_b200 as qas
+    from query_aware_selective_b200 import pipeline, synthetic
+    w = synthetic.FIT_64K
+    inp = synthetic.make_fit_inputs(w, device=dev)
+    ws = torch.empty(qas._abi.fit_workspace_size(w.n_tokens, w.n_tokens, w.hq, w.hkv, w.head_dim, w.d_c,
+                                                 w.oversample) + 256, dtype=torch.uint8, device=dev)
+    graph = pipeline.graph_of(lambda: qas.fit_maps(inp["q"], inp["k"], w.d_c, inp["omega"], ridge=w.ridge,
+                                                   power_iters=w.power_iters, workspace=ws))
+    steps = max(3, args.steps // 3)
+    ms, total = time_steps(graph.replay, steps, args.warmup, flush, dist_max)
+    # the query Gram product alone: n * dq * (dq + 1) flops of symmetric X^T X
+    dq = w.hq * w.head_dim
+    x = inp["q"].view(w.n_tokens, dq)
+    gws = torch.empty(qas._abi.load().esa_gram_workspace_size(w.n_tokens, dq) + 256, dtype=torch.uint8, device=dev)
+    g = torch.empty((dq, dq), dtype=torch.float64, device=dev)
+    gram_graph = pipeline.graph_of(lambda: qas.gram(x, workspace=gws, out=g))
+    gms, gtotal = time_steps(gram_graph.replay, steps, args.warmup, flush, dist_max)
+    flops = w.n_tokens * dq * (dq + 1)
+    ach = flops / (gtotal / steps / 1e3) / 1e12
+    return {"workload": w.name, "value": round(world * w.n_tokens * steps / (total / 1e3), 1),
+            "unit": "calibration tok/s", "ms_per_step": round(total / steps, 3), "steps": steps,
+            "execution": "one CUDA graph per fit (Grams, Cholesky, C, subspace iteration, Rayleigh-Ritz, maps)",
+            "gram_ms": round(gtotal / steps, 4),
+            "roofline": {"bound": "tensor", "kernel": "esa_gram: gram_kernel + fixed-order fp64 sum (query Gram X^T X, 65536 x 4096 bf16)",
+                         "achieved": round(ach, 1), "peak": None, "unit": "TFLOP/s", "frac": None,
+                         "flops_per_launch": flops}}
 
 
 def bench_decode_varlen(args, dev, flush, dist_max, peaks, peak_src, world):

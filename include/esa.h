@@ -389,6 +389,57 @@ esa_status_t esa_sparse_attn_varlen(const void* q, const void* k, const void* v,
 size_t esa_sparse_attn_varlen_workspace_size(int32_t batch, int64_t n_cap, int32_t hq, int32_t hkv,
                                              int32_t head_dim, esa_dtype_t dt, int32_t lists, esa_params_t p);
 
+/* ------------------------------------------- offline fit of the compression maps -- */
+
+/* esa_gram - the Gram matrix G = X^T X of calibration rows X [n, dim] (bf16, rows
+ * contiguous), accumulated in fp32 on the tensor cores (bf16 products are exact in
+ * fp32) and returned in fp64 [dim, dim] (both triangles). The first step of the offline
+ * fit below (ESA write-up, compression paragraph).
+ *   Requires dim a multiple of 128 (<= 16384), 1 <= n < 2^31, x 16-byte aligned.
+ *   workspace: esa_gram_workspace_size(n, dim) bytes, 256-byte aligned (fp32 partial
+ *   sums over slices of the rows, added in a fixed order: the result is deterministic). */
+esa_status_t esa_gram(const void* x, esa_dtype_t dt, int64_t n, int32_t dim, double* g, void* workspace,
+                      size_t ws_bytes, void* stream);
+size_t esa_gram_workspace_size(int64_t n, int32_t dim);
+
+/* esa_fit_maps - the two one-layer compression maps fitted offline from calibration
+ * queries and keys (ESA write-up, compression paragraph: the maps are learned from
+ * queries and keys kept from a calibration run, the model untouched; experiments
+ * paragraph: 4096 -> 128). The loss is not on the pages; this call minimises the plain
+ * least squares of the compressed scores against the merged-head scores over every
+ * (calibration query, calibration key) pair,
+ *     sum_ij ( q~_i . k~_j - sum_h q_i^h . k_j^{h / G} )^2 .
+ * Method: Gram matrices X^T X, Y^T Y (tensor cores, fp32 accumulation) plus a ridge of
+ * ridge * trace / dim on the diagonal, their upper Cholesky factors Rq, Rk (fp64), the
+ * matrix C = Rq E Rk^T (E the GQA expansion), the leading d_c right singular vectors V
+ * of C (the leading eigenvectors of C^T C: subspace iteration with l = d_c + oversample
+ * columns from the caller's Gaussian start omega, power_iters rounds with CholeskyQR2
+ * re-orthonormalisation, then a Rayleigh-Ritz step whose l x l problem is solved by the
+ * cyclic Jacobi method), then W_q = Rq^-1 C V and the folded key map B = Rk^-1 V. The
+ * compressed scores q~ . k~ = x W_q B^T y^T are the least-squares optimum
+ * (Eckart-Young); the maps themselves are one of the equivalent pairs (W_q T, W_k T^-T
+ * for invertible T). The error of the subspace falls like (lambda_{l+1} / lambda_{d_c})
+ * ^ power_iters in the eigenvalues of C^T C.
+ *   xq:    [n_q, hq, head_dim] bf16 calibration queries; yk: [n_k, hkv, head_dim] keys.
+ *   omega: [hkv * head_dim, d_c + oversample] fp64 on the device, standard normal
+ *          entries (the random start is an input: the call draws no random numbers).
+ *   w_q:   [hq * head_dim, d_c] fp32, the query map of esa_compress (n_heads_out = hq).
+ *   w_k:   [hq * head_dim, d_c] fp32, the key map of esa_compress with the keys expanded
+ *          to hq heads (each query head's rows are its KV head's rows of B divided by
+ *          the group size hq / hkv; esa_compress_pack folds it back to B).
+ *   Requires hq * head_dim and hkv * head_dim multiples of 128, d_c >= 1, oversample
+ *   >= 0, d_c + oversample <= min(160, hkv * head_dim), 0 <= power_iters <= 64,
+ *   ridge >= 0 (needed when n_q < hq * head_dim or n_k < hkv * head_dim). A Gram matrix that is not positive definite is reported by
+ *   esa_device_status (a Cholesky pivot was not positive) and the maps are then invalid.
+ *   workspace: esa_fit_workspace_size(...) bytes, 256-byte aligned. Asynchronous on the
+ *   stream; the library allocates nothing. */
+esa_status_t esa_fit_maps(const void* xq, int64_t n_q, const void* yk, int64_t n_k, esa_dtype_t dt, int32_t hq,
+                          int32_t hkv, int32_t head_dim, int32_t d_c, int32_t oversample, double ridge,
+                          int32_t power_iters, const double* omega, float* w_q, float* w_k, void* workspace,
+                          size_t ws_bytes, void* stream);
+size_t esa_fit_workspace_size(int64_t n_q, int64_t n_k, int32_t hq, int32_t hkv, int32_t head_dim, int32_t d_c,
+                              int32_t oversample);
+
 /* ------------------------------------------------------------------- status -- */
 
 /* Message for the last non-OK status returned on this thread ("" if none). */

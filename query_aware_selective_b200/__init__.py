@@ -6,12 +6,12 @@ benchmark inputs; ``cost`` holds the algorithmic byte and flop counts used for
 rooflines.
 """
 from ._abi import (EsaError, EsaParams, cca_attn, compress, compress_pack, compress_pack_size, compress_packed,
-                   compress_packed_varlen, device_status, load, moba_block_attn, moba_block_gate,
+                   compress_packed_varlen, device_status, fit_maps, gram, load, moba_block_attn, moba_block_gate,
                    moba_block_gate_attn, moba_block_means, moba_decode_attn, params, score_select,
                    score_select_heads, score_select_varlen, sparse_attn, sparse_attn_heads, sparse_attn_varlen)
 
 __all__ = ["EsaError", "EsaParams", "cca_attn", "compress", "compress_pack", "compress_pack_size", "compress_packed",
-           "compress_packed_varlen", "device_status", "load", "moba_block_attn", "moba_block_gate",
-           "moba_block_gate_attn", "moba_block_means", "moba_decode_attn", "params",
+           "compress_packed_varlen", "device_status", "fit_maps", "gram", "load", "moba_block_attn",
+           "moba_block_gate", "moba_block_gate_attn", "moba_block_means", "moba_decode_attn", "params",
            "score_select", "score_select_heads", "score_select_varlen", "sparse_attn", "sparse_attn_heads",
            "sparse_attn_varlen"]

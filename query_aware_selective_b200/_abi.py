@@ -70,6 +70,11 @@ SIGNATURES = {
     "cca_attn": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i64, _i32, _i32, _i32, _i32, _i32, _f32, _vp,
                                 _vp, _vp, _sz, _vp]),
     "cca_workspace_size": (_sz, [_i32, _i64, _i32, _i32, _i32]),
+    "esa_gram": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i32, _vp, _vp, _sz, _vp]),
+    "esa_gram_workspace_size": (_sz, [_i64, _i32]),
+    "esa_fit_maps": (ctypes.c_int, [_vp, _i64, _vp, _i64, ctypes.c_int, _i32, _i32, _i32, _i32, _i32,
+                                    ctypes.c_double, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "esa_fit_workspace_size": (_sz, [_i64, _i64, _i32, _i32, _i32, _i32, _i32]),
     "esa_compress_packed_varlen": (ctypes.c_int, [_vp, _i32, _i64, _i32, _i32, _vp, _i32, _vp, _i64, _vp, _vp]),
     "esa_score_select_varlen": (ctypes.c_int, [_vp, _vp, _i32, _i64, _vp, _i32, _i32, EsaParams, _vp, _vp, _vp,
                                                _vp, _sz, _vp]),
@@ -430,6 +435,46 @@ def sparse_attn_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_le
                                          _ptr(lse) if want_lse else None, wp, wn, _stream()),
            "esa_sparse_attn_varlen")
     return out, (lse if want_lse else None)
+
+
+def gram(x: torch.Tensor, workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """esa_gram: G = X^T X (fp64 [dim, dim]) of bf16 rows x [n, dim] (any leading shape
+    flattened to rows)."""
+    _dev(x)
+    dim = x.shape[-1]
+    n = x.numel() // dim
+    if out is None:
+        out = torch.empty((dim, dim), dtype=torch.float64, device=x.device)
+    ws = _workspace(load().esa_gram_workspace_size(n, dim), x.device, workspace)
+    wp, wn = _ws_ptr(ws)
+    _check(load().esa_gram(_ptr(x), _dtype_code(x), n, dim, _ptr(out), wp, wn, _stream()), "esa_gram")
+    return out
+
+
+def fit_workspace_size(n_q, n_k, hq, hkv, d, d_c, oversample) -> int:
+    return load().esa_fit_workspace_size(n_q, n_k, hq, hkv, d, d_c, oversample)
+
+
+def fit_maps(q: torch.Tensor, k: torch.Tensor, d_c: int, omega: torch.Tensor, ridge: float = 0.0,
+             power_iters: int = 8, workspace: Optional[torch.Tensor] = None):
+    """esa_fit_maps: compression maps fitted to calibration queries q [n_q, hq, d] and keys
+    k [n_k, hkv, d] (bf16). omega: [hkv * d, d_c + oversample] float64 standard normal
+    start (its width sets the oversampling). Returns (w_q, w_k), fp32 [hq * d, d_c] each,
+    in the layout esa_compress takes."""
+    _dev(q, k, omega)
+    n_q, hq, d = q.shape
+    n_k, hkv = k.shape[0], k.shape[1]
+    if omega.dtype != torch.float64 or omega.dim() != 2 or omega.shape[0] != hkv * d or omega.shape[1] < d_c:
+        raise ValueError("omega must be a contiguous float64 [hkv * d, d_c + oversample] tensor")
+    oversample = omega.shape[1] - d_c
+    w_q = torch.empty((hq * d, d_c), dtype=torch.float32, device=q.device)
+    w_k = torch.empty((hq * d, d_c), dtype=torch.float32, device=q.device)
+    ws = _workspace(fit_workspace_size(n_q, n_k, hq, hkv, d, d_c, oversample), q.device, workspace)
+    wp, wn = _ws_ptr(ws)
+    _check(load().esa_fit_maps(_ptr(q), n_q, _ptr(k), n_k, _dtype_code(q), hq, hkv, d, d_c, oversample,
+                               float(ridge), int(power_iters), _ptr(omega), _ptr(w_q), _ptr(w_k), wp, wn,
+                               _stream()), "esa_fit_maps")
+    return w_q, w_k
 
 
 def cca_workspace_size(batch, seq, hq, d, group) -> int:

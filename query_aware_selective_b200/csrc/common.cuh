@@ -509,6 +509,12 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* r) {
       "r"(u[25]), "r"(u[26]), "r"(u[27]), "r"(u[28]), "r"(u[29]), "r"(u[30]), "r"(u[31])
       : "memory");
 }
+// Load 8 columns of 32-bit data (lane = thread's row within the warp's quadrant).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* u) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7])
+               : "r"(taddr));
+}
 // Store 8 columns of 32-bit data (lane = thread's row within the warp's quadrant).
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* u) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(u[0]),

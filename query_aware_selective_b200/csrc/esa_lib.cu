@@ -24,6 +24,7 @@
 #include "compress.cuh"
 #include "compress_tc.cuh"
 #include "compress_pk.cuh"
+#include "fit.cuh"
 #include "moba.cuh"
 #include "score.cuh"
 #include "score_tc.cuh"
@@ -399,6 +400,10 @@ esa_status_t esa_device_status(void* stream) {
   if (code == 5u) return fail(ESA_ERR_CUDA, "kernel site %u found its shared memory misaligned and stopped", site);
   if (code == 1u)
     return fail(ESA_ERR_INVALID_ARG, "kernel site %u read a sequence length outside [1, n_cap] (clamped)", site);
+  if (code == 6u)
+    return fail(ESA_ERR_INVALID_ARG,
+                "site %u: a Cholesky pivot was not positive (the matrix is not positive definite; a ridge helps)",
+                site);
   return fail(ESA_ERR_TIMEOUT, "device wait ran out at site %u (status %u)", site, code);
 }
 
@@ -1608,3 +1613,281 @@ esa_status_t esa_score_select_noalloc(const float* q_c, const float* k_c, int32_
 }
 
 size_t esa_score_select_noalloc_capacity(void) { return kNoAllocScratchBytes; }
+
+// ------------------------------------------------------------------ offline fit --
+namespace {
+
+int gram_splits(int dim, int64_t n) {
+  const int tiles = dim / 128;
+  const int64_t pairs = (int64_t)tiles * (tiles + 1) / 2;
+  const int64_t chunks = std::max<int64_t>(1, cdiv(n, esa::kGmRows));
+  return (int)std::max<int64_t>(1, std::min<int64_t>(chunks, 148 / pairs));
+}
+
+size_t gram_part_bytes(int dim, int64_t n) { return up256((size_t)gram_splits(dim, n) * dim * dim * sizeof(double)); }
+
+esa_status_t gram_check(const void* x, esa_dtype_t dt, int64_t n, int32_t dim) {
+  if (dt != ESA_BF16) return fail(ESA_ERR_UNSUPPORTED, "the Gram product takes bf16 rows");
+  if (n <= 0) return fail(ESA_ERR_INVALID_ARG, "n must be >= 1");
+  if (n >= ((int64_t)1 << 31)) return fail(ESA_ERR_UNSUPPORTED, "n must be < 2^31");
+  if (dim <= 0 || dim % 128 || dim > 16384) return fail(ESA_ERR_UNSUPPORTED, "dim %d (a multiple of 128, <= 16384)", dim);
+  if (!x) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(x, 16)) return fail(ESA_ERR_INVALID_ARG, "x needs 16-byte alignment");
+  return ESA_OK;
+}
+
+// G [dim, dim] fp64 = X^T X for X [n, dim] bf16 (rows contiguous); part: scratch.
+esa_status_t gram_launch(const void* x, int64_t n, int32_t dim, double* part, double* g, cudaStream_t s) {
+  static const char what = 0;
+  esa_status_t st = once_per_context(&what, [] {
+    ESA_CUDA(cudaFuncSetAttribute(esa::gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, esa::kGmSmem));
+    return ESA_OK;
+  });
+  if (st != ESA_OK) return st;
+  PFN_cuTensorMapEncodeTiled_v12000 encode;
+  if ((st = get_encoder(&encode)) != ESA_OK) return st;
+  CUtensorMap tm;
+  cuuint64_t dims[2] = {(cuuint64_t)dim, (cuuint64_t)n};
+  cuuint64_t strides[1] = {(cuuint64_t)dim * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)esa::kGmRows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ESA_ERR_CUDA, "cuTensorMapEncodeTiled (Gram rows) failed (%d)", (int)r);
+  const int splits = gram_splits(dim, n);
+  esa::GramArgs a{};
+  a.dim = dim;
+  a.tiles = dim / 128;
+  a.n = n;
+  a.rows_per_split = cdiv(cdiv(n, splits), esa::kGmRows) * esa::kGmRows;
+  a.part = part;
+  const unsigned pairs = (unsigned)(a.tiles * (a.tiles + 1) / 2);
+  esa::gram_kernel<<<dim3(pairs, splits), esa::kGmThreads, esa::kGmSmem, s>>>(tm, a);
+  ESA_LAUNCH_CHECK("gram_kernel");
+  const int64_t count = (int64_t)dim * dim;
+  esa::gram_finish_kernel<<<(unsigned)std::min<int64_t>(4096, cdiv(count, 256)), 256, 0, s>>>(part, splits, count, g);
+  ESA_LAUNCH_CHECK("gram_finish_kernel");
+  return ESA_OK;
+}
+
+esa_status_t gemm64(int m, int n, int k, double alpha, const double* A, int64_t ar, int64_t ac, const double* B,
+                    int64_t br, int64_t bc, double beta, double* C, int64_t ldc, cudaStream_t s) {
+  if (m <= 0 || n <= 0) return ESA_OK;
+  const dim3 grid((unsigned)cdiv(n, esa::kG64Tile), (unsigned)cdiv(m, esa::kG64Tile));
+  esa::gemm64_kernel<<<grid, 256, 0, s>>>(m, n, k, alpha, A, ar, ac, B, br, bc, beta, C, ldc);
+  ESA_LAUNCH_CHECK("gemm64_kernel");
+  return ESA_OK;
+}
+
+esa_status_t fit_kernels_setup() {
+  static const char what = 0;
+  return once_per_context(&what, [] {
+    ESA_CUDA(cudaFuncSetAttribute(esa::chol_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  esa::kCholSmem));
+    ESA_CUDA(cudaFuncSetAttribute(esa::trsm_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  esa::kTrsmSmem));
+    ESA_CUDA(cudaFuncSetAttribute(esa::jacobi_eig_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  esa::kJacobiSmem));
+    return ESA_OK;
+  });
+}
+
+esa_status_t chol_block(double* A, int64_t lda, int nb, unsigned site, cudaStream_t s) {
+  esa::chol_block_kernel<<<1, 256, (size_t)nb * (nb + 1) * sizeof(double), s>>>(A, lda, nb, site);
+  ESA_LAUNCH_CHECK("chol_block_kernel");
+  return ESA_OK;
+}
+
+esa_status_t trsm_block(const double* T, int64_t ldt, int nb, double* X, int64_t xr, int64_t xc, int64_t ncols,
+                        int trans, cudaStream_t s) {
+  if (ncols <= 0) return ESA_OK;
+  const size_t smem = (size_t)nb * esa::kTrsmCols * sizeof(double);
+  esa::trsm_block_kernel<<<(unsigned)cdiv(ncols, esa::kTrsmCols), esa::kTrsmCols, smem, s>>>(T, ldt, nb, X, xr, xc,
+                                                                                              ncols, trans);
+  ESA_LAUNCH_CHECK("trsm_block_kernel");
+  return ESA_OK;
+}
+
+// In place: A [dim, dim] symmetric positive definite -> its upper Cholesky factor R
+// (A = R^T R, strict lower part zeroed). Right-looking, 128-wide blocks: factor the
+// diagonal block, solve its row panel (R_kk^T P = A_k,rest), update the trailing matrix
+// (A_rest -= P^T P) with the fp64 GEMM.
+esa_status_t cholesky(double* A, int dim, unsigned site, cudaStream_t s) {
+  esa_status_t st;
+  const int T = dim / 128;
+  for (int kb = 0; kb < T; ++kb) {
+    double* akk = A + (int64_t)kb * 128 * (dim + 1);
+    if ((st = chol_block(akk, dim, 128, site, s)) != ESA_OK) return st;
+    const int m = dim - (kb + 1) * 128;
+    if (m == 0) break;
+    double* panel = A + (int64_t)kb * 128 * dim + (kb + 1) * 128;
+    if ((st = trsm_block(akk, dim, 128, panel, dim, 1, m, 1, s)) != ESA_OK) return st;
+    if ((st = gemm64(m, m, 128, -1.0, panel, 1, dim, panel, dim, 1, 1.0, A + (int64_t)(kb + 1) * 128 * (dim + 1), dim,
+                     s)) != ESA_OK)
+      return st;
+  }
+  esa::zero_lower_kernel<<<(unsigned)std::min<int64_t>(4096, cdiv((int64_t)dim * dim, 256)), 256, 0, s>>>(A, dim);
+  ESA_LAUNCH_CHECK("zero_lower_kernel");
+  return ESA_OK;
+}
+
+// In place: Y [dim, l] <- R^-1 Y for R [dim, dim] upper (blocked back substitution).
+esa_status_t upper_solve(const double* R, int dim, double* Y, int l, cudaStream_t s) {
+  esa_status_t st;
+  for (int kb = dim / 128 - 1; kb >= 0; --kb) {
+    double* yk = Y + (int64_t)kb * 128 * l;
+    if ((st = trsm_block(R + (int64_t)kb * 128 * (dim + 1), dim, 128, yk, l, 1, l, 0, s)) != ESA_OK) return st;
+    if (kb > 0 &&
+        (st = gemm64(kb * 128, l, 128, -1.0, R + (int64_t)kb * 128, dim, 1, yk, l, 1, 1.0, Y, l, s)) != ESA_OK)
+      return st;
+  }
+  return ESA_OK;
+}
+
+// In place: Y [m, l] <- an orthonormal basis of its columns (CholeskyQR twice: G = Y^T Y,
+// G = R^T R, Y <- Y R^-1, repeated once for accuracy). gs: [l, l] scratch.
+esa_status_t orthonormalize(double* Y, int m, int l, double* gs, unsigned site, cudaStream_t s) {
+  esa_status_t st;
+  for (int pass = 0; pass < 2; ++pass) {
+    if ((st = gemm64(l, l, m, 1.0, Y, 1, l, Y, l, 1, 0.0, gs, l, s)) != ESA_OK) return st;
+    if ((st = chol_block(gs, l, l, site + pass, s)) != ESA_OK) return st;
+    // row y of Y solves x R = y, i.e. R^T x^T = y^T: forward substitution on each row
+    if ((st = trsm_block(gs, l, l, Y, 1, l, m, 1, s)) != ESA_OK) return st;
+  }
+  return ESA_OK;
+}
+
+struct FitWs {
+  double* part;     // Gram row-slice partials
+  double* gq;       // [dq, dq] -> Rq
+  double* gk;       // [dk, dk] -> Rk
+  double* rqe;      // [dq, dk] Rq E
+  double* c;        // [dq, dk] C = Rq E Rk^T
+  double* a;        // [dk, dk] A = C^T C
+  double* v;        // [dk, l] subspace basis
+  double* w;        // [dk, l] A V
+  double* gs;       // [l, l] Gram of the basis / projected problem
+  double* z;        // [L, L] Jacobi rotations (L = l rounded up to even)
+  double* zsel;     // [l, d_c] leading eigenvectors of the projected problem
+  double* vd;       // [dk, d_c] leading right singular vectors of C -> folded key map
+  double* cv;       // [dq, d_c] C V -> query map
+  size_t bytes;
+};
+
+FitWs carve_fit(void* ws, int64_t n_q, int64_t n_k, int dq, int dk, int l, int d_c) {
+  Carver cv{reinterpret_cast<uint8_t*>(ws)};
+  FitWs w{};
+  const size_t part = std::max(gram_part_bytes(dq, n_q), gram_part_bytes(dk, n_k));
+  const int L = l + (l & 1);
+  w.part = cv.take<double>(part / sizeof(double));
+  w.gq = cv.take<double>((size_t)dq * dq);
+  w.gk = cv.take<double>((size_t)dk * dk);
+  w.rqe = cv.take<double>((size_t)dq * dk);
+  w.c = cv.take<double>((size_t)dq * dk);
+  w.a = cv.take<double>((size_t)dk * dk);
+  w.v = cv.take<double>((size_t)dk * l);
+  w.w = cv.take<double>((size_t)dk * l);
+  w.gs = cv.take<double>((size_t)l * l);
+  w.z = cv.take<double>((size_t)L * L);
+  w.zsel = cv.take<double>((size_t)l * d_c);
+  w.vd = cv.take<double>((size_t)dk * d_c);
+  w.cv = cv.take<double>((size_t)dq * d_c);
+  w.bytes = cv.off;
+  return w;
+}
+
+}  // namespace
+
+size_t esa_gram_workspace_size(int64_t n, int32_t dim) {
+  if (n <= 0 || dim <= 0 || dim % 128) return 0;
+  return gram_part_bytes(dim, n);
+}
+
+esa_status_t esa_gram(const void* x, esa_dtype_t dt, int64_t n, int32_t dim, double* g, void* workspace,
+                      size_t ws_bytes, void* stream) {
+  esa_status_t st = gram_check(x, dt, n, dim);
+  if (st != ESA_OK) return st;
+  if (!g) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  const size_t need = gram_part_bytes(dim, n);
+  if (!workspace || ws_bytes < need || !aligned(workspace, 256))
+    return fail(ESA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need, ws_bytes);
+  st = gram_launch(x, n, dim, static_cast<double*>(workspace), g, reinterpret_cast<cudaStream_t>(stream));
+  return st == ESA_OK ? ok() : st;
+}
+
+size_t esa_fit_workspace_size(int64_t n_q, int64_t n_k, int32_t hq, int32_t hkv, int32_t head_dim, int32_t d_c,
+                              int32_t oversample) {
+  if (n_q <= 0 || n_k <= 0 || hq <= 0 || hkv <= 0 || head_dim <= 0 || d_c <= 0 || oversample < 0) return 0;
+  const int dq = hq * head_dim, dk = hkv * head_dim;
+  if (dq % 128 || dk % 128) return 0;
+  return carve_fit(nullptr, n_q, n_k, dq, dk, d_c + oversample, d_c).bytes;
+}
+
+esa_status_t esa_fit_maps(const void* xq, int64_t n_q, const void* yk, int64_t n_k, esa_dtype_t dt, int32_t hq,
+                          int32_t hkv, int32_t head_dim, int32_t d_c, int32_t oversample, double ridge,
+                          int32_t power_iters, const double* omega, float* w_q, float* w_k, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  if (hq <= 0 || hkv <= 0 || hq % hkv) return fail(ESA_ERR_INVALID_ARG, "hq must be a positive multiple of hkv");
+  if (head_dim <= 0) return fail(ESA_ERR_INVALID_ARG, "head_dim must be >= 1");
+  const int dq = hq * head_dim, dk = hkv * head_dim, group = hq / hkv;
+  esa_status_t st = gram_check(xq, dt, n_q, dq);
+  if (st != ESA_OK) return st;
+  if ((st = gram_check(yk, dt, n_k, dk)) != ESA_OK) return st;
+  const int l = d_c + oversample;
+  if (d_c < 1 || oversample < 0 || l > esa::kCholMax || l > dk)
+    return fail(ESA_ERR_UNSUPPORTED, "d_c %d + oversample %d must be in [1, min(%d, hkv * head_dim)]", d_c,
+                oversample, esa::kCholMax);
+  if (!(ridge >= 0.0) || !std::isfinite(ridge)) return fail(ESA_ERR_INVALID_ARG, "ridge must be finite and >= 0");
+  if (power_iters < 0 || power_iters > 64) return fail(ESA_ERR_INVALID_ARG, "power_iters must be in [0, 64]");
+  if (!omega || !w_q || !w_k) return fail(ESA_ERR_INVALID_ARG, "null pointer");
+  const size_t need = carve_fit(nullptr, n_q, n_k, dq, dk, l, d_c).bytes;
+  if (!workspace || ws_bytes < need || !aligned(workspace, 256))
+    return fail(ESA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need, ws_bytes);
+  if ((st = fit_kernels_setup()) != ESA_OK) return st;
+  const FitWs w = carve_fit(workspace, n_q, n_k, dq, dk, l, d_c);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // Gram matrices (+ ridge), then their upper Cholesky factors
+  if ((st = gram_launch(xq, n_q, dq, w.part, w.gq, s)) != ESA_OK) return st;
+  if (ridge > 0.0) {
+    esa::ridge_kernel<<<1, 256, 0, s>>>(w.gq, dq, ridge);
+    ESA_LAUNCH_CHECK("ridge_kernel");
+  }
+  if ((st = gram_launch(yk, n_k, dk, w.part, w.gk, s)) != ESA_OK) return st;
+  if (ridge > 0.0) {
+    esa::ridge_kernel<<<1, 256, 0, s>>>(w.gk, dk, ridge);
+    ESA_LAUNCH_CHECK("ridge_kernel");
+  }
+  if ((st = cholesky(w.gq, dq, 700, s)) != ESA_OK) return st;
+  if ((st = cholesky(w.gk, dk, 701, s)) != ESA_OK) return st;
+  // C = (Rq E) Rk^T and A = C^T C
+  esa::fold_heads_kernel<<<(unsigned)std::min<int64_t>(4096, cdiv((int64_t)dq * dk, 256)), 256, 0, s>>>(
+      w.gq, dq, hkv, group, head_dim, w.rqe);
+  ESA_LAUNCH_CHECK("fold_heads_kernel");
+  if ((st = gemm64(dq, dk, dk, 1.0, w.rqe, dk, 1, w.gk, 1, dk, 0.0, w.c, dk, s)) != ESA_OK) return st;
+  if ((st = gemm64(dk, dk, dq, 1.0, w.c, 1, dk, w.c, dk, 1, 0.0, w.a, dk, s)) != ESA_OK) return st;
+  // subspace iteration: V = orth(A Omega), then power_iters rounds of V = orth(A V)
+  if ((st = gemm64(dk, l, dk, 1.0, w.a, dk, 1, omega, l, 1, 0.0, w.v, l, s)) != ESA_OK) return st;
+  if ((st = orthonormalize(w.v, dk, l, w.gs, 710, s)) != ESA_OK) return st;
+  double* v = w.v;
+  double* t = w.w;
+  for (int it = 0; it < power_iters; ++it) {
+    if ((st = gemm64(dk, l, dk, 1.0, w.a, dk, 1, v, l, 1, 0.0, t, l, s)) != ESA_OK) return st;
+    if ((st = orthonormalize(t, dk, l, w.gs, 720, s)) != ESA_OK) return st;
+    std::swap(v, t);
+  }
+  // Rayleigh-Ritz: H = V^T A V, its leading d_c eigenvectors, V_d = V Z_sel
+  if ((st = gemm64(dk, l, dk, 1.0, w.a, dk, 1, v, l, 1, 0.0, t, l, s)) != ESA_OK) return st;
+  if ((st = gemm64(l, l, dk, 1.0, v, 1, l, t, l, 1, 0.0, w.gs, l, s)) != ESA_OK) return st;
+  esa::jacobi_eig_kernel<<<1, esa::kJacobiThreads, esa::kJacobiSmem, s>>>(w.gs, l, w.z, d_c, w.zsel, 30);
+  ESA_LAUNCH_CHECK("jacobi_eig_kernel");
+  if ((st = gemm64(dk, d_c, l, 1.0, v, l, 1, w.zsel, d_c, 1, 0.0, w.vd, d_c, s)) != ESA_OK) return st;
+  // query map W_q = Rq^-1 C V_d, folded key map B = Rk^-1 V_d
+  if ((st = gemm64(dq, d_c, dk, 1.0, w.c, dk, 1, w.vd, d_c, 1, 0.0, w.cv, d_c, s)) != ESA_OK) return st;
+  if ((st = upper_solve(w.gq, dq, w.cv, d_c, s)) != ESA_OK) return st;
+  if ((st = upper_solve(w.gk, dk, w.vd, d_c, s)) != ESA_OK) return st;
+  esa::emit_maps_kernel<<<(unsigned)std::min<int64_t>(4096, cdiv((int64_t)dq * d_c, 256)), 256, 0, s>>>(
+      w.cv, w.vd, hq, group, head_dim, d_c, w_q, w_k);
+  ESA_LAUNCH_CHECK("emit_maps_kernel");
+  return ok();
+}

@@ -276,6 +276,41 @@ def make_calibration(hq: int, hkv: int, d: int, n_tokens: int, rank: int, seed: 
     return q.reshape(n_tokens, hq, d), k.reshape(n_tokens, hkv, d)
 
 
+@dataclasses.dataclass(frozen=True)
+class FitWorkload:
+    """Offline fit of the compression maps: calibration tokens of one attention layer
+    (make_calibration: rank-`rank` latents plus noise), the compressed width d_c and the
+    fit's knobs (ridge, power iterations of the range finder)."""
+
+    name: str
+    hq: int
+    hkv: int
+    head_dim: int
+    n_tokens: int
+    rank: int
+    d_c: int
+    oversample: int
+    noise: float
+    ridge: float
+    power_iters: int
+    seed: int
+
+
+FIT_64K = FitWorkload("esa_fit_llama3_8b_calib65536_dc128", 32, 8, 128, 65536, 128, 128, 32, 0.1, 0.0, 8, 7)
+
+
+def make_fit_inputs(w: FitWorkload, device="cpu", n_tokens: Optional[int] = None) -> dict:
+    """Calibration queries q [n, hq, d] and keys k [n, hkv, d] in bf16 (make_calibration,
+    rounded), and the subspace iteration's Gaussian start omega [hkv * d, d_c +
+    oversample] (float64, its own generator, seed + 1)."""
+    n = n_tokens or w.n_tokens
+    q, k = make_calibration(w.hq, w.hkv, w.head_dim, n, w.rank, w.seed, w.noise)
+    gen = torch.Generator()
+    gen.manual_seed(w.seed + 1)
+    omega = torch.randn((w.hkv * w.head_dim, w.d_c + w.oversample), generator=gen, dtype=torch.float64)
+    return dict(q=q.to(torch.bfloat16).to(device), k=k.to(torch.bfloat16).to(device), omega=omega.to(device))
+
+
 def varlen_lengths(batch: int, n_max: int, n_min: int, seed: int) -> torch.Tensor:
     """Lengths of a variable-length decode batch: sequence 0 holds n_max tokens, the
     others a seeded uniform draw from [n_min, n_max]. Returns int64 [batch] (host)."""

@@ -227,3 +227,46 @@ def test_cca_rejects_bad_arguments(lib):
 def test_wait_selftest_rejects_out_of_range_limits(lib):
     assert lib.esa_wait_selftest(10, None) == _abi.ESA_ERR_INVALID_ARG
     assert lib.esa_wait_selftest(10 ** 12, None) == _abi.ESA_ERR_INVALID_ARG
+
+
+def test_fit_calls_reject_bad_arguments(lib):
+    # every rejection happens on the host, before a launch
+    before = lib.esa_launch_count()
+    g = lambda dt=1, n=1000, dim=512, x=FAKE, out=FAKE, ws=FAKE, nb=1 << 40: lib.esa_gram(x, dt, n, dim, out, ws, nb,
+                                                                                         None)
+    assert g(dt=0) == _abi.ESA_ERR_UNSUPPORTED                 # fp32 rows
+    assert g(dim=200) == _abi.ESA_ERR_UNSUPPORTED               # not a multiple of 128
+    assert g(n=0) == _abi.ESA_ERR_INVALID_ARG
+    assert g(x=None) == _abi.ESA_ERR_INVALID_ARG
+    assert g(x=FAKE + 2) == _abi.ESA_ERR_INVALID_ARG            # misaligned
+    assert g(out=None) == _abi.ESA_ERR_INVALID_ARG
+    assert g(nb=16) == _abi.ESA_ERR_WORKSPACE
+    f = lambda hq=32, hkv=8, d=128, dc=128, over=32, ridge=0.0, it=8, om=FAKE, nb=1 << 40, dt=1: lib.esa_fit_maps(
+        FAKE, 65536, FAKE, 65536, dt, hq, hkv, d, dc, over, ridge, it, om, FAKE, FAKE, FAKE, nb, None)
+    assert f(hq=30) == _abi.ESA_ERR_INVALID_ARG                 # not a multiple of hkv
+    assert f(d=40) == _abi.ESA_ERR_UNSUPPORTED                  # 8 * 40 = 320 is not a multiple of 128
+    assert f(dc=0) == _abi.ESA_ERR_UNSUPPORTED
+    assert f(dc=129) == _abi.ESA_ERR_UNSUPPORTED                # 129 + 32 > 160
+    assert f(dc=128, over=33) == _abi.ESA_ERR_UNSUPPORTED
+    assert f(over=-1) == _abi.ESA_ERR_UNSUPPORTED
+    assert f(ridge=-1.0) == _abi.ESA_ERR_INVALID_ARG
+    assert f(ridge=math.nan) == _abi.ESA_ERR_INVALID_ARG
+    assert f(it=65) == _abi.ESA_ERR_INVALID_ARG
+    assert f(om=None) == _abi.ESA_ERR_INVALID_ARG
+    assert f(nb=1024) == _abi.ESA_ERR_WORKSPACE
+    assert f(dt=0) == _abi.ESA_ERR_UNSUPPORTED
+    assert lib.esa_launch_count() == before
+
+
+def test_fit_workspace_sizes(lib):
+    # Gram partials: one fp64 [dim, dim] per slice of the rows (slices only when the
+    # upper triangle has fewer than 148 tiles); the fit adds its fp64 matrices
+    assert _abi.load().esa_gram_workspace_size(65536, 4096) == 4096 * 4096 * 8        # 528 tiles: one slice
+    assert _abi.load().esa_gram_workspace_size(65536, 1024) == 4 * 1024 * 1024 * 8    # 36 tiles: 4 slices
+    assert _abi.load().esa_gram_workspace_size(100, 1024) == 1 * 1024 * 1024 * 8      # one 128-row chunk
+    assert _abi.load().esa_gram_workspace_size(100, 1000) == 0
+    need = _abi.fit_workspace_size(65536, 65536, 32, 8, 128, 128, 32)
+    dq, dk, dc, l = 4096, 1024, 128, 160
+    fp64 = 8 * (dq * dq + 2 * dk * dk + 2 * dq * dk + 2 * dk * l + l * l + l * l + l * dc + dk * dc + dq * dc)
+    assert need >= fp64 + dq * dq * 8 and need <= fp64 + dq * dq * 8 + 13 * 256
+    assert _abi.fit_workspace_size(65536, 65536, 32, 8, 40, 128, 32) == 0
