@@ -1702,9 +1702,9 @@ esa_status_t chol_block(double* A, int64_t lda, int nb, unsigned site, cudaStrea
 esa_status_t trsm_block(const double* T, int64_t ldt, int nb, double* X, int64_t xr, int64_t xc, int64_t ncols,
                         int trans, cudaStream_t s) {
   if (ncols <= 0) return ESA_OK;
-  const size_t smem = (size_t)nb * esa::kTrsmCols * sizeof(double);
-  esa::trsm_block_kernel<<<(unsigned)cdiv(ncols, esa::kTrsmCols), esa::kTrsmCols, smem, s>>>(T, ldt, nb, X, xr, xc,
-                                                                                              ncols, trans);
+  const size_t smem = nb <= esa::kTrsmStageMax ? (size_t)nb * nb * sizeof(double) : 0;
+  esa::trsm_block_kernel<<<(unsigned)cdiv(ncols, esa::kTrsmCols), esa::kTrsmThreads, smem, s>>>(T, ldt, nb, X, xr,
+                                                                                                 xc, ncols, trans);
   ESA_LAUNCH_CHECK("trsm_block_kernel");
   return ESA_OK;
 }

@@ -21,6 +21,7 @@
 //   gemm64          C = alpha op(A) op(B) + beta C in fp64 (any strides)
 //   chol_block      Cholesky of one <= 160 x 160 diagonal block in shared memory (fp64)
 //   trsm_block      triangular solve with one <= 160 x 160 upper block, many right sides
+//                   (eight threads per right side)
 //   jacobi_eig      eigenvectors of a symmetric <= 160 x 160 matrix (one CTA), the
 //                   leading d' of them gathered in descending order of eigenvalue
 //   small helpers   trace, diagonal shift, GQA fold of Rq's columns, key-map expansion
@@ -307,15 +308,16 @@ __global__ void __launch_bounds__(256) chol_block_kernel(double* A, int64_t lda,
       }
       break;                                          // every thread reads the same d
     }
-    const double r = sqrt(d);
+    const double r = sqrt(d), inv = 1.0 / r;
     __syncthreads();                                  // all have read cs[k][k]
-    for (int j = k + threadIdx.x; j < nb; j += blockDim.x) cs[k * ld + j] = j == k ? r : cs[k * ld + j] / r;
+    for (int j = k + threadIdx.x; j < nb; j += blockDim.x) cs[k * ld + j] = j == k ? r : cs[k * ld + j] * inv;
     __syncthreads();
     // trailing update of the upper triangle: A[i][j] -= R[k][i] R[k][j], k < i <= j
-    const int m = nb - k - 1;
-    for (int e = threadIdx.x; e < m * m; e += blockDim.x) {
-      const int i = k + 1 + e / m, j = k + 1 + e % m;
-      if (j >= i) cs[i * ld + j] -= cs[k * ld + i] * cs[k * ld + j];
+    // (16 x 16 threads over (i, j), no division in the index arithmetic)
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    for (int i = k + 1 + ty; i < nb; i += 16) {
+      const double rki = cs[k * ld + i];
+      for (int j = i + tx; j < nb; j += 16) cs[i * ld + j] -= rki * cs[k * ld + j];
     }
     __syncthreads();
   }
@@ -330,33 +332,76 @@ __global__ void __launch_bounds__(256) chol_block_kernel(double* A, int64_t lda,
 // ------------------------------------------------------------------ triangular solve --
 // Solves, for the ncols right sides x_c (element i of side c at X[i * xr + c * xc]), in
 // place: trans = 1: R^T x = b (forward substitution), trans = 0: R x = b (back
-// substitution), with R the nb x nb upper block at T (row stride ldt, nb <= 160). A CTA
-// takes 64 right sides, one per thread, staged in shared memory; every thread reads the
-// same element of R at a time (a broadcast served by L1).
-constexpr int kTrsmCols = 64;
-constexpr uint32_t kTrsmSmem = kCholMax * kTrsmCols * sizeof(double);
-__global__ void __launch_bounds__(kTrsmCols) trsm_block_kernel(const double* __restrict__ T, int64_t ldt, int nb,
-                                                                 double* X, int64_t xr, int64_t xc, int64_t ncols,
-                                                                 int trans) {
-  extern __shared__ double bs[];                     // [nb][64]
-  const int64_t c = (int64_t)blockIdx.x * kTrsmCols + threadIdx.x;
+// substitution), with R the nb x nb upper block at T (row stride ldt, nb <= 160).
+// Eight threads of a warp share a right side: thread r holds rows r, r + 8, ... in
+// registers; at step i the owner of row i forms x_i, a shuffle hands it to the other
+// seven, and each updates its own rows. A CTA takes 32 right sides (256 threads); R is
+// staged in shared memory when nb <= 128 (else read as broadcasts through L1).
+constexpr int kTrsmCols = 32;
+constexpr int kTrsmThreads = 8 * kTrsmCols;
+constexpr int kTrsmRowsPer = kCholMax / 8;            // rows a thread holds (nb <= 160)
+constexpr int kTrsmStageMax = 128;
+constexpr uint32_t kTrsmSmem = kTrsmStageMax * kTrsmStageMax * sizeof(double);
+__global__ void __launch_bounds__(kTrsmThreads, 1) trsm_block_kernel(const double* __restrict__ T, int64_t ldt, int nb,
+                                                                    double* X, int64_t xr, int64_t xc, int64_t ncols,
+                                                                    int trans) {
+  extern __shared__ double tsm[];
+  const bool staged = nb <= kTrsmStageMax;
+  const double* tr = staged ? tsm : T;               // R, row stride tl
+  const int64_t tl = staged ? nb : ldt;
+  if (staged)
+    for (int e = threadIdx.x; e < nb * nb; e += blockDim.x) tsm[e] = T[(e / nb) * ldt + e % nb];
+  const int r = threadIdx.x & 7, lane = threadIdx.x & 31;
+  const int src0 = lane & ~7;                        // lane of this side's thread 0
+  const int64_t c = (int64_t)blockIdx.x * kTrsmCols + (threadIdx.x >> 3);
   const bool live = c < ncols;
-  for (int i = 0; i < nb; ++i) bs[i * kTrsmCols + threadIdx.x] = live ? X[i * xr + c * xc] : 0.0;
+  double b[kTrsmRowsPer];
+#pragma unroll
+  for (int t = 0; t < kTrsmRowsPer; ++t) {
+    const int j = r + 8 * t;
+    b[t] = (live && j < nb) ? X[j * xr + c * xc] : 0.0;
+  }
+  __syncthreads();
   if (trans) {
     for (int i = 0; i < nb; ++i) {
-      const double x = bs[i * kTrsmCols + threadIdx.x] / __ldg(T + i * ldt + i);
-      bs[i * kTrsmCols + threadIdx.x] = x;
-      for (int j = i + 1; j < nb; ++j) bs[j * kTrsmCols + threadIdx.x] -= __ldg(T + i * ldt + j) * x;
+      double x = 0.0;
+#pragma unroll
+      for (int t = 0; t < kTrsmRowsPer; ++t)
+        if (r + 8 * t == i) {
+          b[t] = b[t] / tr[i * tl + i];
+          x = b[t];
+        }
+      x = __shfl_sync(0xffffffffu, x, src0 + (i & 7));
+#pragma unroll
+      for (int t = 0; t < kTrsmRowsPer; ++t) {
+        const int j = r + 8 * t;
+        if (j > i && j < nb) b[t] -= tr[i * tl + j] * x;
+      }
     }
   } else {
     for (int i = nb - 1; i >= 0; --i) {
-      const double x = bs[i * kTrsmCols + threadIdx.x] / __ldg(T + i * ldt + i);
-      bs[i * kTrsmCols + threadIdx.x] = x;
-      for (int j = 0; j < i; ++j) bs[j * kTrsmCols + threadIdx.x] -= __ldg(T + j * ldt + i) * x;
+      double x = 0.0;
+#pragma unroll
+      for (int t = 0; t < kTrsmRowsPer; ++t)
+        if (r + 8 * t == i) {
+          b[t] = b[t] / tr[i * tl + i];
+          x = b[t];
+        }
+      x = __shfl_sync(0xffffffffu, x, src0 + (i & 7));
+#pragma unroll
+      for (int t = 0; t < kTrsmRowsPer; ++t) {
+        const int j = r + 8 * t;
+        if (j < i) b[t] -= tr[j * tl + i] * x;
+      }
     }
   }
-  if (live)
-    for (int i = 0; i < nb; ++i) X[i * xr + c * xc] = bs[i * kTrsmCols + threadIdx.x];
+  if (live) {
+#pragma unroll
+    for (int t = 0; t < kTrsmRowsPer; ++t) {
+      const int j = r + 8 * t;
+      if (j < nb) X[j * xr + c * xc] = b[t];
+    }
+  }
 }
 
 // ------------------------------------------------------------------ Jacobi eigensolver --
@@ -369,7 +414,8 @@ __global__ void __launch_bounds__(kTrsmCols) trsm_block_kernel(const double* __r
 // are a sweep, and sweeps stop when the off-diagonal part is below 1e-14 of the whole.
 // Output: zsel [l, d] = the eigenvectors of the d largest eigenvalues, as columns in
 // descending order of eigenvalue (ties to the lower index). One CTA of 512 threads; H
-// lives in shared memory, Z [L, L] (global scratch) accumulates the rotations.
+// lives in shared memory, Z [L, L] (global scratch, stored transposed so that a
+// rotation's two columns are contiguous) accumulates the rotations.
 constexpr int kJacobiThreads = 512;
 constexpr uint32_t kJacobiSmem = (kCholMax * (kCholMax + 1) + 4 * (kCholMax / 2) + kCholMax) * sizeof(double);
 __global__ void __launch_bounds__(kJacobiThreads) jacobi_eig_kernel(const double* __restrict__ H, int l, double* Z,
@@ -387,7 +433,7 @@ __global__ void __launch_bounds__(kJacobiThreads) jacobi_eig_kernel(const double
   for (int e = threadIdx.x; e < L * L; e += blockDim.x) {
     const int i = e / L, j = e % L;
     h[i * ld + j] = (i < l && j < l) ? H[i * l + j] : 0.0;
-    Z[e] = i == j ? 1.0 : 0.0;
+    Z[e] = i == j ? 1.0 : 0.0;                       // stored transposed: Z[p * L + i] = z_ip
   }
   __syncthreads();
   const int P = L / 2;
@@ -461,9 +507,9 @@ __global__ void __launch_bounds__(kJacobiThreads) jacobi_eig_kernel(const double
         const double hp = h[i * ld + p], hq = h[i * ld + q];
         h[i * ld + p] = c * hp - sn * hq;
         h[i * ld + q] = sn * hp + c * hq;
-        const double zp = Z[i * L + p], zq = Z[i * L + q];
-        Z[i * L + p] = c * zp - sn * zq;
-        Z[i * L + q] = sn * zp + c * zq;
+        const double zp = Z[(int64_t)p * L + i], zq = Z[(int64_t)q * L + i];
+        Z[(int64_t)p * L + i] = c * zp - sn * zq;
+        Z[(int64_t)q * L + i] = sn * zp + c * zq;
       }
       __syncthreads();
     }
@@ -476,7 +522,7 @@ __global__ void __launch_bounds__(kJacobiThreads) jacobi_eig_kernel(const double
     int rank = 0;
     for (int j = 0; j < l; ++j) rank += (red[j] > red[i]) || (red[j] == red[i] && j < i);
     if (rank < d)
-      for (int r = 0; r < l; ++r) zsel[r * d + rank] = Z[r * L + i];
+      for (int r = 0; r < l; ++r) zsel[r * d + rank] = Z[(int64_t)i * L + r];
   }
 }
 
