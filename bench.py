@@ -359,17 +359,17 @@ def run_ours(args):
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_host.numel() * out_host.element_size()
 
-    def e2e_step():
-        # the graph reads the input buffers it was captured on: copy the host inputs there
-        for n in ("q", "k", "v"):
-            inp[n].copy_(host[n], non_blocking=True)
-        graph.replay()
-        out_host.copy_(pf.out, non_blocking=True)
-
-    e_ms, e_total = time_steps(e2e_step, args.e2e_steps, 1, flush, dist_max)
+    # the library's own host-buffer entry: chunk by chunk, inputs up on one copy stream
+    # and outputs back on another, overlapping the compute; one CUDA graph per step
+    e2e_graph = pipeline.graph_of(lambda: pf.run_from_host(host["q"], host["k"], host["v"], inp["q"], inp["k"],
+                                                           inp["v"], inp["wq"], inp["wk"], out_host))
+    e_ms, e_total = time_steps(e2e_graph.replay, args.e2e_steps, 1, flush, dist_max)
     e2e = {"value": round(world * tokens * args.e2e_steps / (e_total / 1e3), 1), "unit": "tok/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    del host, out_host
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": round(e_total / args.e2e_steps, 3),
+           "path": "EsaPrefill.run_from_host: per-chunk host-to-device copies on one stream, "
+                   "device-to-host copies on another, overlapping the compute"}
+    del host, out_host, e2e_graph
 
     line = {"metric": METRIC, "value": round(value, 1), "unit": "tok/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 3), "higher_is_better": True,

@@ -231,10 +231,14 @@ SelWs carve_select(void* ws, int32_t batch, int32_t lq, int64_t n_mid, ScorePath
   return w;
 }
 
-// Cluster size of the selection kernel: 16 CTAs when `batch` such clusters (one per
-// sequence) can be resident at once, else the portable 8. Occupancy is queried once per
-// device.
-int select_cluster_size(int32_t batch) {
+// Cluster size of the selection kernel: 16 CTAs only when the middle overflows the
+// shared memory of 8 (8 x kSelUCap keys) and `batch` such clusters (one per sequence)
+// can be resident at once; else the portable 8. A 16-CTA cluster needs 16 free SMs in
+// one GPC, which a chunked prefill's attention (128 CTAs, one per SM) does not leave:
+// its next chunk's selection then waited for the attention to end (8-CTA clusters:
+// 32K prefill 6.05 -> 5.65 ms). Occupancy is queried once per context.
+int select_cluster_size(int32_t batch, int64_t n_mid) {
+  if (n_mid <= (int64_t)8 * esa::kSelUCap) return 8;
   static const char what = 0;
   intptr_t max16 = -1;          // -1: 16-CTA clusters unavailable
   const esa_status_t st = per_context(&what, &max16, [](intptr_t* v) {
@@ -526,7 +530,9 @@ esa_status_t compress_packed_impl(const void* x, int64_t rows, int64_t x_row_str
   int cl = 8;
   esa_status_t st = pk_cluster_size(&cl);
   if (st != ESA_OK) return st;
-  if (K % (64 * cl)) cl = 8;
+  // small calls (a chunk's keys or queries, a decode step) take 8-CTA clusters, which
+  // fit beside a running attention kernel (a 16-CTA cluster needs 16 free SMs in a GPC)
+  if (K % (64 * cl) || rows <= 4096) cl = 8;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   CUtensorMap tw;
   st = make_tmap_kmajor_bf16(&tw, packed, (uint64_t)K, 256, (uint64_t)K);
@@ -789,7 +795,7 @@ esa_status_t score_select_impl(const float* q_c, const float* k_c, int32_t batch
         return sa;
       });
       if (st != ESA_OK) return st;
-      const int cl = select_cluster_size((int32_t)vb);
+      const int cl = select_cluster_size((int32_t)vb, r.n_mid);
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3((unsigned)cl, (unsigned)vb, 1);
       cfg.blockDim = dim3(esa::kSelThreads);

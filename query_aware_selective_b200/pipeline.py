@@ -208,12 +208,17 @@ class EsaPrefill:
         self.front(ci, c0, lq, q, k)
         self.attend(ci, c0, lq, q, k, v, attn_events)
 
-    def run(self, q, k, v, wq, wk, attn_events=None, external_events=False):
+    def run(self, q, k, v, wq, wk, attn_events=None, external_events=False, chunk_ready=None,
+            on_attended=None):
         """q [B, N, Hq, D], k, v [B, N, Hkv, D] (device), wq, wk [Hq*D, d'].
         attn_events: optional list that receives one (start, end) CUDA event pair per
         attention launch (external_events: made to be captured in a graph). Returns
         the output [B, N, Hq, D]. The weights are packed for the tensor-core
         compression at the start of every run.
+        chunk_ready: optional per-chunk CUDA events; work that reads chunk j's rows of
+        q, k, v (and so every later chunk's) waits for event j, so the rows may still be
+        arriving when run() is called. on_attended(ci, c0, lq): called after chunk ci's
+        attention is issued (on the current stream), e.g. to copy its output out.
 
         Three streams: the chunks' key compressions run in order on one, their query
         compression and selection in order on another (chunk j's selection waiting for
@@ -237,6 +242,8 @@ class EsaPrefill:
             nonlocal issued, last_done
             while issued <= upto:
                 b0, b1 = issued * kbatch, min(len(chunks), (issued + 1) * kbatch)
+                if chunk_ready is not None:
+                    self.kside.wait_event(chunk_ready[b1 - 1])
                 with torch.cuda.stream(self.kside):
                     self.compress_keys(chunks[b0][0], chunks[b1 - 1][0] + chunks[b1 - 1][1] - chunks[b0][0], k)
                     last_done = torch.cuda.Event()
@@ -253,18 +260,65 @@ class EsaPrefill:
             with torch.cuda.stream(self.side):
                 if wait is not None:
                     self.side.wait_event(wait)
+                if chunk_ready is not None:
+                    self.side.wait_event(chunk_ready[ci])
                 self.front(ci, c0, lq, q)
                 done.record()
-            main.wait_event(done)
+            main.wait_event(done)                  # (after chunk_ready[ci]: the rows up to c1 are in)
             ev = None
             if attn_events is not None:
                 ev = (_timing_event(external_events), _timing_event(external_events))
                 attn_events.append(ev)
             self.attend(ci, c0, lq, q, k, v, ev)
+            if on_attended is not None:
+                on_attended(ci, c0, lq)
         issue_batches(n_batches - 1)               # the rest complete the compressed cache
         main.wait_stream(self.side)
         main.wait_stream(self.kside)
         return self.out
+
+
+    def run_from_host(self, q_host, k_host, v_host, q, k, v, wq, wk, out_host):
+        """The prefill with its inputs in pinned host memory and its output returned to
+        pinned host memory, the copies overlapping the compute: chunk by chunk, the
+        chunk's rows of q, k, v go up on one copy stream (one copy per tensor and chunk)
+        and each chunk's output comes back on another as soon as its attention is done.
+        q_host, k_host, v_host: pinned host tensors shaped like the device buffers q, k,
+        v, which receive them; out_host: pinned host tensor like the output. Works for
+        batch 1 (a chunk's rows are then contiguous). Returns out_host; the copies are
+        complete once the current stream reaches this point."""
+        if self.batch != 1:
+            raise ValueError("run_from_host streams chunks of one sequence (batch 1)")
+        main = torch.cuda.current_stream()
+        cin, cout = self._copy_streams()
+        cin.wait_stream(main)
+        cout.wait_stream(main)
+        ready = []
+        with torch.cuda.stream(cin):
+            for c0, lq in self.chunks():
+                for dev, host in ((q, q_host), (k, k_host), (v, v_host)):
+                    dev[:, c0:c0 + lq].copy_(host[:, c0:c0 + lq], non_blocking=True)
+                e = torch.cuda.Event()
+                e.record()
+                ready.append(e)
+
+        def copy_out(ci, c0, lq):
+            e = torch.cuda.Event()
+            e.record()
+            cout.wait_event(e)
+            with torch.cuda.stream(cout):
+                out_host[:, c0:c0 + lq].copy_(self.out[:, c0:c0 + lq], non_blocking=True)
+
+        self.run(q, k, v, wq, wk, chunk_ready=ready, on_attended=copy_out)
+        main.wait_stream(cin)
+        main.wait_stream(cout)
+        return out_host
+
+    def _copy_streams(self):
+        if not hasattr(self, "_cin"):
+            self._cin = torch.cuda.Stream(device=self.device)
+            self._cout = torch.cuda.Stream(device=self.device)
+        return self._cin, self._cout
 
 
 class EsaDecode:
