@@ -1229,8 +1229,21 @@ esa_status_t moba_gate_launch(const MobaWs& w, const void* q, const void* k, int
   esa::moba_mean_kernel<__nv_bfloat16><<<dim3(nb, heads, batch), 256, 0, s>>>(
       static_cast<const __nv_bfloat16*>(k), seq, heads, 128, block, 0, nb, w.kbar);
   ESA_LAUNCH_CHECK("moba_mean_kernel");
-  esa::moba_gate_kernel<__nv_bfloat16, 128><<<dim3((unsigned)cdiv(seq, 128), heads, batch), 128, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(q), w.kbar, seq, heads, block, nb, topk, blocks_out);
+  const dim3 ggrid((unsigned)cdiv(seq, 128), heads, batch);
+  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
+  if (topk <= 1)
+    esa::moba_gate_kernel<__nv_bfloat16, 128, 1><<<ggrid, 128, 0, s>>>(qb, w.kbar, seq, heads, block, nb, topk, blocks_out);
+  else if (topk <= 2)
+    esa::moba_gate_kernel<__nv_bfloat16, 128, 2><<<ggrid, 128, 0, s>>>(qb, w.kbar, seq, heads, block, nb, topk, blocks_out);
+  else if (topk <= 3)
+    esa::moba_gate_kernel<__nv_bfloat16, 128, 3><<<ggrid, 128, 0, s>>>(qb, w.kbar, seq, heads, block, nb, topk, blocks_out);
+  else if (topk <= 4)
+    esa::moba_gate_kernel<__nv_bfloat16, 128, 4><<<ggrid, 128, 0, s>>>(qb, w.kbar, seq, heads, block, nb, topk, blocks_out);
+  else if (topk <= 8)
+    esa::moba_gate_kernel<__nv_bfloat16, 128, 8><<<ggrid, 128, 0, s>>>(qb, w.kbar, seq, heads, block, nb, topk, blocks_out);
+  else
+    esa::moba_gate_kernel<__nv_bfloat16, 128, esa::kMobaMaxTopk><<<ggrid, 128, 0, s>>>(qb, w.kbar, seq, heads, block,
+                                                                                         nb, topk, blocks_out);
   ESA_LAUNCH_CHECK("moba_gate_kernel");
   return ESA_OK;
 }

@@ -64,8 +64,10 @@ __global__ void __launch_bounds__(256) moba_mean_kernel(const T* __restrict__ k,
 // grid (ceil(seq / 128), H, B), 128 threads; thread = query position. The query row
 // lives in registers; block means are staged 32 blocks at a time in shared memory and
 // read as broadcasts. Kept list: insertion that never moves an element past an equal
-// one, visiting blocks in ascending order -> ties go to the lower block.
-template <typename T, int D>
+// one, visiting blocks in ascending order -> ties go to the lower block. TK >= topk is
+// the kept list's compile-time length: the insertion runs over TK entries for every
+// block, so the host picks the smallest instantiation that holds topk.
+template <typename T, int D, int TK>
 __global__ void __launch_bounds__(128) moba_gate_kernel(const T* __restrict__ q, const float* __restrict__ kbar,
                                                         int64_t seq, int heads, int block, int n_blocks, int topk,
                                                         int16_t* __restrict__ blocks_out) {
@@ -83,10 +85,10 @@ __global__ void __launch_bounds__(128) moba_gate_kernel(const T* __restrict__ q,
 #pragma unroll
     for (int e = 0; e < D; e += 16 / sizeof(T)) load_vec(qp + e, &qv[e]);
   }
-  float vals[kMobaMaxTopk];
-  int ids[kMobaMaxTopk];
+  float vals[TK];
+  int ids[TK];
 #pragma unroll
-  for (int i = 0; i < kMobaMaxTopk; ++i) { vals[i] = -INFINITY; ids[i] = -1; }
+  for (int i = 0; i < TK; ++i) { vals[i] = -INFINITY; ids[i] = -1; }
   const float* kbh = kbar + ((int64_t)b * heads + h) * n_blocks * D;
   for (int c0 = 0; c0 < cur_max; c0 += CB) {
     __syncthreads();
@@ -111,7 +113,7 @@ __global__ void __launch_bounds__(128) moba_gate_kernel(const T* __restrict__ q,
       float v = acc;
       int id = c0 + c;
 #pragma unroll
-      for (int i = 0; i < kMobaMaxTopk; ++i) {
+      for (int i = 0; i < TK; ++i) {
         if (i < topk && v > vals[i]) {
           const float tv = vals[i]; vals[i] = v; v = tv;
           const int ti = ids[i]; ids[i] = id; id = ti;
@@ -122,9 +124,9 @@ __global__ void __launch_bounds__(128) moba_gate_kernel(const T* __restrict__ q,
   if (!valid) return;
   // ascending block order: small unrolled exchange sort on the kept ids (-1 last)
 #pragma unroll
-  for (int i = 0; i < kMobaMaxTopk; ++i)
+  for (int i = 0; i < TK; ++i)
 #pragma unroll
-    for (int j = 0; j + 1 < kMobaMaxTopk - i; ++j) {
+    for (int j = 0; j + 1 < TK - i; ++j) {
       const int a = ids[j], c = ids[j + 1];
       const bool swap = (a < 0 && c >= 0) || (a >= 0 && c >= 0 && c < a);
       ids[j] = swap ? c : a;
@@ -133,7 +135,7 @@ __global__ void __launch_bounds__(128) moba_gate_kernel(const T* __restrict__ q,
   int16_t* out = blocks_out + ((b * seq + p) * heads + h) * (topk + 1);
   int n = 0;
 #pragma unroll
-  for (int i = 0; i < kMobaMaxTopk; ++i)
+  for (int i = 0; i < TK; ++i)
     if (i < topk && ids[i] >= 0) out[n++] = (int16_t)ids[i];
   out[n++] = (int16_t)cur;
   for (; n < topk + 1; ++n) out[n] = -1;
