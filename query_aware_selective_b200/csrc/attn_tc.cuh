@@ -10,10 +10,10 @@
 // m is the running row maximum used for the exponentials; it is raised (and O, l
 // rescaled in place) only when a tile's maximum exceeds it by more than 2^8, so most
 // tiles skip the rescale and P stays <= 2^8 (exact softmax either way: o = O / l).
-// Roles (608 threads): warps 0-15 softmax (warp w owns TMEM lanes 32 (w % 4) .. + 31,
-// i.e. rows, and key columns 32 (w / 4) .. + 31: four threads per row, exchanging the
-// row max and sum through shared memory), warp 16 issues the MMAs (one lane), warp 17
-// loads Q and the K tiles, warp 18 loads the V tiles.
+// Roles (352 threads): warps 0-7 softmax (warp w owns TMEM lanes 32 (w % 4) .. + 31,
+// i.e. rows, and key columns 64 (w / 4) .. + 63: two threads per row, exchanging the
+// row max and sum through shared memory), warp 8 issues the MMAs (one lane), warp 9
+// loads Q and the K tiles, warp 10 loads the V tiles.
 // Tiles come in by TMA straight into the 128-byte swizzled layout the MMA descriptors
 // name, and the "full" barriers complete on the transaction count. A tile whose 128
 // keys are consecutive tokens (initial tokens, local window, chunk, MoBA blocks) is
@@ -53,7 +53,16 @@
 
 namespace esa {
 
-constexpr int kTcSplit = 4;                                  // softmax threads per row
+// Two softmax threads per row, 64 key columns each: the two warps of a row group on a
+// sub-partition run in lockstep (they agree on the row maximum every tile), and with
+// 64 independent exponentials per thread the pair keeps the MUFU busy where four
+// warps of 32 columns stalled together (kTcSplit = 4: ESA chunk attention 72.3 ->
+// 69.4 us at 2, MoBA 64K 9.27 -> 8.78 ms). 11 warps leave 168 registers a thread.
+#ifndef KTC_SPLIT
+#define KTC_SPLIT 2
+#endif
+constexpr int kTcSplit = KTC_SPLIT;                          // softmax threads per row (2 or 4)
+static_assert(kTcSplit == 4 || kTcSplit == 2, "64 or 32 key columns per softmax thread");
 constexpr int kTcThreads = (4 * kTcSplit + 3) * 32;
 constexpr int kTcMmaWarp = 4 * kTcSplit, kTcKWarp = kTcMmaWarp + 1, kTcVWarp = kTcMmaWarp + 2;
 constexpr int kTcRows = 128;
@@ -286,8 +295,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- softmax (rows)
-    constexpr int HC = kTcKeys / kTcSplit;     // key columns per thread
-    static_assert(HC == 32, "one 32-column TMEM load and two 8-column stores per thread and tile");
+    constexpr int HC = kTcKeys / kTcSplit;     // key columns per thread (32 or 64)
+    // HC columns of 32-bit TMEM data at addr (HC / 32 loads of 32 columns)
+    auto ld_cols = [&](uint32_t addr, float* dst) {
+#pragma unroll
+      for (int c = 0; c < HC / 32; ++c) tmem_ld32(addr + c * 32, dst + c * 32);
+    };
+    auto st_cols = [&](uint32_t addr, const float* src) {
+#pragma unroll
+      for (int c = 0; c < HC / 32; ++c) tmem_st32(addr + c * 32, src + c * 32);
+    };
+    // half a tile's P of this thread: HC / 4 packed bf16 pairs
+    auto st_p = [&](uint32_t addr, const uint32_t* pk) {
+      if constexpr (HC == 32) tmem_st8(addr, pk);
+      else tmem_st16(addr, pk);
+    };
     constexpr uint32_t kGroup = 32 * kTcSplit; // threads sharing a row set (named barrier size)
     const int quad = warp & 3, part = warp >> 2;
     const int r = quad * 32 + lane;            // row = TMEM lane
@@ -313,7 +335,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (got) tc_fence_after();
       return got;
     };
-    auto load_s = [&](int j, float* dst) { tmem_ld32(lane_base + (j % kTcSBufs) * 128 + part * HC, dst); };
+    auto load_s = [&](int j, float* dst) { ld_cols(lane_base + (j % kTcSBufs) * 128 + part * HC, dst); };
     // Masked scores become -inf; returns this part's maximum in log2 units (scale > 0).
     auto mask_max = [&](int rem, float* v) -> float {
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -349,12 +371,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const bool done = mbar_wait_warp(&sm.pv_full[(j - 1) % 3], ((j - 1) / 3) & 1, abort_flag, 110);
         if (!(ok = bar_all(row_bar, kGroup, done))) return false;
         tc_fence_after();
-        float ov[32];
-        tmem_ld32(o_addr, ov);
+        float ov[HC];
+        ld_cols(o_addr, ov);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-        tmem_st32(o_addr, ov);
+        for (int e = 0; e < HC; ++e) ov[e] *= alpha;
+        st_cols(o_addr, ov);
         tmem_wait_st();
         l *= alpha;
       }
@@ -363,13 +385,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     };
     // One tile, software-pipelined: cur holds S_j (masked, m decided). P_j is formed in
     // two halves (MUFU exp2); S_{j+1} is loaded into nxt after the first half (when half
-    // of cur is no longer needed, which keeps the live registers within the 96 a thread
+    // of cur is no longer needed, which keeps the live registers within what a thread
     // has here), and its maximum is taken between the exponentials of the second half,
     // so the ALU reduction hides behind the exp2 unit. P_j goes to
     // the TMEM buffer over S_j (every warp of the row group has read its part of S_j,
-    // the barrier in decide), keys 32 part .. + 31 to columns 16 part .. + 15. Then the
-    // group decides m for tile j + 1. Returns false when there is no next tile or the
-    // group has to stop.
+    // the barrier in decide), keys HC part .. + HC - 1 to columns HC / 2 part .. +
+    // HC / 2 - 1. Then the group decides m for tile j + 1. Returns false when there is
+    // no next tile or the group has to stop.
     auto step = [&](int j, float* cur, float* nxt) -> bool {
       const int s = j % kTcSBufs;
       const bool has_next = j + 1 < nt;
@@ -378,7 +400,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const float m_use = m == -INFINITY ? 0.f : m;
       const float2 scale2 = make_float2(sl2, sl2), shift2 = make_float2(-m_use, -m_use);
       float2 ls2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      uint32_t pk[8];
+      uint32_t pk[HC / 4];
       // P goes to the MMA as bf16, rounded to nearest (unbiased, so l may add the
       // unrounded values)
       auto pair = [&](int e) -> uint32_t {
@@ -390,7 +412,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       };
 #pragma unroll
       for (int e = 0; e < HC / 2; e += 2) pk[e / 2] = pair(e);
-      tmem_st8(lane_base + s * 128 + part * 16, pk);
+      st_p(lane_base + s * 128 + part * (HC / 2), pk);
       float mx_n = -INFINITY;
       if (got_n) {
         load_s(j + 1, nxt);
@@ -413,7 +435,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int e = HC / 2; e < HC; e += 2) pk[(e - HC / 2) / 2] = pair(e);
         if (got_n) mx_n = mask_max(rem_n, nxt);
       }
-      tmem_st8(lane_base + s * 128 + part * 16 + 8, pk);
+      st_p(lane_base + s * 128 + part * (HC / 2) + HC / 4, pk);
       const float2 l2 = __fadd2_rn(ls2[0], ls2[1]);
       l += l2.x + l2.y;
       tmem_wait_st();
@@ -453,7 +475,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (ok) {
       tc_fence_after();
       float o[HC];
-      tmem_ld32(o_addr, o);
+      ld_cols(o_addr, o);
       tmem_wait_ld();
       prob.store(r, part * HC, o, m, l_row);
     }
