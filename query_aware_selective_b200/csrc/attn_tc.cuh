@@ -57,7 +57,8 @@ namespace esa {
 // sub-partition run in lockstep (they agree on the row maximum every tile), and with
 // 64 independent exponentials per thread the pair keeps the MUFU busy where four
 // warps of 32 columns stalled together (kTcSplit = 4: ESA chunk attention 72.3 ->
-// 69.4 us at 2, MoBA 64K 9.27 -> 8.78 ms). 11 warps leave 168 registers a thread.
+// 69.4 us at 2, MoBA 64K 9.27 -> 8.78 ms; one thread per row, with no exchange at
+// all, measured slower: 74.5 us). 11 warps leave 168 registers a thread.
 #ifndef KTC_SPLIT
 #define KTC_SPLIT 2
 #endif
@@ -301,10 +302,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int c = 0; c < HC / 32; ++c) tmem_ld32(addr + c * 32, dst + c * 32);
     };
-    auto st_cols = [&](uint32_t addr, const float* src) {
-#pragma unroll
-      for (int c = 0; c < HC / 32; ++c) tmem_st32(addr + c * 32, src + c * 32);
-    };
     // half a tile's P of this thread: HC / 4 packed bf16 pairs
     auto st_p = [&](uint32_t addr, const uint32_t* pk) {
       if constexpr (HC == 32) tmem_st8(addr, pk);
@@ -316,6 +313,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t o_addr = lane_base + kTmemO + part * HC;
     const uint32_t row_bar = 1 + quad;         // named barrier of the kTcSplit warps of this quadrant
+    // O *= alpha for this thread's columns, 32 at a time (few live registers)
+    auto rescale_o = [&](float alpha) {
+#pragma unroll 1
+      for (int c = 0; c < HC / 32; ++c) {
+        float ov[32];
+        tmem_ld32(o_addr + c * 32, ov);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+        tmem_st32(o_addr + c * 32, ov);
+      }
+      tmem_wait_st();
+    };
     if constexpr (HasPrefetch<Problem>::value) prob.prefetch(r, part * (kTcD / kTcSplit));
     const int64_t lim = prob.limit(r);
     const float sl2 = prob.scale_log2();
@@ -371,13 +381,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const bool done = mbar_wait_warp(&sm.pv_full[(j - 1) % 3], ((j - 1) / 3) & 1, abort_flag, 110);
         if (!(ok = bar_all(row_bar, kGroup, done))) return false;
         tc_fence_after();
-        float ov[HC];
-        ld_cols(o_addr, ov);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < HC; ++e) ov[e] *= alpha;
-        st_cols(o_addr, ov);
-        tmem_wait_st();
+        rescale_o(alpha);
         l *= alpha;
       }
       m = m_new;
