@@ -110,14 +110,16 @@ __device__ __forceinline__ void gather_tile(uint32_t dst, const CUtensorMap* tm,
   tma_gather4(d + kBlkBytes, tm, 64, r[0], r[1], r[2], r[3], bar);
 }
 
-// One loader warp streams the key tiles of one operand (K or V) through its NST
-// stages (tile j in stage j % NST, the barrier's j / NST-th phase). The rows of tile j + 1 are looked up (4 per lane, consecutive keys, so a
-// gathered index list is read coalesced) while tile j waits for its stage.
+// One loader warp streams the key tiles j0 .. j0 + nt - 1 of one operand (K or V)
+// through its NST stages (the u-th of them, tile j0 + u, in stage u % NST, the
+// barrier's u / NST-th phase). The rows of the next tile are looked up (4 per lane,
+// consecutive keys, so a gathered index list is read coalesced) while the current one
+// waits for its stage.
 template <int NST, class Problem>
 __device__ __forceinline__ void stream_kv(const Problem& prob, const CUtensorMap* tm_rows, const CUtensorMap* tm_box,
                                           const CUtensorMap* tm_staged, uint32_t stage0, uint64_t* full,
                                           uint64_t* empty, int nt, int64_t n_keys, int lane,
-                                          volatile int* abort_flag, unsigned site) {
+                                          volatile int* abort_flag, unsigned site, int j0 = 0) {
   int32_t cur[4], nxt[4];
   auto fetch = [&](int j, int32_t* out) {
 #pragma unroll
@@ -129,18 +131,18 @@ __device__ __forceinline__ void stream_kv(const Problem& prob, const CUtensorMap
   if (nt == 0) return;
   const int32_t fallback = prob.kv_row(0);
   int by = 0, bz = 0;
-  int box_next = prob.kv_box(0, &by, &bz);        // 0: gather, 1: cache box, 2: staged box
-  if (!box_next) fetch(0, nxt);
-  for (int j = 0; j < nt; ++j) {
-    const int s = j % NST;
-    const int ph = (j / NST) & 1;
+  int box_next = prob.kv_box(j0, &by, &bz);       // 0: gather, 1: cache box, 2: staged box
+  if (!box_next) fetch(j0, nxt);
+  for (int u = 0; u < nt; ++u) {
+    const int s = u % NST;
+    const int ph = (u / NST) & 1;
     const int box = box_next;
     const int y = by, z = bz;
 #pragma unroll
     for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
-    if (j + 1 < nt) {
-      box_next = prob.kv_box(j + 1, &by, &bz);
-      if (!box_next) fetch(j + 1, nxt);
+    if (u + 1 < nt) {
+      box_next = prob.kv_box(j0 + u + 1, &by, &bz);
+      if (!box_next) fetch(j0 + u + 1, nxt);
     }
     bool ok = mbar_wait(&empty[s], ph ^ 1, abort_flag, site);
     if (!__all_sync(0xffffffffu, ok)) return;
@@ -509,8 +511,9 @@ struct EsaTcProblem {
   int b, g, tile, cnt, list;
   int64_t n_prior, nk;
 
-  __device__ bool setup() {
-    tile = blockIdx.x;
+  __device__ bool setup() { return setup_at(blockIdx.x); }
+  __device__ bool setup_at(int t) {
+    tile = t;
     g = blockIdx.y;
     b = blockIdx.z;
     list = lists > 1 ? b * lists + g : b;

@@ -249,6 +249,8 @@ def test_sparse_attn_decode_parity(batch, n_cap, hq, hkv, n_init, window, topk):
     (2, 64, 700, 0, 4, 4, 16, 256, 64),           # first chunk: causal only
     (1, 512, 5000, 4488, 32, 8, 128, 2048, 1024), # a full chunk, several key tiles
     (1, 96, 4000, 333, 16, 4, 128, 512, 2048),    # short middle: full causal attention
+    (10, 64, 1500, 1000, 32, 8, 16, 256, 256),    # 80 tile pairs: no key split
+    (5, 64, 2500, 2000, 32, 8, 64, 512, 512),     # 40 tile pairs: three key parts per pair
 ])
 def test_sparse_attn_tensor_core_parity(batch, lq, n_cap, c0, hq, hkv, n_init, window, topk):
     p = qas.params(n_init, window, topk, 2, 10.0)
@@ -258,6 +260,8 @@ def test_sparse_attn_tensor_core_parity(batch, lq, n_cap, c0, hq, hkv, n_init, w
     _, (m0, m1), _ = oesa.regions(c0, c0 + lq, n_init, window)
     idx, cnt = synthetic.random_index_list(batch, m0, m1, topk, seed=24)
     o, lse = qas.sparse_attn(q.to(DEV), k.to(DEV), v.to(DEV), c0, idx.to(DEV), cnt.to(DEV), p, want_lse=True)
+    o2, lse2 = qas.sparse_attn(q.to(DEV), k.to(DEV), v.to(DEV), c0, idx.to(DEV), cnt.to(DEV), p, want_lse=True)
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)     # the key-split merge is deterministic
     ref_o, ref_lse = oesa.sparse_attn(_np(q), _np(k), _np(v), c0, idx.numpy(), cnt.numpy(), n_init, window)
     assert max_abs(_np(o), ref_o) <= ATOL_BF16
     assert max_abs(lse.cpu().numpy(), ref_lse) <= 2e-2
