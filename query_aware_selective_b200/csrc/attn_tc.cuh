@@ -110,16 +110,16 @@ __device__ __forceinline__ void gather_tile(uint32_t dst, const CUtensorMap* tm,
   tma_gather4(d + kBlkBytes, tm, 64, r[0], r[1], r[2], r[3], bar);
 }
 
-// One loader warp streams the key tiles j0 .. j0 + nt - 1 of one operand (K or V)
-// through its NST stages (the u-th of them, tile j0 + u, in stage u % NST, the
-// barrier's u / NST-th phase). The rows of the next tile are looked up (4 per lane,
+// One loader warp streams nt key tiles of one operand (K or V), tiles j0, j0 + js,
+// j0 + 2 js, ..., through its NST stages (the u-th of them, tile j0 + u js, in stage
+// u % NST, the barrier's u / NST-th phase). The rows of the next tile are looked up (4 per lane,
 // consecutive keys, so a gathered index list is read coalesced) while the current one
 // waits for its stage.
 template <int NST, class Problem>
 __device__ __forceinline__ void stream_kv(const Problem& prob, const CUtensorMap* tm_rows, const CUtensorMap* tm_box,
                                           const CUtensorMap* tm_staged, uint32_t stage0, uint64_t* full,
                                           uint64_t* empty, int nt, int64_t n_keys, int lane,
-                                          volatile int* abort_flag, unsigned site, int j0 = 0) {
+                                          volatile int* abort_flag, unsigned site, int j0 = 0, int js = 1) {
   int32_t cur[4], nxt[4];
   auto fetch = [&](int j, int32_t* out) {
 #pragma unroll
@@ -141,8 +141,8 @@ __device__ __forceinline__ void stream_kv(const Problem& prob, const CUtensorMap
 #pragma unroll
     for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
     if (u + 1 < nt) {
-      box_next = prob.kv_box(j0 + u + 1, &by, &bz);
-      if (!box_next) fetch(j0 + u + 1, nxt);
+      box_next = prob.kv_box(j0 + (u + 1) * js, &by, &bz);
+      if (!box_next) fetch(j0 + (u + 1) * js, nxt);
     }
     bool ok = mbar_wait(&empty[s], ph ^ 1, abort_flag, site);
     if (!__all_sync(0xffffffffu, ok)) return;

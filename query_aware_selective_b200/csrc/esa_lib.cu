@@ -1219,7 +1219,7 @@ MobaWs carve_moba(void* ws, int which, int32_t batch, int64_t seq, int32_t heads
   const int64_t nb = cdiv(seq, block);
   w.n_lists = (int64_t)batch * heads * nb;
   w.pairs = moba_pairs(seq, block, topk) * batch * heads;
-  w.max_tiles = cdiv(w.pairs, esa::kTcRows) + w.n_lists;
+  w.max_tiles = cdiv(w.pairs, 2 * esa::kTcRows) + w.n_lists;   // units of a pair of 128-row tiles
   if (which == 0 || which == 2) w.kbar = c.take<float>((size_t)batch * heads * nb * d);
   if (which == 2) w.blocks = c.take<int16_t>((size_t)batch * seq * heads * (topk + 1));
   if (which >= 1) {
@@ -1285,8 +1285,8 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
   const float sl2 = scale * 1.4426950408889634f;
   static const char what = 0;
   const esa_status_t sa = once_per_context(&what, [] {
-    esa_status_t st = set_max_smem(esa::attn_tc_kernel<esa::MobaPastProblem>, esa::kTcSmemBytes);
-    if (st == ESA_OK) st = set_max_smem(esa::attn_tc_kernel<esa::MobaCurrentProblem>, esa::kTcSmemBytes);
+    esa_status_t st = set_max_smem(esa::attn_pp_kernel<esa::MobaPastProblem>, esa::kPpSmemBytes);
+    if (st == ESA_OK) st = set_max_smem(esa::attn_pp_kernel<esa::MobaCurrentProblem>, esa::kPpSmemBytes);
     return st;
   });
   if (sa != ESA_OK) return sa;
@@ -1305,7 +1305,7 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
     esa::moba_list_kernel<<<lgrid, esa::kMobaListThreads, lsmem, s>>>(blocks, seq, heads, block, nb, topk, 0, w.cnt,
                                                                       w.off, w.fill, w.list);
     ESA_LAUNCH_CHECK("moba_list_kernel(count)");
-    esa::moba_scan_kernel<<<1, 1024, 0, s>>>(w.cnt, w.n_lists, w.off, w.tile_off, w.totals);
+    esa::moba_scan_kernel<<<1, 1024, 0, s>>>(w.cnt, w.n_lists, w.off, w.tile_off, w.totals, 2 * esa::kTcRows);
     ESA_LAUNCH_CHECK("moba_scan_kernel");
     esa::moba_list_kernel<<<lgrid, esa::kMobaListThreads, lsmem, s>>>(blocks, seq, heads, block, nb, topk, 1, w.cnt,
                                                                       w.off, w.fill, w.list);
@@ -1327,9 +1327,9 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
     pp.topk = topk;
     pp.n_lists = w.n_lists;
     pp.sl2 = sl2;
-    esa::attn_tc_kernel<esa::MobaPastProblem><<<(unsigned)w.max_tiles, esa::kTcThreads, esa::kTcSmemBytes, s>>>(
-        tq, tk, tv, bq, bk, bv, bk, bv, pp);
-    ESA_LAUNCH_CHECK("attn_tc_kernel<moba past>");
+    esa::attn_pp_kernel<esa::MobaPastProblem><<<(unsigned)w.max_tiles, esa::kPpThreads, esa::kPpSmemBytes, s>>>(
+        tq, tk, tv, bq, bk, bv, bk, bv, pp, 1);
+    ESA_LAUNCH_CHECK("attn_pp_kernel<moba past>");
   }
   esa::MobaCurrentProblem cp{};
   cp.q = static_cast<const __nv_bfloat16*>(q);
@@ -1346,10 +1346,10 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
   cp.topk = topk;
   cp.tiles_per_block = (int)cdiv(block, esa::kTcRows);
   cp.sl2 = sl2;
-  esa::attn_tc_kernel<esa::MobaCurrentProblem>
-      <<<dim3(cp.tiles_per_block * nb, heads, batch), esa::kTcThreads, esa::kTcSmemBytes, s>>>(tq, tk, tv, bq, bk, bv,
-                                                                                            bk, bv, cp);
-  ESA_LAUNCH_CHECK("attn_tc_kernel<moba current>");
+  esa::attn_pp_kernel<esa::MobaCurrentProblem>
+      <<<dim3((unsigned)(cdiv(cp.tiles_per_block, 2) * nb), heads, batch), esa::kPpThreads, esa::kPpSmemBytes, s>>>(
+          tq, tk, tv, bq, bk, bv, bk, bv, cp, 1);
+  ESA_LAUNCH_CHECK("attn_pp_kernel<moba current>");
   return ESA_OK;
 }
 

@@ -196,10 +196,11 @@ __global__ void __launch_bounds__(kMobaListThreads) moba_list_kernel(const int16
   }
 }
 
-// Exclusive scans over all lists: entry offsets and 128-row tile offsets. One CTA.
+// Exclusive scans over all lists: entry offsets and offsets of units of unit_rows rows
+// (a pair of 128-row tiles: 256). One CTA.
 __global__ void __launch_bounds__(1024) moba_scan_kernel(const uint32_t* __restrict__ cnt, int64_t n_lists,
                                                          uint32_t* __restrict__ off, uint32_t* __restrict__ tile_off,
-                                                         uint32_t* __restrict__ totals) {
+                                                         uint32_t* __restrict__ totals, uint32_t unit_rows) {
   using Scan = cub::BlockScan<uint32_t, 1024>;
   __shared__ typename Scan::TempStorage t1, t2;
   __shared__ uint32_t carry_e, carry_t;
@@ -208,7 +209,7 @@ __global__ void __launch_bounds__(1024) moba_scan_kernel(const uint32_t* __restr
   for (int64_t base = 0; base < n_lists; base += 1024) {
     const int64_t i = base + threadIdx.x;
     const uint32_t c = i < n_lists ? cnt[i] : 0u;
-    const uint32_t t = (c + kTcRows - 1) / kTcRows;
+    const uint32_t t = (c + unit_rows - 1) / unit_rows;
     uint32_t ec, tc, es, ts;
     Scan(t1).ExclusiveSum(c, ec, es);
     Scan(t2).ExclusiveSum(t, tc, ts);
@@ -236,7 +237,7 @@ struct MobaPastProblem {
   const __nv_bfloat16* v;
   __nv_bfloat16* part_o;
   float* part_lse;
-  const uint32_t* tile_off;   // [n_lists + 1]
+  const uint32_t* tile_off;   // [n_lists + 1], in pairs of 128-row tiles
   const uint32_t* off;        // [n_lists]
   const uint32_t* cnt;        // [n_lists]
   const uint32_t* list;       // packed (p << 4 | slot)
@@ -248,21 +249,23 @@ struct MobaPastProblem {
   int b, h, blk;
   uint32_t e0, n_rows;
 
-  __device__ bool setup() {
-    const uint32_t tile = blockIdx.x;
-    if (tile >= tile_off[n_lists]) return false;
-    int64_t lo = 0, hi = n_lists - 1;       // last list with tile_off <= tile
+  // tile = 2 pair + t: half t of the pair-th 256-row unit (units numbered over the lists)
+  __device__ bool setup_at(int tile) {
+    const uint32_t pair = (uint32_t)tile >> 1, t = (uint32_t)tile & 1u;
+    if (pair >= tile_off[n_lists]) return false;
+    int64_t lo = 0, hi = n_lists - 1;       // last list with tile_off <= pair
     while (lo < hi) {
       const int64_t mid = (lo + hi + 1) / 2;
-      if (tile_off[mid] <= tile) lo = mid; else hi = mid - 1;
+      if (tile_off[mid] <= pair) lo = mid; else hi = mid - 1;
     }
     const int64_t li = lo;
+    const uint32_t start = (pair - tile_off[li]) * 2 * kTcRows + t * kTcRows;
+    if (start >= cnt[li]) return false;
     blk = (int)(li % n_blocks);
     h = (int)((li / n_blocks) % heads);
     b = (int)(li / ((int64_t)n_blocks * heads));
-    const uint32_t t_in = tile - tile_off[li];
-    e0 = off[li] + t_in * kTcRows;
-    n_rows = min((uint32_t)kTcRows, cnt[li] - t_in * kTcRows);
+    e0 = off[li] + start;
+    n_rows = min((uint32_t)kTcRows, cnt[li] - start);
     return true;
   }
   __device__ int32_t q_row(int r) const {
@@ -303,8 +306,9 @@ struct MobaPastProblem {
   }
 };
 
-// Current block: grid (tiles_per_block * n_blocks, H, B); rows = 128 consecutive
-// queries of one head inside one block; keys = the block up to each query (causal).
+// Current block: grid (pairs_per_block * n_blocks, H, B), a pair = two consecutive
+// 128-row tiles of one block; rows = 128 consecutive queries of one head inside one
+// block; keys = the block up to each query (causal).
 struct MobaCurrentProblem {
   const __nv_bfloat16* q;
   const __nv_bfloat16* k;
@@ -319,9 +323,13 @@ struct MobaCurrentProblem {
   int b, h, blk;
   int64_t p0, kb0, nrows;
 
-  __device__ bool setup() {
-    blk = blockIdx.x / tiles_per_block;
-    const int t = blockIdx.x % tiles_per_block;
+  // tile = 2 pair + t: tile 2 (pair % pairs_per_block) + t of block pair / pairs_per_block
+  __device__ bool setup_at(int tile) {
+    const int ppb = (tiles_per_block + 1) / 2;
+    const int pair = tile >> 1;
+    blk = pair / ppb;
+    const int t = (pair % ppb) * 2 + (tile & 1);
+    if (t >= tiles_per_block) return false;
     h = blockIdx.y;
     b = blockIdx.z;
     kb0 = (int64_t)blk * block;

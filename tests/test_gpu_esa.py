@@ -250,7 +250,7 @@ def test_sparse_attn_decode_parity(batch, n_cap, hq, hkv, n_init, window, topk):
     (1, 512, 5000, 4488, 32, 8, 128, 2048, 1024), # a full chunk, several key tiles
     (1, 96, 4000, 333, 16, 4, 128, 512, 2048),    # short middle: full causal attention
     (10, 64, 1500, 1000, 32, 8, 16, 256, 256),    # 80 tile pairs: no key split
-    (5, 64, 2500, 2000, 32, 8, 64, 512, 512),     # 40 tile pairs: three key parts per pair
+    (5, 64, 2500, 2000, 32, 8, 64, 512, 512),     # 40 tile pairs: two key parts per pair
 ])
 def test_sparse_attn_tensor_core_parity(batch, lq, n_cap, c0, hq, hkv, n_init, window, topk):
     p = qas.params(n_init, window, topk, 2, 10.0)
