@@ -2,7 +2,7 @@
 // in ping-pong (sm_100a tcgen05).
 //
 // One CTA computes two tiles of 128 query rows (Q0, Q1: consecutive row tiles that
-// share their key list) against the key tiles of its part of that list, 128 keys a step.
+// share their key list) against that list, 128 keys a step.
 // Each key tile is loaded once and used by both query tiles:
 //   S_t = Q_t K_j^T          tcgen05.mma kind::f16 (bf16 in, fp32 accumulate), TMEM
 //   P_t = exp2(S_t c - m)    softmax warpgroup t reads S_t from TMEM, writes bf16 P_t
@@ -31,20 +31,10 @@
 // (and O, l rescaled) only when a tile's maximum exceeds it by more than 2^8, so most
 // tiles skip the rescale and P stays <= 2^8 (exact softmax either way: o = O / l).
 //
-// Key split: with n_split > 1 (2 or 4) the n_split CTAs of one tile pair form a
-// cluster and share the pair's key tiles (part s takes tiles s, s + n_split, ...: each
-// part gets its share of the masked tiles at the end of the list, so the parts finish
-// together). At the end each part owns 256 / n_split of the pair's rows:
-// the other parts stage their unnormalised (O, m, l) for those rows in their own shared
-// memory and send each part's block with one bulk copy into that part's shared memory
-// (into the tile buffers, free by then; an mbarrier counts the bytes in), and it merges
-// the parts by log-sum-exp, in part order, and stores the rows. This fills the 148 SMs
-// when there are fewer tile pairs than SMs.
-//
 // The problem policy is the one of attn_tc_kernel (attn_tc.cuh), with
 // `bool setup_at(int tile)` in place of setup(): per-CTA fields for row tile `tile`
-// (blockIdx.y, blockIdx.z as in attn_tc_kernel), false = no such tile. store() takes
-// 64 columns at a time.
+// (2 blockIdx.x or 2 blockIdx.x + 1; blockIdx.y, blockIdx.z as the policy defines
+// them), false = no such tile. store() takes 64 columns at a time.
 #pragma once
 #include <cuda.h>
 
@@ -63,22 +53,11 @@ constexpr uint32_t kPpCtrlBytes = 1024;
 constexpr uint32_t kPpSmemBytes = (2 + kPpKStages + kPpVStages) * kTileBytes + kPpCtrlBytes;
 static_assert(kPpSmemBytes <= 232448, "exceeds the 227 KB of shared memory per CTA");
 static_assert(kTcD / kTcSplit == 64, "store() takes 64 columns");
-// one row sent to the merging part: O (128 floats), m, l, two floats of padding
-// (16-byte rows, 33 of them: a warp's 16-byte stores to 32 rows meet no bank conflict)
-constexpr int kPpPartStride = kTcD + 4;
-// the received blocks, then the staged ones: 2 (n_split - 1) blocks of 256 / n_split
-// rows each
-// (then the merge coefficients, 8 floats a merged row)
-static_assert(2 * 1 * 128 * kPpPartStride * 4 + 128 * 32 <= (2 + kPpKStages + kPpVStages) * kTileBytes &&
-                  2 * 3 * 64 * kPpPartStride * 4 + 64 * 32 <= (2 + kPpKStages + kPpVStages) * kTileBytes,
-              "the blocks fit in the tile buffers");
-
 struct PpSmem {
   uint64_t q_full;
   uint64_t k_full[kPpKStages], k_empty[kPpKStages], v_full[kPpVStages], v_empty[kPpVStages];
   uint64_t s_full[2], p_full[2], pv_full[2];
   uint64_t mma_done;
-  uint64_t recv_full;                                // the other parts' blocks are in
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -90,7 +69,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tb_q,
                    const __grid_constant__ CUtensorMap tb_k, const __grid_constant__ CUtensorMap tb_v,
                    const __grid_constant__ CUtensorMap ts_k, const __grid_constant__ CUtensorMap ts_v,
-                   Problem prob0, int n_split) {
+                   Problem prob0) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   if (smem_u32(smem) & 1023u) {
@@ -103,7 +82,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   PpSmem& sm = *reinterpret_cast<PpSmem*>(smem + (2 + kPpKStages + kPpVStages) * kTileBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = blockIdx.x / n_split, part = blockIdx.x % n_split;   // part = rank in the cluster
+  const int pair = blockIdx.x;
   // pk: the policy of the pair's later tile (it sees the most keys), which the loaders
   // use for the key list; each role sets up its own copy for its tile below
   Problem pk = prob0;
@@ -116,7 +95,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   }
   const int64_t n_keys = pk.n_keys();
   const int nt = (int)((n_keys + kTcKeys - 1) / kTcKeys);
-  const int n = nt > part ? (nt - part + n_split - 1) / n_split : 0;   // tiles part + u n_split
+  const int n = nt;
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
@@ -134,7 +113,6 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       mbar_init(&sm.pv_full[t], 1);
     }
     mbar_init(&sm.mma_done, 1);
-    mbar_init(&sm.recv_full, 1);
     sm.abort_flag = 0;
     fence_barrier_init();
   }
@@ -174,12 +152,10 @@ __global__ void __launch_bounds__(kPpThreads, 1)
           }
         }
       }
-      stream_kv<kPpKStages>(pk, &tm_k, &tb_k, &ts_k, sK, sm.k_full, sm.k_empty, n, n_keys, lane, abort_flag, 121,
-                            part, n_split);
+      stream_kv<kPpKStages>(pk, &tm_k, &tb_k, &ts_k, sK, sm.k_full, sm.k_empty, n, n_keys, lane, abort_flag, 121);
     } else if (warp == kPpVWarp) {
       // -------------------------------------------------------------- V loader
-      stream_kv<kPpVStages>(pk, &tm_v, &tb_v, &ts_v, sV, sm.v_full, sm.v_empty, n, n_keys, lane, abort_flag, 122,
-                            part, n_split);
+      stream_kv<kPpVStages>(pk, &tm_v, &tb_v, &ts_v, sV, sm.v_full, sm.v_empty, n, n_keys, lane, abort_flag, 122);
     } else if (warp == kPpMmaWarp && n > 0) {
       // -------------------------------------------------------------- MMA issuer
       // The whole warp runs the loop (converged: the warp-uniform descriptors stay in
@@ -255,10 +231,6 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       mbar_wait(&sm.mma_done, 0, abort_flag, 128, /*respect_abort=*/false);
     }
     __syncwarp();
-    if (n_split > 1) {                               // the epilogue's two cluster barriers
-      cluster_sync_all();
-      cluster_sync_all();
-    }
   } else {
     setmaxnreg_inc<kPpRegsSoftmax>();
     // ---------------------------------------------------------------- softmax (rows)
@@ -285,12 +257,10 @@ __global__ void __launch_bounds__(kPpThreads, 1)
         lim = pr.limit(r);
         sl2 = pr.scale_log2();
       }
-      // key tiles j < j_mask have no masked key for any row of this warp (keys
-      // j * 128 + e with e <= limit - j * 128 are visible; limits are below 2^31); this
-      // part's u-th tile is j = part + u n_split
+      // key tiles u < u_mask have no masked key for any row of this warp (keys
+      // u * 128 + e with e <= limit - u * 128 are visible; limits are below 2^31)
       const int lim_min = __reduce_min_sync(0xffffffffu, (int)lim);
-      const int j_mask = lim_min >= kTcKeys - 1 ? (lim_min - (kTcKeys - 1)) / kTcKeys + 1 : 0;
-      const int u_mask = j_mask > part ? (j_mask - part + n_split - 1) / n_split : 0;
+      const int u_mask = lim_min >= kTcKeys - 1 ? (lim_min - (kTcKeys - 1)) / kTcKeys + 1 : 0;
       if constexpr (HasPrefetch<Problem>::value) {
         Problem pf = prob0;
         pf.setup_at(2 * pair + t);
@@ -366,7 +336,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
         float lt;
         if (u >= u_mask) {
           // the causal cut: keys j * 128 + e with e <= rem are visible (rem >= 127: all)
-          const int64_t rem64 = lim - (int64_t)(part + u * n_split) * kTcKeys;
+          const int64_t rem64 = lim - (int64_t)u * kTcKeys;
           const int rem = rem64 < 0 ? -1 : (rem64 >= kTcKeys ? kTcKeys : (int)rem64);
 #pragma unroll
           for (int e = 0; e < kTcKeys; ++e) v[e] = e <= rem ? v[e] : -INFINITY;
@@ -388,140 +358,19 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     __syncwarp();
 
     // -------------------------------------------------------------- epilogue
-    // O_t complete, then store the rows, or merge the key parts
-    bool fin = active && ok;
-    if (fin && n > 0) fin = mbar_wait_warp(&sm.pv_full[t], (n - 1) & 1, abort_flag, 130);
-    const bool have_o = fin && n > 0;                // warp-uniform (the tcgen05.ld below)
-    if (have_o) tc_fence_after();
-    if (!fin) {
-      m = -INFINITY;
-      l = 0.f;
-    }
-    // 64 columns of this thread's O row (zero when there is none)
-    auto load_half = [&](int h, float* o) {
-      if (have_o) {
+    // O_t complete, then the rows are stored, 64 columns at a time from TMEM
+    if (active && ok && n > 0 && mbar_wait_warp(&sm.pv_full[t], (n - 1) & 1, abort_flag, 130)) {
+      tc_fence_after();
+      Problem pr = prob0;
+      pr.setup_at(2 * pair + t);
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float o[64];
         tmem_ld32(o_addr + h * 64, o);
         tmem_ld32(o_addr + h * 64 + 32, o + 32);
         tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int e = 0; e < 64; ++e) o[e] = 0.f;
+        pr.store(r, h * 64, o, m, l);
       }
-    };
-    if (n_split == 1) {
-      Problem pr = prob0;
-      pr.setup_at(2 * pair + t);
-      if (fin) {
-#pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          float o[64];
-          load_half(h, o);
-          pr.store(r, h * 64, o, m, l);
-        }
-      }
-    } else {
-      // every role of every part is done with its tile buffers (the MMA warp waited for
-      // its last MMA, every load was consumed): they take the blocks now. Both
-      // warpgroups work on every row here, warpgroup w on columns 64 w .. + 63 (a warp
-      // reads the TMEM lanes of its quadrant, whichever tile they belong to).
-      // the rows this part merges: tile tm, quadrants of rows part R .. + R - 1 (its
-      // policy set up before the barrier: the setup's loads wait beside it)
-      const int R = 256 / n_split;                   // rows each part merges (a multiple of 32)
-      const int tm = part * R / 128;
-      Problem pm = prob0;
-      pm.setup_at(2 * pair + tm);
-      cluster_sync_all();
-      tc_fence_after();                              // (every MMA completed before the barrier)
-      const uint32_t block = (uint32_t)R * kPpPartStride * 4;
-      const uint32_t recv = sQ, stage = sQ + (n_split - 1) * block;
-      float* coef = reinterpret_cast<float*>(smem + 2 * (n_split - 1) * block);   // [R][8]: M, L, a_q
-      const int w = t;                               // this thread's column half
-      const bool o_ok = __all_sync(0xffffffffu, n > 0 && *abort_flag == 0);   // O_0, O_1 hold results
-      auto ld_half = [&](int tt, float* o) {         // columns 64 w .. + 63 of O_tt, this row
-        if (o_ok) {
-          const uint32_t a = lane_base + 256 + tt * 128 + w * 64;
-          tmem_ld32(a, o);
-          tmem_ld32(a + 32, o + 32);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 64; ++e) o[e] = 0.f;
-        }
-      };
-      // stage the rows of the other parts: row tt * 128 + r goes to part (row / R)
-      for (int tt = 0; tt < (has1 ? 2 : 1); ++tt) {
-        const int row = tt * 128 + r, dest = row / R;              // warp-uniform
-        if (dest == part) continue;
-        const uint32_t dst = stage + (dest < part ? dest : dest - 1) * block + (row - dest * R) * kPpPartStride * 4;
-        float o[64];
-        ld_half(tt, o);
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          st_shared_f4(dst + (w * 16 + c) * 16, o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-        if (w == tt) st_shared_f4(dst + kTcD * 4, m, l, 0.f, 0.f);  // this thread's own row
-      }
-      fence_proxy_async();                           // the staged rows, to the bulk copies
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(&sm.recv_full, (n_split - 1) * block);
-        for (int d = 0; d < n_split; ++d) {
-          if (d == part) continue;
-          const uint32_t src = stage + (d < part ? d : d - 1) * block;
-          const uint32_t dst = recv + (part < d ? part : part - 1) * block;   // part's slot at d
-          bulk_copy_to_cluster(dsmem_map(dst, d), src, block, dsmem_map(smem_u32(&sm.recv_full), d));
-        }
-      }
-      const int row = tm * 128 + r;
-      const bool mine = row / R == part && (tm == 0 || has1);     // warp-uniform
-      const bool got = mbar_wait_warp(&sm.recv_full, 0, abort_flag, 131);
-      // part q's row: this thread's own for q == part, else received slot q (- 1 past part)
-      const float* rv = reinterpret_cast<const float*>(smem) + (row - part * R) * kPpPartStride;
-      auto slot = [&](int q) { return rv + (q < part ? q : q - 1) * R * kPpPartStride; };
-      float* cf = coef + (row - part * R) * 8;
-      if (mine && got && w == tm) {
-        // the merge coefficients, from the thread that holds this row's own m and l
-        float M = m;
-        for (int q = 0; q < n_split; ++q)
-          if (q != part) M = fmaxf(M, slot(q)[kTcD]);
-        const float M_use = M == -INFINITY ? 0.f : M;
-        float L = 0.f;
-        for (int q = 0; q < n_split; ++q) {         // part order: the same sum whatever the timing
-          const float a = q == part ? fast_exp2(m - M_use) : fast_exp2(slot(q)[kTcD] - M_use);   // -inf: 0
-          L += a * (q == part ? l : slot(q)[kTcD + 1]);
-          cf[2 + q] = a;
-        }
-        cf[0] = M;
-        cf[1] = L;
-      }
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (mine && got) {
-        float own[64], o[64];
-        ld_half(tm, own);
-#pragma unroll
-        for (int e = 0; e < 64; ++e) o[e] = 0.f;
-#pragma unroll 1
-        for (int q = 0; q < n_split; ++q) {
-          const float a = cf[2 + q];
-          if (q == part) {
-#pragma unroll
-            for (int e = 0; e < 64; ++e) o[e] += a * own[e];
-          } else {
-            const float4* s4 = reinterpret_cast<const float4*>(slot(q) + w * 64);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const float4 x = s4[c];
-              o[4 * c] += a * x.x;
-              o[4 * c + 1] += a * x.y;
-              o[4 * c + 2] += a * x.z;
-              o[4 * c + 3] += a * x.w;
-            }
-          }
-        }
-        pm.store(r, w * 64, o, cf[0], cf[1]);
-      }
-      // no part leaves while a copy may still read its staged blocks or write its own
-      // (every part has waited for its blocks when it gets here)
-      cluster_sync_all();
     }
   }
   tc_fence_before();

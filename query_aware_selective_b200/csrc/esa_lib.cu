@@ -835,21 +835,6 @@ struct AttnPlan {
   size_t ws_bytes;
 };
 
-// Grid of the paired-tile attention: tile pairs per (KV head, sequence), and the key
-// parts (1, 2 or 4: the CTAs of a pair form a cluster) each pair is split into, the
-// most that keep the CTAs within one wave on the 148 SMs.
-struct PpGrid {
-  int n_pairs;
-  int n_split;
-};
-PpGrid pp_grid(int64_t batch, int64_t lq, int g, int64_t hkv) {
-  PpGrid pg{};
-  pg.n_pairs = (int)cdiv(cdiv(lq * g, esa::kTcRows), 2);
-  const int64_t pairs = (int64_t)pg.n_pairs * hkv * batch;
-  pg.n_split = pairs * 4 <= 148 ? 4 : (pairs * 2 <= 148 ? 2 : 1);
-  return pg;
-}
-
 AttnPlan plan_attn(int32_t batch, int32_t lq, int64_t c0, int32_t hq, int32_t hkv, int32_t head_dim, esa_dtype_t dt,
                    const esa_params_t& p) {
   AttnPlan pl{};
@@ -1022,7 +1007,7 @@ esa_status_t sparse_attn_impl(const void* q, const void* k, const void* v, esa_d
   }
   if (pl.tc) {
     static const char what = 0;
-    st = once_per_context(&what, [] { return set_max_smem(esa::attn_pp_kernel<esa::EsaTcProblem>, esa::kPpSmemBytes); });
+    st = once_per_context(&what, [] { return set_max_smem(esa::attn_tc_kernel<esa::EsaTcProblem>, esa::kTcSmemBytes); });
     if (st != ESA_OK) return st;
     esa::EsaTcProblem pr{};
     pr.q = static_cast<const __nv_bfloat16*>(q);
@@ -1063,22 +1048,10 @@ esa_status_t sparse_attn_impl(const void* q, const void* k, const void* v, esa_d
     if ((st = make_tmap_box_bf16(&bq, q, hq, (uint64_t)batch * lq, g, esa::kTcRows / g)) != ESA_OK) return st;
     if ((st = make_tmap_box_bf16(&bk, k, hkv, (uint64_t)batch * n_cap, 1, esa::kTcKeys)) != ESA_OK) return st;
     if ((st = make_tmap_box_bf16(&bv, v, hkv, (uint64_t)batch * n_cap, 1, esa::kTcKeys)) != ESA_OK) return st;
-    const PpGrid pg = pp_grid(batch, lq, g, hkv);    // (one query per sequence never takes this path)
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(pg.n_pairs * pg.n_split), (unsigned)hkv, (unsigned)batch);
-    cfg.blockDim = dim3(esa::kPpThreads);
-    cfg.dynamicSmemBytes = esa::kPpSmemBytes;
-    cfg.stream = s;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = (unsigned)pg.n_split;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, esa::attn_pp_kernel<esa::EsaTcProblem>, tq, tk, tv, bq, bk, bv, sk, sv, pr,
-                       pg.n_split);
-    ESA_LAUNCH_CHECK("attn_pp_kernel<esa>");
+    dim3 grid((unsigned)cdiv((int64_t)lq * g, esa::kTcRows), hkv, batch);
+    esa::attn_tc_kernel<esa::EsaTcProblem><<<grid, esa::kTcThreads, esa::kTcSmemBytes, s>>>(tq, tk, tv, bq, bk, bv,
+                                                                                           sk, sv, pr);
+    ESA_LAUNCH_CHECK("attn_tc_kernel<esa>");
     return ok();
   }
   if (pl.dec) {
@@ -1328,7 +1301,7 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
     pp.n_lists = w.n_lists;
     pp.sl2 = sl2;
     esa::attn_pp_kernel<esa::MobaPastProblem><<<(unsigned)w.max_tiles, esa::kPpThreads, esa::kPpSmemBytes, s>>>(
-        tq, tk, tv, bq, bk, bv, bk, bv, pp, 1);
+        tq, tk, tv, bq, bk, bv, bk, bv, pp);
     ESA_LAUNCH_CHECK("attn_pp_kernel<moba past>");
   }
   esa::MobaCurrentProblem cp{};
@@ -1348,7 +1321,7 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
   cp.sl2 = sl2;
   esa::attn_pp_kernel<esa::MobaCurrentProblem>
       <<<dim3((unsigned)(cdiv(cp.tiles_per_block, 2) * nb), heads, batch), esa::kPpThreads, esa::kPpSmemBytes, s>>>(
-          tq, tk, tv, bq, bk, bv, bk, bv, cp, 1);
+          tq, tk, tv, bq, bk, bv, bk, bv, cp);
   ESA_LAUNCH_CHECK("attn_pp_kernel<moba current>");
   return ESA_OK;
 }
