@@ -100,23 +100,35 @@ __global__ void __launch_bounds__(128) moba_gate_kernel(const T* __restrict__ q,
     __syncthreads();
     if (!valid) continue;
     const int cend = min(CB, cur - c0);
-    for (int c = 0; c < cend; ++c) {
-      float acc = 0.f;
+    // two blocks at a time, four partial sums each: eight independent FMA chains (one
+    // chain of D dependent FMAs per block left the FMA pipe waiting on its latency)
+    for (int c = 0; c < cend; c += 2) {
+      float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+      const int c1 = c + 1 < CB ? c + 1 : c;       // (a block past cend is computed, not kept)
 #pragma unroll
       for (int e = 0; e < D / 4; ++e) {
-        const float4 w = kb[c][e];
-        acc = fmaf(qv[4 * e], w.x, acc);
-        acc = fmaf(qv[4 * e + 1], w.y, acc);
-        acc = fmaf(qv[4 * e + 2], w.z, acc);
-        acc = fmaf(qv[4 * e + 3], w.w, acc);
+        const float4 w = kb[c][e], x = kb[c1][e];
+        a0[0] = fmaf(qv[4 * e], w.x, a0[0]);
+        a0[1] = fmaf(qv[4 * e + 1], w.y, a0[1]);
+        a0[2] = fmaf(qv[4 * e + 2], w.z, a0[2]);
+        a0[3] = fmaf(qv[4 * e + 3], w.w, a0[3]);
+        a1[0] = fmaf(qv[4 * e], x.x, a1[0]);
+        a1[1] = fmaf(qv[4 * e + 1], x.y, a1[1]);
+        a1[2] = fmaf(qv[4 * e + 2], x.z, a1[2]);
+        a1[3] = fmaf(qv[4 * e + 3], x.w, a1[3]);
       }
-      float v = acc;
-      int id = c0 + c;
+      const float s2[2] = {(a0[0] + a0[1]) + (a0[2] + a0[3]), (a1[0] + a1[1]) + (a1[2] + a1[3])};
 #pragma unroll
-      for (int i = 0; i < TK; ++i) {
-        if (i < topk && v > vals[i]) {
-          const float tv = vals[i]; vals[i] = v; v = tv;
-          const int ti = ids[i]; ids[i] = id; id = ti;
+      for (int q2 = 0; q2 < 2; ++q2) {
+        if (c + q2 >= cend) break;
+        float v = s2[q2];
+        int id = c0 + c + q2;
+#pragma unroll
+        for (int i = 0; i < TK; ++i) {
+          if (i < topk && v > vals[i]) {
+            const float tv = vals[i]; vals[i] = v; v = tv;
+            const int ti = ids[i]; ids[i] = id; id = ti;
+          }
         }
       }
     }
