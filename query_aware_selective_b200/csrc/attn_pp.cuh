@@ -96,9 +96,14 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   const int64_t n_keys = pk.n_keys();
   const int nt = (int)((n_keys + kTcKeys - 1) / kTcKeys);
   const int n = nt;
+  // Q tiles as TMA boxes (consecutive queries), or gathered rows: then each softmax
+  // thread copies its own row with 16-byte cp.async (a TMA gather4 moves 4 rows an
+  // instruction, and the 128 instructions of two tiles took about 11 us to land)
+  int qy = 0, qz = 0;
+  const bool q_tma = pk.q_box(&qy, &qz);
 
   if (threadIdx.x == 0) {
-    mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.q_full, q_tma ? 1 : 256);          // the TMA's arrival, or every softmax thread's
     for (int s = 0; s < kPpKStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
@@ -130,26 +135,16 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     setmaxnreg_dec<kPpRegsOther>();
     if (warp == kPpKWarp) {
       // -------------------------------------------------------------- Q + K loader
-      if (n > 0) {
-        if (lane == 0) mbar_arrive_expect_tx(&sm.q_full, (has1 ? 2u : 1u) * kTileBytes);
-        __syncwarp();
+      if (n > 0 && q_tma && lane == 0) {
+        mbar_arrive_expect_tx(&sm.q_full, (has1 ? 2u : 1u) * kTileBytes);
         for (int tq = 0; tq < (has1 ? 2 : 1); ++tq) {
           Problem pq = prob0;
           pq.setup_at(2 * pair + tq);
+          int y = 0, z = 0;
+          pq.q_box(&y, &z);
           const uint32_t dst = sQ + tq * kTileBytes;
-          int qy = 0, qz = 0;
-          if (pq.q_box(&qy, &qz)) {
-            if (lane == 0) {
-              tma_load_3d(dst, &tb_q, 0, qy, qz, &sm.q_full);
-              tma_load_3d(dst + kBlkBytes, &tb_q, 64, qy, qz, &sm.q_full);
-            }
-          } else {
-            int32_t qr[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) qr[q] = pq.q_row(lane * 4 + q);
-            const int32_t q_fallback = __shfl_sync(0xffffffffu, qr[0], 0);  // row 0 is always a real query
-            gather_tile(dst, &tm_q, qr, q_fallback, &sm.q_full, lane);
-          }
+          tma_load_3d(dst, &tb_q, 0, y, z, &sm.q_full);
+          tma_load_3d(dst + kBlkBytes, &tb_q, 64, y, z, &sm.q_full);
         }
       }
       stream_kv<kPpKStages>(pk, &tm_k, &tb_k, &ts_k, sK, sm.k_full, sm.k_empty, n, n_keys, lane, abort_flag, 121);
@@ -241,6 +236,24 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     const uint32_t s_addr = lane_base + t * 128, o_addr = lane_base + 256 + t * 128;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+    if (!q_tma) {
+      // this thread's query row into the 128-byte-swizzled Q tile (row r: 16-byte chunk c
+      // of 64-column block c / 8 at sw128_off(r, c % 8)); padding rows copy the tile's
+      // first row (a real query; its scores are never stored)
+      if (n > 0 && active) {
+        Problem pq = prob0;
+        pq.setup_at(2 * pair + t);
+        int32_t row = pq.q_row(r);
+        if (row < 0) row = pq.q_row(0);
+        const __nv_bfloat16* src = pq.q + (int64_t)row * kTcD;
+        const uint32_t dst = sQ + t * kTileBytes;
+#pragma unroll
+        for (int c = 0; c < kTcD / 8; ++c) cp_async16(dst + (c >> 3) * kBlkBytes + sw128_off(r, c & 7), src + c * 8, 16);
+        cp_async_wait_all();
+        fence_proxy_async();                         // written through the generic proxy, read by the MMA
+      }
+      mbar_arrive(&sm.q_full);
+    }
     // The tile maximum is needed only to decide a rescale (tile max > m + 2^8 in log2
     // units), so it is computed only when that can be the case: while m is not set yet,
     // in tiles with masked keys, or when the tile's sum of exp2(s c - m) exceeds 2^8
