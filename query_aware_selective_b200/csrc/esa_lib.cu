@@ -1169,6 +1169,7 @@ struct MobaWs {
   uint32_t* off;
   uint32_t* tile_off;
   uint32_t* totals;
+  uint32_t* unit_list;     // [max_tiles]: the list of each 256-row unit (n_lists past the last)
   uint32_t* list;
   __nv_bfloat16* part_o;   // past partials: [B, seq, H, topk, D] bf16, lse [B, seq, H, topk]
   float* part_lse;
@@ -1203,6 +1204,7 @@ MobaWs carve_moba(void* ws, int which, int32_t batch, int64_t seq, int32_t heads
     w.off = c.take<uint32_t>(w.n_lists);
     w.tile_off = c.take<uint32_t>(w.n_lists + 1);
     w.totals = c.take<uint32_t>(2);
+    w.unit_list = c.take<uint32_t>(w.max_tiles);
     w.list = c.take<uint32_t>(std::max<int64_t>(1, w.pairs));
     w.part_o = c.take<__nv_bfloat16>((size_t)batch * seq * heads * topk * d);
     w.part_lse = c.take<float>((size_t)batch * seq * heads * topk);
@@ -1278,7 +1280,8 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
     esa::moba_list_kernel<<<lgrid, esa::kMobaListThreads, lsmem, s>>>(blocks, seq, heads, block, nb, topk, 0, w.cnt,
                                                                       w.off, w.fill, w.list);
     ESA_LAUNCH_CHECK("moba_list_kernel(count)");
-    esa::moba_scan_kernel<<<1, 1024, 0, s>>>(w.cnt, w.n_lists, w.off, w.tile_off, w.totals, 2 * esa::kTcRows);
+    esa::moba_scan_kernel<<<1, 1024, 0, s>>>(w.cnt, w.n_lists, w.off, w.tile_off, w.totals, 2 * esa::kTcRows,
+                                             w.unit_list, w.max_tiles);
     ESA_LAUNCH_CHECK("moba_scan_kernel");
     esa::moba_list_kernel<<<lgrid, esa::kMobaListThreads, lsmem, s>>>(blocks, seq, heads, block, nb, topk, 1, w.cnt,
                                                                       w.off, w.fill, w.list);
@@ -1290,6 +1293,7 @@ esa_status_t moba_attn_launch(const MobaWs& w, const void* q, const void* k, con
     pp.part_o = w.part_o;
     pp.part_lse = w.part_lse;
     pp.tile_off = w.tile_off;
+    pp.unit_list = w.unit_list;
     pp.off = w.off;
     pp.cnt = w.cnt;
     pp.list = w.list;

@@ -209,10 +209,12 @@ __global__ void __launch_bounds__(kMobaListThreads) moba_list_kernel(const int16
 }
 
 // Exclusive scans over all lists: entry offsets and offsets of units of unit_rows rows
-// (a pair of 128-row tiles: 256). One CTA.
+// (a pair of 128-row tiles: 256); then unit_list[u] = the list of unit u (n_lists for
+// u past the last unit, up to n_units), so that a CTA finds its list with one load. One CTA.
 __global__ void __launch_bounds__(1024) moba_scan_kernel(const uint32_t* __restrict__ cnt, int64_t n_lists,
                                                          uint32_t* __restrict__ off, uint32_t* __restrict__ tile_off,
-                                                         uint32_t* __restrict__ totals, uint32_t unit_rows) {
+                                                         uint32_t* __restrict__ totals, uint32_t unit_rows,
+                                                         uint32_t* __restrict__ unit_list, int64_t n_units) {
   using Scan = cub::BlockScan<uint32_t, 1024>;
   __shared__ typename Scan::TempStorage t1, t2;
   __shared__ uint32_t carry_e, carry_t;
@@ -238,6 +240,10 @@ __global__ void __launch_bounds__(1024) moba_scan_kernel(const uint32_t* __restr
     totals[0] = carry_e;
     totals[1] = carry_t;
   }
+  __syncthreads();                                   // tile_off complete (this CTA wrote it)
+  for (int64_t i = threadIdx.x; i < n_lists; i += 1024)
+    for (uint32_t u = tile_off[i]; u < tile_off[i + 1] && u < n_units; ++u) unit_list[u] = (uint32_t)i;
+  for (int64_t u = (int64_t)carry_t + threadIdx.x; u < n_units; u += 1024) unit_list[u] = (uint32_t)n_lists;
 }
 
 // ------------------------------------------------------------------ TC problems --
@@ -250,6 +256,7 @@ struct MobaPastProblem {
   __nv_bfloat16* part_o;
   float* part_lse;
   const uint32_t* tile_off;   // [n_lists + 1], in pairs of 128-row tiles
+  const uint32_t* unit_list;  // [grid]: list of each pair (n_lists past the last)
   const uint32_t* off;        // [n_lists]
   const uint32_t* cnt;        // [n_lists]
   const uint32_t* list;       // packed (p << 4 | slot)
@@ -264,13 +271,8 @@ struct MobaPastProblem {
   // tile = 2 pair + t: half t of the pair-th 256-row unit (units numbered over the lists)
   __device__ bool setup_at(int tile) {
     const uint32_t pair = (uint32_t)tile >> 1, t = (uint32_t)tile & 1u;
-    if (pair >= tile_off[n_lists]) return false;
-    int64_t lo = 0, hi = n_lists - 1;       // last list with tile_off <= pair
-    while (lo < hi) {
-      const int64_t mid = (lo + hi + 1) / 2;
-      if (tile_off[mid] <= pair) lo = mid; else hi = mid - 1;
-    }
-    const int64_t li = lo;
+    const int64_t li = unit_list[pair];
+    if (li >= n_lists) return false;
     const uint32_t start = (pair - tile_off[li]) * 2 * kTcRows + t * kTcRows;
     if (start >= cnt[li]) return false;
     blk = (int)(li % n_blocks);
